@@ -1,0 +1,79 @@
+"""Byte accounting for the FlashLoop cross-loop cache and its decode kernels.
+
+Two parts:
+
+* the storage arithmetic the flozi guide "FlashLoop: store changes between
+  repeated passes" prints (section 1, Cell 1: bytes per (token, loop) of a BF16
+  cross-loop cache; section 3: ideal INT4 payload with a 64-token BF16 tail),
+  restated here so the figures can be checked;
+* the algorithmic bytes of one launch of each decode kernel: what must cross
+  HBM at least once, used as the numerator of achieved GB/s.
+
+Per-token costs of the packed INT4 layout (head dim 128, group 64): 64 B of key
+codes, 64 B of value codes, 8 B of value (scale, zero) and 8 B of key
+(scale, zero) amortised over the 64 tokens of a key group: 144 B per stored
+row, base or residual.  A BF16 tail row is 256 B of key plus 256 B of value.
+"""
+from __future__ import annotations
+
+GIB = 1024 ** 3
+HEAD_DIM = 128
+GROUP = 64
+CODE_ROW = HEAD_DIM // 2          # 64 B of packed 4-bit codes per row
+VSZ_ROW = 8                       # two (scale, zero) fp16 pairs per value row
+KSZ_GROUP = HEAD_DIM * 4          # (scale, zero) fp16 pair per channel per key group
+ROW_BYTES = 2 * CODE_ROW + VSZ_ROW + KSZ_GROUP // GROUP   # 144
+TAIL_ROW = 2 * HEAD_DIM * 2       # K + V in BF16
+
+
+def bf16_bytes_per_token_loop(layers: int, heads: int, head_dim: int = HEAD_DIM) -> int:
+    """K and V of one token in one loop, all layers, BF16."""
+    return layers * heads * head_dim * 2 * 2
+
+
+def bf16_cache_bytes(layers: int, heads: int, context: int, loops: int, head_dim: int = HEAD_DIM) -> int:
+    """A separate BF16 (K, V) per loop for every token."""
+    return bf16_bytes_per_token_loop(layers, heads, head_dim) * context * loops
+
+
+def ideal_int4_payload(bf16_total: float, loops: int, retained) -> float:
+    """INT4 codes only (no scales): a quarter of each loop's BF16 share, times the rows kept."""
+    return bf16_total / loops * (4 / 16) * sum(retained)
+
+
+def bf16_tail_extra(bf16_total: float, context: int, tail: int = 64) -> float:
+    """Extra bytes of keeping ``tail`` recent tokens in BF16 rather than INT4, every loop."""
+    return bf16_total * (tail / context) * (1 - 4 / 16)
+
+
+# ----------------------------------------------------------------------------
+# Algorithmic bytes per launch (one layer, all heads)
+# ----------------------------------------------------------------------------
+def dense_bytes(heads: int, n_q: int, n_tail: int, res_rows: int, keep_scores: bool) -> int:
+    """One dense-reader launch of loop r.
+
+    n_q quantised columns read their base rows, ``res_rows`` is the number of
+    residual rows of loops 2..r that belong to those columns, the tail rows are
+    BF16.  Plus q (BF16), o (fp32), and with ``keep_scores`` the per-column
+    log-score (fp32) and loop tag (u8) written for the selector.
+    """
+    per_head = (n_q + res_rows) * ROW_BYTES + n_tail * TAIL_ROW + HEAD_DIM * 2 + HEAD_DIM * 4
+    if keep_scores:
+        per_head += (n_q + n_tail) * 5
+    return heads * per_head
+
+
+def sparse_bytes(heads: int, cols_quant: int, res_rows: int, key_groups: int, cols_tail: int) -> int:
+    """One sparse-reader launch, summed over heads.
+
+    ``cols_quant``: selected quantised columns (over all heads); ``res_rows``:
+    residual rows those columns carry up to this loop; ``key_groups``: distinct
+    (store, key group) pairs the selected rows touch (512 B of key scales each);
+    ``cols_tail``: selected tail columns.  Each selected column also reads its
+    index (4 B), writes its new log-score and loop tag (5 B); per head q, m, u
+    and o are read or written.
+    """
+    row = 2 * CODE_ROW + VSZ_ROW
+    cols = cols_quant + cols_tail
+    return ((cols_quant + res_rows) * row + key_groups * KSZ_GROUP + cols_tail * TAIL_ROW
+            + cols * (4 + 5) + heads * (HEAD_DIM * 2 + 4 + HEAD_DIM * 4 * 2))
