@@ -1,0 +1,476 @@
+"""Benchmark of the FlashLoop decode hot path on B200 (one JSON line on rank 0).
+
+Workload (default): a 48-layer x 16-head x head-dim-128 cross-loop cache at 32K
+context with 4 loops (Ouro-2.6B-shaped), INT4 base + nested 25 % / 10 % residuals
++ BF16 tail, synthetic seeded data.  A *step* decodes one token through every
+layer and loop in loop-major order (loop r runs all layers before loop r+1):
+
+    append / flush tail -> loop 1 dense (48) -> loop 2 dense (48, keeps scores)
+    -> select for loop 3 (all layers, one launch) -> loop 3 sparse (48)
+    -> select for loop 4 (one launch) -> loop 4 sparse (48)
+
+Metric: sparse loop-4 decode attention (the loop-4 selection launch plus the 48
+loop-4 sparse-reader launches), microseconds per step.  Also reported: the whole
+step, the per-kernel averages measured with CUDA events on the launch stream, the
+achieved HBM bandwidth against the measured peak, the oracle on the host cores,
+and the same metric end to end from pinned host buffers.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {flashloop,reference}]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from quantized_kv_attention_int4_b200 import bytemodel  # noqa: E402
+
+METRIC = "sparse loop-4 decode attention µs/step at 32K ctx; achieved HBM GB/s vs peak"
+UNIT = "us/step"
+DEFAULT_WORKLOAD = "cache_l48_h16_n32768"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the GPU path
+# ----------------------------------------------------------------------------
+def build_cache(w: synth.Workload, layers: int, rank: int, device):
+    from quantized_kv_attention_int4_b200.cache import FlashLoopCache, round_up
+
+    n = w.n_ctx
+    sets = synth.active_sets(w, n)
+    extra = 64 * 4 + 64
+    cap = round_up(n + extra)
+    res_cap = {r: round_up(min(cap, int((sets[r] < n).sum()) + extra + 64 * 4)) for r in range(2, w.loops + 1)}
+    cache = FlashLoopCache(layers, w.heads, w.loops, cap, res_capacity=res_cap,
+                           max_select=w.k_sel(cap), device=device)
+    wr = synth.Workload(**{**w.__dict__, "seed": w.seed + 100003 * rank})
+    info = None
+    for layer in range(layers):
+        d = synth.prefill_layer(wr, layer, device=device, sets=sets)
+        info = cache.prefill_layer(layer, d["K"], d["V"], sets)
+        del d
+    n_q, n_tail, tail_depth = info
+    cache.set_timeline(n_q, n_tail, tail_depth)
+    torch.cuda.synchronize()
+    return cache, wr
+
+
+def step_inputs(w: synth.Workload, layers: int, steps: int, device):
+    """Per step: queries and the new token's k/v, BF16 [R+1][L][H][128] (slice 0 unused)."""
+    out = []
+    for s in range(steps):
+        q = torch.stack([synth.queries(w, l, s + 1, device=device) for l in range(layers)], dim=1)
+        toks = [synth.decode_token(w, l, s, device=device) for l in range(layers)]
+        kn = torch.stack([torch.stack([torch.zeros_like(t["k"][1])] + t["k"][1:]) for t in toks], dim=1)
+        vn = torch.stack([torch.stack([torch.zeros_like(t["v"][1])] + t["v"][1:]) for t in toks], dim=1)
+        out.append((q.contiguous(), kn.contiguous(), vn.contiguous()))
+    return out
+
+
+class Step:
+    """One decode step: flush the tail if full (Python bookkeeping, native encoders), then the
+    native loop-major executor over every layer and loop."""
+
+    def __init__(self, cache, w, layers, device):
+        self.c, self.w, self.L = cache, w, layers
+        self.O = torch.zeros(w.loops + 1, layers, w.heads, 128, dtype=torch.float32, device=device)
+
+    def launches(self, flushed: bool) -> int:
+        w, L = self.w, self.L
+        sparse = w.loops - w.dense_loops
+        return (L * w.loops if flushed else 0) + L * w.loops + sparse
+
+    def run(self, q, kn, vn, ev=None, loop_first=1, loop_last=None):
+        c, w = self.c, self.w
+        if ev is not None:
+            ev["start"].record()
+        flushed = False
+        if loop_first == 1:
+            flushed = c.n_tail == 64
+            c.begin_token()
+        seg = [ev[k] for k in EXEC_EVENTS] if ev is not None else None
+        c.step(w.dense_loops, w.k_sel(c.n_cols), q, self.O, kn, vn, loop_first=loop_first,
+               loop_last=loop_last or w.loops, events=seg)
+        return self.launches(flushed)
+
+
+EXEC_EVENTS = ("flushed", "sel1", "loop1", "sel2", "loop2", "select3", "loop3", "select4", "loop4")
+SEGMENTS = ("start",) + EXEC_EVENTS
+
+
+def sparse_bytes_from_state(cache, w, layers, loop, k_sel):
+    """Algorithmic bytes of the loop-`loop` sparse readers, from the selections now in the cache."""
+    H, n_q, N = cache.H, cache.n_q, cache.n_cols
+    C = cache.capacity
+    total = 0
+    ms = cache.dims.max_select
+    for l in range(layers):
+        S = cache.raw("sel", l).view(torch.int32)[: H * ms].view(H, ms)[:, :k_sel].cpu().numpy()
+        depth = cache.raw("depth", l)[:C].cpu().numpy().astype(np.int64)
+        mask = cache.raw("mask", l).view(torch.int64)[: (w.loops + 1) * (C // 64)].view(w.loops + 1, C // 64)
+        first = cache.raw("first", l).view(torch.int32)[: (w.loops + 1) * (C // 64)].view(w.loops + 1, C // 64)
+        mask = mask.cpu().numpy().view(np.uint64)
+        first = first.cpu().numpy()
+        quant = S[S < n_q]
+        cols_tail = int((S >= n_q).sum())
+        dep = np.minimum(depth[quant], loop)
+        res_rows = int(np.maximum(dep - 1, 0).sum())
+        groups = 0
+        for h in range(H):
+            s = S[h][S[h] < n_q]
+            groups += len(np.unique(s // 64))  # base key groups
+            for rp in range(2, loop + 1):
+                act = s[depth[s] >= rp]
+                if act.size == 0:
+                    continue
+                b = act // 64
+                t = (act % 64).astype(np.uint64)
+                mk = mask[rp, b]
+                low = mk & ((np.uint64(1) << t) - np.uint64(1))
+                cnt = np.array([bin(int(x)).count("1") for x in low])
+                gs = cache.layout.slot_base[rp] + first[rp, b] + cnt
+                groups += len(np.unique(gs // 64))
+        total += bytemodel.sparse_bytes(H, int(quant.size), res_rows, groups, cols_tail)
+    return total / layers
+
+
+def dense_bytes_avg(cache, w, layers, loop):
+    H = cache.H
+    tot = 0
+    for l in range(layers):
+        res_rows = sum(cache.n_rows[l][rp] for rp in range(2, loop + 1))
+        tot += bytemodel.dense_bytes(H, cache.n_q, cache.n_tail, res_rows, keep_scores=(loop == w.dense_loops))
+    return tot / layers
+
+
+def run_gpu(args, rank, world):
+    from quantized_kv_attention_int4_b200 import abi  # noqa: F401  (fails loudly without the library)
+
+    device = torch.device("cuda", torch.cuda.current_device())
+    w = synth.WORKLOADS[args.workload]
+    layers = args.layers or w.layers
+    t0 = time.time()
+    cache, wr = build_cache(w, layers, rank, device)
+    total_steps = args.warmup + args.steps
+    inputs = step_inputs(wr, layers, total_steps + args.e2e_steps, device)
+    step = Step(cache, wr, layers, device)
+    setup_s = time.time() - t0
+
+    for s in range(args.warmup):
+        step.run(*inputs[s])
+    torch.cuda.synchronize()
+    st, info = cache.status()
+    if st != 0:
+        raise RuntimeError(f"device error during warm-up: {info}")
+
+    evs = [{k: torch.cuda.Event(enable_timing=True) for k in SEGMENTS} for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()]))
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    launches = 0
+    for s in range(args.steps):
+        launches += step.run(*inputs[args.warmup + s], ev=evs[s])
+    t_end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+
+    seg = {k: [] for k in ("flush", "loop1", "loop2", "select3", "loop3", "select4", "loop4")}
+    for e in evs:
+        seg["flush"].append(e["start"].elapsed_time(e["flushed"]))
+        seg["loop1"].append(e["flushed"].elapsed_time(e["loop1"]))
+        seg["loop2"].append(e["loop1"].elapsed_time(e["loop2"]))
+        seg["select3"].append(e["loop2"].elapsed_time(e["select3"]))
+        seg["loop3"].append(e["select3"].elapsed_time(e["loop3"]))
+        seg["select4"].append(e["loop3"].elapsed_time(e["select4"]))
+        seg["loop4"].append(e["select4"].elapsed_time(e["loop4"]))
+    mean = {k: float(np.mean(v)) for k, v in seg.items()}
+    metric_us = (mean["select4"] + mean["loop4"]) * 1e3
+    step_ms = total_ms / args.steps
+
+    # max over ranks
+    vals = torch.tensor([metric_us, step_ms, mean["loop4"], mean["loop1"] + mean["loop2"]], device=device,
+                        dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    metric_us, step_ms, loop4_ms, dense_ms = [float(x) for x in vals.tolist()]
+
+    N = cache.n_cols
+    k_sel = wr.k_sel(N)
+    hbm, peak_kind = _peaks()
+    sp_bytes = sparse_bytes_from_state(cache, wr, layers, 4, k_sel)
+    sp_launch_us = loop4_ms * 1e3 / layers
+    sp_gbs = sp_bytes / (sp_launch_us * 1e-6) / 1e9
+    d_bytes = (dense_bytes_avg(cache, wr, layers, 1) + dense_bytes_avg(cache, wr, layers, 2)) / 2
+    d_launch_us = dense_ms * 1e3 / (2 * layers)
+    d_gbs = d_bytes / (d_launch_us * 1e-6) / 1e9
+
+    e2e = run_e2e(step, cache, wr, layers, inputs[total_steps:], device) if args.e2e_steps else None
+    return dict(metric_us=metric_us, step_ms=step_ms, seg=mean, clocks=clocks, launches=launches / args.steps,
+                sp_bytes=sp_bytes, sp_launch_us=sp_launch_us, sp_gbs=sp_gbs, d_bytes=d_bytes,
+                d_launch_us=d_launch_us, d_gbs=d_gbs, hbm=hbm, peak_kind=peak_kind, N=N, k_sel=k_sel,
+                layers=layers, setup_s=setup_s, e2e=e2e, w=wr)
+
+
+def run_e2e(step, cache, w, layers, inputs, device):
+    """The metric end to end through the C ABI: each step runs loops 1-3 untimed, then times
+    the loop-4 inputs copied from pinned host memory, the loop-4 selection and sparse
+    readers, and the loop-4 outputs read back to pinned host memory."""
+    res = []
+    H = w.heads
+    for q, kn, vn in inputs:
+        hq = q[4].cpu().pin_memory()
+        hk = kn[4].cpu().pin_memory()
+        hv = vn[4].cpu().pin_memory()
+        hout = torch.empty(layers, H, 128, dtype=torch.float32).pin_memory()
+        q[4].zero_()
+        kn[4].zero_()
+        vn[4].zero_()
+        step.run(q, kn, vn, loop_first=1, loop_last=3)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        q[4].copy_(hq, non_blocking=True)
+        kn[4].copy_(hk, non_blocking=True)
+        vn[4].copy_(hv, non_blocking=True)
+        step.run(q, kn, vn, loop_first=4, loop_last=4)
+        hout.copy_(step.O[4], non_blocking=True)
+        b.record()
+        b.synchronize()
+        res.append(a.elapsed_time(b) * 1e3)
+    h2d = 3 * layers * H * 128 * 2
+    d2h = layers * H * 128 * 4
+    return {"value": float(np.mean(res)), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ----------------------------------------------------------------------------
+# the oracle on the host cores
+# ----------------------------------------------------------------------------
+def oracle_loop4_sample(w: synth.Workload, budget_s: float, heads=(0,)):
+    """Time the oracle's loop-4 selection + sparse attention for one (layer, head) sample.
+
+    Setup (encoding, loops 1-3) is untimed; the loop-4 step is repeated until about
+    ``budget_s`` seconds have been spent.  Returns (seconds per (layer, head), reps).
+    """
+    from oracle import flashloop_oracle as fo
+
+    n = w.n_ctx
+    sets = synth.active_sets(w, n)
+    d = synth.prefill_layer(w, 0, device="cpu", sets=sets)
+    n_q, n_tail = synth.split_prefill(n)
+    hs = list(heads)
+    f = lambda t: t.float().numpy()
+    lay = fo.OracleLayer(len(hs), w.loops, n + 64)
+    lay.encode_base(0, f(d["K"][1][hs, :n_q]), f(d["V"][1][hs, :n_q]))
+    for r in range(2, w.loops + 1):
+        rows = sets[r][sets[r] < n_q].numpy()
+        lay.encode_residual(r, rows, f(d["K"][r][hs][:, rows]), f(d["V"][r][hs][:, rows]))
+    depth = synth.depth_of(sets, n).numpy()
+    lay.set_tail([None] + [f(d["K"][r][hs, n_q:]) for r in range(1, w.loops + 1)],
+                 [None] + [f(d["V"][r][hs, n_q:]) for r in range(1, w.loops + 1)], depth[n_q:])
+    del d
+    q = synth.queries(w, 0, 0).float().numpy()[:, hs]
+    k = w.k_sel(lay.n_cols)
+    for r in range(1, 4):
+        if r <= w.dense_loops:
+            lay.dense_loop(r, q[r])
+        else:
+            S, _, _ = lay.select(k)
+            lay.sparse_loop(r, q[r], S)
+    p_save, lam_save = lay.p_tilde.copy(), lay.lam.copy()
+    times = []
+    t_all = time.perf_counter()
+    while True:
+        lay.p_tilde, lay.lam = p_save.copy(), lam_save.copy()
+        t = time.perf_counter()
+        S = fo.select_topk(lay.p_tilde, k)
+        lay.sparse_loop(4, q[4], S)
+        times.append(time.perf_counter() - t)
+        if time.perf_counter() - t_all > budget_s and len(times) >= 2:
+            break
+    return float(np.mean(times)) / len(hs), len(times)
+
+
+def cpu_baseline(w: synth.Workload, layers: int, budget_s: float):
+    per_lh, reps = oracle_loop4_sample(w, budget_s)
+    us = per_lh * layers * w.heads * 1e6
+    return {"value": us, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"oracle (NumPy, fp64) loop-4 top-K selection + sparse attention for 1 of "
+                      f"{layers}x{w.heads} (layer, head) pairs at N={w.n_ctx}, {reps} reps, scaled by "
+                      f"{layers * w.heads}"}
+
+
+# ----------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("flashloop", "reference"), default="flashloop")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.WORKLOADS[args.workload]
+    layers = args.layers or w.layers
+    config = {"workload": args.workload, "layers": layers, "heads": w.heads, "head_dim": 128,
+              "context": w.n_ctx, "loops": w.loops, "dense_loops": w.dense_loops, "key_pct": w.key_pct,
+              "retention": "100/100/25/10 %", "storage": "int4 base+residual, bf16 tail",
+              "l2": "inputs larger than L2: loop-major over all layers, ~1.3 GB read between reuses of a layer"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per_step = []
+        for _ in range(args.warmup + args.steps):
+            per_lh, _ = oracle_loop4_sample(w, 0.0)
+            per_step.append(per_lh * layers * w.heads * 1e6)
+        v = float(np.mean(per_step[args.warmup:]))
+        line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3, "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                 "sample": "oracle loop-4 selection + sparse attention, 1 (layer, head) per step, "
+                                           f"scaled by {layers * w.heads}"},
+                "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+
+    r = run_gpu(args, rank, world)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline(w, layers, args.cpu_budget)
+    hbm = r["hbm"]
+    line = {
+        "metric": METRIC, "value": r["metric_us"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": {**config, "context_at_end": r["N"],
+                                                                          "k_sel": r["k_sel"]},
+        "roofline": {"bound": "hbm", "kernel": "fl_decode_attn_sparse (loop 4)", "achieved": r["sp_gbs"],
+                     "peak": hbm, "unit": "GB/s", "frac": r["sp_gbs"] / hbm, "traffic": None,
+                     "peak_kind": peak_kind_str(r["peak_kind"]), "bytes_per_launch": r["sp_bytes"],
+                     "us_per_launch": r["sp_launch_us"]},
+        "roofline_dense": {"bound": "hbm", "kernel": "fl_decode_attn_dense (loops 1-2)", "achieved": r["d_gbs"],
+                           "peak": hbm, "unit": "GB/s", "frac": r["d_gbs"] / hbm, "traffic": None,
+                           "bytes_per_launch": r["d_bytes"], "us_per_launch": r["d_launch_us"]},
+        "segments_ms": r["seg"], "clocks": r["clocks"], "gpu_launches": r["launches"],
+        "e2e": r["e2e"], "cpu_baseline": cpu, "setup_s": r["setup_s"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+def peak_kind_str(kind):
+    return "of measured" if kind == "measured" else "of fallback"
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,245 @@
+/*
+ * flashloop.h -- C ABI of libflashloop_b200.so, the B200 (sm_100a) decode path of
+ * FlashLoop: single-query attention over a cross-loop INT4 KV cache with
+ * loop-aware sparse attention in late loops.
+ *
+ * Sources (page title, then section):
+ *   [PyPI]    "flashloop 0.1.0" project description, "Configuration and supported scope":
+ *             four loops, dense loops 1-2, 25 % / 10 % token retention in loops 3-4,
+ *             10 % key retention in sparse late loops, 4-bit K/V with group size 64,
+ *             a 64-token BF16 tail; head dimension 128, equal query/KV head counts.
+ *   [Project] "FlashLoop: Fast and Memory-Efficient Looped Transformers via Lazy
+ *             Updates" project page, "The Method": Step 01 (inactive tokens reuse the
+ *             preceding loop's KV), Step 02 (recompute a few columns chosen from the
+ *             preceding loop and keep their global probability mass), Step 03 (a
+ *             quantised loop-1 base plus per-loop residuals against the reconstructed
+ *             preceding state), and the closing paragraph on compact gather buffers and
+ *             fusing KV updates into the attention kernel.
+ *   [Guide]   flozi.net "FlashLoop: store changes between repeated passes", section 3:
+ *             per-channel (post-RoPE) key groups, per-token value groups, residuals of
+ *             active tokens only; sparse loops are a rank-K correction of the previous
+ *             loop's output.
+ *
+ * Conventions for every entry point
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates, frees or keeps device memory, and keeps no global mutable state.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
+ *     enqueues work on it and returns; calls on one cache must be stream-ordered.
+ *   - BF16 tensors are passed as uint16_t bit patterns.
+ *   - Arguments are validated on the host before any launch: a bad value returns
+ *     FL_ERR_INVALID / FL_ERR_UNSUPPORTED / FL_ERR_WORKSPACE and enqueues nothing.
+ *     A failed launch returns FL_ERR_CUDA.  Data errors found on the device (rows
+ *     out of order, sets that do not nest, a selected index out of range) are
+ *     recorded in the cache's status words, read with fl_read_status(); kernels
+ *     never trap and never spin-wait.
+ *   - Numbers: codes, scales and zero points are exact (the quantiser below, fp32
+ *     with one IEEE rounding per operation); attention runs in fp32 and returns fp32.
+ *
+ * The 4-bit quantiser (a group of values x):
+ *     s = fp16_rn(fp32_rn(max - min) / 15),  z = fp16_rn(min),
+ *     code = clamp(rint_even(fp32_rn(x - z) / s), 0, 15)   (0 when s == 0),
+ *     x_hat = fma(code, s, z).
+ *   Key groups are (64-token block, channel) in the base and (64 consecutive
+ *   slots of one encode call, channel) in a residual store; value groups are
+ *   (token or slot, 64-channel half).
+ *
+ * Packed cache layout (one buffer of fl_cache_layout().total_bytes; every array
+ * starts on a 256-byte boundary; L layers, H heads, C = capacity, T = total slots,
+ * R loops; "sz" = a (scale, zero) fp16 pair stored as scale in the low half of a
+ * 32-bit word):
+ *   kcode  u8  [L][H][C][64]       base key codes; byte b = channel 2b (low nibble), 2b+1 (high)
+ *   vcode  u8  [L][H][C][64]       base value codes, same packing
+ *   ksz    u32 [L][H][C/64][128]   base key sz per (block, channel)
+ *   vsz    u32 [L][H][C][2]        base value sz per (token, half)
+ *   rkcode u8  [L][H][T][64]       residual key codes of every loop; loop r owns slots
+ *                                   [slot_base[r], slot_base[r] + res_capacity[r])
+ *   rvcode u8  [L][H][T][64]
+ *   rksz   u32 [L][H][T/64][128]   residual key sz per (slot group, channel)
+ *   rvsz   u32 [L][H][T][2]
+ *   mask   u64 [L][R+1][C/64]      bit t of mask[r][b]: token 64b+t has a loop-r residual
+ *   first  i32 [L][R+1][C/64]      slot (within loop r's store) of block b's first loop-r row;
+ *                                   the block's rows occupy consecutive slots in token order
+ *   depth  u8  [L][C]              last loop in which the token was active (1 = base only)
+ *   tail_k bf16[L][R][H][64][128]  BF16 tail of loop r at index r-1
+ *   tail_v bf16[L][R][H][64][128]
+ *   score  f32 [L][H][C]           log2-domain score of each column from the loop that last
+ *                                   computed it (tag); log2 p~_j = score_j - offset[tag_j]
+ *   tag    u8  [L][H][C]
+ *   offset f32 [L][H][33]          per-loop log2 normaliser
+ *   sel    i32 [L][H][max_select]  selected columns S, ascending
+ *   mass   f32 [L][H]              m = sum over S of p~
+ *   unsel  f32 [L][H][128]         u = sum over columns not in S of p~_j * v_j (at loop tag_j)
+ *   status i32 [16]                [0] first device error code (0 = none), [1] its detail,
+ *                                   [2] number of device errors
+ */
+#ifndef FLASHLOOP_H
+#define FLASHLOOP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FL_HEAD_DIM 128
+#define FL_GROUP 64
+#define FL_TAIL 64
+#define FL_MAX_LOOPS 32
+/* The selector holds every column's score of one (layer, head) in shared memory. */
+#define FL_MAX_SELECT_COLS 49152
+
+typedef enum fl_status {
+  FL_OK = 0,
+  FL_ERR_INVALID = -1,     /* null pointer, index out of range, inconsistent sizes */
+  FL_ERR_UNSUPPORTED = -2, /* a shape the kernels do not implement (head_dim != 128, group != 64, ...) */
+  FL_ERR_CUDA = -3,        /* a CUDA runtime call or kernel launch failed */
+  FL_ERR_WORKSPACE = -4,   /* workspace pointer null or smaller than fl_workspace_bytes() */
+  FL_ERR_DEVICE = -6       /* fl_read_status: a kernel recorded a data error */
+} fl_status;
+
+/* Device error codes recorded in status[0] (status[1] holds the offending index). */
+#define FL_DEV_ROWS_ORDER 1   /* encode rows not strictly ascending */
+#define FL_DEV_ROWS_RANGE 2   /* encode row outside [row0, row0 + n_span) */
+#define FL_DEV_NOT_NESTED 3   /* loop-r row not active in loop r-1 */
+#define FL_DEV_SEL_RANGE 4    /* selected column outside [0, N) */
+#define FL_DEV_TAG_RANGE 5    /* a column's loop tag outside [1, R] */
+
+typedef struct fl_dims {
+  int32_t layers;      /* L >= 1 */
+  int32_t heads;       /* H >= 1 (MHA: query heads == KV heads) */
+  int32_t head_dim;    /* must be 128 */
+  int32_t group;       /* must be 64 */
+  int32_t loops;       /* R in [1, 32] */
+  int32_t capacity;    /* max columns N = quantised + tail; a positive multiple of 64 */
+  int32_t max_select;  /* capacity of the selected-column list per (layer, head), >= 1 */
+  int32_t res_capacity[FL_MAX_LOOPS + 1]; /* slots of loop r's residual store, r = 2..R, multiples of 64 */
+} fl_dims;
+
+typedef struct fl_layout {
+  uint64_t total_bytes;
+  uint64_t kcode, vcode, ksz, vsz;
+  uint64_t rkcode, rvcode, rksz, rvsz;
+  uint64_t mask, first, depth;
+  uint64_t tail_k, tail_v;
+  uint64_t score, tag, offset;
+  uint64_t sel, mass, unsel;
+  uint64_t status;
+  /* bytes from one layer to the next inside each array above (same order) */
+  uint64_t layer_stride[19];
+  int32_t slot_base[FL_MAX_LOOPS + 1]; /* first global slot of loop r's residual store */
+  int32_t total_slots;                 /* T */
+} fl_layout;
+
+/* Library version string. */
+const char* fl_version(void);
+
+/* Human-readable name of a status code (static storage). */
+const char* fl_status_string(fl_status st);
+
+/* Byte offsets of every cache array for `dims` (host-only, no CUDA call).
+ * Returns FL_ERR_INVALID / FL_ERR_UNSUPPORTED for bad dims. */
+fl_status fl_cache_layout(const fl_dims* dims, fl_layout* out);
+
+/* Zero the whole cache buffer (`cache` has fl_cache_layout().total_bytes) on `stream`. */
+fl_status fl_cache_init(const fl_dims* dims, void* cache, void* stream);
+
+/* Workspace the readers need for split-K partials and their completion counters. */
+size_t fl_workspace_bytes(const fl_dims* dims);
+
+/* Zero the workspace counters; required once before the first reader call. */
+fl_status fl_workspace_init(const fl_dims* dims, void* ws, size_t ws_bytes, void* stream);
+
+/* Copy `n_rows` BF16 rows [H][n_rows][128] (head stride `head_stride` elements) into
+ * rows [row0, row0 + n_rows) of layer `layer`'s loop-`loop` tail.  Used to load the
+ * prompt's last 1..64 columns.  0 <= row0, row0 + n_rows <= 64. */
+fl_status fl_write_tail(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,
+                        int32_t row0, int32_t n_rows, const uint16_t* k, const uint16_t* v,
+                        int64_t head_stride, void* stream);
+
+/* [Project] Step 03 base; [Guide] section 3.  Quantise loop-1 keys/values of tokens
+ * [row0, row0 + n_rows) (both multiples of 64) into the base.  k, v: BF16
+ * [H][n_rows][128] with `head_stride` elements between heads (row i = token row0 + i).
+ * Sets depth = 1 and clears every loop's residual mask/first entries for those blocks. */
+fl_status fl_encode_base(const fl_dims* dims, void* cache, int32_t layer, int32_t row0,
+                         int32_t n_rows, const uint16_t* k, const uint16_t* v,
+                         int64_t head_stride, void* stream);
+
+/* [Project] Step 01 + Step 03; [Guide] section 3.  Store loop-`loop` (2..R) residuals
+ * of the active tokens `rows` (device int32, strictly ascending, inside
+ * [row0, row0 + n_span), each active in loop `loop`-1 as well: the sets nest) against the reconstructed
+ * loop-(loop-1) state.  row0 and n_span are multiples of 64 and cover whole blocks that
+ * are already in the base; the call owns those blocks' loop-`loop` metadata (cleared,
+ * then rebuilt).  Rows go to slots [slot0, slot0 + n_rows) of the loop's store; slot0
+ * is a multiple of 64 and slot0 + n_rows <= res_capacity[loop].  Inputs are BF16
+ * [H][.][128]: with `compact` = 1 row i of k/v is token rows[i]; with `compact` = 0
+ * it is token row0 + i.  n_rows may be 0 (clears the blocks' metadata only). */
+fl_status fl_encode_residual(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,
+                             int32_t row0, int32_t n_span, int32_t slot0,
+                             const int32_t* rows, int32_t n_rows,
+                             const uint16_t* k, const uint16_t* v, int64_t head_stride,
+                             int32_t compact, void* stream);
+
+/* [Project] Step 02 (dense loops); [PyPI] "dense loops 1-2".  Full single-query
+ * attention of loop `loop` over N = n_q + n_tail columns (n_q a multiple of 64,
+ * n_tail in [1, 64]): keys/values are the base plus the column's residuals of loops
+ * 2..loop, or the loop's BF16 tail row.  q: BF16 [H][128]; o: fp32 [H][128]
+ * (softmax(q K^T / sqrt(128)) V).  If k_new/v_new (BF16 [H][128]) are non-NULL they
+ * are the current token's loop-`loop` key/value: they are used as column N-1 and
+ * stored into tail row n_tail-1.  With keep_scores != 0 every column's score and tag
+ * (and the loop's offset) are written for the selector. */
+fl_status fl_decode_attn_dense(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,
+                               int32_t n_q, int32_t n_tail, const uint16_t* q,
+                               const uint16_t* k_new, const uint16_t* v_new, float* o,
+                               int32_t keep_scores, void* ws, size_t ws_bytes, void* stream);
+
+/* [Project] Step 02; [Guide] section 3.  For layers [layer0, layer0 + n_layers) and
+ * every head: S = the k_sel columns of largest p~ (the distribution the preceding loop
+ * left: scores/tags/offsets), ties to the smaller index, written ascending; the mass
+ * m = sum over S of p~; and the unselected contribution u = o_prev - sum over S of
+ * p~_j v_j, v_j taken at the loop that last computed column j.  o_prev: fp32
+ * [n_layers][H][128], the preceding loop's outputs.  N = n_q + n_tail <=
+ * FL_MAX_SELECT_COLS and 1 <= k_sel <= min(N, max_select). */
+fl_status fl_select_topk(const fl_dims* dims, void* cache, int32_t layer0, int32_t n_layers,
+                         int32_t n_q, int32_t n_tail, int32_t k_sel, const float* o_prev,
+                         void* stream);
+
+/* [Project] Step 02; [Guide] section 3.  Sparse attention of loop `loop` over the
+ * columns fl_select_topk chose (same k_sel, n_q, n_tail):
+ *   o = u + m * softmax_S(q K_S^T / sqrt(128)) V_S,
+ * keys/values at loop `loop`.  Then splices the state: score/tag of j in S become this
+ * loop's, and offset[loop] makes p~_j = m * softmax_S(.)_j.  q, k_new, v_new, o as in
+ * fl_decode_attn_dense. */
+fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,
+                                int32_t n_q, int32_t n_tail, int32_t k_sel, const uint16_t* q,
+                                const uint16_t* k_new, const uint16_t* v_new, float* o,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Native executor of one decode step for layers [0, L) in loop-major order (every
+ * layer runs loop r before any layer runs loop r+1), for loops loop_first..loop_last:
+ * loops up to dense_loops call the dense reader (the last dense loop keeps scores);
+ * every later loop first selects k_sel columns for all layers in one launch
+ * (fl_select_topk, o_prev = that loop's previous outputs) and then runs each layer's
+ * sparse reader.  Same arguments and semantics as the individual calls; validated once.
+ *   q, k_new, v_new: BF16 [R+1][L][H][128] (slice r = loop r, slice 0 unused;
+ *                    k_new/v_new may be NULL)
+ *   o: fp32 [R+1][L][H][128]   (o[r] = loop r's outputs; o[loop_first-1] must hold the
+ *                               previous loop's outputs when loop_first is sparse)
+ *   events: NULL, or 2*R+1 cudaEvent_t; events[0] is recorded before loop_first, and
+ *           for each loop r in range events[2r-1] after its selection (right away for a
+ *           dense loop) and events[2r] after its readers. */
+fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail,
+                         int32_t dense_loops, int32_t k_sel, int32_t loop_first, int32_t loop_last,
+                         const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new, float* o,
+                         void* ws, size_t ws_bytes, void* const* events, void* stream);
+
+/* Synchronise `stream`, copy the cache's status words to host `out[0..2]`, and return
+ * FL_ERR_DEVICE if a kernel recorded an error (FL_OK otherwise).  With `clear` != 0
+ * the words are zeroed afterwards. */
+fl_status fl_read_status(const fl_dims* dims, void* cache, int32_t* out, int32_t clear,
+                         void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLASHLOOP_H */

@@ -1,0 +1,243 @@
+"""ctypes binding of libflashloop_b200.so: the C ABI of include/flashloop.h, same names.
+
+Argument marshalling only: every wrapper checks tensor placement, dtype and
+contiguity, passes raw device pointers and the current CUDA stream, and raises
+FlashLoopError on a non-OK status.  All compute runs in the library's kernels.
+Importing this module without the built library raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LIB_PATH = _build.LIB_PATH
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing; build it with `python -m quantized_kv_attention_int4_b200.build`")
+lib = ctypes.CDLL(LIB_PATH)
+
+MAX_LOOPS = 32
+HEAD_DIM = 128
+GROUP = 64
+TAIL = 64
+MAX_SELECT_COLS = 49152
+N_ARRAYS = 19
+ARRAY_NAMES = ("kcode", "vcode", "ksz", "vsz", "rkcode", "rvcode", "rksz", "rvsz", "mask", "first",
+               "depth", "tail_k", "tail_v", "score", "tag", "offset", "sel", "mass", "unsel")
+
+FL_OK, FL_ERR_INVALID, FL_ERR_UNSUPPORTED, FL_ERR_CUDA, FL_ERR_WORKSPACE, FL_ERR_DEVICE = 0, -1, -2, -3, -4, -6
+EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init", "fl_workspace_bytes",
+            "fl_workspace_init", "fl_write_tail", "fl_encode_base", "fl_encode_residual",
+            "fl_decode_attn_dense", "fl_select_topk", "fl_decode_attn_sparse", "fl_decode_step",
+            "fl_read_status")
+
+
+class fl_dims(ctypes.Structure):
+    _fields_ = [("layers", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("group", ctypes.c_int32), ("loops", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("max_select", ctypes.c_int32), ("res_capacity", ctypes.c_int32 * (MAX_LOOPS + 1))]
+
+
+class fl_layout(ctypes.Structure):
+    _fields_ = ([("total_bytes", ctypes.c_uint64)]
+                + [(n, ctypes.c_uint64) for n in ARRAY_NAMES]
+                + [("status", ctypes.c_uint64), ("layer_stride", ctypes.c_uint64 * N_ARRAYS),
+                   ("slot_base", ctypes.c_int32 * (MAX_LOOPS + 1)), ("total_slots", ctypes.c_int32)])
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_L = ctypes.c_int64
+_DP = ctypes.POINTER(fl_dims)
+
+
+def _sig(name, res, *args):
+    f = getattr(lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_c_version = _sig("fl_version", ctypes.c_char_p)
+_c_status_string = _sig("fl_status_string", ctypes.c_char_p, _I)
+_c_cache_layout = _sig("fl_cache_layout", _I, _DP, ctypes.POINTER(fl_layout))
+_c_cache_init = _sig("fl_cache_init", _I, _DP, _P, _P)
+_c_workspace_bytes = _sig("fl_workspace_bytes", ctypes.c_size_t, _DP)
+_c_workspace_init = _sig("fl_workspace_init", _I, _DP, _P, ctypes.c_size_t, _P)
+_c_write_tail = _sig("fl_write_tail", _I, _DP, _P, _I, _I, _I, _I, _P, _P, _L, _P)
+_c_encode_base = _sig("fl_encode_base", _I, _DP, _P, _I, _I, _I, _P, _P, _L, _P)
+_c_encode_residual = _sig("fl_encode_residual", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _L, _I, _P)
+_c_dense = _sig("fl_decode_attn_dense", _I, _DP, _P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P,
+                ctypes.c_size_t, _P)
+_c_select = _sig("fl_select_topk", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _P)
+_c_sparse = _sig("fl_decode_attn_sparse", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                 ctypes.c_size_t, _P)
+_c_step = _sig("fl_decode_step", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                ctypes.POINTER(ctypes.c_void_p), _P)
+_c_read_status = _sig("fl_read_status", _I, _DP, _P, ctypes.POINTER(ctypes.c_int32), _I, _P)
+
+
+class FlashLoopError(RuntimeError):
+    def __init__(self, where: str, status: int):
+        super().__init__(f"{where}: {fl_status_string(status)}")
+        self.status = status
+
+
+def _check(where: str, st: int):
+    if st != FL_OK:
+        raise FlashLoopError(where, st)
+
+
+def Dims(layers: int, heads: int, loops: int, capacity: int, max_select: int, res_capacity) -> fl_dims:
+    """fl_dims with head_dim 128 / group 64; res_capacity[r] for r = 2..loops (mapping or list)."""
+    d = fl_dims()
+    d.layers, d.heads, d.head_dim, d.group = layers, heads, HEAD_DIM, GROUP
+    d.loops, d.capacity, d.max_select = loops, capacity, max_select
+    items = res_capacity.items() if isinstance(res_capacity, dict) else enumerate(res_capacity)
+    for r, v in items:
+        d.res_capacity[r] = int(v)
+    return d
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _rows_tensor(x, name):
+    """BF16 [H][n][128] with a unit-stride last dimension; returns (ptr, head_stride)."""
+    if x.dim() != 3 or x.shape[2] != HEAD_DIM or x.stride(2) != 1 or x.stride(1) != HEAD_DIM:
+        raise ValueError(f"{name} must be [H][n][128] with contiguous rows")
+    return _ptr(x, torch.bfloat16, name), x.stride(0)
+
+
+# ---------------------------------------------------------------------------
+def fl_version() -> str:
+    return _c_version().decode()
+
+
+def fl_status_string(st: int) -> str:
+    return _c_status_string(int(st)).decode()
+
+
+def fl_cache_layout(dims: fl_dims) -> fl_layout:
+    out = fl_layout()
+    _check("fl_cache_layout", _c_cache_layout(ctypes.byref(dims), ctypes.byref(out)))
+    return out
+
+
+def fl_cache_init(dims, cache, stream=None):
+    _check("fl_cache_init", _c_cache_init(ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), _stream(stream)))
+
+
+def fl_workspace_bytes(dims) -> int:
+    return int(_c_workspace_bytes(ctypes.byref(dims)))
+
+
+def fl_workspace_init(dims, ws, stream=None):
+    _check("fl_workspace_init", _c_workspace_init(ctypes.byref(dims), _ptr(ws, torch.uint8, "ws"),
+                                                  ws.numel(), _stream(stream)))
+
+
+def fl_write_tail(dims, cache, layer, loop, row0, k, v, stream=None):
+    kp, ks = _rows_tensor(k, "k")
+    vp, vs = _rows_tensor(v, "v")
+    if ks != vs or k.shape != v.shape:
+        raise ValueError("k and v must have the same shape and strides")
+    _check("fl_write_tail", _c_write_tail(ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer, loop,
+                                          row0, k.shape[1], kp, vp, ks, _stream(stream)))
+
+
+def fl_encode_base(dims, cache, layer, row0, k, v, stream=None):
+    kp, ks = _rows_tensor(k, "k")
+    vp, vs = _rows_tensor(v, "v")
+    if ks != vs or k.shape != v.shape:
+        raise ValueError("k and v must have the same shape and strides")
+    _check("fl_encode_base", _c_encode_base(ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer, row0,
+                                            k.shape[1], kp, vp, ks, _stream(stream)))
+
+
+def fl_encode_residual(dims, cache, layer, loop, row0, n_span, slot0, rows, k, v, compact, stream=None):
+    n = 0 if rows is None else rows.numel()
+    if n:
+        kp, ks = _rows_tensor(k, "k")
+        vp, vs = _rows_tensor(v, "v")
+        if ks != vs or k.shape != v.shape:
+            raise ValueError("k and v must have the same shape and strides")
+        rp = _ptr(rows, torch.int32, "rows")
+    else:
+        kp = vp = rp = None
+        ks = 0
+    _check("fl_encode_residual", _c_encode_residual(ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer,
+                                                    loop, row0, n_span, slot0, rp, n, kp, vp, ks,
+                                                    1 if compact else 0, _stream(stream)))
+
+
+def fl_decode_attn_dense(dims, cache, layer, loop, n_q, n_tail, q, k_new, v_new, o, keep_scores, ws, stream=None):
+    _check("fl_decode_attn_dense", _c_dense(
+        ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer, loop, n_q, n_tail,
+        _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        _ptr(o, torch.float32, "o"), 1 if keep_scores else 0, _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)))
+
+
+def fl_select_topk(dims, cache, layer0, n_layers, n_q, n_tail, k_sel, o_prev, stream=None):
+    _check("fl_select_topk", _c_select(ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer0, n_layers,
+                                       n_q, n_tail, k_sel, _ptr(o_prev, torch.float32, "o_prev"), _stream(stream)))
+
+
+def fl_decode_attn_sparse(dims, cache, layer, loop, n_q, n_tail, k_sel, q, k_new, v_new, o, ws, stream=None):
+    _check("fl_decode_attn_sparse", _c_sparse(
+        ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer, loop, n_q, n_tail, k_sel,
+        _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        _ptr(o, torch.float32, "o"), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def fl_decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, k_new, v_new, o, ws,
+                   events=None, stream=None):
+    """One loop-major decode step over every layer; q/k_new/v_new BF16 and o fp32, all [R+1][L][H][128].
+
+    ``events``: None or a list of 2R+1 torch.cuda.Event (enable_timing) recorded at segment boundaries.
+    """
+    ev = None
+    if events is not None:
+        for e in events:
+            e.record()  # materialise the underlying cudaEvent_t
+        ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    for t, name in ((q, "q"), (k_new, "k_new"), (v_new, "v_new")):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [R+1][L][H][128]")
+    if not o.is_contiguous():
+        raise ValueError("o must be contiguous [R+1][L][H][128]")
+    _check("fl_decode_step", _c_step(
+        ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), n_q, n_tail, dense_loops, k_sel, loop_first, loop_last,
+        _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        _ptr(o, torch.float32, "o"), _ptr(ws, torch.uint8, "ws"), ws.numel(), ev, _stream(stream)))
+
+
+def fl_read_status(dims, cache, clear=True, stream=None):
+    """(status, [first error code, detail, count]); synchronises the stream."""
+    out = (ctypes.c_int32 * 3)()
+    st = _c_read_status(ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), out, 1 if clear else 0,
+                        _stream(stream))
+    if st not in (FL_OK, FL_ERR_DEVICE):
+        raise FlashLoopError("fl_read_status", st)
+    return st, [out[0], out[1], out[2]]

@@ -1,0 +1,425 @@
+// Host side of the C ABI declared in include/flashloop.h: layout arithmetic, argument
+// validation and kernel launches.  Nothing here allocates device memory.
+#include <cstring>
+
+#include "kernels.h"
+
+using namespace fl;
+
+namespace {
+
+constexpr uint64_t kAlign = 256;
+
+inline uint64_t align_up(uint64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+fl_status check_dims(const fl_dims* d) {
+  if (!d) return FL_ERR_INVALID;
+  if (d->head_dim != FL_HEAD_DIM || d->group != FL_GROUP) return FL_ERR_UNSUPPORTED;
+  if (d->layers < 1 || d->heads < 1 || d->loops < 1 || d->loops > FL_MAX_LOOPS) return FL_ERR_INVALID;
+  if (d->capacity < FL_GROUP || d->capacity % FL_GROUP != 0) return FL_ERR_INVALID;
+  if (d->max_select < 1) return FL_ERR_INVALID;
+  for (int r = 2; r <= d->loops; ++r)
+    if (d->res_capacity[r] < 0 || d->res_capacity[r] % FL_GROUP != 0) return FL_ERR_INVALID;
+  return FL_OK;
+}
+
+// Per-layer byte sizes of every array, in fl_layout order.
+void layer_sizes(const fl_dims* d, uint64_t* sz, int32_t* slot_base, int32_t* total_slots) {
+  const uint64_t H = d->heads, C = d->capacity, R = d->loops;
+  uint64_t T = 0;
+  for (int r = 0; r <= FL_MAX_LOOPS; ++r) slot_base[r] = 0;
+  for (int r = 2; r <= d->loops; ++r) {
+    slot_base[r] = (int32_t)T;
+    T += (uint64_t)d->res_capacity[r];
+  }
+  *total_slots = (int32_t)T;
+  sz[A_KCODE] = H * C * 64;
+  sz[A_VCODE] = H * C * 64;
+  sz[A_KSZ] = H * (C / 64) * 128 * 4;
+  sz[A_VSZ] = H * C * 2 * 4;
+  sz[A_RKCODE] = H * T * 64;
+  sz[A_RVCODE] = H * T * 64;
+  sz[A_RKSZ] = H * (T / 64) * 128 * 4;
+  sz[A_RVSZ] = H * T * 2 * 4;
+  sz[A_MASK] = (R + 1) * (C / 64) * 8;
+  sz[A_FIRST] = (R + 1) * (C / 64) * 4;
+  sz[A_DEPTH] = C;
+  sz[A_TAILK] = R * H * 64 * 128 * 2;
+  sz[A_TAILV] = R * H * 64 * 128 * 2;
+  sz[A_SCORE] = H * C * 4;
+  sz[A_TAG] = H * C;
+  sz[A_OFFSET] = H * (FL_MAX_LOOPS + 1) * 4;
+  sz[A_SEL] = H * (uint64_t)d->max_select * 4;
+  sz[A_MASS] = H * 4;
+  sz[A_UNSEL] = H * 128 * 4;
+}
+
+fl_status make_layout(const fl_dims* d, fl_layout* L) {
+  fl_status st = check_dims(d);
+  if (st != FL_OK) return st;
+  std::memset(L, 0, sizeof(*L));
+  uint64_t sz[A_COUNT];
+  layer_sizes(d, sz, L->slot_base, &L->total_slots);
+  uint64_t* offs[A_COUNT] = {&L->kcode, &L->vcode, &L->ksz, &L->vsz, &L->rkcode, &L->rvcode,
+                             &L->rksz, &L->rvsz, &L->mask, &L->first, &L->depth, &L->tail_k,
+                             &L->tail_v, &L->score, &L->tag, &L->offset, &L->sel, &L->mass,
+                             &L->unsel};
+  uint64_t cur = 0;
+  for (int i = 0; i < A_COUNT; ++i) {
+    const uint64_t stride = align_up(sz[i]);
+    *offs[i] = cur;
+    L->layer_stride[i] = stride;
+    cur += stride * (uint64_t)d->layers;
+  }
+  L->status = cur;
+  cur += align_up(16 * sizeof(int32_t));
+  L->total_bytes = cur;
+  return FL_OK;
+}
+
+CacheView make_view(const fl_dims* d, const fl_layout& L, void* cache) {
+  CacheView v;
+  std::memset(&v, 0, sizeof(v));
+  v.base = static_cast<uint8_t*>(cache);
+  const uint64_t offs[A_COUNT] = {L.kcode, L.vcode, L.ksz, L.vsz, L.rkcode, L.rvcode, L.rksz,
+                                  L.rvsz, L.mask, L.first, L.depth, L.tail_k, L.tail_v,
+                                  L.score, L.tag, L.offset, L.sel, L.mass, L.unsel};
+  for (int i = 0; i < A_COUNT; ++i) {
+    v.off[i] = offs[i];
+    v.lstride[i] = L.layer_stride[i];
+  }
+  for (int r = 0; r <= FL_MAX_LOOPS; ++r) v.slot_base[r] = L.slot_base[r];
+  v.status = reinterpret_cast<int32_t*>(v.base + L.status);
+  v.H = d->heads;
+  v.R = d->loops;
+  v.cap = d->capacity;
+  v.total_slots = L.total_slots;
+  v.max_select = d->max_select;
+  return v;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FL_OK : FL_ERR_CUDA; }
+
+uint64_t ws_part_bytes(const fl_dims* d) {
+  return (uint64_t)d->heads * kMaxSplits * kPartStride * sizeof(float);
+}
+
+fl_status check_reader(const fl_dims* d, void* cache, int layer, int loop, int n_q, int n_tail,
+                       const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new, float* o,
+                       void* ws, size_t ws_bytes) {
+  fl_status st = check_dims(d);
+  if (st != FL_OK) return st;
+  if (!cache || !q || !o) return FL_ERR_INVALID;
+  if (layer < 0 || layer >= d->layers || loop < 1 || loop > d->loops) return FL_ERR_INVALID;
+  if (n_q < 0 || n_q % FL_GROUP != 0 || n_tail < 1 || n_tail > FL_TAIL) return FL_ERR_INVALID;
+  if ((int64_t)n_q + n_tail > d->capacity) return FL_ERR_INVALID;
+  if ((k_new == nullptr) != (v_new == nullptr)) return FL_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(o) || (k_new && (!aligned16(k_new) || !aligned16(v_new))))
+    return FL_ERR_INVALID;
+  if (!ws || ws_bytes < fl_workspace_bytes(d)) return FL_ERR_WORKSPACE;
+  return FL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fl_version(void) { return "flashloop-b200 0.1.0 (sm_100a)"; }
+
+const char* fl_status_string(fl_status st) {
+  switch (st) {
+    case FL_OK: return "FL_OK";
+    case FL_ERR_INVALID: return "FL_ERR_INVALID: invalid argument";
+    case FL_ERR_UNSUPPORTED: return "FL_ERR_UNSUPPORTED: unsupported shape";
+    case FL_ERR_CUDA: return "FL_ERR_CUDA: CUDA runtime or launch error";
+    case FL_ERR_WORKSPACE: return "FL_ERR_WORKSPACE: workspace missing or too small";
+    case FL_ERR_DEVICE: return "FL_ERR_DEVICE: a kernel recorded a data error";
+  }
+  return "unknown fl_status";
+}
+
+fl_status fl_cache_layout(const fl_dims* dims, fl_layout* out) {
+  if (!out) return FL_ERR_INVALID;
+  return make_layout(dims, out);
+}
+
+fl_status fl_cache_init(const fl_dims* dims, void* cache, void* stream) {
+  fl_layout L;
+  fl_status st = make_layout(dims, &L);
+  if (st != FL_OK) return st;
+  if (!cache) return FL_ERR_INVALID;
+  return cuda_status(cudaMemsetAsync(cache, 0, L.total_bytes, (cudaStream_t)stream));
+}
+
+size_t fl_workspace_bytes(const fl_dims* dims) {
+  if (check_dims(dims) != FL_OK) return 0;
+  return ws_part_bytes(dims) + align_up((uint64_t)dims->heads * sizeof(int32_t));
+}
+
+fl_status fl_workspace_init(const fl_dims* dims, void* ws, size_t ws_bytes, void* stream) {
+  fl_status st = check_dims(dims);
+  if (st != FL_OK) return st;
+  if (!ws || ws_bytes < fl_workspace_bytes(dims)) return FL_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(static_cast<uint8_t*>(ws) + ws_part_bytes(dims), 0,
+                                     (size_t)dims->heads * sizeof(int32_t), (cudaStream_t)stream));
+}
+
+fl_status fl_write_tail(const fl_dims* dims, void* cache, int32_t layer, int32_t loop, int32_t row0,
+                        int32_t n_rows, const uint16_t* k, const uint16_t* v, int64_t head_stride,
+                        void* stream) {
+  fl_layout L;
+  fl_status st = make_layout(dims, &L);
+  if (st != FL_OK) return st;
+  if (!cache || !k || !v) return FL_ERR_INVALID;
+  if (layer < 0 || layer >= dims->layers || loop < 1 || loop > dims->loops) return FL_ERR_INVALID;
+  if (row0 < 0 || n_rows < 0 || row0 + n_rows > FL_TAIL || head_stride < (int64_t)n_rows * FL_HEAD_DIM)
+    return FL_ERR_INVALID;
+  if (n_rows == 0) return FL_OK;
+  uint8_t* base = static_cast<uint8_t*>(cache);
+  const size_t row_bytes = FL_HEAD_DIM * 2;
+  const size_t dpitch = (size_t)FL_TAIL * row_bytes;
+  const size_t per_loop = (size_t)dims->heads * dpitch;
+  for (int which = 0; which < 2; ++which) {
+    uint8_t* dst = base + (which ? L.tail_v : L.tail_k) + L.layer_stride[which ? A_TAILV : A_TAILK] * layer +
+                   per_loop * (loop - 1) + (size_t)row0 * row_bytes;
+    const uint16_t* src = which ? v : k;
+    cudaError_t e = cudaMemcpy2DAsync(dst, dpitch, src, (size_t)head_stride * 2, (size_t)n_rows * row_bytes,
+                                      dims->heads, cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+    if (e != cudaSuccess) return FL_ERR_CUDA;
+  }
+  return FL_OK;
+}
+
+fl_status fl_encode_base(const fl_dims* dims, void* cache, int32_t layer, int32_t row0, int32_t n_rows,
+                         const uint16_t* k, const uint16_t* v, int64_t head_stride, void* stream) {
+  fl_layout L;
+  fl_status st = make_layout(dims, &L);
+  if (st != FL_OK) return st;
+  if (!cache || !k || !v) return FL_ERR_INVALID;
+  if (layer < 0 || layer >= dims->layers) return FL_ERR_INVALID;
+  if (row0 < 0 || row0 % FL_GROUP || n_rows < 0 || n_rows % FL_GROUP) return FL_ERR_INVALID;
+  if ((int64_t)row0 + n_rows > dims->capacity) return FL_ERR_INVALID;
+  if (!aligned16(k) || !aligned16(v) || head_stride % 8 || head_stride < (int64_t)n_rows * FL_HEAD_DIM)
+    return FL_ERR_INVALID;
+  if (n_rows == 0) return FL_OK;
+  EncodeBaseArgs a;
+  a.c = make_view(dims, L, cache);
+  a.layer = layer;
+  a.row0 = row0;
+  a.n_rows = n_rows;
+  a.k = k;
+  a.v = v;
+  a.head_stride = head_stride;
+  return cuda_status(launch_encode_base(a, (cudaStream_t)stream));
+}
+
+fl_status fl_encode_residual(const fl_dims* dims, void* cache, int32_t layer, int32_t loop, int32_t row0,
+                             int32_t n_span, int32_t slot0, const int32_t* rows, int32_t n_rows,
+                             const uint16_t* k, const uint16_t* v, int64_t head_stride, int32_t compact,
+                             void* stream) {
+  fl_layout L;
+  fl_status st = make_layout(dims, &L);
+  if (st != FL_OK) return st;
+  if (!cache) return FL_ERR_INVALID;
+  if (layer < 0 || layer >= dims->layers || loop < 2 || loop > dims->loops) return FL_ERR_INVALID;
+  if (row0 < 0 || row0 % FL_GROUP || n_span < 0 || n_span % FL_GROUP) return FL_ERR_INVALID;
+  if ((int64_t)row0 + n_span > dims->capacity) return FL_ERR_INVALID;
+  if (n_rows < 0 || n_rows > n_span) return FL_ERR_INVALID;
+  if (slot0 < 0 || slot0 % FL_GROUP || (int64_t)slot0 + n_rows > dims->res_capacity[loop]) return FL_ERR_INVALID;
+  if (n_rows > 0) {
+    if (!rows || !k || !v || !aligned16(k) || !aligned16(v) || head_stride % 8) return FL_ERR_INVALID;
+    const int64_t rows_in = compact ? n_rows : n_span;
+    if (head_stride < rows_in * FL_HEAD_DIM) return FL_ERR_INVALID;
+  }
+  const int ncb = dims->capacity / FL_GROUP;
+  uint8_t* base = static_cast<uint8_t*>(cache);
+  const int b0 = row0 / FL_GROUP, nbk = n_span / FL_GROUP;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (nbk > 0) {
+    uint8_t* m = base + L.mask + L.layer_stride[A_MASK] * layer + ((size_t)loop * ncb + b0) * 8;
+    uint8_t* f = base + L.first + L.layer_stride[A_FIRST] * layer + ((size_t)loop * ncb + b0) * 4;
+    if (cudaMemsetAsync(m, 0, (size_t)nbk * 8, s) != cudaSuccess) return FL_ERR_CUDA;
+    if (cudaMemsetAsync(f, 0xff, (size_t)nbk * 4, s) != cudaSuccess) return FL_ERR_CUDA;
+  }
+  EncodeResArgs a;
+  a.c = make_view(dims, L, cache);
+  a.layer = layer;
+  a.r = loop;
+  a.row0 = row0;
+  a.n_span = n_span;
+  a.slot0 = slot0;
+  a.n_rows = n_rows;
+  a.compact = compact ? 1 : 0;
+  a.rows = rows;
+  a.k = k;
+  a.v = v;
+  a.head_stride = head_stride;
+  return cuda_status(launch_encode_residual(a, s));
+}
+
+fl_status fl_decode_attn_dense(const fl_dims* dims, void* cache, int32_t layer, int32_t loop, int32_t n_q,
+                               int32_t n_tail, const uint16_t* q, const uint16_t* k_new,
+                               const uint16_t* v_new, float* o, int32_t keep_scores, void* ws,
+                               size_t ws_bytes, void* stream) {
+  fl_status st = check_reader(dims, cache, layer, loop, n_q, n_tail, q, k_new, v_new, o, ws, ws_bytes);
+  if (st != FL_OK) return st;
+  fl_layout L;
+  make_layout(dims, &L);
+  ReaderArgs a;
+  a.c = make_view(dims, L, cache);
+  a.layer = layer;
+  a.r = loop;
+  a.n_q = n_q;
+  a.n_tail = n_tail;
+  a.k_sel = 0;
+  a.n_splits = 1;
+  a.keep = keep_scores ? 1 : 0;
+  a.q = q;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.o = o;
+  a.part = static_cast<float*>(ws);
+  a.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_part_bytes(dims));
+  return cuda_status(launch_dense(a, (cudaStream_t)stream));
+}
+
+fl_status fl_select_topk(const fl_dims* dims, void* cache, int32_t layer0, int32_t n_layers, int32_t n_q,
+                         int32_t n_tail, int32_t k_sel, const float* o_prev, void* stream) {
+  fl_layout L;
+  fl_status st = make_layout(dims, &L);
+  if (st != FL_OK) return st;
+  if (!cache || !o_prev) return FL_ERR_INVALID;
+  if (layer0 < 0 || n_layers < 1 || (int64_t)layer0 + n_layers > dims->layers) return FL_ERR_INVALID;
+  if (n_q < 0 || n_q % FL_GROUP != 0 || n_tail < 1 || n_tail > FL_TAIL) return FL_ERR_INVALID;
+  const int64_t N = (int64_t)n_q + n_tail;
+  if (N > dims->capacity) return FL_ERR_INVALID;
+  if (N > FL_MAX_SELECT_COLS) return FL_ERR_UNSUPPORTED;
+  if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
+  SelectArgs a;
+  a.c = make_view(dims, L, cache);
+  a.layer0 = layer0;
+  a.n_q = n_q;
+  a.n_tail = n_tail;
+  a.k_sel = k_sel;
+  a.o_prev = o_prev;
+  return cuda_status(launch_select(a, n_layers, (cudaStream_t)stream));
+}
+
+fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer, int32_t loop, int32_t n_q,
+                                int32_t n_tail, int32_t k_sel, const uint16_t* q, const uint16_t* k_new,
+                                const uint16_t* v_new, float* o, void* ws, size_t ws_bytes, void* stream) {
+  fl_status st = check_reader(dims, cache, layer, loop, n_q, n_tail, q, k_new, v_new, o, ws, ws_bytes);
+  if (st != FL_OK) return st;
+  const int64_t N = (int64_t)n_q + n_tail;
+  if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
+  fl_layout L;
+  make_layout(dims, &L);
+  ReaderArgs a;
+  a.c = make_view(dims, L, cache);
+  a.layer = layer;
+  a.r = loop;
+  a.n_q = n_q;
+  a.n_tail = n_tail;
+  a.k_sel = k_sel;
+  a.n_splits = 1;
+  a.keep = 1;
+  a.q = q;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.o = o;
+  a.part = static_cast<float*>(ws);
+  a.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_part_bytes(dims));
+  return cuda_status(launch_sparse(a, (cudaStream_t)stream));
+}
+
+fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
+                         int32_t k_sel, int32_t loop_first, int32_t loop_last, const uint16_t* q,
+                         const uint16_t* k_new, const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,
+                         void* const* events, void* stream) {
+  fl_status st = check_reader(dims, cache, 0, 1, n_q, n_tail, q, k_new, v_new, o, ws, ws_bytes);
+  if (st != FL_OK) return st;
+  const int R = dims->loops, L = dims->layers, H = dims->heads;
+  if (dense_loops < 0 || dense_loops > R || loop_first < 1 || loop_last > R || loop_first > loop_last)
+    return FL_ERR_INVALID;
+  const int64_t N = (int64_t)n_q + n_tail;
+  const bool any_sparse = loop_last > dense_loops;
+  if (any_sparse) {
+    if (N > FL_MAX_SELECT_COLS) return FL_ERR_UNSUPPORTED;
+    if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
+    if (loop_first == 1 && dense_loops == 0) return FL_ERR_INVALID;  // a sparse loop needs a predecessor
+  }
+  fl_layout lay;
+  make_layout(dims, &lay);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t row = (size_t)H * FL_HEAD_DIM;              // one (loop, layer) slice
+  const size_t ostride_r = (size_t)L * row;                // elements between loops
+  auto rec = [&](int i) -> bool {
+    return !events || cudaEventRecord((cudaEvent_t)events[i], s) == cudaSuccess;
+  };
+  ReaderArgs a;
+  a.c = make_view(dims, lay, cache);
+  a.n_q = n_q;
+  a.n_tail = n_tail;
+  a.k_sel = k_sel;
+  a.n_splits = 1;
+  a.part = static_cast<float*>(ws);
+  a.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_part_bytes(dims));
+  if (!rec(0)) return FL_ERR_CUDA;
+  for (int r = loop_first; r <= loop_last; ++r) {
+    a.r = r;
+    if (r <= dense_loops) {
+      if (!rec(2 * r - 1)) return FL_ERR_CUDA;
+      a.keep = r == dense_loops ? 1 : 0;
+      for (int l = 0; l < L; ++l) {
+        const size_t qo = (size_t)r * ostride_r + (size_t)l * row;
+        a.layer = l;
+        a.q = q + qo;
+        a.k_new = k_new ? k_new + qo : nullptr;
+        a.v_new = v_new ? v_new + qo : nullptr;
+        a.o = o + qo;
+        if (launch_dense(a, s) != cudaSuccess) return FL_ERR_CUDA;
+      }
+    } else {
+      SelectArgs sa;
+      sa.c = a.c;
+      sa.layer0 = 0;
+      sa.n_q = n_q;
+      sa.n_tail = n_tail;
+      sa.k_sel = k_sel;
+      sa.o_prev = o + (size_t)(r - 1) * ostride_r;
+      if (launch_select(sa, L, s) != cudaSuccess) return FL_ERR_CUDA;
+      if (!rec(2 * r - 1)) return FL_ERR_CUDA;
+      a.keep = 1;
+      for (int l = 0; l < L; ++l) {
+        const size_t qo = (size_t)r * ostride_r + (size_t)l * row;
+        a.layer = l;
+        a.q = q + qo;
+        a.k_new = k_new ? k_new + qo : nullptr;
+        a.v_new = v_new ? v_new + qo : nullptr;
+        a.o = o + qo;
+        if (launch_sparse(a, s) != cudaSuccess) return FL_ERR_CUDA;
+      }
+    }
+    if (!rec(2 * r)) return FL_ERR_CUDA;
+  }
+  return FL_OK;
+}
+
+fl_status fl_read_status(const fl_dims* dims, void* cache, int32_t* out, int32_t clear, void* stream) {
+  fl_layout L;
+  fl_status st = make_layout(dims, &L);
+  if (st != FL_OK) return st;
+  if (!cache || !out) return FL_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* dev = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(cache) + L.status);
+  if (cudaMemcpyAsync(out, dev, 3 * sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FL_ERR_CUDA;
+  if (clear) {
+    if (cudaMemsetAsync(dev, 0, 16 * sizeof(int32_t), s) != cudaSuccess) return FL_ERR_CUDA;
+  }
+  return out[0] != 0 ? FL_ERR_DEVICE : FL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,343 @@
+// Dense decode reader: single-query attention of one loop over every column.
+//
+// FlashLoop project page, "The Method": dense loops attend over all columns; a
+// column's key/value in loop r is the loop-1 base plus its residuals of loops 2..r
+// (Step 03), or the loop's BF16 tail row (flashloop 0.1.0 PyPI description,
+// "Configuration and supported scope": 64-token BF16 tail).
+//
+// Work split: grid (splits, heads); a CTA of 8 warps owns a contiguous range of
+// 64-token blocks ("units", plus one unit for the tail).  A warp processes one unit
+// at a time entirely on its own:
+//   1. the block's key (scale, zero) record becomes 128 pre-scaled query weights
+//      (qs'_c = 128 q_c s_c, one constant per group) in the warp's shared slice;
+//   2. 8 coalesced 512-byte loads bring the 64 key rows; lane (row tr, quarter qq)
+//      dots its 32 nibbles with 32 weights, a quad shuffle finishes each logit;
+//   3. each residual loop's rows of the block (consecutive slots) add their logit
+//      contribution through a slot->token map, one group's weights at a time;
+//   4. online softmax (base-2, running max per warp);
+//   5. the value rows (base, then residuals) are accumulated with per-token weights
+//      128 p s and a per-half correction sum(p z - 128 p s).
+// Warps merge in shared memory, CTAs write (M, L, o) partials, and the last CTA of
+// each head (an atomic ticket, no waiting) combines them by log-sum-exp.
+#include "kernels.h"
+
+namespace fl {
+namespace {
+
+constexpr int kWarps = 8;
+
+__global__ void __launch_bounds__(kWarps * 32, 2) dense_kernel(ReaderArgs a) {
+  const int h = blockIdx.y, split = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, qq = lane & 3, tr = lane >> 2;
+  const CacheView& c = a.c;
+  const int H = c.H, cap = c.cap, ncb = cap / kG, T = c.total_slots, r = a.r;
+
+  const uint8_t* kcode = arr<uint8_t>(c, A_KCODE, a.layer) + (size_t)h * cap * 64;
+  const uint8_t* vcode = arr<uint8_t>(c, A_VCODE, a.layer) + (size_t)h * cap * 64;
+  const uint32_t* ksz = arr<uint32_t>(c, A_KSZ, a.layer) + (size_t)h * ncb * kD;
+  const uint32_t* vsz = arr<uint32_t>(c, A_VSZ, a.layer) + (size_t)h * cap * 2;
+  const uint8_t* rkcode = arr<uint8_t>(c, A_RKCODE, a.layer) + (size_t)h * T * 64;
+  const uint8_t* rvcode = arr<uint8_t>(c, A_RVCODE, a.layer) + (size_t)h * T * 64;
+  const uint32_t* rksz = arr<uint32_t>(c, A_RKSZ, a.layer) + (size_t)h * (T / kG) * kD;
+  const uint32_t* rvsz = arr<uint32_t>(c, A_RVSZ, a.layer) + (size_t)h * T * 2;
+  const unsigned long long* mask = arr<unsigned long long>(c, A_MASK, a.layer);
+  const int32_t* first = arr<int32_t>(c, A_FIRST, a.layer);
+  uint16_t* tail_k = arr<uint16_t>(c, A_TAILK, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
+  uint16_t* tail_v = arr<uint16_t>(c, A_TAILV, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
+  float* score = arr<float>(c, A_SCORE, a.layer) + (size_t)h * cap;
+  uint8_t* tag = arr<uint8_t>(c, A_TAG, a.layer) + (size_t)h * cap;
+
+  __shared__ __align__(16) float q_s[kD];
+  __shared__ __align__(16) float qs_w[kWarps][kD];
+  __shared__ float lg_w[kWarps][kG];
+  __shared__ uint8_t tok_w[kWarps][kG];
+  __shared__ float m_w[kWarps], l_w[kWarps];
+  __shared__ __align__(16) float o_w[kWarps][kD];
+  __shared__ int last_cta;
+
+  if (tid < kD) q_s[tid] = __uint_as_float((uint32_t)a.q[(size_t)h * kD + tid] << 16) * kQScale;
+  __syncthreads();
+
+  const int nb = a.n_q / kG;
+  const int n_units = nb + 1;
+  const int u0 = (int)((long long)split * n_units / a.n_splits);
+  const int u1 = (int)((long long)(split + 1) * n_units / a.n_splits);
+  const bool has_new = a.k_new != nullptr;
+
+  float acc[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+  float corr = 0.f, M = -INFINITY, Ls = 0.f;
+  float* qsw = qs_w[warp];
+  float* lgw = lg_w[warp];
+  uint8_t* tokw = tok_w[warp];
+
+  for (int u = u0 + warp; u < u1; u += kWarps) {
+    float qsr[32];
+    if (u < nb) {
+      const int b = u;
+      // ---- keys: base ----
+      __syncwarp();
+      float cb = group_weights(ksz + (size_t)b * kD, q_s, qsw, lane);
+      __syncwarp();
+      load32(qsw + 32 * qq, qsr);
+      const uint4* kc = reinterpret_cast<const uint4*>(kcode + (size_t)b * kG * 64);
+      uint4 w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __ldg(kc + 32 * i + lane);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float p = dot32(w[i], qsr);
+        p += __shfl_xor_sync(kFull, p, 1);
+        p += __shfl_xor_sync(kFull, p, 2);
+        if (qq == 0) lgw[8 * i + tr] = p + cb;
+      }
+      // ---- keys: residual loops 2..r ----
+      for (int rp = 2; rp <= r; ++rp) {
+        const unsigned long long mk = mask[(size_t)rp * ncb + b];
+        if (mk == 0ull) continue;
+        const int na = __popcll(mk);
+        const int gs0 = c.slot_base[rp] + first[(size_t)rp * ncb + b];
+        __syncwarp();
+        for (int tt = lane; tt < kG; tt += 32)
+          if ((mk >> tt) & 1ull) tokw[__popcll(mk & ((1ull << tt) - 1ull))] = (uint8_t)tt;
+        int row = 0;
+        while (row < na) {
+          const int grp = (gs0 + row) >> 6;
+          const int row_end = min(na, ((grp + 1) << 6) - gs0);
+          __syncwarp();
+          const float cg = group_weights(rksz + (size_t)grp * kD, q_s, qsw, lane);
+          __syncwarp();
+          load32(qsw + 32 * qq, qsr);
+          for (int i0 = row; i0 < row_end; i0 += 8) {
+            const int rw = i0 + tr;
+            const bool act = rw < row_end;
+            uint4 x = make_uint4(0u, 0u, 0u, 0u);
+            if (act) x = __ldg(reinterpret_cast<const uint4*>(rkcode + (size_t)(gs0 + rw) * 64) + qq);
+            float p = dot32(x, qsr);
+            p += __shfl_xor_sync(kFull, p, 1);
+            p += __shfl_xor_sync(kFull, p, 2);
+            if (act && qq == 0) lgw[tokw[rw]] += p + cg;
+          }
+          row = row_end;
+        }
+      }
+      __syncwarp();
+      // ---- online softmax over the block ----
+      const float l0 = lgw[lane], l1 = lgw[lane + 32];
+      if (a.keep) {
+        score[(size_t)b * kG + lane] = l0;
+        score[(size_t)b * kG + lane + 32] = l1;
+        tag[(size_t)b * kG + lane] = (uint8_t)r;
+        tag[(size_t)b * kG + lane + 32] = (uint8_t)r;
+      }
+      const float mb = warp_max(fmaxf(l0, l1));
+      if (mb > M) {
+        const float al = ex2(M - mb);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) acc[k] *= al;
+        corr *= al;
+        Ls *= al;
+        M = mb;
+      }
+      const float p0 = ex2(l0 - M), p1 = ex2(l1 - M);
+      Ls += p0 + p1;
+      __syncwarp();
+      lgw[lane] = p0;
+      lgw[lane + 32] = p1;
+      __syncwarp();
+      // ---- values: base ----
+      {
+        const uint4* vc = reinterpret_cast<const uint4*>(vcode + (size_t)b * kG * 64);
+        const uint32_t* vs = vsz + (size_t)b * kG * 2;
+        uint4 vw[8];
+        uint32_t sw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          vw[i] = __ldg(vc + 32 * i + lane);
+          sw[i] = __ldg(vs + 2 * (8 * i + tr) + (qq >> 1));
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float p = lgw[8 * i + tr];
+          const float2 sz = unpack_sz(sw[i]);
+          const float P = 128.f * (p * sz.x);
+          corr += fmaf(p, sz.y, -P);
+          axpy32(vw[i], P, acc);
+        }
+      }
+      // ---- values: residual loops ----
+      for (int rp = 2; rp <= r; ++rp) {
+        const unsigned long long mk = mask[(size_t)rp * ncb + b];
+        if (mk == 0ull) continue;
+        const int na = __popcll(mk);
+        const int gs0 = c.slot_base[rp] + first[(size_t)rp * ncb + b];
+        __syncwarp();
+        for (int tt = lane; tt < kG; tt += 32)
+          if ((mk >> tt) & 1ull) tokw[__popcll(mk & ((1ull << tt) - 1ull))] = (uint8_t)tt;
+        __syncwarp();
+        for (int i0 = 0; i0 < na; i0 += 8) {
+          const int rw = i0 + tr;
+          if (rw < na) {
+            const int gs = gs0 + rw;
+            const uint4 x = __ldg(reinterpret_cast<const uint4*>(rvcode + (size_t)gs * 64) + qq);
+            const float2 sz = unpack_sz(__ldg(rvsz + (size_t)gs * 2 + (qq >> 1)));
+            const float p = lgw[tokw[rw]];
+            const float P = 128.f * (p * sz.x);
+            corr += fmaf(p, sz.y, -P);
+            axpy32(x, P, acc);
+          }
+        }
+      }
+    } else {
+      // ---- BF16 tail unit: rows [0, n_tail) of this loop; row n_tail-1 may be new ----
+      const int nt = a.n_tail;
+      if (has_new) {
+        __syncwarp();
+        const uint2* kn = reinterpret_cast<const uint2*>(a.k_new + (size_t)h * kD);
+        const uint2* vn = reinterpret_cast<const uint2*>(a.v_new + (size_t)h * kD);
+        reinterpret_cast<uint2*>(tail_k + (size_t)(nt - 1) * kD)[lane] = kn[lane];
+        reinterpret_cast<uint2*>(tail_v + (size_t)(nt - 1) * kD)[lane] = vn[lane];
+      }
+      load32(q_s + 32 * qq, qsr);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = 8 * i + tr;
+        const bool act = t < nt;
+        float p = 0.f;
+        if (act) {
+          const uint16_t* row = (has_new && t == nt - 1) ? a.k_new + (size_t)h * kD : tail_k + (size_t)t * kD;
+          p = dot_bf16_32(row + 32 * qq, qsr);
+        }
+        p += __shfl_xor_sync(kFull, p, 1);
+        p += __shfl_xor_sync(kFull, p, 2);
+        if (qq == 0) lgw[t] = act ? p : -INFINITY;
+      }
+      __syncwarp();
+      const float l0 = lgw[lane], l1 = lgw[lane + 32];
+      if (a.keep) {
+        if (lane < nt) {
+          score[(size_t)a.n_q + lane] = l0;
+          tag[(size_t)a.n_q + lane] = (uint8_t)r;
+        }
+        if (lane + 32 < nt) {
+          score[(size_t)a.n_q + lane + 32] = l1;
+          tag[(size_t)a.n_q + lane + 32] = (uint8_t)r;
+        }
+      }
+      const float mb = warp_max(fmaxf(l0, l1));
+      if (mb > M) {
+        const float al = ex2(M - mb);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) acc[k] *= al;
+        corr *= al;
+        Ls *= al;
+        M = mb;
+      }
+      const float p0 = ex2(l0 - M), p1 = ex2(l1 - M);
+      Ls += p0 + p1;
+      __syncwarp();
+      lgw[lane] = p0;
+      lgw[lane + 32] = p1;
+      __syncwarp();
+      for (int i = 0; i < 8; ++i) {
+        const int t = 8 * i + tr;
+        if (t < nt) {
+          const uint16_t* row = (has_new && t == nt - 1) ? a.v_new + (size_t)h * kD : tail_v + (size_t)t * kD;
+          axpy_bf16_32(row + 32 * qq, lgw[t], acc);
+        }
+      }
+    }
+  }
+
+  // ---- warp reduction: lanes sharing a channel quarter ----
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    acc[k] += __shfl_xor_sync(kFull, acc[k], 4);
+    acc[k] += __shfl_xor_sync(kFull, acc[k], 8);
+    acc[k] += __shfl_xor_sync(kFull, acc[k], 16);
+  }
+  corr += __shfl_xor_sync(kFull, corr, 4);
+  corr += __shfl_xor_sync(kFull, corr, 8);
+  corr += __shfl_xor_sync(kFull, corr, 16);
+  Ls = warp_sum(Ls);
+  if (tr == 0) {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) o_w[warp][32 * qq + k] = acc[k] + corr;
+  }
+  if (lane == 0) {
+    m_w[warp] = M;
+    l_w[warp] = Ls;
+  }
+  __syncthreads();
+
+  // ---- CTA partial (M, L, o) ----
+  float* part = a.part + ((size_t)h * a.n_splits + split) * kPartStride;
+  if (tid < kD) {
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) Mx = fmaxf(Mx, m_w[w]);
+    float Lt = 0.f, ot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      if (m_w[w] != -INFINITY) {
+        const float e = ex2(m_w[w] - Mx);
+        Lt = fmaf(l_w[w], e, Lt);
+        ot = fmaf(o_w[w][tid], e, ot);
+      }
+    }
+    part[4 + tid] = ot;
+    if (tid == 0) {
+      part[0] = Mx;
+      part[1] = Lt;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last_cta = (atomicAdd(&a.counter[h], 1) == a.n_splits - 1);
+  __syncthreads();
+  if (!last_cta) return;
+  __threadfence();
+
+  // ---- last CTA of this head: log-sum-exp combine of every split ----
+  if (tid < kD) {
+    const float* hp = a.part + (size_t)h * a.n_splits * kPartStride;
+    float Mx = -INFINITY;
+    for (int s = 0; s < a.n_splits; ++s) Mx = fmaxf(Mx, __ldcg(hp + (size_t)s * kPartStride));
+    float Lt = 0.f, ot = 0.f;
+    for (int s = 0; s < a.n_splits; ++s) {
+      const float ms = __ldcg(hp + (size_t)s * kPartStride);
+      if (ms == -INFINITY) continue;
+      const float e = ex2(ms - Mx);
+      Lt = fmaf(__ldcg(hp + (size_t)s * kPartStride + 1), e, Lt);
+      ot = fmaf(__ldcg(hp + (size_t)s * kPartStride + 4 + tid), e, ot);
+    }
+    a.o[(size_t)h * kD + tid] = ot / Lt;
+    if (tid == 0) {
+      arr<float>(c, A_OFFSET, a.layer)[(size_t)h * kOffStride + r] = Mx + log2f(Lt);
+      a.counter[h] = 0;
+    }
+  }
+}
+
+}  // namespace
+
+int dense_splits(int heads, int n_q) {
+  const int n_units = n_q / kG + 1;
+  int by_work = (n_units + 2 * kWarps - 1) / (2 * kWarps);  // >= ~2 units per warp
+  int by_sms = (148 * 2) / heads;                            // one wave at 2 CTAs per SM
+  int s = by_work < by_sms ? by_work : by_sms;
+  if (s < 1) s = 1;
+  if (s > n_units) s = n_units;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return s;
+}
+
+cudaError_t launch_dense(ReaderArgs a, cudaStream_t s) {
+  a.n_splits = dense_splits(a.c.H, a.n_q);
+  dim3 grid(a.n_splits, a.c.H);
+  dense_kernel<<<grid, kWarps * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fl

@@ -1,0 +1,51 @@
+// Internal launcher declarations shared by the CUDA translation units.
+#pragma once
+
+#include "common.cuh"
+
+namespace fl {
+
+struct EncodeBaseArgs {
+  CacheView c;
+  int layer, row0, n_rows;
+  const uint16_t* k;
+  const uint16_t* v;
+  int64_t head_stride;
+};
+
+struct EncodeResArgs {
+  CacheView c;
+  int layer, r, row0, n_span, slot0, n_rows, compact;
+  const int32_t* rows;
+  const uint16_t* k;
+  const uint16_t* v;
+  int64_t head_stride;
+};
+
+struct ReaderArgs {
+  CacheView c;
+  int layer, r, n_q, n_tail, k_sel, n_splits, keep;
+  const uint16_t* q;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  float* o;
+  float* part;
+  int32_t* counter;
+};
+
+struct SelectArgs {
+  CacheView c;
+  int layer0, n_q, n_tail, k_sel;
+  const float* o_prev;
+};
+
+cudaError_t launch_encode_base(const EncodeBaseArgs& a, cudaStream_t s);
+cudaError_t launch_encode_residual(const EncodeResArgs& a, cudaStream_t s);
+cudaError_t launch_dense(ReaderArgs a, cudaStream_t s);
+cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s);
+cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s);
+
+int dense_splits(int heads, int n_q);
+int sparse_splits(int heads, int k_sel);
+
+}  // namespace fl

@@ -1,0 +1,260 @@
+// Column selector for sparse loops: top-K of the preceding loop's distribution, the
+// selected mass m, and the unselected columns' contribution u.
+//
+// FlashLoop project page, "The Method", Step 02: the preceding loop identifies the
+// columns to recompute, and their global probability mass under the preceding loop's
+// full distribution is cached so the sparse softmax is not renormalised to 1.
+// flozi guide "FlashLoop: store changes between repeated passes", section 3: each
+// sparse loop ranks key columns by the previous loop's attention statistics.
+//
+// One CTA (1024 threads) per (layer, head), launched for a range of layers at once.
+//   keys:     log2 p~_j = score_j - offset[tag_j], mapped to an order-preserving u32
+//             and kept in shared memory (N <= FL_MAX_SELECT_COLS);
+//   select:   radix select of the K-th largest key, digits 12 + 12 + 8 bits, each
+//             pass a shared-memory histogram over the keys that still match the
+//             prefix and a block-wide scan from the top bin;
+//   compact:  keys above the threshold plus the lowest-index ties, written in index
+//             order (per-warp ballots and a block prefix), so S is ascending;
+//   m, u:     m = sum_S p~_j; u = o_prev - sum_S p~_j v_j with v_j the column's value
+//             at loop tag_j (base plus residuals up to min(tag_j, depth_j), or the
+//             tail row of loop tag_j).
+#include "kernels.h"
+
+namespace fl {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kWarpsSel = kThreads / 32;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// Inclusive block scan of one value per thread (1024 threads).
+__device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* wtot, int lane, int warp) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += n;
+  }
+  __syncthreads();
+  if (lane == 31) wtot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t t = wtot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(kFull, t, o);
+      if (lane >= o) t += n;
+    }
+    wtot[lane] = t;
+  }
+  __syncthreads();
+  return v + (warp > 0 ? wtot[warp - 1] : 0u);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
+  extern __shared__ uint32_t keys[];
+  __shared__ __align__(16) uint32_t hist[4096];
+  __shared__ float offs[kOffStride];
+  __shared__ uint32_t wtot[32];
+  __shared__ uint32_t sh_digit, sh_krem;
+  __shared__ float red[32];
+
+  const int h = blockIdx.x, layer = a.layer0 + blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const CacheView& c = a.c;
+  const int H = c.H, cap = c.cap, ncb = cap / kG, T = c.total_slots, R = c.R;
+  const int n_q = a.n_q, N = a.n_q + a.n_tail, K = a.k_sel;
+
+  const float* score = arr<float>(c, A_SCORE, layer) + (size_t)h * cap;
+  const uint8_t* tag = arr<uint8_t>(c, A_TAG, layer) + (size_t)h * cap;
+  int32_t* sel = arr<int32_t>(c, A_SEL, layer) + (size_t)h * c.max_select;
+
+  if (tid < kOffStride) offs[tid] = arr<float>(c, A_OFFSET, layer)[(size_t)h * kOffStride + tid];
+  __syncthreads();
+  for (int j = tid; j < N; j += kThreads) {
+    int t = tag[j];
+    if (t < 1 || t > R) {
+      record_error(c.status, FL_DEV_TAG_RANGE, j);
+      t = t < 1 ? 1 : R;
+    }
+    keys[j] = order_key(score[j] - offs[t]);
+  }
+  __syncthreads();
+
+  // ---- radix select of the K-th largest key ----
+  uint32_t prefix = 0u, pmask = 0u, krem = (uint32_t)K;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
+    const int nbins = pass < 2 ? 4096 : 256;
+    const uint32_t dmask = (uint32_t)nbins - 1u;
+    for (int i = tid; i < nbins; i += kThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int j = tid; j < N; j += kThreads) {
+      const uint32_t u = keys[j];
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    // thread t owns bins [nbins - per*(t+1), nbins - per*t), i.e. descending order
+    const int per = nbins / kThreads > 0 ? nbins / kThreads : 1;
+    const int owners = nbins / per;
+    uint32_t local = 0u;
+    if (tid < owners)
+      for (int i = 0; i < per; ++i) local += hist[nbins - per * tid - 1 - i];
+    const uint32_t incl = block_scan(local, wtot, lane, warp);
+    const uint32_t excl = incl - local;
+    if (tid < owners && excl < krem && krem <= incl) {
+      uint32_t cum = excl;
+      for (int i = 0; i < per; ++i) {
+        const int bin = nbins - per * tid - 1 - i;
+        if (cum + hist[bin] >= krem) {
+          sh_digit = (uint32_t)bin;
+          sh_krem = krem - cum;
+          break;
+        }
+        cum += hist[bin];
+      }
+    }
+    __syncthreads();
+    prefix |= sh_digit << shift;
+    pmask |= dmask << shift;
+    krem = sh_krem;
+    __syncthreads();
+  }
+  const uint32_t thr = prefix;  // the K-th largest key; take krem of the keys equal to it
+
+  // ---- compaction in index order ----
+  const int chunk = ((((N + kWarpsSel - 1) / kWarpsSel) + 31) / 32) * 32;
+  const int wbeg = warp * chunk;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t eqc = 0u;
+  for (int i = 0; i < chunk; i += 32) {
+    const int j = wbeg + i + lane;
+    eqc += __popc(__ballot_sync(kFull, j < N && keys[j] == thr));
+  }
+  if (lane == 0) wtot[warp] = eqc;
+  __syncthreads();
+  uint32_t eq_base = 0u;
+  for (int w = 0; w < warp; ++w) eq_base += wtot[w];
+  __syncthreads();
+  uint32_t selc = 0u, eqrun = eq_base;
+  for (int i = 0; i < chunk; i += 32) {
+    const int j = wbeg + i + lane;
+    const uint32_t u = j < N ? keys[j] : 0u;
+    const unsigned be = __ballot_sync(kFull, j < N && u == thr);
+    const bool s = (j < N && u > thr) || (j < N && u == thr && eqrun + __popc(be & lt) < krem);
+    eqrun += __popc(be);
+    selc += __popc(__ballot_sync(kFull, s));
+  }
+  if (lane == 0) wtot[warp] = selc;
+  __syncthreads();
+  uint32_t pos = 0u;
+  for (int w = 0; w < warp; ++w) pos += wtot[w];
+  eqrun = eq_base;
+  float mpart = 0.f;
+  for (int i = 0; i < chunk; i += 32) {
+    const int j = wbeg + i + lane;
+    const uint32_t u = j < N ? keys[j] : 0u;
+    const unsigned be = __ballot_sync(kFull, j < N && u == thr);
+    const bool s = (j < N && u > thr) || (j < N && u == thr && eqrun + __popc(be & lt) < krem);
+    eqrun += __popc(be);
+    const unsigned bs = __ballot_sync(kFull, s);
+    if (s) {
+      sel[pos + __popc(bs & lt)] = j;
+      mpart += ex2(key_value(u));
+    }
+    pos += __popc(bs);
+  }
+  mpart = warp_sum(mpart);
+  if (lane == 0) red[warp] = mpart;
+  __syncthreads();
+
+  // ---- u = o_prev - sum_S p~_j v_j(tag_j) ----
+  const uint8_t* vcode = arr<uint8_t>(c, A_VCODE, layer) + (size_t)h * cap * 64;
+  const uint32_t* vsz = arr<uint32_t>(c, A_VSZ, layer) + (size_t)h * cap * 2;
+  const uint8_t* rvcode = arr<uint8_t>(c, A_RVCODE, layer) + (size_t)h * T * 64;
+  const uint32_t* rvsz = arr<uint32_t>(c, A_RVSZ, layer) + (size_t)h * T * 2;
+  const unsigned long long* mask = arr<unsigned long long>(c, A_MASK, layer);
+  const int32_t* first = arr<int32_t>(c, A_FIRST, layer);
+  const uint8_t* depth = arr<uint8_t>(c, A_DEPTH, layer);
+  const uint16_t* tail_v = arr<uint16_t>(c, A_TAILV, layer);
+  const int qq = tid & 3;
+  float acc[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+  float corr = 0.f;
+  for (int task = tid; task < 4 * K; task += kThreads) {
+    const int j = sel[task >> 2];
+    const float p = ex2(key_value(keys[j]));
+    int lam = tag[j];
+    lam = lam < 1 ? 1 : (lam > R ? R : lam);
+    if (j < n_q) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(vcode + (size_t)j * 64) + qq);
+      const float2 sz = unpack_sz(__ldg(vsz + (size_t)j * 2 + (qq >> 1)));
+      const float P = 128.f * (p * sz.x);
+      corr += fmaf(p, sz.y, -P);
+      axpy32(x, P, acc);
+      const int dep = depth[j];
+      const int top = lam < dep ? lam : dep;
+      const int b = j >> 6, jt = j & 63;
+      for (int rp = 2; rp <= top; ++rp) {
+        const unsigned long long mk = mask[(size_t)rp * ncb + b];
+        const int gs = c.slot_base[rp] + first[(size_t)rp * ncb + b] + __popcll(mk & ((1ull << jt) - 1ull));
+        const uint4 y = __ldg(reinterpret_cast<const uint4*>(rvcode + (size_t)gs * 64) + qq);
+        const float2 s2 = unpack_sz(__ldg(rvsz + (size_t)gs * 2 + (qq >> 1)));
+        const float P2 = 128.f * (p * s2.x);
+        corr += fmaf(p, s2.y, -P2);
+        axpy32(y, P2, acc);
+      }
+    } else {
+      const uint16_t* row = tail_v + (((size_t)(lam - 1) * H + h) * kTail + (j - n_q)) * kD;
+      axpy_bf16_32(row + 32 * qq, p, acc);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    acc[k] += __shfl_xor_sync(kFull, acc[k], 4);
+    acc[k] += __shfl_xor_sync(kFull, acc[k], 8);
+    acc[k] += __shfl_xor_sync(kFull, acc[k], 16);
+  }
+  corr += __shfl_xor_sync(kFull, corr, 4);
+  corr += __shfl_xor_sync(kFull, corr, 8);
+  corr += __shfl_xor_sync(kFull, corr, 16);
+  float* ored = reinterpret_cast<float*>(hist);  // [32 warps][128]
+  if (lane < 4) {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) ored[warp * kD + 32 * qq + k] = acc[k] + corr;
+  }
+  __syncthreads();
+  if (tid < kD) {
+    float s = 0.f;
+    for (int w = 0; w < kWarpsSel; ++w) s += ored[w * kD + tid];
+    const float op = a.o_prev[((size_t)blockIdx.y * H + h) * kD + tid];
+    arr<float>(c, A_UNSEL, layer)[(size_t)h * kD + tid] = op - s;
+  }
+  if (tid == 0) {
+    float m = 0.f;
+    for (int w = 0; w < kWarpsSel; ++w) m += red[w];
+    arr<float>(c, A_MASS, layer)[h] = m;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s) {
+  const int N = a.n_q + a.n_tail;
+  const size_t smem = (size_t)N * sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(FL_MAX_SELECT_COLS * sizeof(uint32_t)));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.c.H, n_layers);
+  select_kernel<<<grid, kThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fl

@@ -1,0 +1,195 @@
+"""Test-side helpers: unpack the library's packed cache into logical arrays, build a
+GPU cache and an oracle from the same synthetic inputs, and compare them."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synth
+from oracle import flashloop_oracle as fo
+from quantized_kv_attention_int4_b200 import abi
+from quantized_kv_attention_int4_b200.cache import FlashLoopCache, round_up, split_prefill
+
+TOL = 2e-3
+
+
+def f32(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy()
+
+
+def nibbles(raw: np.ndarray) -> np.ndarray:
+    """[..., 64] packed bytes -> [..., 128] codes (byte b = channels 2b low, 2b+1 high)."""
+    out = np.empty(raw.shape[:-1] + (raw.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = raw & 15
+    out[..., 1::2] = raw >> 4
+    return out
+
+
+def split_sz(raw: np.ndarray):
+    """uint32 (scale | zero << 16) -> (scale f16, zero f16)."""
+    return (raw & 0xFFFF).astype(np.uint16).view(np.float16), (raw >> 16).astype(np.uint16).view(np.float16)
+
+
+class Unpacked:
+    """Logical views of one layer of a FlashLoopCache (CPU copies)."""
+
+    def __init__(self, cache: FlashLoopCache, layer: int = 0):
+        H, C, R = cache.H, cache.capacity, cache.R
+        T = cache.layout.total_slots
+        g = lambda n: cache.raw(n, layer).cpu().numpy()
+        self.kc = nibbles(g("kcode")[: H * C * 64].reshape(H, C, 64))
+        self.vc = nibbles(g("vcode")[: H * C * 64].reshape(H, C, 64))
+        self.ks, self.kz = split_sz(g("ksz").view(np.uint32)[: H * (C // 64) * 128].reshape(H, C // 64, 128))
+        self.vs, self.vz = split_sz(g("vsz").view(np.uint32)[: H * C * 2].reshape(H, C, 2))
+        self.rkc = nibbles(g("rkcode")[: H * T * 64].reshape(H, T, 64))
+        self.rvc = nibbles(g("rvcode")[: H * T * 64].reshape(H, T, 64))
+        self.rks, self.rkz = split_sz(g("rksz").view(np.uint32)[: H * (T // 64) * 128].reshape(H, T // 64, 128))
+        self.rvs, self.rvz = split_sz(g("rvsz").view(np.uint32)[: H * T * 2].reshape(H, T, 2))
+        self.mask = g("mask").view(np.uint64)[: (R + 1) * (C // 64)].reshape(R + 1, C // 64)
+        self.first = g("first").view(np.int32)[: (R + 1) * (C // 64)].reshape(R + 1, C // 64)
+        self.depth = g("depth")[:C]
+        self.slot_base = list(cache.layout.slot_base)
+
+
+def selection(cache: FlashLoopCache, layer: int, k_sel: int):
+    H, ms = cache.H, cache.dims.max_select
+    S = cache.raw("sel", layer).view(torch.int32)[: H * ms].view(H, ms)[:, :k_sel].cpu().numpy().astype(np.int64)
+    m = cache.raw("mass", layer).view(torch.float32)[:H].cpu().numpy().astype(np.float64)
+    u = cache.raw("unsel", layer).view(torch.float32)[: H * 128].view(H, 128).cpu().numpy().astype(np.float64)
+    return S, m, u
+
+
+def rel_err(got, ref) -> float:
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    num = np.abs(got - ref).reshape(ref.shape[0], -1).max(axis=1)
+    den = np.abs(ref).reshape(ref.shape[0], -1).max(axis=1)
+    return float((num / np.maximum(den, 1e-30)).max())
+
+
+def check_topk_valid(S, p_tilde, k):
+    """S (per head, ascending, unique) is a top-k of p_tilde up to tau = 1e-5 * max p_tilde."""
+    H, N = p_tilde.shape
+    for h in range(H):
+        s = S[h]
+        assert s.shape == (k,) and np.all(np.diff(s) > 0) and s[0] >= 0 and s[-1] < N
+        tau = 1e-5 * p_tilde[h].max()
+        inside = np.zeros(N, bool)
+        inside[s] = True
+        if k < N:
+            assert p_tilde[h][inside].min() >= p_tilde[h][~inside].max() - tau
+
+
+class Pair:
+    """A one-layer GPU cache and its oracle, built from the same synthetic prompt."""
+
+    def __init__(self, w: synth.Workload, heads=None, extra_tokens: int = 0, layer: int = 0, data=None):
+        self.w = w
+        self.layer = layer
+        n = w.n_ctx
+        self.heads = list(range(w.heads)) if heads is None else list(heads)
+        cap = round_up(n + extra_tokens + 64)
+        self.cache = FlashLoopCache(1, w.heads, w.loops, cap, max_select=cap)
+        d = synth.prefill_layer(w, layer, device="cuda") if data is None else data
+        self.sets = d["sets"]
+        n_q, n_tail, tail_depth = self.cache.prefill_layer(0, d["K"], d["V"], self.sets)
+        self.cache.set_timeline(n_q, n_tail, tail_depth)
+        hs = self.heads
+        self.oracle = fo.OracleLayer(len(hs), w.loops, cap)
+        lay = self.oracle
+        lay.encode_base(0, f32(d["K"][1][hs, :n_q]), f32(d["V"][1][hs, :n_q]))
+        self.calls = {r: [] for r in range(2, w.loops + 1)}
+        for r in range(2, w.loops + 1):
+            rows = self.sets[r][self.sets[r] < n_q].numpy()
+            lay.encode_residual(r, rows, f32(d["K"][r][hs][:, rows]), f32(d["V"][r][hs][:, rows]))
+            self.calls[r].append((0, len(rows)))
+        lay.set_tail([None] + [f32(d["K"][r][hs, n_q:]) for r in range(1, w.loops + 1)],
+                     [None] + [f32(d["V"][r][hs, n_q:]) for r in range(1, w.loops + 1)], np.array(tail_depth))
+        del d
+
+    # -- decode --------------------------------------------------------------------
+    def begin_token(self, step: int):
+        """Append decode token ``step`` (flushing a full tail first) on both sides."""
+        w, hs = self.w, self.heads
+        if self.cache.n_tail == 64:
+            for r in range(2, w.loops + 1):
+                slot0 = round_up(self.cache.n_slots[0][r])
+                self.calls[r].append((slot0, sum(1 for dep in self.cache.tail_depth if dep >= r)))
+        self.cache.begin_token()
+        tok = synth.decode_token(w, self.layer, step, device="cuda")
+        self.oracle.append_token([None] + [f32(tok["k"][r][hs]) for r in range(1, w.loops + 1)],
+                                 [None] + [f32(tok["v"][r][hs]) for r in range(1, w.loops + 1)])
+        return tok
+
+    def run_loops(self, q, tok=None, k_sel=None, loops=None, check=True):
+        """Every loop of one decode step on the GPU and in the oracle; returns per-loop errors."""
+        w, hs, c, lay = self.w, self.heads, self.cache, self.oracle
+        H = w.heads
+        N = c.n_cols
+        k_sel = w.k_sel(N) if k_sel is None else k_sel
+        errs = {}
+        o_prev = None
+        for r in range(1, (loops or w.loops) + 1):
+            o = torch.empty(H, 128, dtype=torch.float32, device="cuda")
+            kn = tok["k"][r] if tok else None
+            vn = tok["v"][r] if tok else None
+            qr = q[r].contiguous()
+            if r <= w.dense_loops:
+                c.dense(0, r, qr, o, kn, vn, keep_scores=True)
+                ref = lay.dense_loop(r, f32(q[r][hs]))
+                errs[r] = rel_err(o.cpu().numpy()[hs], ref["o"])
+            else:
+                c.select(0, 1, k_sel, o_prev.view(1, H, 128))
+                S, m, u = selection(c, 0, k_sel)
+                if check:
+                    check_topk_valid(S[hs], lay.p_tilde, k_sel)
+                c.sparse(0, r, k_sel, qr, o, kn, vn)
+                ref = lay.sparse_loop(r, f32(q[r][hs]), S[hs])
+                errs[(r, "m")] = float(np.max(np.abs(m[hs] - ref["m"]) / ref["m"]))
+                scale = np.maximum(np.abs(ref["u"]).max(axis=1), np.abs(ref["o"]).max(axis=1))
+                errs[(r, "u")] = float((np.abs(u[hs] - ref["u"]).max(axis=1) / scale).max())
+                errs[r] = rel_err(o.cpu().numpy()[hs], ref["o"])
+            o_prev = o
+        st, info = c.status()
+        assert st == abi.FL_OK, info
+        return errs
+
+
+def compare_encoding(pair: Pair):
+    """Codes, scales and zero points of base and residual stores are bit-exact; the
+    block masks / first slots / depths address exactly the oracle's slots."""
+    U = Unpacked(pair.cache)
+    lay, hs, n_q = pair.oracle, pair.heads, pair.cache.n_q
+    nb = n_q // 64
+    u16 = lambda a: np.ascontiguousarray(a).view(np.uint16)
+    assert np.array_equal(U.kc[hs, :n_q], lay.base["kc"][:, :n_q])
+    assert np.array_equal(U.vc[hs, :n_q], lay.base["vc"][:, :n_q])
+    assert np.array_equal(u16(U.ks[hs, :nb]), u16(lay.base["ks"][:, :nb]))
+    assert np.array_equal(u16(U.kz[hs, :nb]), u16(lay.base["kz"][:, :nb]))
+    assert np.array_equal(u16(U.vs[hs, :n_q]), u16(lay.base["vs"][:, :n_q]))
+    assert np.array_equal(u16(U.vz[hs, :n_q]), u16(lay.base["vz"][:, :n_q]))
+    assert np.array_equal(U.depth[:n_q], lay.depth[:n_q])
+    for r in range(2, pair.w.loops + 1):
+        assert len(pair.calls[r]) == len(lay.calls[r])
+        for (slot0, n), call in zip(pair.calls[r], lay.calls[r]):
+            enc = call["enc"]
+            g0 = U.slot_base[r] + slot0
+            ng = -(-n // 64)
+            assert np.array_equal(U.rkc[hs, g0:g0 + n], enc["kc"])
+            assert np.array_equal(U.rvc[hs, g0:g0 + n], enc["vc"])
+            assert not U.rkc[hs, g0 + n:g0 + ng * 64].any()
+            assert np.array_equal(u16(U.rks[hs, g0 // 64:g0 // 64 + ng]), u16(enc["ks"]))
+            assert np.array_equal(u16(U.rkz[hs, g0 // 64:g0 // 64 + ng]), u16(enc["kz"]))
+            assert np.array_equal(u16(U.rvs[hs, g0:g0 + n]), u16(enc["vs"]))
+            assert np.array_equal(u16(U.rvz[hs, g0:g0 + n]), u16(enc["vz"]))
+            rows = call["rows"]
+            for i, j in enumerate(rows.tolist()):
+                b, t = j // 64, j % 64
+                mk = int(U.mask[r, b])
+                assert (mk >> t) & 1
+                assert U.first[r, b] + bin(mk & ((1 << t) - 1)).count("1") == slot0 + i
+        act = lay.depth[:n_q] >= r
+        bits = np.zeros(nb, np.uint64)
+        for j in np.nonzero(act)[0].tolist():
+            bits[j // 64] |= np.uint64(1 << (j % 64))
+        assert np.array_equal(U.mask[r, :nb], bits)

@@ -1,0 +1,137 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol the header
+declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_kv_attention_int4_b200 import abi
+from quantized_kv_attention_int4_b200.cache import round_up, split_prefill
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "flashloop.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:fl_status|size_t|const char\*)\s+(fl_\w+)\s*\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) == 14
+    for n in names:
+        assert hasattr(abi.lib, n), n
+    assert set(names) == set(abi.EXPORTED)
+    assert "sm_100a" in abi.fl_version()
+
+
+def _dims(**kw):
+    base = dict(layers=2, heads=4, loops=4, capacity=1024, max_select=128,
+                res_capacity={2: 1024, 3: 256, 4: 128})
+    base.update(kw)
+    return abi.Dims(**base)
+
+
+def test_layout_is_aligned_and_consistent():
+    d = _dims()
+    L = abi.fl_cache_layout(d)
+    offs = [getattr(L, n) for n in abi.ARRAY_NAMES] + [L.status]
+    assert all(o % 256 == 0 for o in offs)
+    assert offs == sorted(offs) and len(set(offs)) == len(offs)
+    assert list(L.slot_base)[2:5] == [0, 1024, 1280] and L.total_slots == 1408
+    H, C, T = 4, 1024, 1408
+    assert L.layer_stride[0] == H * C * 64                      # kcode
+    assert L.layer_stride[2] == H * (C // 64) * 128 * 4         # ksz
+    assert L.layer_stride[6] == H * (T // 64) * 128 * 4         # rksz
+    assert L.layer_stride[11] == 4 * H * 64 * 128 * 2           # tail_k
+    for i, name in enumerate(abi.ARRAY_NAMES[:-1]):
+        nxt = getattr(L, abi.ARRAY_NAMES[i + 1])
+        assert getattr(L, name) + 2 * L.layer_stride[i] == nxt
+    assert L.total_bytes >= L.status + 64
+
+
+@pytest.mark.parametrize("kw,st", [
+    (dict(capacity=1000), abi.FL_ERR_INVALID),
+    (dict(loops=33), abi.FL_ERR_INVALID),
+    (dict(max_select=0), abi.FL_ERR_INVALID),
+    (dict(res_capacity={2: 100}), abi.FL_ERR_INVALID),
+])
+def test_bad_dims_are_rejected(kw, st):
+    out = abi.fl_layout()
+    assert abi._c_cache_layout(ctypes.byref(_dims(**kw)), ctypes.byref(out)) == st
+
+
+def test_unsupported_head_dim_and_group():
+    d = _dims()
+    d.head_dim = 64
+    assert abi._c_cache_layout(ctypes.byref(d), ctypes.byref(abi.fl_layout())) == abi.FL_ERR_UNSUPPORTED
+    d = _dims()
+    d.group = 32
+    assert abi._c_workspace_bytes(ctypes.byref(d)) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails validation first
+
+
+def test_reader_arguments_are_validated_before_launch():
+    d = _dims()
+    ws = abi.fl_workspace_bytes(d)
+    dense = lambda **k: abi._c_dense(ctypes.byref(d), k.get("cache", FAKE), k.get("layer", 0), k.get("loop", 1),
+                                     k.get("n_q", 64), k.get("n_tail", 1), FAKE, k.get("kn"), k.get("vn"), FAKE,
+                                     1, FAKE, k.get("ws", ws), None)
+    assert dense(cache=None) == abi.FL_ERR_INVALID
+    assert dense(layer=2) == abi.FL_ERR_INVALID
+    assert dense(loop=5) == abi.FL_ERR_INVALID
+    assert dense(loop=0) == abi.FL_ERR_INVALID
+    assert dense(n_q=65) == abi.FL_ERR_INVALID
+    assert dense(n_tail=0) == abi.FL_ERR_INVALID
+    assert dense(n_tail=65) == abi.FL_ERR_INVALID
+    assert dense(n_q=1024) == abi.FL_ERR_INVALID          # exceeds capacity
+    assert dense(kn=FAKE) == abi.FL_ERR_INVALID            # k_new without v_new
+    assert dense(ws=ws - 1) == abi.FL_ERR_WORKSPACE
+    sparse = lambda k_sel: abi._c_sparse(ctypes.byref(d), FAKE, 0, 3, 64, 1, k_sel, FAKE, None, None, FAKE,
+                                         FAKE, ws, None)
+    assert sparse(0) == abi.FL_ERR_INVALID
+    assert sparse(66) == abi.FL_ERR_INVALID               # more than N
+    sel = lambda **k: abi._c_select(ctypes.byref(d), FAKE, k.get("l0", 0), k.get("nl", 1), k.get("n_q", 64), 1,
+                                    k.get("k_sel", 10), FAKE, None)
+    assert sel(nl=3) == abi.FL_ERR_INVALID
+    assert sel(k_sel=129) == abi.FL_ERR_INVALID           # above max_select
+    step = lambda **k: abi._c_step(ctypes.byref(d), FAKE, 64, 1, k.get("dl", 2), k.get("k_sel", 10),
+                                   k.get("lf", 1), k.get("ll", 4), FAKE, None, None, FAKE, FAKE, ws, None, None)
+    assert step(dl=5) == abi.FL_ERR_INVALID
+    assert step(lf=3, ll=2) == abi.FL_ERR_INVALID
+    assert step(ll=5) == abi.FL_ERR_INVALID
+    assert step(k_sel=0) == abi.FL_ERR_INVALID
+    assert step(dl=0, lf=1) == abi.FL_ERR_INVALID         # first loop cannot be sparse
+    big = _dims(capacity=65536, max_select=10)
+    assert abi._c_select(ctypes.byref(big), FAKE, 0, 1, 49152, 1, 10, FAKE, None) == abi.FL_ERR_UNSUPPORTED
+
+
+def test_encoder_arguments_are_validated_before_launch():
+    d = _dims()
+    base = lambda row0, n: abi._c_encode_base(ctypes.byref(d), FAKE, 0, row0, n, FAKE, FAKE, 128 * 64, None)
+    assert base(32, 64) == abi.FL_ERR_INVALID
+    assert base(0, 100) == abi.FL_ERR_INVALID
+    assert base(1024, 64) == abi.FL_ERR_INVALID
+    res = lambda **k: abi._c_encode_residual(ctypes.byref(d), FAKE, 0, k.get("loop", 3), 0, 256,
+                                             k.get("slot0", 0), FAKE, k.get("n", 10), FAKE, FAKE,
+                                             128 * 256, 0, None)
+    assert res(loop=1) == abi.FL_ERR_INVALID
+    assert res(slot0=32) == abi.FL_ERR_INVALID
+    assert res(slot0=192, n=100) == abi.FL_ERR_INVALID    # beyond loop 3's 256 slots
+    assert res(n=300) == abi.FL_ERR_INVALID               # more rows than the span
+    tail = abi._c_write_tail(ctypes.byref(d), FAKE, 0, 1, 60, 8, FAKE, FAKE, 128 * 8, None)
+    assert tail == abi.FL_ERR_INVALID
+
+
+def test_status_strings():
+    for st in (abi.FL_OK, abi.FL_ERR_INVALID, abi.FL_ERR_UNSUPPORTED, abi.FL_ERR_CUDA, abi.FL_ERR_WORKSPACE,
+               abi.FL_ERR_DEVICE):
+        assert abi.fl_status_string(st).startswith("FL_")
+
+
+def test_host_bookkeeping_helpers():
+    assert [round_up(x) for x in (0, 1, 64, 65, 8176)] == [0, 64, 64, 128, 8192]
+    assert split_prefill(32768) == (32704, 64) and split_prefill(100) == (64, 36)
