@@ -46,16 +46,17 @@
  * Packed cache layout (one buffer of fl_cache_layout().total_bytes; every array
  * starts on a 256-byte boundary; L layers, H heads, C = capacity, T = total slots,
  * R loops; "sz" = a (scale, zero) fp16 pair stored as scale in the low half of a
- * 32-bit word):
- *   kcode  u8  [L][H][C][64]       base key codes; byte b = channel 2b (low nibble), 2b+1 (high)
- *   vcode  u8  [L][H][C][64]       base value codes, same packing
- *   ksz    u32 [L][H][C/64][128]   base key sz per (block, channel)
- *   vsz    u32 [L][H][C][2]        base value sz per (token, half)
- *   rkcode u8  [L][H][T][64]       residual key codes of every loop; loop r owns slots
+ * 32-bit word).  Codes and scales live in 9216-byte GROUP RECORDS, one per 64 rows
+ * of a store (a 64-token block of the base, or 64 consecutive slots of a residual
+ * store):
+ *     bytes [0, 8192)     64 rows x 128 B: row i = 64 B of key codes then 64 B of
+ *                         value codes; code byte b holds channel 2b (low nibble) and
+ *                         2b+1 (high nibble)
+ *     bytes [8192, 8704)  64 x 2 value sz: row i, half h (channels 64h..64h+63)
+ *     bytes [8704, 9216)  128 key sz: one per channel of the group
+ *   brec   u8  [L][H][C/64][9216]  base group records (loop 1), block b = tokens 64b..64b+63
+ *   rrec   u8  [L][H][T/64][9216]  residual group records of every loop; loop r owns slots
  *                                   [slot_base[r], slot_base[r] + res_capacity[r])
- *   rvcode u8  [L][H][T][64]
- *   rksz   u32 [L][H][T/64][128]   residual key sz per (slot group, channel)
- *   rvsz   u32 [L][H][T][2]
  *   mask   u64 [L][R+1][C/64]      bit t of mask[r][b]: token 64b+t has a loop-r residual
  *   first  i32 [L][R+1][C/64]      slot (within loop r's store) of block b's first loop-r row;
  *                                   the block's rows occupy consecutive slots in token order
@@ -69,6 +70,11 @@
  *   sel    i32 [L][H][max_select]  selected columns S, ascending
  *   mass   f32 [L][H]              m = sum over S of p~
  *   unsel  f32 [L][H][128]         u = sum over columns not in S of p~_j * v_j (at loop tag_j)
+ *   plan   i32 [L][H][max_select][P] gather plan of S, P = plan_stride = roundup(R + 2, 4):
+ *                                   [0] column j, [1] tag_j | (stores << 8) where stores =
+ *                                   min(loop, depth_j) for a quantised column and 0 for a tail
+ *                                   column, [2] p~_j as fp32 bits, [3 + (r - 2)] the global
+ *                                   residual slot of column j in loop r's store, r = 2..stores
  *   status i32 [16]                [0] first device error code (0 = none), [1] its detail,
  *                                   [2] number of device errors
  */
@@ -104,6 +110,8 @@ typedef enum fl_status {
 #define FL_DEV_NOT_NESTED 3   /* loop-r row not active in loop r-1 */
 #define FL_DEV_SEL_RANGE 4    /* selected column outside [0, N) */
 #define FL_DEV_TAG_RANGE 5    /* a column's loop tag outside [1, R] */
+#define FL_DEV_TIMEOUT 6      /* a bounded wait for staged data ran out (the kernel returned early) */
+#define FL_GROUP_RECORD 9216  /* bytes of one group record */
 
 typedef struct fl_dims {
   int32_t layers;      /* L >= 1 */
@@ -118,15 +126,15 @@ typedef struct fl_dims {
 
 typedef struct fl_layout {
   uint64_t total_bytes;
-  uint64_t kcode, vcode, ksz, vsz;
-  uint64_t rkcode, rvcode, rksz, rvsz;
+  uint64_t brec, rrec;
   uint64_t mask, first, depth;
   uint64_t tail_k, tail_v;
   uint64_t score, tag, offset;
-  uint64_t sel, mass, unsel;
+  uint64_t sel, mass, unsel, plan;
   uint64_t status;
   /* bytes from one layer to the next inside each array above (same order) */
-  uint64_t layer_stride[19];
+  uint64_t layer_stride[14];
+  int32_t plan_stride;                 /* int32 words per plan entry */
   int32_t slot_base[FL_MAX_LOOPS + 1]; /* first global slot of loop r's residual store */
   int32_t total_slots;                 /* T */
 } fl_layout;
@@ -193,34 +201,35 @@ fl_status fl_decode_attn_dense(const fl_dims* dims, void* cache, int32_t layer, 
                                const uint16_t* k_new, const uint16_t* v_new, float* o,
                                int32_t keep_scores, void* ws, size_t ws_bytes, void* stream);
 
-/* [Project] Step 02; [Guide] section 3.  For layers [layer0, layer0 + n_layers) and
- * every head: S = the k_sel columns of largest p~ (the distribution the preceding loop
- * left: scores/tags/offsets), ties to the smaller index, written ascending; the mass
- * m = sum over S of p~; and the unselected contribution u = o_prev - sum over S of
- * p~_j v_j, v_j taken at the loop that last computed column j.  o_prev: fp32
- * [n_layers][H][128], the preceding loop's outputs.  N = n_q + n_tail <=
- * FL_MAX_SELECT_COLS and 1 <= k_sel <= min(N, max_select). */
+/* [Project] Step 02; [Guide] section 3.  Prepares sparse loop `loop` for layers
+ * [layer0, layer0 + n_layers) and every head: S = the k_sel columns of largest p~ (the
+ * distribution the preceding loop left: scores/tags/offsets), ties to the smaller
+ * index, written ascending; the selected mass m = sum over S of p~; and the gather
+ * plan of S (its layout is above).  N = n_q + n_tail <= FL_MAX_SELECT_COLS and
+ * 1 <= k_sel <= min(N, max_select); 2 <= loop <= R. */
 fl_status fl_select_topk(const fl_dims* dims, void* cache, int32_t layer0, int32_t n_layers,
-                         int32_t n_q, int32_t n_tail, int32_t k_sel, const float* o_prev,
-                         void* stream);
+                         int32_t loop, int32_t n_q, int32_t n_tail, int32_t k_sel, void* stream);
 
 /* [Project] Step 02; [Guide] section 3.  Sparse attention of loop `loop` over the
- * columns fl_select_topk chose (same k_sel, n_q, n_tail):
+ * columns fl_select_topk chose for this loop (same k_sel, n_q, n_tail):
  *   o = u + m * softmax_S(q K_S^T / sqrt(128)) V_S,
- * keys/values at loop `loop`.  Then splices the state: score/tag of j in S become this
- * loop's, and offset[loop] makes p~_j = m * softmax_S(.)_j.  q, k_new, v_new, o as in
+ *   u = o_prev - sum over S of p~_j v_j   (v_j at the loop that last computed column j),
+ * i.e. u is the unselected columns' contribution to the preceding loop's output o_prev
+ * (fp32 [H][128]).  Keys/values are those of loop `loop`.  The pass also records m and u
+ * in the cache and splices the state: score/tag of j in S become this loop's, and
+ * offset[loop] makes p~_j = m * softmax_S(.)_j.  q, k_new, v_new, o as in
  * fl_decode_attn_dense. */
 fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,
                                 int32_t n_q, int32_t n_tail, int32_t k_sel, const uint16_t* q,
-                                const uint16_t* k_new, const uint16_t* v_new, float* o,
-                                void* ws, size_t ws_bytes, void* stream);
+                                const uint16_t* k_new, const uint16_t* v_new, const float* o_prev,
+                                float* o, void* ws, size_t ws_bytes, void* stream);
 
 /* Native executor of one decode step for layers [0, L) in loop-major order (every
  * layer runs loop r before any layer runs loop r+1), for loops loop_first..loop_last:
  * loops up to dense_loops call the dense reader (the last dense loop keeps scores);
  * every later loop first selects k_sel columns for all layers in one launch
- * (fl_select_topk, o_prev = that loop's previous outputs) and then runs each layer's
- * sparse reader.  Same arguments and semantics as the individual calls; validated once.
+ * (fl_select_topk) and then runs each layer's sparse reader with o_prev = that
+ * layer's output of the previous loop.  Same arguments and semantics as the individual calls; validated once.
  *   q, k_new, v_new: BF16 [R+1][L][H][128] (slice r = loop r, slice 0 unused;
  *                    k_new/v_new may be NULL)
  *   o: fp32 [R+1][L][H][128]   (o[r] = loop r's outputs; o[loop_first-1] must hold the

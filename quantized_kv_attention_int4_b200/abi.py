@@ -24,9 +24,10 @@ HEAD_DIM = 128
 GROUP = 64
 TAIL = 64
 MAX_SELECT_COLS = 49152
-N_ARRAYS = 19
-ARRAY_NAMES = ("kcode", "vcode", "ksz", "vsz", "rkcode", "rvcode", "rksz", "rvsz", "mask", "first",
-               "depth", "tail_k", "tail_v", "score", "tag", "offset", "sel", "mass", "unsel")
+N_ARRAYS = 14
+ARRAY_NAMES = ("brec", "rrec", "mask", "first", "depth", "tail_k", "tail_v", "score", "tag", "offset", "sel",
+               "mass", "unsel", "plan")
+GROUP_RECORD = 9216
 
 FL_OK, FL_ERR_INVALID, FL_ERR_UNSUPPORTED, FL_ERR_CUDA, FL_ERR_WORKSPACE, FL_ERR_DEVICE = 0, -1, -2, -3, -4, -6
 EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init", "fl_workspace_bytes",
@@ -45,7 +46,8 @@ class fl_layout(ctypes.Structure):
     _fields_ = ([("total_bytes", ctypes.c_uint64)]
                 + [(n, ctypes.c_uint64) for n in ARRAY_NAMES]
                 + [("status", ctypes.c_uint64), ("layer_stride", ctypes.c_uint64 * N_ARRAYS),
-                   ("slot_base", ctypes.c_int32 * (MAX_LOOPS + 1)), ("total_slots", ctypes.c_int32)])
+                   ("plan_stride", ctypes.c_int32), ("slot_base", ctypes.c_int32 * (MAX_LOOPS + 1)),
+                   ("total_slots", ctypes.c_int32)])
 
 
 _P = ctypes.c_void_p
@@ -72,8 +74,8 @@ _c_encode_base = _sig("fl_encode_base", _I, _DP, _P, _I, _I, _I, _P, _P, _L, _P)
 _c_encode_residual = _sig("fl_encode_residual", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _L, _I, _P)
 _c_dense = _sig("fl_decode_attn_dense", _I, _DP, _P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P,
                 ctypes.c_size_t, _P)
-_c_select = _sig("fl_select_topk", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _P)
-_c_sparse = _sig("fl_decode_attn_sparse", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+_c_select = _sig("fl_select_topk", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P)
+_c_sparse = _sig("fl_decode_attn_sparse", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                  ctypes.c_size_t, _P)
 _c_step = _sig("fl_decode_step", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t,
                 ctypes.POINTER(ctypes.c_void_p), _P)
@@ -199,16 +201,18 @@ def fl_decode_attn_dense(dims, cache, layer, loop, n_q, n_tail, q, k_new, v_new,
         _stream(stream)))
 
 
-def fl_select_topk(dims, cache, layer0, n_layers, n_q, n_tail, k_sel, o_prev, stream=None):
+def fl_select_topk(dims, cache, layer0, n_layers, loop, n_q, n_tail, k_sel, stream=None):
     _check("fl_select_topk", _c_select(ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer0, n_layers,
-                                       n_q, n_tail, k_sel, _ptr(o_prev, torch.float32, "o_prev"), _stream(stream)))
+                                       loop, n_q, n_tail, k_sel, _stream(stream)))
 
 
-def fl_decode_attn_sparse(dims, cache, layer, loop, n_q, n_tail, k_sel, q, k_new, v_new, o, ws, stream=None):
+def fl_decode_attn_sparse(dims, cache, layer, loop, n_q, n_tail, k_sel, q, k_new, v_new, o_prev, o, ws,
+                          stream=None):
     _check("fl_decode_attn_sparse", _c_sparse(
         ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer, loop, n_q, n_tail, k_sel,
         _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
-        _ptr(o, torch.float32, "o"), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+        _ptr(o_prev, torch.float32, "o_prev"), _ptr(o, torch.float32, "o"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)))
 
 
 def fl_decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, k_new, v_new, o, ws,

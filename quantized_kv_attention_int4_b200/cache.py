@@ -145,12 +145,12 @@ class FlashLoopCache:
         abi.fl_decode_attn_dense(self.dims, self.buf, layer, loop, self.n_q, self.n_tail, q, k_new, v_new, o,
                                  keep_scores, self.ws, stream)
 
-    def select(self, layer0, n_layers, k_sel, o_prev, stream=None):
-        abi.fl_select_topk(self.dims, self.buf, layer0, n_layers, self.n_q, self.n_tail, k_sel, o_prev, stream)
+    def select(self, layer0, n_layers, loop, k_sel, stream=None):
+        abi.fl_select_topk(self.dims, self.buf, layer0, n_layers, loop, self.n_q, self.n_tail, k_sel, stream)
 
-    def sparse(self, layer, loop, k_sel, q, o, k_new=None, v_new=None, stream=None):
+    def sparse(self, layer, loop, k_sel, q, o_prev, o, k_new=None, v_new=None, stream=None):
         abi.fl_decode_attn_sparse(self.dims, self.buf, layer, loop, self.n_q, self.n_tail, k_sel, q, k_new, v_new,
-                                  o, self.ws, stream)
+                                  o_prev, o, self.ws, stream)
 
     def step(self, dense_loops, k_sel, q, o, k_new=None, v_new=None, loop_first=1, loop_last=None, events=None,
              stream=None):

@@ -23,6 +23,8 @@ fl_status check_dims(const fl_dims* d) {
   return FL_OK;
 }
 
+inline int plan_stride(const fl_dims* d) { return (d->loops + 2 + 3) / 4 * 4; }
+
 // Per-layer byte sizes of every array, in fl_layout order.
 void layer_sizes(const fl_dims* d, uint64_t* sz, int32_t* slot_base, int32_t* total_slots) {
   const uint64_t H = d->heads, C = d->capacity, R = d->loops;
@@ -33,14 +35,8 @@ void layer_sizes(const fl_dims* d, uint64_t* sz, int32_t* slot_base, int32_t* to
     T += (uint64_t)d->res_capacity[r];
   }
   *total_slots = (int32_t)T;
-  sz[A_KCODE] = H * C * 64;
-  sz[A_VCODE] = H * C * 64;
-  sz[A_KSZ] = H * (C / 64) * 128 * 4;
-  sz[A_VSZ] = H * C * 2 * 4;
-  sz[A_RKCODE] = H * T * 64;
-  sz[A_RVCODE] = H * T * 64;
-  sz[A_RKSZ] = H * (T / 64) * 128 * 4;
-  sz[A_RVSZ] = H * T * 2 * 4;
+  sz[A_BREC] = H * (C / 64) * (uint64_t)FL_GROUP_RECORD;
+  sz[A_RREC] = H * (T / 64) * (uint64_t)FL_GROUP_RECORD;
   sz[A_MASK] = (R + 1) * (C / 64) * 8;
   sz[A_FIRST] = (R + 1) * (C / 64) * 4;
   sz[A_DEPTH] = C;
@@ -52,6 +48,7 @@ void layer_sizes(const fl_dims* d, uint64_t* sz, int32_t* slot_base, int32_t* to
   sz[A_SEL] = H * (uint64_t)d->max_select * 4;
   sz[A_MASS] = H * 4;
   sz[A_UNSEL] = H * 128 * 4;
+  sz[A_PLAN] = H * (uint64_t)d->max_select * plan_stride(d) * 4;
 }
 
 fl_status make_layout(const fl_dims* d, fl_layout* L) {
@@ -60,10 +57,9 @@ fl_status make_layout(const fl_dims* d, fl_layout* L) {
   std::memset(L, 0, sizeof(*L));
   uint64_t sz[A_COUNT];
   layer_sizes(d, sz, L->slot_base, &L->total_slots);
-  uint64_t* offs[A_COUNT] = {&L->kcode, &L->vcode, &L->ksz, &L->vsz, &L->rkcode, &L->rvcode,
-                             &L->rksz, &L->rvsz, &L->mask, &L->first, &L->depth, &L->tail_k,
-                             &L->tail_v, &L->score, &L->tag, &L->offset, &L->sel, &L->mass,
-                             &L->unsel};
+  uint64_t* offs[A_COUNT] = {&L->brec,  &L->rrec,   &L->mask,  &L->first, &L->depth,
+                             &L->tail_k, &L->tail_v, &L->score, &L->tag,   &L->offset,
+                             &L->sel,   &L->mass,   &L->unsel, &L->plan};
   uint64_t cur = 0;
   for (int i = 0; i < A_COUNT; ++i) {
     const uint64_t stride = align_up(sz[i]);
@@ -74,6 +70,7 @@ fl_status make_layout(const fl_dims* d, fl_layout* L) {
   L->status = cur;
   cur += align_up(16 * sizeof(int32_t));
   L->total_bytes = cur;
+  L->plan_stride = plan_stride(d);
   return FL_OK;
 }
 
@@ -81,9 +78,8 @@ CacheView make_view(const fl_dims* d, const fl_layout& L, void* cache) {
   CacheView v;
   std::memset(&v, 0, sizeof(v));
   v.base = static_cast<uint8_t*>(cache);
-  const uint64_t offs[A_COUNT] = {L.kcode, L.vcode, L.ksz, L.vsz, L.rkcode, L.rvcode, L.rksz,
-                                  L.rvsz, L.mask, L.first, L.depth, L.tail_k, L.tail_v,
-                                  L.score, L.tag, L.offset, L.sel, L.mass, L.unsel};
+  const uint64_t offs[A_COUNT] = {L.brec,  L.rrec, L.mask, L.first, L.depth, L.tail_k, L.tail_v,
+                                  L.score, L.tag,  L.offset, L.sel, L.mass, L.unsel, L.plan};
   for (int i = 0; i < A_COUNT; ++i) {
     v.off[i] = offs[i];
     v.lstride[i] = L.layer_stride[i];
@@ -95,6 +91,7 @@ CacheView make_view(const fl_dims* d, const fl_layout& L, void* cache) {
   v.cap = d->capacity;
   v.total_slots = L.total_slots;
   v.max_select = d->max_select;
+  v.plan_stride = L.plan_stride;
   return v;
 }
 
@@ -279,19 +276,21 @@ fl_status fl_decode_attn_dense(const fl_dims* dims, void* cache, int32_t layer, 
   a.q = q;
   a.k_new = k_new;
   a.v_new = v_new;
+  a.o_prev = nullptr;
   a.o = o;
   a.part = static_cast<float*>(ws);
   a.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_part_bytes(dims));
   return cuda_status(launch_dense(a, (cudaStream_t)stream));
 }
 
-fl_status fl_select_topk(const fl_dims* dims, void* cache, int32_t layer0, int32_t n_layers, int32_t n_q,
-                         int32_t n_tail, int32_t k_sel, const float* o_prev, void* stream) {
+fl_status fl_select_topk(const fl_dims* dims, void* cache, int32_t layer0, int32_t n_layers, int32_t loop,
+                         int32_t n_q, int32_t n_tail, int32_t k_sel, void* stream) {
   fl_layout L;
   fl_status st = make_layout(dims, &L);
   if (st != FL_OK) return st;
-  if (!cache || !o_prev) return FL_ERR_INVALID;
+  if (!cache) return FL_ERR_INVALID;
   if (layer0 < 0 || n_layers < 1 || (int64_t)layer0 + n_layers > dims->layers) return FL_ERR_INVALID;
+  if (loop < 2 || loop > dims->loops) return FL_ERR_INVALID;
   if (n_q < 0 || n_q % FL_GROUP != 0 || n_tail < 1 || n_tail > FL_TAIL) return FL_ERR_INVALID;
   const int64_t N = (int64_t)n_q + n_tail;
   if (N > dims->capacity) return FL_ERR_INVALID;
@@ -300,18 +299,20 @@ fl_status fl_select_topk(const fl_dims* dims, void* cache, int32_t layer0, int32
   SelectArgs a;
   a.c = make_view(dims, L, cache);
   a.layer0 = layer0;
+  a.r = loop;
   a.n_q = n_q;
   a.n_tail = n_tail;
   a.k_sel = k_sel;
-  a.o_prev = o_prev;
   return cuda_status(launch_select(a, n_layers, (cudaStream_t)stream));
 }
 
 fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer, int32_t loop, int32_t n_q,
                                 int32_t n_tail, int32_t k_sel, const uint16_t* q, const uint16_t* k_new,
-                                const uint16_t* v_new, float* o, void* ws, size_t ws_bytes, void* stream) {
+                                const uint16_t* v_new, const float* o_prev, float* o, void* ws, size_t ws_bytes,
+                                void* stream) {
   fl_status st = check_reader(dims, cache, layer, loop, n_q, n_tail, q, k_new, v_new, o, ws, ws_bytes);
   if (st != FL_OK) return st;
+  if (!o_prev || loop < 2) return FL_ERR_INVALID;
   const int64_t N = (int64_t)n_q + n_tail;
   if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
   fl_layout L;
@@ -328,6 +329,7 @@ fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer,
   a.q = q;
   a.k_new = k_new;
   a.v_new = v_new;
+  a.o_prev = o_prev;
   a.o = o;
   a.part = static_cast<float*>(ws);
   a.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_part_bytes(dims));
@@ -360,6 +362,7 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
   };
   ReaderArgs a;
   a.c = make_view(dims, lay, cache);
+  a.o_prev = nullptr;
   a.n_q = n_q;
   a.n_tail = n_tail;
   a.k_sel = k_sel;
@@ -385,10 +388,10 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
       SelectArgs sa;
       sa.c = a.c;
       sa.layer0 = 0;
+      sa.r = r;
       sa.n_q = n_q;
       sa.n_tail = n_tail;
       sa.k_sel = k_sel;
-      sa.o_prev = o + (size_t)(r - 1) * ostride_r;
       if (launch_select(sa, L, s) != cudaSuccess) return FL_ERR_CUDA;
       if (!rec(2 * r - 1)) return FL_ERR_CUDA;
       a.keep = 1;
@@ -399,6 +402,7 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
         a.k_new = k_new ? k_new + qo : nullptr;
         a.v_new = v_new ? v_new + qo : nullptr;
         a.o = o + qo;
+        a.o_prev = o + qo - ostride_r;
         if (launch_sparse(a, s) != cudaSuccess) return FL_ERR_CUDA;
       }
     }

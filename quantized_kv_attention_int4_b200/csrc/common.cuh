@@ -17,15 +17,20 @@ constexpr int kG = 64;      // group size / block of tokens
 constexpr int kTail = 64;   // BF16 tail rows
 constexpr int kOffStride = FL_MAX_LOOPS + 1;  // offset[L][H][33]
 constexpr int kMaxSplits = 256;
-constexpr int kPartStride = 132;  // M, L, pad, pad, o[128]
+constexpr int kPartStride = 260;  // M, L, m, pad, o[128], u[128]
 constexpr unsigned kFull = 0xffffffffu;
 
 // Array ids, in fl_layout order.
 enum Arr {
-  A_KCODE = 0, A_VCODE, A_KSZ, A_VSZ, A_RKCODE, A_RVCODE, A_RKSZ, A_RVSZ,
-  A_MASK, A_FIRST, A_DEPTH, A_TAILK, A_TAILV, A_SCORE, A_TAG, A_OFFSET,
-  A_SEL, A_MASS, A_UNSEL, A_COUNT
+  A_BREC = 0, A_RREC, A_MASK, A_FIRST, A_DEPTH, A_TAILK, A_TAILV, A_SCORE, A_TAG, A_OFFSET,
+  A_SEL, A_MASS, A_UNSEL, A_PLAN, A_COUNT
 };
+
+// Group record: 64 rows of (64 B key codes, 64 B value codes), then 64 x 2 value
+// (scale, zero) words, then 128 key (scale, zero) words.
+constexpr int kRec = FL_GROUP_RECORD;
+constexpr int kRecVsz = 8192;
+constexpr int kRecKsz = 8704;
 
 // Device view of one cache buffer: base pointer, array offsets and per-layer strides.
 struct CacheView {
@@ -34,7 +39,7 @@ struct CacheView {
   uint64_t lstride[A_COUNT];
   int32_t slot_base[FL_MAX_LOOPS + 1];
   int32_t* status;
-  int32_t H, R, cap, total_slots, max_select;
+  int32_t H, R, cap, total_slots, max_select, plan_stride;
 };
 
 template <class T>
@@ -186,6 +191,23 @@ __device__ __forceinline__ float group_weights(const uint32_t* rec, const float*
   return warp_sum(cpart);
 }
 
+// group_weights for a record already in shared memory, rewritten in place as fp32
+// weights qs'_c; returns the record's additive constant.
+__device__ __forceinline__ float group_weights_smem(uint32_t* rec, const float* q_s, int lane) {
+  const uint4 r = *reinterpret_cast<const uint4*>(rec + 4 * lane);
+  const float4 qv = *reinterpret_cast<const float4*>(q_s + 4 * lane);
+  const float2 a = unpack_sz(r.x), b = unpack_sz(r.y), c = unpack_sz(r.z), d = unpack_sz(r.w);
+  float4 w;
+  w.x = 128.f * (qv.x * a.x);
+  w.y = 128.f * (qv.y * b.x);
+  w.z = 128.f * (qv.z * c.x);
+  w.w = 128.f * (qv.w * d.x);
+  const float cpart = fmaf(qv.x, a.y, -w.x) + fmaf(qv.y, b.y, -w.y) + fmaf(qv.z, c.y, -w.z) +
+                      fmaf(qv.w, d.y, -w.w);
+  *reinterpret_cast<float4*>(rec + 4 * lane) = w;
+  return warp_sum(cpart);
+}
+
 __device__ __forceinline__ void load32(const float* src, float* dst) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -195,6 +217,141 @@ __device__ __forceinline__ void load32(const float* src, float* dst) {
     dst[4 * i + 2] = v.z;
     dst[4 * i + 3] = v.w;
   }
+}
+
+// ---- asynchronous bulk copies (TMA engine) into shared memory, mbarrier completion ----
+__device__ __forceinline__ unsigned smem_addr(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1; }" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+// global -> shared bulk copy; dst, src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for phase `parity` of `bar`; false if the bound ran out.
+constexpr long long kWaitBound = 1ll << 22;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  for (long long i = 0; i < kWaitBound; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// fp32 accumulate of an fp16 product: acc += a * b with a, b binary16 (exact product).
+__device__ __forceinline__ void hfma_f32(float& acc, unsigned short a, unsigned short b) {
+  asm("{ .reg .f16 x, y; mov.b16 x, %1; mov.b16 y, %2; fma.rn.f32.f16 %0, x, y, %0; }"
+      : "+f"(acc)
+      : "h"(a), "h"(b));
+}
+
+// acc[k] += code_k * (weight) over the 8 nibbles of one code word, with the nibbles
+// turned into binary16 values 1024 + n (even channels, weight we) and 1024 + 16 n (odd
+// channels, weight wo = we / 16); the constant 1024 * weight per channel is removed by
+// the caller's correction terms.  Channel order follows the code word: nibble k at
+// bits 4k..4k+3 is channel k.
+__device__ __forceinline__ void axpy8_h(uint32_t w, unsigned short we, unsigned short wo, float* acc) {
+  const uint32_t a = (w & 0x000F000Fu) | 0x64006400u;          // ch 0, 4
+  const uint32_t b = (w & 0x00F000F0u) | 0x64006400u;          // ch 1, 5 (x16)
+  const uint32_t w8 = w >> 8;
+  const uint32_t c = (w8 & 0x000F000Fu) | 0x64006400u;         // ch 2, 6
+  const uint32_t d = (w8 & 0x00F000F0u) | 0x64006400u;         // ch 3, 7 (x16)
+  hfma_f32(acc[0], (unsigned short)a, we);
+  hfma_f32(acc[4], (unsigned short)(a >> 16), we);
+  hfma_f32(acc[1], (unsigned short)b, wo);
+  hfma_f32(acc[5], (unsigned short)(b >> 16), wo);
+  hfma_f32(acc[2], (unsigned short)c, we);
+  hfma_f32(acc[6], (unsigned short)(c >> 16), we);
+  hfma_f32(acc[3], (unsigned short)d, wo);
+  hfma_f32(acc[7], (unsigned short)(d >> 16), wo);
+}
+
+// ---- exact integer key dots (dp4a) against fixed-point query weights ----
+// A group's weights qs_c = q_c * s_c become Q_c = rint(qs_c * 2^E), |Q_c| <= 32767,
+// split into an unsigned low byte and a signed high byte.  For code word w (channels
+// 8w..8w+7) the limbs are 4 words: low bytes of the even channels (8w, 8w+2, 8w+4,
+// 8w+6), high bytes of the even channels, low bytes of the odd channels, high bytes of
+// the odd channels -- matching the low / high nibbles of the code word's bytes.
+__device__ __forceinline__ void dp4a_word(uint32_t w, uint4 limb, int& lo, int& hi) {
+  const uint32_t ne = w & 0x0F0F0F0Fu;
+  const uint32_t no = (w >> 4) & 0x0F0F0F0Fu;
+  asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(lo) : "r"(ne), "r"(limb.x));
+  asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(hi) : "r"(ne), "r"(limb.y));
+  asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(lo) : "r"(no), "r"(limb.z));
+  asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(hi) : "r"(no), "r"(limb.w));
+}
+
+// One warp turns a key (scale, zero) record (128 words) into dp4a limbs in place:
+// words 0..63 = limbs, word 64 = E, word 65 = C = sum_c q_c z_c (fp32 bits).
+__device__ __forceinline__ void record_to_limbs(uint32_t* rec, const float* q_s, int lane) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(rec + 4 * lane);
+  const float4 qv = *reinterpret_cast<const float4*>(q_s + 4 * lane);
+  const float2 s0 = unpack_sz(raw.x), s1 = unpack_sz(raw.y), s2 = unpack_sz(raw.z), s3 = unpack_sz(raw.w);
+  const float qs0 = qv.x * s0.x, qs1 = qv.y * s1.x, qs2 = qv.z * s2.x, qs3 = qv.w * s3.x;
+  float cz = fmaf(qv.x, s0.y, fmaf(qv.y, s1.y, fmaf(qv.z, s2.y, qv.w * s3.y)));
+  float mx = fmaxf(fmaxf(fabsf(qs0), fabsf(qs1)), fmaxf(fabsf(qs2), fabsf(qs3)));
+  mx = warp_max(mx);
+  cz = warp_sum(cz);
+  int e2 = 0;
+  if (mx > 0.f) frexpf(mx, &e2);        // mx = f * 2^e2, f in [0.5, 1)
+  const int E = 15 - e2;                 // |qs| * 2^E < 2^15
+  const float sc = ldexpf(1.0f, E);
+  auto fix = [&](float v) {
+    int qv_ = __float2int_rn(v * sc);
+    return qv_ > 32767 ? 32767 : (qv_ < -32767 ? -32767 : qv_);
+  };
+  const int Q0 = fix(qs0), Q1 = fix(qs1), Q2 = fix(qs2), Q3 = fix(qs3);
+  __syncwarp();
+  // lane l holds channels 4l..4l+3 of code word w = l/2; even channels 4l, 4l+2 and odd
+  // channels 4l+1, 4l+3 fill bytes 2*(l&1), 2*(l&1)+1 of the word's four limb words.
+  const int w = lane >> 1, hb = (lane & 1) * 2;
+  uint8_t* lb = reinterpret_cast<uint8_t*>(rec + 4 * w);
+  lb[0 * 4 + hb] = (uint8_t)(Q0 & 0xff);
+  lb[0 * 4 + hb + 1] = (uint8_t)(Q2 & 0xff);
+  lb[1 * 4 + hb] = (uint8_t)((Q0 >> 8) & 0xff);
+  lb[1 * 4 + hb + 1] = (uint8_t)((Q2 >> 8) & 0xff);
+  lb[2 * 4 + hb] = (uint8_t)(Q1 & 0xff);
+  lb[2 * 4 + hb + 1] = (uint8_t)(Q3 & 0xff);
+  lb[3 * 4 + hb] = (uint8_t)((Q1 >> 8) & 0xff);
+  lb[3 * 4 + hb + 1] = (uint8_t)((Q3 >> 8) & 0xff);
+  if (lane == 0) {
+    rec[64] = (uint32_t)E;
+    rec[65] = __float_as_uint(cz);
+  }
+}
+
+// The record's limb dot over one 32-channel quarter qq of a key code row (4 code words).
+__device__ __forceinline__ float limb_dot_quarter(const uint32_t* rec, uint4 code, int qq) {
+  const uint4* lw = reinterpret_cast<const uint4*>(rec) + 4 * qq;
+  int lo = 0, hi = 0;
+  dp4a_word(code.x, lw[0], lo, hi);
+  dp4a_word(code.y, lw[1], lo, hi);
+  dp4a_word(code.z, lw[2], lo, hi);
+  dp4a_word(code.w, lw[3], lo, hi);
+  const int E = (int)rec[64];
+  return (float)(hi * 256 + lo) * __int_as_float((127 - E) << 23);
 }
 
 // log2(e) / sqrt(128): scores are kept in the base-2 domain.

@@ -32,14 +32,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_kernel(ReaderArgs a) {
   const CacheView& c = a.c;
   const int H = c.H, cap = c.cap, ncb = cap / kG, T = c.total_slots, r = a.r;
 
-  const uint8_t* kcode = arr<uint8_t>(c, A_KCODE, a.layer) + (size_t)h * cap * 64;
-  const uint8_t* vcode = arr<uint8_t>(c, A_VCODE, a.layer) + (size_t)h * cap * 64;
-  const uint32_t* ksz = arr<uint32_t>(c, A_KSZ, a.layer) + (size_t)h * ncb * kD;
-  const uint32_t* vsz = arr<uint32_t>(c, A_VSZ, a.layer) + (size_t)h * cap * 2;
-  const uint8_t* rkcode = arr<uint8_t>(c, A_RKCODE, a.layer) + (size_t)h * T * 64;
-  const uint8_t* rvcode = arr<uint8_t>(c, A_RVCODE, a.layer) + (size_t)h * T * 64;
-  const uint32_t* rksz = arr<uint32_t>(c, A_RKSZ, a.layer) + (size_t)h * (T / kG) * kD;
-  const uint32_t* rvsz = arr<uint32_t>(c, A_RVSZ, a.layer) + (size_t)h * T * 2;
+  const uint8_t* brec = arr<uint8_t>(c, A_BREC, a.layer) + (size_t)h * ncb * kRec;
+  const uint8_t* rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * kRec;
+  // residual slot gs: row (gs & 63) of group record (gs >> 6)
+  auto rrow = [&](int gs) { return rrec + (size_t)(gs >> 6) * kRec + (size_t)(gs & 63) * 128; };
   const unsigned long long* mask = arr<unsigned long long>(c, A_MASK, a.layer);
   const int32_t* first = arr<int32_t>(c, A_FIRST, a.layer);
   uint16_t* tail_k = arr<uint16_t>(c, A_TAILK, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
@@ -78,13 +74,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_kernel(ReaderArgs a) {
       const int b = u;
       // ---- keys: base ----
       __syncwarp();
-      float cb = group_weights(ksz + (size_t)b * kD, q_s, qsw, lane);
+      const uint8_t* rec = brec + (size_t)b * kRec;
+      float cb = group_weights(reinterpret_cast<const uint32_t*>(rec + kRecKsz), q_s, qsw, lane);
       __syncwarp();
       load32(qsw + 32 * qq, qsr);
-      const uint4* kc = reinterpret_cast<const uint4*>(kcode + (size_t)b * kG * 64);
+      const uint4* kc = reinterpret_cast<const uint4*>(rec);
       uint4 w[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] = __ldg(kc + 32 * i + lane);
+      for (int i = 0; i < 8; ++i) w[i] = __ldg(kc + (8 * i + tr) * 8 + qq);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float p = dot32(w[i], qsr);
@@ -106,14 +103,15 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_kernel(ReaderArgs a) {
           const int grp = (gs0 + row) >> 6;
           const int row_end = min(na, ((grp + 1) << 6) - gs0);
           __syncwarp();
-          const float cg = group_weights(rksz + (size_t)grp * kD, q_s, qsw, lane);
+          const float cg = group_weights(
+              reinterpret_cast<const uint32_t*>(rrec + (size_t)grp * kRec + kRecKsz), q_s, qsw, lane);
           __syncwarp();
           load32(qsw + 32 * qq, qsr);
           for (int i0 = row; i0 < row_end; i0 += 8) {
             const int rw = i0 + tr;
             const bool act = rw < row_end;
             uint4 x = make_uint4(0u, 0u, 0u, 0u);
-            if (act) x = __ldg(reinterpret_cast<const uint4*>(rkcode + (size_t)(gs0 + rw) * 64) + qq);
+            if (act) x = __ldg(reinterpret_cast<const uint4*>(rrow(gs0 + rw)) + qq);
             float p = dot32(x, qsr);
             p += __shfl_xor_sync(kFull, p, 1);
             p += __shfl_xor_sync(kFull, p, 2);
@@ -148,13 +146,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_kernel(ReaderArgs a) {
       __syncwarp();
       // ---- values: base ----
       {
-        const uint4* vc = reinterpret_cast<const uint4*>(vcode + (size_t)b * kG * 64);
-        const uint32_t* vs = vsz + (size_t)b * kG * 2;
+        const uint8_t* rec = brec + (size_t)b * kRec;
+        const uint4* vc = reinterpret_cast<const uint4*>(rec);
+        const uint32_t* vs = reinterpret_cast<const uint32_t*>(rec + kRecVsz);
         uint4 vw[8];
         uint32_t sw[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          vw[i] = __ldg(vc + 32 * i + lane);
+          vw[i] = __ldg(vc + (8 * i + tr) * 8 + 4 + qq);
           sw[i] = __ldg(vs + 2 * (8 * i + tr) + (qq >> 1));
         }
 #pragma unroll
@@ -180,8 +179,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_kernel(ReaderArgs a) {
           const int rw = i0 + tr;
           if (rw < na) {
             const int gs = gs0 + rw;
-            const uint4 x = __ldg(reinterpret_cast<const uint4*>(rvcode + (size_t)gs * 64) + qq);
-            const float2 sz = unpack_sz(__ldg(rvsz + (size_t)gs * 2 + (qq >> 1)));
+            const uint4 x = __ldg(reinterpret_cast<const uint4*>(rrow(gs)) + 4 + qq);
+            const float2 sz = unpack_sz(__ldg(reinterpret_cast<const uint32_t*>(
+                rrec + (size_t)(gs >> 6) * kRec + kRecVsz) + (gs & 63) * 2 + (qq >> 1)));
             const float p = lgw[tokw[rw]];
             const float P = 128.f * (p * sz.x);
             corr += fmaf(p, sz.y, -P);

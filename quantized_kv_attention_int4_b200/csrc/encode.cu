@@ -80,10 +80,9 @@ __global__ void __launch_bounds__(256) encode_base_kernel(EncodeBaseArgs a) {
   __shared__ float sk[kD], zk[kD];
   __shared__ float sv[kG][2], zv[kG][2];
 
-  uint8_t* kcode = arr<uint8_t>(c, A_KCODE, a.layer) + ((size_t)h * cap + tok0) * 64;
-  uint8_t* vcode = arr<uint8_t>(c, A_VCODE, a.layer) + ((size_t)h * cap + tok0) * 64;
-  uint32_t* ksz = arr<uint32_t>(c, A_KSZ, a.layer) + ((size_t)h * ncb + gb) * kD;
-  uint32_t* vsz = arr<uint32_t>(c, A_VSZ, a.layer) + ((size_t)h * cap + tok0) * 2;
+  uint8_t* rec = arr<uint8_t>(c, A_BREC, a.layer) + ((size_t)h * ncb + gb) * kRec;
+  uint32_t* ksz = reinterpret_cast<uint32_t*>(rec + kRecKsz);
+  uint32_t* vsz = reinterpret_cast<uint32_t*>(rec + kRecVsz);
   const size_t in_off = (size_t)h * a.head_stride + (size_t)blk * kG * kD;
   const int t = tid >> 2, qq = tid & 3;
 
@@ -103,7 +102,7 @@ __global__ void __launch_bounds__(256) encode_base_kernel(EncodeBaseArgs a) {
     ksz[tid] = pack_sz(hs, hz);
   }
   __syncthreads();
-  reinterpret_cast<uint4*>(kcode + (size_t)t * 64)[qq] =
+  reinterpret_cast<uint4*>(rec + (size_t)t * 128)[qq] =
       pack_quarter(xs, t, qq, [&](int, int ch) { return make_float2(sk[ch], zk[ch]); });
   __syncthreads();
 
@@ -124,7 +123,7 @@ __global__ void __launch_bounds__(256) encode_base_kernel(EncodeBaseArgs a) {
     vsz[tt * 2 + hf] = pack_sz(hs, hz);
   }
   __syncthreads();
-  reinterpret_cast<uint4*>(vcode + (size_t)t * 64)[qq] =
+  reinterpret_cast<uint4*>(rec + (size_t)t * 128 + 64)[qq] =
       pack_quarter(xs, t, qq, [&](int tt, int ch) { return make_float2(sv[tt][ch >> 6], zv[tt][ch >> 6]); });
 
   if (h == 0) {
@@ -174,16 +173,15 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
   __syncthreads();
 
   const int gslot0 = c.slot_base[r] + a.slot0 + i0;  // a multiple of 64
-  const size_t hT = (size_t)h * T;
   const int t = tid >> 2, qq = tid & 3;
+  const uint8_t* brec = arr<uint8_t>(c, A_BREC, a.layer) + (size_t)h * ncb * kRec;
+  uint8_t* rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * kRec;
+  uint8_t* orec = rrec + (size_t)(gslot0 >> 6) * kRec;  // this CTA's output group record
 
   for (int part = 0; part < 2; ++part) {
     const bool is_v = part == 1;
     const uint16_t* src = is_v ? a.v : a.k;
-    const uint8_t* bcode = arr<uint8_t>(c, is_v ? A_VCODE : A_KCODE, a.layer) + (size_t)h * cap * 64;
-    const uint32_t* bsz = arr<uint32_t>(c, is_v ? A_VSZ : A_KSZ, a.layer);
-    const uint8_t* rcode = arr<uint8_t>(c, is_v ? A_RVCODE : A_RKCODE, a.layer) + hT * 64;
-    const uint32_t* rsz = arr<uint32_t>(c, is_v ? A_RVSZ : A_RKSZ, a.layer);
+    const int code_off = is_v ? 64 : 0;
 
     // residual E = X^(r) - X_hat^(r-1) for 8 channels per item
     for (int item = tid; item < kG * 16; item += 256) {
@@ -201,11 +199,13 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
       const int b = j >> 6, jt = j & 63;
       float xh[8];
       {
-        const uint32_t cw = *reinterpret_cast<const uint32_t*>(bcode + (size_t)j * 64 + c8 / 2);
+        const uint8_t* g = brec + (size_t)b * kRec;
+        const uint32_t cw = *reinterpret_cast<const uint32_t*>(g + (size_t)jt * 128 + code_off + c8 / 2);
+        const uint32_t* ks = reinterpret_cast<const uint32_t*>(g + kRecKsz);
+        const uint32_t* vs = reinterpret_cast<const uint32_t*>(g + kRecVsz);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const uint32_t szw = is_v ? bsz[((size_t)h * cap + j) * 2 + (c8 >> 6)]
-                                    : bsz[((size_t)h * ncb + b) * kD + c8 + e];
+          const uint32_t szw = is_v ? vs[jt * 2 + (c8 >> 6)] : ks[c8 + e];
           xh[e] = deq((cw >> (4 * e)) & 15u, unpack_sz(szw));
         }
       }
@@ -213,11 +213,14 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
         const unsigned long long mk = mask[(size_t)rp * ncb + b];
         const int gs = c.slot_base[rp] + first[(size_t)rp * ncb + b] +
                        __popcll(mk & ((1ull << jt) - 1ull));
-        const uint32_t cw = *reinterpret_cast<const uint32_t*>(rcode + (size_t)gs * 64 + c8 / 2);
+        const uint8_t* g = rrec + (size_t)(gs >> 6) * kRec;
+        const int rw = gs & 63;
+        const uint32_t cw = *reinterpret_cast<const uint32_t*>(g + (size_t)rw * 128 + code_off + c8 / 2);
+        const uint32_t* ks = reinterpret_cast<const uint32_t*>(g + kRecKsz);
+        const uint32_t* vs = reinterpret_cast<const uint32_t*>(g + kRecVsz);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const uint32_t szw = is_v ? rsz[(hT + gs) * 2 + (c8 >> 6)]
-                                    : rsz[((size_t)h * (T / kG) + (gs >> 6)) * kD + c8 + e];
+          const uint32_t szw = is_v ? vs[rw * 2 + (c8 >> 6)] : ks[c8 + e];
           xh[e] = __fadd_rn(xh[e], deq((cw >> (4 * e)) & 15u, unpack_sz(szw)));
         }
       }
@@ -226,8 +229,8 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
     }
     __syncthreads();
 
-    uint8_t* ocode = arr<uint8_t>(c, is_v ? A_RVCODE : A_RKCODE, a.layer) + (hT + gslot0) * 64;
-    uint32_t* osz = arr<uint32_t>(c, is_v ? A_RVSZ : A_RKSZ, a.layer);
+    uint32_t* oks = reinterpret_cast<uint32_t*>(orec + kRecKsz);
+    uint32_t* ovs = reinterpret_cast<uint32_t*>(orec + kRecVsz);
     if (!is_v) {
       if (tid < kD) {  // one group per (64 consecutive slots, channel), rows present only
         float mn = xs[0][tid], mx = mn;
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
         group_sz(mn, mx, hs, hz);
         sk[tid] = __half2float(hs);
         zk[tid] = __half2float(hz);
-        osz[((size_t)h * (T / kG) + (gslot0 >> 6)) * kD + tid] = pack_sz(hs, hz);
+        oks[tid] = pack_sz(hs, hz);
       }
     } else if (tid < 2 * kG) {  // one group per (slot, half)
       const int tt = tid >> 1, hf = tid & 1;
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
       }
       sv[tt][hf] = sval;
       zv[tt][hf] = zval;
-      osz[(hT + gslot0 + tt) * 2 + hf] = packed;
+      ovs[tt * 2 + hf] = packed;
     }
     __syncthreads();
     uint4 w = make_uint4(0u, 0u, 0u, 0u);
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
       else
         w = pack_quarter(xs, t, qq, [&](int tt, int ch) { return make_float2(sv[tt][ch >> 6], zv[tt][ch >> 6]); });
     }
-    reinterpret_cast<uint4*>(ocode + (size_t)t * 64)[qq] = w;
+    reinterpret_cast<uint4*>(orec + (size_t)t * 128 + code_off)[qq] = w;
     __syncthreads();
   }
 

@@ -28,6 +28,7 @@ struct ReaderArgs {
   const uint16_t* q;
   const uint16_t* k_new;
   const uint16_t* v_new;
+  const float* o_prev;
   float* o;
   float* part;
   int32_t* counter;
@@ -35,8 +36,7 @@ struct ReaderArgs {
 
 struct SelectArgs {
   CacheView c;
-  int layer0, n_q, n_tail, k_sel;
-  const float* o_prev;
+  int layer0, r, n_q, n_tail, k_sel;
 };
 
 cudaError_t launch_encode_base(const EncodeBaseArgs& a, cudaStream_t s);
@@ -46,6 +46,6 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s);
 
 int dense_splits(int heads, int n_q);
-int sparse_splits(int heads, int k_sel);
+int sparse_splits(int heads, int k_sel, int loops);
 
 }  // namespace fl

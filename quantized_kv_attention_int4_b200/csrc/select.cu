@@ -1,5 +1,5 @@
 // Column selector for sparse loops: top-K of the preceding loop's distribution, the
-// selected mass m, and the unselected columns' contribution u.
+// selected mass m, and the gather plan the sparse reader follows.
 //
 // FlashLoop project page, "The Method", Step 02: the preceding loop identifies the
 // columns to recompute, and their global probability mass under the preceding loop's
@@ -15,9 +15,10 @@
 //             prefix and a block-wide scan from the top bin;
 //   compact:  keys above the threshold plus the lowest-index ties, written in index
 //             order (per-warp ballots and a block prefix), so S is ascending;
-//   m, u:     m = sum_S p~_j; u = o_prev - sum_S p~_j v_j with v_j the column's value
-//             at loop tag_j (base plus residuals up to min(tag_j, depth_j), or the
-//             tail row of loop tag_j).
+//   m, plan:  m = sum_S p~_j; for every j in S its tag, p~_j, the number of stores it
+//             has in loop r (min(r, depth_j); 0 for a BF16 tail column) and its slot in
+//             each residual store (block first slot + popcount of the block mask), so the
+//             sparse reader can issue all of a column's loads at once.
 #include "kernels.h"
 
 namespace fl {
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int h = blockIdx.x, layer = a.layer0 + blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const CacheView& c = a.c;
-  const int H = c.H, cap = c.cap, ncb = cap / kG, T = c.total_slots, R = c.R;
+  const int cap = c.cap, ncb = cap / kG, R = c.R;
   const int n_q = a.n_q, N = a.n_q + a.n_tail, K = a.k_sel;
 
   const float* score = arr<float>(c, A_SCORE, layer) + (size_t)h * cap;
@@ -174,68 +175,31 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   if (lane == 0) red[warp] = mpart;
   __syncthreads();
 
-  // ---- u = o_prev - sum_S p~_j v_j(tag_j) ----
-  const uint8_t* vcode = arr<uint8_t>(c, A_VCODE, layer) + (size_t)h * cap * 64;
-  const uint32_t* vsz = arr<uint32_t>(c, A_VSZ, layer) + (size_t)h * cap * 2;
-  const uint8_t* rvcode = arr<uint8_t>(c, A_RVCODE, layer) + (size_t)h * T * 64;
-  const uint32_t* rvsz = arr<uint32_t>(c, A_RVSZ, layer) + (size_t)h * T * 2;
+  // ---- gather plan of S: column, tag, stores, p~, residual slots ----
   const unsigned long long* mask = arr<unsigned long long>(c, A_MASK, layer);
   const int32_t* first = arr<int32_t>(c, A_FIRST, layer);
   const uint8_t* depth = arr<uint8_t>(c, A_DEPTH, layer);
-  const uint16_t* tail_v = arr<uint16_t>(c, A_TAILV, layer);
-  const int qq = tid & 3;
-  float acc[32];
-#pragma unroll
-  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-  float corr = 0.f;
-  for (int task = tid; task < 4 * K; task += kThreads) {
-    const int j = sel[task >> 2];
-    const float p = ex2(key_value(keys[j]));
+  const int ps = c.plan_stride;
+  int32_t* plan = arr<int32_t>(c, A_PLAN, layer) + (size_t)h * c.max_select * ps;
+  const int r = a.r;
+  for (int k = tid; k < K; k += kThreads) {
+    const int j = sel[k];
     int lam = tag[j];
     lam = lam < 1 ? 1 : (lam > R ? R : lam);
+    int stores = 0;
     if (j < n_q) {
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(vcode + (size_t)j * 64) + qq);
-      const float2 sz = unpack_sz(__ldg(vsz + (size_t)j * 2 + (qq >> 1)));
-      const float P = 128.f * (p * sz.x);
-      corr += fmaf(p, sz.y, -P);
-      axpy32(x, P, acc);
       const int dep = depth[j];
-      const int top = lam < dep ? lam : dep;
-      const int b = j >> 6, jt = j & 63;
-      for (int rp = 2; rp <= top; ++rp) {
-        const unsigned long long mk = mask[(size_t)rp * ncb + b];
-        const int gs = c.slot_base[rp] + first[(size_t)rp * ncb + b] + __popcll(mk & ((1ull << jt) - 1ull));
-        const uint4 y = __ldg(reinterpret_cast<const uint4*>(rvcode + (size_t)gs * 64) + qq);
-        const float2 s2 = unpack_sz(__ldg(rvsz + (size_t)gs * 2 + (qq >> 1)));
-        const float P2 = 128.f * (p * s2.x);
-        corr += fmaf(p, s2.y, -P2);
-        axpy32(y, P2, acc);
-      }
-    } else {
-      const uint16_t* row = tail_v + (((size_t)(lam - 1) * H + h) * kTail + (j - n_q)) * kD;
-      axpy_bf16_32(row + 32 * qq, p, acc);
+      stores = dep < r ? dep : r;
     }
-  }
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    acc[k] += __shfl_xor_sync(kFull, acc[k], 4);
-    acc[k] += __shfl_xor_sync(kFull, acc[k], 8);
-    acc[k] += __shfl_xor_sync(kFull, acc[k], 16);
-  }
-  corr += __shfl_xor_sync(kFull, corr, 4);
-  corr += __shfl_xor_sync(kFull, corr, 8);
-  corr += __shfl_xor_sync(kFull, corr, 16);
-  float* ored = reinterpret_cast<float*>(hist);  // [32 warps][128]
-  if (lane < 4) {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) ored[warp * kD + 32 * qq + k] = acc[k] + corr;
-  }
-  __syncthreads();
-  if (tid < kD) {
-    float s = 0.f;
-    for (int w = 0; w < kWarpsSel; ++w) s += ored[w * kD + tid];
-    const float op = a.o_prev[((size_t)blockIdx.y * H + h) * kD + tid];
-    arr<float>(c, A_UNSEL, layer)[(size_t)h * kD + tid] = op - s;
+    int32_t* e = plan + (size_t)k * ps;
+    e[0] = j;
+    e[1] = lam | (stores << 8);
+    e[2] = __float_as_int(ex2(key_value(keys[j])));
+    const int b = j >> 6, jt = j & 63;
+    for (int rp = 2; rp <= stores; ++rp) {
+      const unsigned long long mk = mask[(size_t)rp * ncb + b];
+      e[1 + rp] = c.slot_base[rp] + first[(size_t)rp * ncb + b] + __popcll(mk & ((1ull << jt) - 1ull));
+    }
   }
   if (tid == 0) {
     float m = 0.f;

@@ -30,6 +30,17 @@ def split_sz(raw: np.ndarray):
     return (raw & 0xFFFF).astype(np.uint16).view(np.float16), (raw >> 16).astype(np.uint16).view(np.float16)
 
 
+def _split_records(raw: np.ndarray, H: int, G: int):
+    """Group records [H][G][9216] -> key codes, value codes [H][G*64][128], key sz [H][G][128], value sz [H][G*64][2]."""
+    rec = raw[: H * G * 9216].reshape(H, G, 9216)
+    rows = rec[:, :, :8192].reshape(H, G, 64, 128)
+    kc = nibbles(rows[..., :64].reshape(H, G * 64, 64))
+    vc = nibbles(rows[..., 64:].reshape(H, G * 64, 64))
+    vsz = np.ascontiguousarray(rec[:, :, 8192:8704]).view(np.uint32).reshape(H, G * 64, 2)
+    ksz = np.ascontiguousarray(rec[:, :, 8704:]).view(np.uint32).reshape(H, G, 128)
+    return kc, vc, ksz, vsz
+
+
 class Unpacked:
     """Logical views of one layer of a FlashLoopCache (CPU copies)."""
 
@@ -37,14 +48,12 @@ class Unpacked:
         H, C, R = cache.H, cache.capacity, cache.R
         T = cache.layout.total_slots
         g = lambda n: cache.raw(n, layer).cpu().numpy()
-        self.kc = nibbles(g("kcode")[: H * C * 64].reshape(H, C, 64))
-        self.vc = nibbles(g("vcode")[: H * C * 64].reshape(H, C, 64))
-        self.ks, self.kz = split_sz(g("ksz").view(np.uint32)[: H * (C // 64) * 128].reshape(H, C // 64, 128))
-        self.vs, self.vz = split_sz(g("vsz").view(np.uint32)[: H * C * 2].reshape(H, C, 2))
-        self.rkc = nibbles(g("rkcode")[: H * T * 64].reshape(H, T, 64))
-        self.rvc = nibbles(g("rvcode")[: H * T * 64].reshape(H, T, 64))
-        self.rks, self.rkz = split_sz(g("rksz").view(np.uint32)[: H * (T // 64) * 128].reshape(H, T // 64, 128))
-        self.rvs, self.rvz = split_sz(g("rvsz").view(np.uint32)[: H * T * 2].reshape(H, T, 2))
+        self.kc, self.vc, ksz, vsz = _split_records(g("brec"), H, C // 64)
+        self.ks, self.kz = split_sz(ksz)
+        self.vs, self.vz = split_sz(vsz)
+        self.rkc, self.rvc, rksz, rvsz = _split_records(g("rrec"), H, T // 64)
+        self.rks, self.rkz = split_sz(rksz)
+        self.rvs, self.rvz = split_sz(rvsz)
         self.mask = g("mask").view(np.uint64)[: (R + 1) * (C // 64)].reshape(R + 1, C // 64)
         self.first = g("first").view(np.int32)[: (R + 1) * (C // 64)].reshape(R + 1, C // 64)
         self.depth = g("depth")[:C]
@@ -139,11 +148,12 @@ class Pair:
                 ref = lay.dense_loop(r, f32(q[r][hs]))
                 errs[r] = rel_err(o.cpu().numpy()[hs], ref["o"])
             else:
-                c.select(0, 1, k_sel, o_prev.view(1, H, 128))
-                S, m, u = selection(c, 0, k_sel)
+                c.select(0, 1, r, k_sel)
+                S, _, _ = selection(c, 0, k_sel)
                 if check:
                     check_topk_valid(S[hs], lay.p_tilde, k_sel)
-                c.sparse(0, r, k_sel, qr, o, kn, vn)
+                c.sparse(0, r, k_sel, qr, o_prev, o, kn, vn)
+                _, m, u = selection(c, 0, k_sel)
                 ref = lay.sparse_loop(r, f32(q[r][hs]), S[hs])
                 errs[(r, "m")] = float(np.max(np.abs(m[hs] - ref["m"]) / ref["m"]))
                 scale = np.maximum(np.abs(ref["u"]).max(axis=1), np.abs(ref["o"]).max(axis=1))

@@ -37,14 +37,14 @@ def test_layout_is_aligned_and_consistent():
     d = _dims()
     L = abi.fl_cache_layout(d)
     offs = [getattr(L, n) for n in abi.ARRAY_NAMES] + [L.status]
+    assert L.plan_stride == 8
     assert all(o % 256 == 0 for o in offs)
     assert offs == sorted(offs) and len(set(offs)) == len(offs)
     assert list(L.slot_base)[2:5] == [0, 1024, 1280] and L.total_slots == 1408
     H, C, T = 4, 1024, 1408
-    assert L.layer_stride[0] == H * C * 64                      # kcode
-    assert L.layer_stride[2] == H * (C // 64) * 128 * 4         # ksz
-    assert L.layer_stride[6] == H * (T // 64) * 128 * 4         # rksz
-    assert L.layer_stride[11] == 4 * H * 64 * 128 * 2           # tail_k
+    assert L.layer_stride[0] == H * (C // 64) * 9216            # base group records
+    assert L.layer_stride[1] == H * (T // 64) * 9216            # residual group records
+    assert L.layer_stride[5] == 4 * H * 64 * 128 * 2            # tail_k
     for i, name in enumerate(abi.ARRAY_NAMES[:-1]):
         nxt = getattr(L, abi.ARRAY_NAMES[i + 1])
         assert getattr(L, name) + 2 * L.layer_stride[i] == nxt
@@ -90,13 +90,15 @@ def test_reader_arguments_are_validated_before_launch():
     assert dense(n_q=1024) == abi.FL_ERR_INVALID          # exceeds capacity
     assert dense(kn=FAKE) == abi.FL_ERR_INVALID            # k_new without v_new
     assert dense(ws=ws - 1) == abi.FL_ERR_WORKSPACE
-    sparse = lambda k_sel: abi._c_sparse(ctypes.byref(d), FAKE, 0, 3, 64, 1, k_sel, FAKE, None, None, FAKE,
-                                         FAKE, ws, None)
+    sparse = lambda k_sel, prev=FAKE: abi._c_sparse(ctypes.byref(d), FAKE, 0, 3, 64, 1, k_sel, FAKE, None, None,
+                                                    prev, FAKE, FAKE, ws, None)
     assert sparse(0) == abi.FL_ERR_INVALID
     assert sparse(66) == abi.FL_ERR_INVALID               # more than N
-    sel = lambda **k: abi._c_select(ctypes.byref(d), FAKE, k.get("l0", 0), k.get("nl", 1), k.get("n_q", 64), 1,
-                                    k.get("k_sel", 10), FAKE, None)
+    assert sparse(10, prev=None) == abi.FL_ERR_INVALID    # o_prev is required
+    sel = lambda **k: abi._c_select(ctypes.byref(d), FAKE, k.get("l0", 0), k.get("nl", 1), k.get("loop", 3),
+                                    k.get("n_q", 64), 1, k.get("k_sel", 10), None)
     assert sel(nl=3) == abi.FL_ERR_INVALID
+    assert sel(loop=1) == abi.FL_ERR_INVALID              # a selection prepares a sparse loop >= 2
     assert sel(k_sel=129) == abi.FL_ERR_INVALID           # above max_select
     step = lambda **k: abi._c_step(ctypes.byref(d), FAKE, 64, 1, k.get("dl", 2), k.get("k_sel", 10),
                                    k.get("lf", 1), k.get("ll", 4), FAKE, None, None, FAKE, FAKE, ws, None, None)
@@ -106,7 +108,7 @@ def test_reader_arguments_are_validated_before_launch():
     assert step(k_sel=0) == abi.FL_ERR_INVALID
     assert step(dl=0, lf=1) == abi.FL_ERR_INVALID         # first loop cannot be sparse
     big = _dims(capacity=65536, max_select=10)
-    assert abi._c_select(ctypes.byref(big), FAKE, 0, 1, 49152, 1, 10, FAKE, None) == abi.FL_ERR_UNSUPPORTED
+    assert abi._c_select(ctypes.byref(big), FAKE, 0, 1, 3, 49152, 1, 10, None) == abi.FL_ERR_UNSUPPORTED
 
 
 def test_encoder_arguments_are_validated_before_launch():

@@ -72,13 +72,14 @@ def test_full_retention_sparse_equals_dense():
         c.dense(0, r, q[r].contiguous(), o, keep_scores=True)
         lay.dense_loop(r, f32(q[r]))
         o_prev = o
-    c.select(0, 1, N, o_prev.view(1, 16, 128))
-    S, m, u = selection(c, 0, N)
+    c.select(0, 1, 3, N)
+    S, _, _ = selection(c, 0, N)
     assert np.array_equal(S, np.tile(np.arange(N), (16, 1)))
+    o = torch.empty(16, 128, device="cuda")
+    c.sparse(0, 3, N, q[3].contiguous(), o_prev, o)
+    _, m, u = selection(c, 0, N)
     assert np.all(np.abs(m - 1) < 1e-5)
     assert np.abs(u).max() < 1e-5 * np.abs(o_prev.cpu().numpy()).max() * 10
-    o = torch.empty(16, 128, device="cuda")
-    c.sparse(0, 3, N, q[3].contiguous(), o)
     ref = fo.attention_dense(f32(q[3]), *lay.columns(3))[0]
     assert rel_err(o.cpu().numpy(), ref) < TOL
 
@@ -96,7 +97,7 @@ def test_decode_steps_across_two_flushes():
         tok = pair.begin_token(step)
         q = synth.queries(w, 0, step + 1, device="cuda")
         _assert_errs(pair.run_loops(q, tok))
-    assert pair.cache.n_q == 192 + 128
+    assert pair.cache.n_q == 192 + 3 * 64  # flushes at steps 0, 64 and 128
     compare_encoding(pair)
 
 
@@ -154,14 +155,17 @@ def test_device_errors_are_recorded_not_trapped():
                            compact=False)
     st, info = c.status()
     assert st == abi.FL_ERR_DEVICE and info[0] == 3 and info[1] == inactive3
-    # a selected column out of range is skipped and reported
+    # a selected column out of range is skipped and reported (on a fresh, consistent cache)
+    pair = Pair(w)
+    c = pair.cache
     q = synth.queries(w, 0, 0, device="cuda")
     o = torch.empty(2, 128, device="cuda")
-    pair.cache.set_timeline(pair.cache.n_q, pair.cache.n_tail, pair.cache.tail_depth)
     c.dense(0, 1, q[1].contiguous(), o, keep_scores=True)
-    c.select(0, 1, 10, o.view(1, 2, 128))
-    c.raw("sel", 0).view(torch.int32)[3] = 100000
-    c.sparse(0, 2, 10, q[2].contiguous(), o)
+    c.select(0, 1, 2, 10)
+    ps = c.layout.plan_stride
+    c.raw("plan", 0).view(torch.int32)[3 * ps] = 100000   # head 0, fourth selected column
+    o2 = torch.empty(2, 128, device="cuda")
+    c.sparse(0, 2, 10, q[2].contiguous(), o, o2)
     st, info = c.status()
     assert st == abi.FL_ERR_DEVICE and info[0] == 4 and info[1] == 100000
-    assert torch.isfinite(o).all()
+    assert torch.isfinite(o2).all()
