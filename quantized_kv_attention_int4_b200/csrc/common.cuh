@@ -289,22 +289,18 @@ __device__ __forceinline__ void axpy8_h(uint32_t w, unsigned short we, unsigned 
 }
 
 // ---- exact integer key dots (dp4a) against fixed-point query weights ----
-// A group's weights qs_c = q_c * s_c become Q_c = rint(qs_c * 2^E), |Q_c| <= 32767,
-// split into an unsigned low byte and a signed high byte.  For code word w (channels
-// 8w..8w+7) the limbs are 4 words: low bytes of the even channels (8w, 8w+2, 8w+4,
-// 8w+6), high bytes of the even channels, low bytes of the odd channels, high bytes of
-// the odd channels -- matching the low / high nibbles of the code word's bytes.
-__device__ __forceinline__ void dp4a_word(uint32_t w, uint4 limb, int& lo, int& hi) {
-  const uint32_t ne = w & 0x0F0F0F0Fu;
-  const uint32_t no = (w >> 4) & 0x0F0F0F0Fu;
-  asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(lo) : "r"(ne), "r"(limb.x));
-  asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(hi) : "r"(ne), "r"(limb.y));
-  asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(lo) : "r"(no), "r"(limb.z));
-  asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(hi) : "r"(no), "r"(limb.w));
-}
+// A key group's weights qs_c = q_c * s_c become Q_c = rint(qs_c * 2^E) with
+// |Q_c| < 2^23 (24-bit fixed point, E per record from the largest |qs_c|), split into
+// bytes b0, b1 (unsigned) and b2 (signed): Q = b2 * 2^16 + b1 * 2^8 + b0.  For code
+// word w (channels 8w..8w+7, nibble k = channel 8w + k) the limbs are 6 words:
+// b0, b1, b2 of the even channels (8w, 8w+2, 8w+4, 8w+6), then b0, b1, b2 of the odd
+// channels -- matching the low / high nibbles of the code word's four bytes.
+constexpr int kLimbWords = 6;
+constexpr int kLimbE = 16 * kLimbWords;   // record word holding E
+constexpr int kLimbC = kLimbE + 1;        // record word holding C = sum_c q_c z_c (fp32 bits)
 
-// One warp turns a key (scale, zero) record (128 words) into dp4a limbs in place:
-// words 0..63 = limbs, word 64 = E, word 65 = C = sum_c q_c z_c (fp32 bits).
+// One warp turns a key (scale, zero) record (128 words: channel c at word c, scale in
+// the low half) into limbs in place: words 0..95 limbs, word 96 E, word 97 C.
 __device__ __forceinline__ void record_to_limbs(uint32_t* rec, const float* q_s, int lane) {
   const uint4 raw = *reinterpret_cast<const uint4*>(rec + 4 * lane);
   const float4 qv = *reinterpret_cast<const float4*>(q_s + 4 * lane);
@@ -314,44 +310,67 @@ __device__ __forceinline__ void record_to_limbs(uint32_t* rec, const float* q_s,
   float mx = fmaxf(fmaxf(fabsf(qs0), fabsf(qs1)), fmaxf(fabsf(qs2), fabsf(qs3)));
   mx = warp_max(mx);
   cz = warp_sum(cz);
-  int e2 = 0;
-  if (mx > 0.f) frexpf(mx, &e2);        // mx = f * 2^e2, f in [0.5, 1)
-  const int E = 15 - e2;                 // |qs| * 2^E < 2^15
+  int E = 0;
+  if (mx > 0.f) {
+    int e2;
+    frexpf(mx, &e2);  // mx = f * 2^e2, f in [0.5, 1)
+    E = min(23 - e2, 126);
+  }
   const float sc = ldexpf(1.0f, E);
   auto fix = [&](float v) {
-    int qv_ = __float2int_rn(v * sc);
-    return qv_ > 32767 ? 32767 : (qv_ < -32767 ? -32767 : qv_);
+    const int x = __float2int_rn(v * sc);
+    return x > 8388607 ? 8388607 : (x < -8388607 ? -8388607 : x);
   };
   const int Q0 = fix(qs0), Q1 = fix(qs1), Q2 = fix(qs2), Q3 = fix(qs3);
   __syncwarp();
-  // lane l holds channels 4l..4l+3 of code word w = l/2; even channels 4l, 4l+2 and odd
-  // channels 4l+1, 4l+3 fill bytes 2*(l&1), 2*(l&1)+1 of the word's four limb words.
+  // lane l holds channels 4l..4l+3 of code word w = l/2: even channels 4l, 4l+2 and odd
+  // channels 4l+1, 4l+3 fill bytes 2*(l&1), 2*(l&1)+1 of the word's limb words.
   const int w = lane >> 1, hb = (lane & 1) * 2;
-  uint8_t* lb = reinterpret_cast<uint8_t*>(rec + 4 * w);
-  lb[0 * 4 + hb] = (uint8_t)(Q0 & 0xff);
-  lb[0 * 4 + hb + 1] = (uint8_t)(Q2 & 0xff);
-  lb[1 * 4 + hb] = (uint8_t)((Q0 >> 8) & 0xff);
-  lb[1 * 4 + hb + 1] = (uint8_t)((Q2 >> 8) & 0xff);
-  lb[2 * 4 + hb] = (uint8_t)(Q1 & 0xff);
-  lb[2 * 4 + hb + 1] = (uint8_t)(Q3 & 0xff);
-  lb[3 * 4 + hb] = (uint8_t)((Q1 >> 8) & 0xff);
-  lb[3 * 4 + hb + 1] = (uint8_t)((Q3 >> 8) & 0xff);
+  uint16_t* lh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(rec + kLimbWords * w) + hb);
+  auto pair = [](int a, int b, int sh) { return (uint16_t)(((a >> sh) & 0xff) | (((b >> sh) & 0xff) << 8)); };
+  lh[0] = pair(Q0, Q2, 0);
+  lh[2] = pair(Q0, Q2, 8);
+  lh[4] = pair(Q0, Q2, 16);
+  lh[6] = pair(Q1, Q3, 0);
+  lh[8] = pair(Q1, Q3, 8);
+  lh[10] = pair(Q1, Q3, 16);
   if (lane == 0) {
-    rec[64] = (uint32_t)E;
-    rec[65] = __float_as_uint(cz);
+    rec[kLimbE] = (uint32_t)E;
+    rec[kLimbC] = __float_as_uint(cz);
   }
 }
 
-// The record's limb dot over one 32-channel quarter qq of a key code row (4 code words).
-__device__ __forceinline__ float limb_dot_quarter(const uint32_t* rec, uint4 code, int qq) {
-  const uint4* lw = reinterpret_cast<const uint4*>(rec) + 4 * qq;
-  int lo = 0, hi = 0;
-  dp4a_word(code.x, lw[0], lo, hi);
-  dp4a_word(code.y, lw[1], lo, hi);
-  dp4a_word(code.z, lw[2], lo, hi);
-  dp4a_word(code.w, lw[3], lo, hi);
-  const int E = (int)rec[64];
-  return (float)(hi * 256 + lo) * __int_as_float((127 - E) << 23);
+// Dot of one 32-channel quarter of a code row (4 code words) with the record's 24 limb
+// words of that quarter (words 24*qq.., held in registers), in units of 2^-E.  Odd
+// channels are taken in place (their nibble x16) and scaled back here.
+__device__ __forceinline__ float limb_dot(uint4 code, const uint32_t* L) {
+  int e0 = 0, e1 = 0, e2 = 0, o0 = 0, o1 = 0, o2 = 0;
+  const uint32_t cw[4] = {code.x, code.y, code.z, code.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t ne = cw[i] & 0x0F0F0F0Fu, no = cw[i] & 0xF0F0F0F0u;
+    asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(e0) : "r"(ne), "r"(L[6 * i + 0]));
+    asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(e1) : "r"(ne), "r"(L[6 * i + 1]));
+    asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(e2) : "r"(ne), "r"(L[6 * i + 2]));
+    asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(o0) : "r"(no), "r"(L[6 * i + 3]));
+    asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(o1) : "r"(no), "r"(L[6 * i + 4]));
+    asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(o2) : "r"(no), "r"(L[6 * i + 5]));
+  }
+  const int le = e1 * 256 + e0, lo = o1 * 256 + o0;
+  return fmaf((float)e2, 65536.f, (float)le) + 0.0625f * fmaf((float)o2, 65536.f, (float)lo);
+}
+
+// The 24 limb words of quarter qq of a converted record, into registers.
+__device__ __forceinline__ void load_limbs(const uint32_t* rec, int qq, uint32_t* L) {
+  const uint4* p = reinterpret_cast<const uint4*>(rec) + 6 * qq;
+#pragma unroll
+  for (int j = 0; j < 6; ++j) {
+    const uint4 x = p[j];
+    L[4 * j + 0] = x.x;
+    L[4 * j + 1] = x.y;
+    L[4 * j + 2] = x.z;
+    L[4 * j + 3] = x.w;
+  }
 }
 
 // log2(e) / sqrt(128): scores are kept in the base-2 domain.

@@ -1,4 +1,6 @@
-// Dense decode reader: single-query attention of one loop over every column.
+// Dense decode reader, direct-load form: single-query attention of one loop over every
+// column.  The staged reader (dense_staged.cu) covers loops whose residual rows come from
+// at most two stores; this form serves every other loop.
 //
 // FlashLoop project page, "The Method": dense loops attend over all columns; a
 // column's key/value in loop r is the loop-1 base plus its residuals of loops 2..r
@@ -26,7 +28,7 @@ namespace {
 
 constexpr int kWarps = 8;
 
-__global__ void __launch_bounds__(kWarps * 32, 2) dense_kernel(ReaderArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs a) {
   const int h = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, qq = lane & 3, tr = lane >> 2;
   const CacheView& c = a.c;
@@ -333,10 +335,10 @@ int dense_splits(int heads, int n_q) {
   return s;
 }
 
-cudaError_t launch_dense(ReaderArgs a, cudaStream_t s) {
+cudaError_t launch_dense_direct(ReaderArgs a, cudaStream_t s) {
   a.n_splits = dense_splits(a.c.H, a.n_q);
   dim3 grid(a.n_splits, a.c.H);
-  dense_kernel<<<grid, kWarps * 32, 0, s>>>(a);
+  dense_direct_kernel<<<grid, kWarps * 32, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,693 @@
+// Dense decode reader, staged form: single-query attention of one loop r <= 3 over
+// every column, with the block's bytes staged in shared memory by bulk copies.
+//
+// FlashLoop project page, "The Method": dense loops attend over all columns; a
+// column's key/value in loop r is the loop-1 base plus its residuals of loops 2..r
+// (Step 03), or the loop's BF16 tail row (flashloop 0.1.0 PyPI description,
+// "Configuration and supported scope": 64-token BF16 tail).
+//
+// Grid: one persistent CTA per SM, kWS warps each.  The units of all heads (each
+// head's 64-token blocks, then its tail unit) are numbered head-major and cut into one
+// contiguous range per CTA (at most two heads per range); warp w takes units w,
+// w + kWS, ... of its CTA's range and owns a ring of shared memory.  Ahead of use it
+// stages into the ring, for each block, one span:
+//   [0, 9216)   the block's base group record (one bulk copy);
+//   per residual store s of loops 2..r, if the block has rows there: the rows' code
+//               lines (128 B each, from one or two group records), then per group record
+//               its key (scale, zero) record (512 B) and the value (scale, zero) words of
+//               the rows (rounded out to an even slot so the copy is 16-byte aligned).
+// The copies of one span complete on one mbarrier (kSlots per warp, round robin).
+//
+// Per block, all on the staged bytes:
+//   keys    every key (scale, zero) record becomes 24-bit fixed-point query weights
+//           Q_c = rint(q_c s_c 2^E) split into byte limbs; a code row is dotted with
+//           them by dp4a (exact integer sums), then scaled by 2^-E, plus sum_c q_c z_c;
+//           residual rows add their dot to the logit of their token;
+//   softmax p'_t = 2^(l_t - m_b) with m_b the block maximum; the warp's running (M, L)
+//           and output are rescaled once per block;
+//   values  row weights W = p' s_h per 64-channel half h become 24-bit fixed point
+//           numbers (E_h from the block's largest weight); the code words of four rows are
+//           transposed by byte permutes into per-channel nibble quadruples and dotted
+//           by dp4a with the four rows' weight limbs; plus Z_h = sum_t p'_t z_t,h.
+// The tail unit reads its BF16 rows from global memory in fp32.
+// Warps' partials merge per CTA; the last CTA of each head (atomic ticket) combines the
+// CTA partials by log-sum-exp and writes o and offset[r] = M + log2 L.
+#include "kernels.h"
+
+namespace fl {
+namespace {
+
+constexpr int kWS = 7;                           // warps per CTA
+constexpr int kThreads = kWS * 32;
+constexpr int kSlots = 4;                        // staged blocks in flight per warp
+constexpr int kStores = 2;                       // residual stores staged (loops 2, 3)
+constexpr int kMaxGroups = 16 + kStores * 16;    // 4-row weight groups of one block
+constexpr int kSmemTotal = 232448;               // opt-in shared memory per CTA
+constexpr int kHdr = 64 + 2 * kD * 4;            // flags + the CTA's two queries
+
+struct alignas(16) WarpCtl {
+  uint64_t bar[kSlots];
+  int32_t slot_off[kSlots];
+  int32_t slot_gs0[kSlots][kStores];
+  unsigned long long slot_mk[kSlots][kStores];
+  float lg[kG];                  // logits of the block, then p'
+  uint8_t tok[kStores][kG];      // token of each residual row
+  uint4 wl[kMaxGroups][2];       // weight limbs (bytes 0, 1, 2 of four rows) per group, half
+  float part0[2 + kD];           // (M, L, o) of the warp's first head
+  int32_t has[2];
+};
+
+constexpr int kRing = ((kSmemTotal - kHdr - kWS * (int)sizeof(WarpCtl)) / kWS) & ~15;
+// largest span: base record + 2 stores x (64 code rows + 2 key records + 66 value words)
+constexpr int kMaxSpan = kRec + kStores * (kG * 128 + 2 * 512 + (kG + 2) * 8);
+static_assert(kRing >= kMaxSpan, "ring must hold the largest span");
+
+// Geometry of one block's rows in one residual store, as staged in the span.
+struct StoreGeom {
+  int na, n1;          // rows, rows in the first group record
+  int off_codes;       // code rows 0..na-1, 128 B each (rows past na read padding)
+  int off_k0, off_k1;  // key (scale, zero) records, turned into limbs in place
+  int off_v0, off_v1;  // value (scale, zero) words: row i of piece p at off_vp + (vskip_p + i) * 8
+  int vskip0;
+};
+
+__device__ __forceinline__ int store_geom(unsigned long long mk, int gs0, int pos, StoreGeom& g) {
+  g.na = __popcll(mk);
+  g.n1 = 0;
+  g.off_codes = g.off_k0 = g.off_k1 = g.off_v0 = g.off_v1 = pos;
+  g.vskip0 = 0;
+  if (g.na == 0) return pos;
+  const int s0 = gs0 & 63;
+  g.n1 = min(g.na, kG - s0);
+  g.off_codes = pos;
+  pos += g.na * 128;
+  g.off_k0 = pos;
+  pos += 512;
+  g.off_v0 = pos;
+  g.vskip0 = s0 & 1;
+  pos += (((s0 + g.n1 + 1) & ~1) - (s0 & ~1)) * 8;
+  g.off_k1 = g.off_k0;
+  g.off_v1 = g.off_v0;
+  if (g.n1 < g.na) {
+    const int n2 = g.na - g.n1;
+    g.off_k1 = pos;
+    pos += 512;
+    g.off_v1 = pos;
+    pos += ((n2 + 1) & ~1) * 8;
+  }
+  return pos;
+}
+
+// Bulk copies of one span (lane 0 only); `bytes` is the span size.
+__device__ __forceinline__ void issue_span(uint8_t* sp, const uint8_t* brec_b, const uint8_t* rrec,
+                                           const StoreGeom* g, const int* gs0, int bytes, uint64_t* bar) {
+  fence_proxy_async();
+  mbar_expect_tx(bar, (unsigned)bytes);
+  bulk_g2s(sp, brec_b, kRec, bar);
+#pragma unroll
+  for (int s = 0; s < kStores; ++s) {
+    const StoreGeom& G = g[s];
+    if (G.na == 0) continue;
+    const int s0 = gs0[s] & 63;
+    const uint8_t* R0 = rrec + (size_t)(gs0[s] >> 6) * kRec;
+    bulk_g2s(sp + G.off_codes, R0 + s0 * 128, G.n1 * 128, bar);
+    bulk_g2s(sp + G.off_k0, R0 + kRecKsz, 512, bar);
+    const int a0 = s0 & ~1, a1 = (s0 + G.n1 + 1) & ~1;
+    bulk_g2s(sp + G.off_v0, R0 + kRecVsz + a0 * 8, (a1 - a0) * 8, bar);
+    if (G.n1 < G.na) {
+      const int n2 = G.na - G.n1;
+      const uint8_t* R1 = R0 + kRec;
+      bulk_g2s(sp + G.off_codes + G.n1 * 128, R1, n2 * 128, bar);
+      bulk_g2s(sp + G.off_k1, R1 + kRecKsz, 512, bar);
+      bulk_g2s(sp + G.off_v1, R1 + kRecVsz, ((n2 + 1) & ~1) * 8, bar);
+    }
+  }
+}
+
+__device__ __forceinline__ void dp4a_u(int& acc, uint32_t a, uint32_t b) {
+  asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(acc) : "r"(a), "r"(b));
+}
+
+// Four rows' code words x0..x3 (same word, channels 8w..8w+7) against the four rows'
+// weight limbs (byte 0, 1, 2 words): a0/a1/a2[c] accumulate channel 8w + c (odd
+// channels x16).
+__device__ __forceinline__ void v_group(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint4 wq,
+                                        int* a0, int* a1, int* a2) {
+  const uint32_t a_lo = __byte_perm(x0, x1, 0x5140), a_hi = __byte_perm(x0, x1, 0x7362);
+  const uint32_t b_lo = __byte_perm(x2, x3, 0x5140), b_hi = __byte_perm(x2, x3, 0x7362);
+  uint32_t T[4];
+  T[0] = __byte_perm(a_lo, b_lo, 0x5410);  // byte 0 of rows 0..3
+  T[1] = __byte_perm(a_lo, b_lo, 0x7632);  // byte 1
+  T[2] = __byte_perm(a_hi, b_hi, 0x5410);  // byte 2
+  T[3] = __byte_perm(a_hi, b_hi, 0x7632);  // byte 3
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t ev = T[b] & 0x0F0F0F0Fu, od = T[b] & 0xF0F0F0F0u;
+    dp4a_u(a0[2 * b], ev, wq.x);
+    dp4a_u(a1[2 * b], ev, wq.y);
+    dp4a_u(a2[2 * b], ev, wq.z);
+    dp4a_u(a0[2 * b + 1], od, wq.x);
+    dp4a_u(a1[2 * b + 1], od, wq.y);
+    dp4a_u(a2[2 * b + 1], od, wq.z);
+  }
+}
+
+// CTA holding unit x when U units are cut into n contiguous ranges floor(cU/n).
+__device__ __forceinline__ int cta_of(long long x, long long U, int n) {
+  return (int)(((x + 1) * n + U - 1) / U) - 1;
+}
+
+__device__ __forceinline__ uint32_t fix24(float w, float sc) {
+  const uint32_t q = __float2uint_rn(w * sc);
+  return q > 16777215u ? 16777215u : q;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a, int n_cta) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  int* last = reinterpret_cast<int*>(smem);
+  float* q_all = reinterpret_cast<float*>(smem + 64);
+  WarpCtl* ctl = reinterpret_cast<WarpCtl*>(smem + kHdr);
+  uint8_t* rings = smem + kHdr + kWS * sizeof(WarpCtl);
+
+  const CacheView& c = a.c;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int qq = lane & 3, tr = lane >> 2;        // key mapping: row tr of 8, quarter qq
+  const int wv = lane & 15, gv = lane >> 4, hv = wv >> 3;  // value mapping: word, row parity
+  const int H = c.H, cap = c.cap, ncb = cap / kG, T = c.total_slots, r = a.r;
+  const int nb = a.n_q / kG, nbp = nb + 1;
+  const long long U = (long long)H * nbp;
+  const int cta = blockIdx.x;
+  const int U0 = (int)((long long)cta * U / n_cta), U1 = (int)((long long)(cta + 1) * U / n_cta);
+  const int h0 = U0 / nbp, h1 = (U1 - 1) / nbp;
+  const int nst = r - 1;
+
+  for (int i = tid; i < 2 * kD; i += kThreads) {
+    const int hh = h0 + i / kD;
+    q_all[i] = hh <= h1 ? __uint_as_float((uint32_t)a.q[(size_t)hh * kD + (i % kD)] << 16) * kQScale : 0.f;
+  }
+  WarpCtl& w = ctl[warp];
+  uint8_t* ring = rings + (size_t)warp * kRing;
+  if (lane == 0) {
+    for (int i = 0; i < kSlots; ++i) mbar_init(&w.bar[i], 1);
+    fence_mbar_init();
+    w.has[0] = w.has[1] = 0;
+  }
+  __syncthreads();
+
+  const unsigned long long* mask = arr<unsigned long long>(c, A_MASK, a.layer);
+  const int32_t* first = arr<int32_t>(c, A_FIRST, a.layer);
+  const uint8_t* brec_l = arr<uint8_t>(c, A_BREC, a.layer);
+  const uint8_t* rrec_l = arr<uint8_t>(c, A_RREC, a.layer);
+  const int n_my = U1 - U0 > warp ? (U1 - U0 - warp + kWS - 1) / kWS : 0;
+  const bool has_new = a.k_new != nullptr;
+
+  // metadata window: lane (k_off = lane >> 1, s = lane & 1) holds store 2+s of unit iss_k + k_off
+  const int ms = lane & 1;
+  auto load_meta = [&](int k, unsigned long long& mk, int& g0) {
+    mk = 0ull;
+    g0 = 0;
+    if (k < n_my && ms < nst) {
+      const int u = U0 + warp + k * kWS, b = u % nbp;
+      if (b < nb) {
+        const int rp = 2 + ms;
+        mk = __ldg(mask + (size_t)rp * ncb + b);
+        g0 = c.slot_base[rp] + __ldg(first + (size_t)rp * ncb + b);
+      }
+    }
+  };
+  unsigned long long m_mk;
+  int m_gs;
+  load_meta(lane >> 1, m_mk, m_gs);
+
+  int iss_k = 0, iss_seq = 0, con_seq = 0, wpos = 0;
+  bool failed = false;
+
+  float acc[8];
+  float M = -INFINITY, Ls = 0.f;
+  int cur_hs = -1;
+
+  auto flush = [&](int hs) {
+    float* dst = hs == 0 ? w.part0 : reinterpret_cast<float*>(ring);
+    float o8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o8[k] = acc[k] + __shfl_xor_sync(kFull, acc[k], 16);
+    const float Lw = warp_sum(Ls);
+    if (gv == 0) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) dst[2 + 8 * wv + k] = o8[k];
+    }
+    if (lane == 0) {
+      dst[0] = M;
+      dst[1] = Lw;
+      w.has[hs] = 1;
+    }
+  };
+  // merge one block's (max, per-lane sum, per-channel values) into the running state
+  auto merge = [&](float mb, float bs, const float* val) {
+    const float Mn = fmaxf(M, mb);
+    const float ao = ex2(M - Mn), ab = ex2(mb - Mn);
+    Ls = fmaf(Ls, ao, bs * ab);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = fmaf(acc[k], ao, ab * val[k]);
+    M = Mn;
+  };
+
+  for (int k = 0; k < n_my; ++k) {
+    // ---- stage ahead: issue spans while a slot and ring space are free ----
+    while (!failed && iss_k < n_my) {
+      const int u = U0 + warp + iss_k * kWS, b = u % nbp;
+      if (b < nb) {
+        if (iss_seq - con_seq >= kSlots) break;
+        unsigned long long mk2[kStores];
+        int gs[kStores];
+        mk2[0] = __shfl_sync(kFull, m_mk, 0);
+        mk2[1] = __shfl_sync(kFull, m_mk, 1);
+        gs[0] = __shfl_sync(kFull, m_gs, 0);
+        gs[1] = __shfl_sync(kFull, m_gs, 1);
+        StoreGeom g[kStores];
+        int pos = store_geom(mk2[0], gs[0], kRec, g[0]);
+        pos = store_geom(mk2[1], gs[1], pos, g[1]);
+        int start = -1;
+        if (iss_seq == con_seq) {
+          start = 0;
+        } else {
+          const int rp = w.slot_off[con_seq % kSlots];
+          if (wpos > rp) {
+            if (wpos + pos <= kRing) start = wpos;
+            else if (pos <= rp) start = 0;
+          } else if (wpos + pos <= rp) {
+            start = wpos;
+          }
+        }
+        if (start < 0) break;
+        wpos = start + pos;
+        const int slot = iss_seq % kSlots;
+        __syncwarp();
+        if (lane == 0) {
+          w.slot_off[slot] = start;
+          w.slot_mk[slot][0] = mk2[0];
+          w.slot_mk[slot][1] = mk2[1];
+          w.slot_gs0[slot][0] = gs[0];
+          w.slot_gs0[slot][1] = gs[1];
+          const int h = u / nbp;
+          issue_span(ring + start, brec_l + ((size_t)h * ncb + b) * kRec,
+                     rrec_l + (size_t)h * (T / kG) * kRec, g, gs, pos, &w.bar[slot]);
+        }
+        ++iss_seq;
+      }
+      ++iss_k;
+      // slide the metadata window by one unit
+      const unsigned lo_m = __shfl_down_sync(kFull, (unsigned)m_mk, 2);
+      const unsigned hi_m = __shfl_down_sync(kFull, (unsigned)(m_mk >> 32), 2);
+      m_gs = __shfl_down_sync(kFull, m_gs, 2);
+      m_mk = ((unsigned long long)hi_m << 32) | lo_m;
+      if (lane >= 30) load_meta(iss_k + 15, m_mk, m_gs);
+    }
+    __syncwarp();
+    if (failed) break;
+
+    const int u = U0 + warp + k * kWS, h = u / nbp, b = u % nbp, hs = h - h0;
+    if (hs != cur_hs) {
+      if (cur_hs >= 0) flush(cur_hs);
+      cur_hs = hs;
+      M = -INFINITY;
+      Ls = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    }
+    const float* qh = q_all + hs * kD;
+    float* score = arr<float>(c, A_SCORE, a.layer) + (size_t)h * cap;
+    uint8_t* tag = arr<uint8_t>(c, A_TAG, a.layer) + (size_t)h * cap;
+
+    if (b < nb) {
+      // ================= staged block =================
+      const int slot = con_seq % kSlots;
+      const bool ok = __any_sync(kFull, mbar_wait(&w.bar[slot], (unsigned)(con_seq / kSlots) & 1u));
+      if (!ok) {
+        if (lane == 0) record_error(c.status, FL_DEV_TIMEOUT, b);
+        failed = true;
+        break;
+      }
+      uint8_t* sp = ring + w.slot_off[slot];
+      StoreGeom g[kStores];
+      const unsigned long long mkA = w.slot_mk[slot][0], mkB = w.slot_mk[slot][1];
+      {
+        const int pos = store_geom(mkA, w.slot_gs0[slot][0], kRec, g[0]);
+        store_geom(mkB, w.slot_gs0[slot][1], pos, g[1]);
+      }
+
+      // ---- key limbs of the base record and of every residual group record ----
+      record_to_limbs(reinterpret_cast<uint32_t*>(sp + kRecKsz), qh, lane);
+#pragma unroll
+      for (int s = 0; s < kStores; ++s) {
+        if (g[s].na == 0) continue;
+        record_to_limbs(reinterpret_cast<uint32_t*>(sp + g[s].off_k0), qh, lane);
+        if (g[s].n1 < g[s].na) record_to_limbs(reinterpret_cast<uint32_t*>(sp + g[s].off_k1), qh, lane);
+      }
+      __syncwarp();
+
+      // ---- base logits ----
+      {
+        const uint32_t* lim = reinterpret_cast<const uint32_t*>(sp + kRecKsz);
+        uint32_t lw[24];
+        load_limbs(lim, qq, lw);
+        const float sc = ldexpf(1.f, -(int)lim[kLimbE]);
+        const float C = __uint_as_float(lim[kLimbC]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int t = 8 * i + tr;
+          const uint4 code = *reinterpret_cast<const uint4*>(sp + t * 128 + 16 * qq);
+          float v = limb_dot(code, lw) * sc;
+          v += __shfl_xor_sync(kFull, v, 1);
+          v += __shfl_xor_sync(kFull, v, 2);
+          if (qq == 0) w.lg[t] = v + C;
+        }
+      }
+      // ---- residual logits, added to their tokens ----
+#pragma unroll
+      for (int s = 0; s < kStores; ++s) {
+        const StoreGeom& G = g[s];
+        if (G.na == 0) continue;
+        const unsigned long long mk = s == 0 ? mkA : mkB;
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tt = lane + 32 * e;
+          if ((mk >> tt) & 1ull) w.tok[s][__popcll(mk & ((1ull << tt) - 1ull))] = (uint8_t)tt;
+        }
+        __syncwarp();
+        for (int i0 = 0; i0 < G.na; i0 += 8) {
+          const int i = i0 + tr;
+          const bool act = i < G.na;
+          const int ii = act ? i : G.na - 1;
+          const uint32_t* lim = reinterpret_cast<const uint32_t*>(sp + (ii < G.n1 ? G.off_k0 : G.off_k1));
+          uint32_t lw[24];
+          load_limbs(lim, qq, lw);
+          const uint4 code = *reinterpret_cast<const uint4*>(sp + G.off_codes + ii * 128 + 16 * qq);
+          float v = limb_dot(code, lw) * ldexpf(1.f, -(int)lim[kLimbE]);
+          v += __shfl_xor_sync(kFull, v, 1);
+          v += __shfl_xor_sync(kFull, v, 2);
+          if (act && qq == 0) w.lg[w.tok[s][i]] += v + __uint_as_float(lim[kLimbC]);
+        }
+      }
+      __syncwarp();
+
+      // ---- block softmax ----
+      const float l0 = w.lg[lane], l1 = w.lg[lane + 32];
+      if (a.keep) {
+        score[(size_t)b * kG + lane] = l0;
+        score[(size_t)b * kG + lane + 32] = l1;
+        tag[(size_t)b * kG + lane] = (uint8_t)r;
+        tag[(size_t)b * kG + lane + 32] = (uint8_t)r;
+      }
+      const float mb = warp_max(fmaxf(l0, l1));
+      const float p0 = ex2(l0 - mb), p1 = ex2(l1 - mb);
+      __syncwarp();
+      w.lg[lane] = p0;
+      w.lg[lane + 32] = p1;
+      __syncwarp();
+
+      // ---- value weights: W = p' s_h as 16-bit fixed point per half ----
+      const int pad0 = (g[0].na + 3) & ~3, pad1 = (g[1].na + 3) & ~3;
+      const int nvr = kG + pad0 + pad1;
+      float W0[6], W1[6];
+      float z0 = 0.f, z1 = 0.f, mx0 = 0.f, mx1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 6; ++i) {
+        W0[i] = W1[i] = 0.f;
+        if (32 * i >= nvr) break;
+        const int v = lane + 32 * i;
+        float p = 0.f;
+        uint2 sz = make_uint2(0u, 0u);
+        if (v < kG) {
+          p = w.lg[v];
+          sz = *reinterpret_cast<const uint2*>(sp + kRecVsz + v * 8);
+        } else if (v < nvr) {
+          int vv = v - kG;
+          const int s = vv >= pad0 ? 1 : 0;
+          if (s) vv -= pad0;
+          const int na = s ? g[1].na : g[0].na, n1 = s ? g[1].n1 : g[0].n1;
+          if (vv < na) {
+            p = w.lg[w.tok[s][vv]];
+            const int off = vv < n1 ? (s ? g[1].off_v0 : g[0].off_v0) + ((s ? g[1].vskip0 : g[0].vskip0) + vv) * 8
+                                    : (s ? g[1].off_v1 : g[0].off_v1) + (vv - n1) * 8;
+            sz = *reinterpret_cast<const uint2*>(sp + off);
+          }
+        }
+        const float2 e0 = unpack_sz(sz.x), e1 = unpack_sz(sz.y);
+        W0[i] = p * e0.x;
+        W1[i] = p * e1.x;
+        z0 = fmaf(p, e0.y, z0);
+        z1 = fmaf(p, e1.y, z1);
+        mx0 = fmaxf(mx0, W0[i]);
+        mx1 = fmaxf(mx1, W1[i]);
+      }
+      mx0 = warp_max(mx0);
+      mx1 = warp_max(mx1);
+      z0 = warp_sum(z0);
+      z1 = warp_sum(z1);
+      int E0 = 0, E1 = 0;
+      if (mx0 > 0.f) { int e; frexpf(mx0, &e); E0 = min(24 - e, 126); }
+      if (mx1 > 0.f) { int e; frexpf(mx1, &e); E1 = min(24 - e, 126); }
+      const float sc0 = ldexpf(1.f, E0), sc1 = ldexpf(1.f, E1);
+#pragma unroll
+      for (int i = 0; i < 6; ++i) {
+        if (32 * i >= nvr) break;
+        const int v = lane + 32 * i;
+        const uint32_t Q0 = fix24(W0[i], sc0), Q1 = fix24(W1[i], sc1);
+        // lane 4m gathers rows 4m..4m+3 and writes their three limb words per half
+        const uint32_t Q0b = __shfl_down_sync(kFull, Q0, 1), Q0c = __shfl_down_sync(kFull, Q0, 2),
+                       Q0d = __shfl_down_sync(kFull, Q0, 3);
+        const uint32_t Q1b = __shfl_down_sync(kFull, Q1, 1), Q1c = __shfl_down_sync(kFull, Q1, 2),
+                       Q1d = __shfl_down_sync(kFull, Q1, 3);
+        if ((lane & 3) == 0 && v < nvr) {
+          uint32_t A = __byte_perm(Q0, Q0b, 0x5140), B = __byte_perm(Q0c, Q0d, 0x5140);
+          uint32_t C = __byte_perm(Q0, Q0b, 0x7362), D = __byte_perm(Q0c, Q0d, 0x7362);
+          w.wl[v >> 2][0] = make_uint4(__byte_perm(A, B, 0x5410), __byte_perm(A, B, 0x7632),
+                                       __byte_perm(C, D, 0x5410), 0u);
+          A = __byte_perm(Q1, Q1b, 0x5140);
+          B = __byte_perm(Q1c, Q1d, 0x5140);
+          C = __byte_perm(Q1, Q1b, 0x7362);
+          D = __byte_perm(Q1c, Q1d, 0x7362);
+          w.wl[v >> 2][1] = make_uint4(__byte_perm(A, B, 0x5410), __byte_perm(A, B, 0x7632),
+                                       __byte_perm(C, D, 0x5410), 0u);
+        }
+      }
+      __syncwarp();
+
+      // ---- values: dp4a over transposed nibbles ----
+      int a0[8], a1[8], a2[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a0[i] = a1[i] = a2[i] = 0;
+      {
+        const uint8_t* vb = sp + 64 + 4 * wv;
+#pragma unroll
+        for (int kg = gv; kg < 16; kg += 2) {
+          const uint8_t* rp = vb + kg * 512;
+          v_group(*reinterpret_cast<const uint32_t*>(rp), *reinterpret_cast<const uint32_t*>(rp + 128),
+                  *reinterpret_cast<const uint32_t*>(rp + 256), *reinterpret_cast<const uint32_t*>(rp + 384),
+                  w.wl[kg][hv], a0, a1, a2);
+        }
+      }
+#pragma unroll
+      for (int s = 0; s < kStores; ++s) {
+        const int ng = (s ? pad1 : pad0) >> 2;
+        const int kb = 16 + (s ? (pad0 >> 2) : 0);
+        const uint8_t* vb = sp + (s ? g[1].off_codes : g[0].off_codes) + 64 + 4 * wv;
+        for (int kg = gv; kg < ng; kg += 2) {
+          const uint8_t* rp = vb + kg * 512;
+          v_group(*reinterpret_cast<const uint32_t*>(rp), *reinterpret_cast<const uint32_t*>(rp + 128),
+                  *reinterpret_cast<const uint32_t*>(rp + 256), *reinterpret_cast<const uint32_t*>(rp + 384),
+                  w.wl[kb + kg][hv], a0, a1, a2);
+        }
+      }
+      const float isc = ldexpf(1.f, -(hv ? E1 : E0));
+      const float zh = gv == 0 ? (hv ? z1 : z0) : 0.f;
+      float val[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        val[i] = fmaf(fmaf((float)a2[i], 65536.f, fmaf((float)a1[i], 256.f, (float)a0[i])),
+                      (i & 1) ? isc * 0.0625f : isc, zh);
+      merge(mb, p0 + p1, val);
+      fence_proxy_async();  // this span's generic reads and writes precede its reuse by bulk copies
+      __syncwarp();
+      ++con_seq;
+    } else {
+      // ================= BF16 tail unit (global loads) =================
+      const int nt = a.n_tail;
+      uint16_t* tail_k = arr<uint16_t>(c, A_TAILK, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
+      uint16_t* tail_v = arr<uint16_t>(c, A_TAILV, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
+      const uint16_t* kn = has_new ? a.k_new + (size_t)h * kD : nullptr;
+      const uint16_t* vn = has_new ? a.v_new + (size_t)h * kD : nullptr;
+      if (has_new) {
+        reinterpret_cast<uint2*>(tail_k + (size_t)(nt - 1) * kD)[lane] = reinterpret_cast<const uint2*>(kn)[lane];
+        reinterpret_cast<uint2*>(tail_v + (size_t)(nt - 1) * kD)[lane] = reinterpret_cast<const uint2*>(vn)[lane];
+      }
+      float qsr[32];
+      load32(qh + 32 * qq, qsr);
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = 8 * i + tr;
+        const bool act = t < nt;
+        float p = 0.f;
+        if (act) {
+          const uint16_t* row = (has_new && t == nt - 1) ? kn : tail_k + (size_t)t * kD;
+          p = dot_bf16_32(row + 32 * qq, qsr);
+        }
+        p += __shfl_xor_sync(kFull, p, 1);
+        p += __shfl_xor_sync(kFull, p, 2);
+        if (qq == 0) w.lg[t] = act ? p : -INFINITY;
+      }
+      __syncwarp();
+      const float l0 = w.lg[lane], l1 = w.lg[lane + 32];
+      if (a.keep) {
+        if (lane < nt) {
+          score[(size_t)a.n_q + lane] = l0;
+          tag[(size_t)a.n_q + lane] = (uint8_t)r;
+        }
+        if (lane + 32 < nt) {
+          score[(size_t)a.n_q + lane + 32] = l1;
+          tag[(size_t)a.n_q + lane + 32] = (uint8_t)r;
+        }
+      }
+      const float mb = warp_max(fmaxf(l0, l1));
+      if (mb != -INFINITY) {
+        const float p0 = ex2(l0 - mb), p1 = ex2(l1 - mb);
+        __syncwarp();
+        w.lg[lane] = p0;
+        w.lg[lane + 32] = p1;
+        __syncwarp();
+        float val[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) val[i] = 0.f;
+        for (int t = gv; t < nt; t += 2) {
+          const uint16_t* row = (has_new && t == nt - 1) ? vn : tail_v + (size_t)t * kD;
+          const uint4 x = __ldg(reinterpret_cast<const uint4*>(row) + wv);
+          const float pt = w.lg[t];
+          val[0] = fmaf(pt, bf16_lo(x.x), val[0]);
+          val[1] = fmaf(pt, bf16_hi(x.x), val[1]);
+          val[2] = fmaf(pt, bf16_lo(x.y), val[2]);
+          val[3] = fmaf(pt, bf16_hi(x.y), val[3]);
+          val[4] = fmaf(pt, bf16_lo(x.z), val[4]);
+          val[5] = fmaf(pt, bf16_hi(x.z), val[5]);
+          val[6] = fmaf(pt, bf16_lo(x.w), val[6]);
+          val[7] = fmaf(pt, bf16_hi(x.w), val[7]);
+        }
+        merge(mb, p0 + p1, val);
+      }
+      __syncwarp();
+    }
+  }
+
+  if (failed) {
+    // staged copies still in flight land before the ring is reused below
+    for (int s = con_seq; s < iss_seq; ++s) mbar_wait(&w.bar[s % kSlots], (unsigned)(s / kSlots) & 1u);
+    __syncwarp();
+  }
+  if (cur_hs >= 0) flush(cur_hs);
+  __syncthreads();
+
+  // ---- CTA partials per head, then the last CTA of each head combines ----
+  for (int hs = 0; hs <= h1 - h0; ++hs) {
+    const int h = h0 + hs;
+    const int c_lo = cta_of((long long)h * nbp, U, n_cta);
+    float* part = a.part + ((size_t)h * kMaxSplits + (cta - c_lo)) * kPartStride;
+    if (tid < kD) {
+      float Mx = -INFINITY;
+      for (int v = 0; v < kWS; ++v)
+        if (ctl[v].has[hs]) {
+          const float* src = hs == 0 ? ctl[v].part0 : reinterpret_cast<const float*>(rings + (size_t)v * kRing);
+          Mx = fmaxf(Mx, src[0]);
+        }
+      float Lt = 0.f, ot = 0.f;
+      for (int v = 0; v < kWS; ++v)
+        if (ctl[v].has[hs]) {
+          const float* src = hs == 0 ? ctl[v].part0 : reinterpret_cast<const float*>(rings + (size_t)v * kRing);
+          if (src[0] == -INFINITY) continue;
+          const float e = ex2(src[0] - Mx);
+          Lt = fmaf(src[1], e, Lt);
+          ot = fmaf(src[2 + tid], e, ot);
+        }
+      part[4 + tid] = ot;
+      if (tid == 0) {
+        part[0] = Mx;
+        part[1] = Lt;
+      }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    for (int hs = 0; hs < 2; ++hs) {
+      last[hs] = 0;
+      if (hs > h1 - h0) continue;
+      const int h = h0 + hs;
+      const int n_parts = cta_of((long long)(h + 1) * nbp - 1, U, n_cta) - cta_of((long long)h * nbp, U, n_cta) + 1;
+      last[hs] = atomicAdd(&a.counter[h], 1) == n_parts - 1;
+    }
+  }
+  __syncthreads();
+  for (int hs = 0; hs <= h1 - h0; ++hs) {
+    if (!last[hs]) continue;
+    __threadfence();
+    const int h = h0 + hs;
+    const int c_lo = cta_of((long long)h * nbp, U, n_cta);
+    const int n_parts = cta_of((long long)(h + 1) * nbp - 1, U, n_cta) - c_lo + 1;
+    if (tid < kD) {
+      const float* hp = a.part + (size_t)h * kMaxSplits * kPartStride;
+      float Mx = -INFINITY;
+      for (int s = 0; s < n_parts; ++s) Mx = fmaxf(Mx, __ldcg(hp + (size_t)s * kPartStride));
+      float Lt = 0.f, ot = 0.f;
+      for (int s = 0; s < n_parts; ++s) {
+        const float m_s = __ldcg(hp + (size_t)s * kPartStride);
+        if (m_s == -INFINITY) continue;
+        const float e = ex2(m_s - Mx);
+        Lt = fmaf(__ldcg(hp + (size_t)s * kPartStride + 1), e, Lt);
+        ot = fmaf(__ldcg(hp + (size_t)s * kPartStride + 4 + tid), e, ot);
+      }
+      a.o[(size_t)h * kD + tid] = ot / Lt;
+      if (tid == 0) {
+        arr<float>(c, A_OFFSET, a.layer)[(size_t)h * kOffStride + r] = Mx + log2f(Lt);
+        a.counter[h] = 0;
+      }
+    }
+  }
+}
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace
+
+cudaError_t launch_dense(ReaderArgs a, cudaStream_t s) {
+  const int sms = num_sms();
+  const long long U = (long long)a.c.H * (a.n_q / kG + 1);
+  long long n = sms < U ? sms : U;
+  if (n < a.c.H) n = a.c.H;  // every CTA range then touches at most two heads
+  if (a.r > 3 || sms == 0 || n > kMaxSplits) return launch_dense_direct(a, s);
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(dense_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  a.n_splits = (int)n;
+  dense_staged_kernel<<<(int)n, kThreads, kSmemTotal, s>>>(a, (int)n);
+  return cudaGetLastError();
+}
+
+}  // namespace fl
