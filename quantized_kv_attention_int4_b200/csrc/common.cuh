@@ -252,12 +252,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for phase `parity` of `bar`; false if the bound ran out.
-constexpr long long kWaitBound = 1ll << 22;
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// try_wait that lets the hardware suspend the thread for up to `ns` nanoseconds while
+// the phase is incomplete (no issue slots are spent meanwhile).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, unsigned parity, unsigned ns) {
+  unsigned ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for phase `parity` of `bar` (2 s of device time); false if the bound ran out.
+constexpr uint64_t kWaitNs = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
-  for (long long i = 0; i < kWaitBound; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+  if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait_sleep(bar, parity, 1000000u))
+    if (global_ns() - t0 > kWaitNs) return false;
+  return true;
 }
 
 // fp32 accumulate of an fp16 product: acc += a * b with a, b binary16 (exact product).
