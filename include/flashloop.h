@@ -224,6 +224,32 @@ fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer,
                                 const uint16_t* k_new, const uint16_t* v_new, const float* o_prev,
                                 float* o, void* ws, size_t ws_bytes, void* stream);
 
+/* Largest scratch of fl_decode_attn_sparse_noalloc, in bytes (a static device array of
+ * the library). */
+#define FL_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* fl_decode_attn_sparse for callers that cannot allocate device memory -- an engine
+ * whose allocator is frozen after start-up, or a host ABI with no way to hand over a
+ * workspace.  Same arguments, validation and results as fl_decode_attn_sparse except
+ * that there is no ws/ws_bytes: the reader's scratch (one ticket per head, which this
+ * call clears on `stream` before the launch, and heads x splits x 1040 bytes of split
+ * partials) lives in a file-scope device array of FL_NOALLOC_SCRATCH_BYTES owned by the
+ * library.  Nothing is allocated by this call.
+ *   - The first call on a device looks the array's address up (cudaGetSymbolAddress,
+ *     with that device current) and caches it; make that first call before any stream
+ *     capture that is to contain this call.
+ *   - The array keeps its contents between calls and is shared by every caller in the
+ *     process on that device: calls that can overlap (different streams, threads)
+ *     race on it and must be serialised by the caller.
+ *   - FL_ERR_UNSUPPORTED when the scratch would exceed FL_NOALLOC_SCRATCH_BYTES (many
+ *     heads or a large k_sel); use fl_decode_attn_sparse with a workspace then.
+ * The FlashLoop pages have no counterpart: this is a deployment convenience of this
+ * library, not a step of the method. */
+fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,
+                                        int32_t n_q, int32_t n_tail, int32_t k_sel, const uint16_t* q,
+                                        const uint16_t* k_new, const uint16_t* v_new,
+                                        const float* o_prev, float* o, void* stream);
+
 /* Native executor of one decode step for layers [0, L) in loop-major order (every
  * layer runs loop r before any layer runs loop r+1), for loops loop_first..loop_last:
  * loops up to dense_loops call the dense reader (the last dense loop keeps scores);

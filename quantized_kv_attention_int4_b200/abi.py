@@ -33,7 +33,7 @@ FL_OK, FL_ERR_INVALID, FL_ERR_UNSUPPORTED, FL_ERR_CUDA, FL_ERR_WORKSPACE, FL_ERR
 EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init", "fl_workspace_bytes",
             "fl_workspace_init", "fl_write_tail", "fl_encode_base", "fl_encode_residual",
             "fl_decode_attn_dense", "fl_select_topk", "fl_decode_attn_sparse", "fl_decode_step",
-            "fl_read_status")
+            "fl_read_status", "fl_decode_attn_sparse_noalloc")
 
 
 class fl_dims(ctypes.Structure):
@@ -77,6 +77,8 @@ _c_dense = _sig("fl_decode_attn_dense", _I, _DP, _P, _I, _I, _I, _I, _P, _P, _P,
 _c_select = _sig("fl_select_topk", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P)
 _c_sparse = _sig("fl_decode_attn_sparse", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                  ctypes.c_size_t, _P)
+_c_sparse_noalloc = _sig("fl_decode_attn_sparse_noalloc", _I, _DP, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                         _P)
 _c_step = _sig("fl_decode_step", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t,
                 ctypes.POINTER(ctypes.c_void_p), _P)
 _c_read_status = _sig("fl_read_status", _I, _DP, _P, ctypes.POINTER(ctypes.c_int32), _I, _P)
@@ -213,6 +215,15 @@ def fl_decode_attn_sparse(dims, cache, layer, loop, n_q, n_tail, k_sel, q, k_new
         _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
         _ptr(o_prev, torch.float32, "o_prev"), _ptr(o, torch.float32, "o"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _stream(stream)))
+
+
+def fl_decode_attn_sparse_noalloc(dims, cache, layer, loop, n_q, n_tail, k_sel, q, k_new, v_new, o_prev, o,
+                                  stream=None):
+    """fl_decode_attn_sparse with the library's static scratch instead of a workspace."""
+    _check("fl_decode_attn_sparse_noalloc", _c_sparse_noalloc(
+        ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), layer, loop, n_q, n_tail, k_sel,
+        _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        _ptr(o_prev, torch.float32, "o_prev"), _ptr(o, torch.float32, "o"), _stream(stream)))
 
 
 def fl_decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, k_new, v_new, o, ws,

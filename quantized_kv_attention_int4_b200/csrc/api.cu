@@ -336,6 +336,68 @@ fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer,
   return cuda_status(launch_sparse(a, (cudaStream_t)stream));
 }
 
+// ---- sparse reader with library-owned scratch (for callers that cannot allocate) ----
+// The scratch is one file-scope device array; its address is looked up once per device
+// (cudaGetSymbolAddress, with that device current) and cached here.  Nothing is
+// allocated: the array is part of the library's loaded module.
+}  // extern "C"
+namespace {
+__device__ __align__(256) uint8_t g_noalloc_scratch[FL_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_ptr[64] = {nullptr};
+}  // namespace
+extern "C" {
+
+fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,
+                                        int32_t n_q, int32_t n_tail, int32_t k_sel, const uint16_t* q,
+                                        const uint16_t* k_new, const uint16_t* v_new, const float* o_prev,
+                                        float* o, void* stream) {
+  fl_status st = check_dims(dims);
+  if (st != FL_OK) return st;
+  if (!cache || !q || !o || !o_prev) return FL_ERR_INVALID;
+  if (layer < 0 || layer >= dims->layers || loop < 2 || loop > dims->loops) return FL_ERR_INVALID;
+  if (n_q < 0 || n_q % FL_GROUP != 0 || n_tail < 1 || n_tail > FL_TAIL) return FL_ERR_INVALID;
+  const int64_t N = (int64_t)n_q + n_tail;
+  if (N > dims->capacity) return FL_ERR_INVALID;
+  if ((k_new == nullptr) != (v_new == nullptr)) return FL_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(o) || (k_new && (!aligned16(k_new) || !aligned16(v_new))))
+    return FL_ERR_INVALID;
+  if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
+  // scratch: per-head tickets (must start at zero), then the split partials
+  const int n_splits = sparse_splits(dims->heads, k_sel, dims->loops);
+  const uint64_t ticket_bytes = ((uint64_t)dims->heads * sizeof(int32_t) + 255) / 256 * 256;
+  const uint64_t need = ticket_bytes + (uint64_t)dims->heads * n_splits * kPartStride * sizeof(float);
+  if (need > FL_NOALLOC_SCRATCH_BYTES) return FL_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FL_ERR_CUDA;
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return FL_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  uint8_t* scratch = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(scratch, 0, (size_t)dims->heads * sizeof(int32_t), s) != cudaSuccess) return FL_ERR_CUDA;
+  fl_layout L;
+  make_layout(dims, &L);
+  ReaderArgs a;
+  a.c = make_view(dims, L, cache);
+  a.layer = layer;
+  a.r = loop;
+  a.n_q = n_q;
+  a.n_tail = n_tail;
+  a.k_sel = k_sel;
+  a.n_splits = 1;
+  a.keep = 1;
+  a.q = q;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.o_prev = o_prev;
+  a.o = o;
+  a.counter = reinterpret_cast<int32_t*>(scratch);
+  a.part = reinterpret_cast<float*>(scratch + ticket_bytes);
+  return cuda_status(launch_sparse(a, s));
+}
+
 fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
                          int32_t k_sel, int32_t loop_first, int32_t loop_last, const uint16_t* q,
                          const uint16_t* k_new, const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,

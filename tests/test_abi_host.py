@@ -19,7 +19,7 @@ def _declared():
 
 def test_every_declared_symbol_is_exported():
     names = _declared()
-    assert len(names) == 14
+    assert len(names) == 15
     for n in names:
         assert hasattr(abi.lib, n), n
     assert set(names) == set(abi.EXPORTED)
@@ -137,3 +137,18 @@ def test_status_strings():
 def test_host_bookkeeping_helpers():
     assert [round_up(x) for x in (0, 1, 64, 65, 8176)] == [0, 64, 64, 128, 8192]
     assert split_prefill(32768) == (32704, 64) and split_prefill(100) == (64, 36)
+
+
+def test_noalloc_sparse_validation():
+    """The no-workspace sparse entry point validates on the host like the workspace one
+    and refuses a scratch larger than its static array (no compute: null cache)."""
+    d = abi.Dims(layers=1, heads=4, loops=4, capacity=1024, res_capacity={2: 1024, 3: 256, 4: 128}, max_select=128)
+    code = abi._c_sparse_noalloc(ctypes.byref(d), None, 0, 3, 960, 1, 10, None, None, None, None, None, None)
+    assert code == abi.FL_ERR_INVALID
+    # a scratch beyond the static array is refused before any CUDA call
+    buf = ctypes.create_string_buffer(256)
+    p = (ctypes.addressof(buf) + 15) // 16 * 16
+    big = abi.Dims(layers=1, heads=1100, loops=4, capacity=1024, res_capacity={2: 1024, 3: 256, 4: 128},
+                   max_select=128)
+    code = abi._c_sparse_noalloc(ctypes.byref(big), p, 0, 3, 960, 1, 10, p, None, None, p, p, None)
+    assert code == abi.FL_ERR_UNSUPPORTED
