@@ -43,6 +43,24 @@ DEFAULT_WORKLOAD = "cache_l48_h16_n32768"
 FALLBACK_HBM_GBS = 6650.0
 
 
+def _kernel_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu record, or None when the
+    kernel's sources changed since that capture (the counters no longer describe it)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "kernel_traffic.json")) as f:
+            rec = json.load(f)[kernel]
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, "quantized_kv_attention_int4_b200", "csrc", src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        return int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"])
+    except Exception:
+        return None
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -112,6 +130,21 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # the GPU path
 # ----------------------------------------------------------------------------
+def replica_workload(w: synth.Workload, rank: int) -> synth.Workload:
+    """Rank `rank`'s independent replica of the workload (weak scaling: same shapes,
+    its own seeds, no data shared between ranks)."""
+    return synth.Workload(**{**w.__dict__, "seed": w.seed + 100003 * rank})
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of `values` over all ranks (the job's time is its slowest rank)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() and \
+            torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def build_cache(w: synth.Workload, layers: int, rank: int, device):
     from quantized_kv_attention_int4_b200.cache import FlashLoopCache, round_up
 
@@ -122,7 +155,7 @@ def build_cache(w: synth.Workload, layers: int, rank: int, device):
     res_cap = {r: round_up(min(cap, int((sets[r] < n).sum()) + extra + 64 * 4)) for r in range(2, w.loops + 1)}
     cache = FlashLoopCache(layers, w.heads, w.loops, cap, res_capacity=res_cap,
                            max_select=w.k_sel(cap), device=device)
-    wr = synth.Workload(**{**w.__dict__, "seed": w.seed + 100003 * rank})
+    wr = replica_workload(w, rank)
     info = None
     for layer in range(layers):
         d = synth.prefill_layer(wr, layer, device=device, sets=sets)
@@ -276,12 +309,8 @@ def run_gpu(args, rank, world):
     metric_us = (mean["select4"] + mean["loop4"]) * 1e3
     step_ms = total_ms / args.steps
 
-    # max over ranks
-    vals = torch.tensor([metric_us, step_ms, mean["loop4"], mean["loop1"] + mean["loop2"]], device=device,
-                        dtype=torch.float64)
-    if world > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
-    metric_us, step_ms, loop4_ms, dense_ms = [float(x) for x in vals.tolist()]
+    metric_us, step_ms, loop4_ms, dense_ms = max_over_ranks(
+        [metric_us, step_ms, mean["loop4"], mean["loop1"] + mean["loop2"]], device)
 
     N = cache.n_cols
     k_sel = wr.k_sel(N)
@@ -335,49 +364,70 @@ def run_e2e(step, cache, w, layers, inputs, device):
 # ----------------------------------------------------------------------------
 # the oracle on the host cores
 # ----------------------------------------------------------------------------
-def oracle_loop4_sample(w: synth.Workload, budget_s: float, heads=(0,)):
-    """Time the oracle's loop-4 selection + sparse attention for one (layer, head) sample.
+class OracleLoop4:
+    """The oracle's loop-4 selection + sparse attention for one (layer, head) sample.
 
-    Setup (encoding, loops 1-3) is untimed; the loop-4 step is repeated until about
-    ``budget_s`` seconds have been spent.  Returns (seconds per (layer, head), reps).
+    Construction (untimed) encodes the prompt and runs loops 1-3; `run_once()` times one
+    loop-4 step (top-K selection from the spliced distribution, then the sparse loop)
+    from the same state and returns its seconds per (layer, head).
     """
-    from oracle import flashloop_oracle as fo
 
-    n = w.n_ctx
-    sets = synth.active_sets(w, n)
-    d = synth.prefill_layer(w, 0, device="cpu", sets=sets)
-    n_q, n_tail = synth.split_prefill(n)
-    hs = list(heads)
-    f = lambda t: t.float().numpy()
-    lay = fo.OracleLayer(len(hs), w.loops, n + 64)
-    lay.encode_base(0, f(d["K"][1][hs, :n_q]), f(d["V"][1][hs, :n_q]))
-    for r in range(2, w.loops + 1):
-        rows = sets[r][sets[r] < n_q].numpy()
-        lay.encode_residual(r, rows, f(d["K"][r][hs][:, rows]), f(d["V"][r][hs][:, rows]))
-    depth = synth.depth_of(sets, n).numpy()
-    lay.set_tail([None] + [f(d["K"][r][hs, n_q:]) for r in range(1, w.loops + 1)],
-                 [None] + [f(d["V"][r][hs, n_q:]) for r in range(1, w.loops + 1)], depth[n_q:])
-    del d
-    q = synth.queries(w, 0, 0).float().numpy()[:, hs]
-    k = w.k_sel(lay.n_cols)
-    for r in range(1, 4):
-        if r <= w.dense_loops:
-            lay.dense_loop(r, q[r])
-        else:
-            S, _, _ = lay.select(k)
-            lay.sparse_loop(r, q[r], S)
-    p_save, lam_save = lay.p_tilde.copy(), lay.lam.copy()
+    def __init__(self, w: synth.Workload, heads=(0,)):
+        from oracle import flashloop_oracle as fo
+
+        self.fo = fo
+        n = w.n_ctx
+        sets = synth.active_sets(w, n)
+        d = synth.prefill_layer(w, 0, device="cpu", sets=sets)
+        n_q, n_tail = synth.split_prefill(n)
+        hs = list(heads)
+        self.nh = len(hs)
+        f = lambda t: t.float().numpy()
+        lay = fo.OracleLayer(len(hs), w.loops, n + 64)
+        lay.encode_base(0, f(d["K"][1][hs, :n_q]), f(d["V"][1][hs, :n_q]))
+        for r in range(2, w.loops + 1):
+            rows = sets[r][sets[r] < n_q].numpy()
+            lay.encode_residual(r, rows, f(d["K"][r][hs][:, rows]), f(d["V"][r][hs][:, rows]))
+        depth = synth.depth_of(sets, n).numpy()
+        lay.set_tail([None] + [f(d["K"][r][hs, n_q:]) for r in range(1, w.loops + 1)],
+                     [None] + [f(d["V"][r][hs, n_q:]) for r in range(1, w.loops + 1)], depth[n_q:])
+        del d
+        self.q = synth.queries(w, 0, 0).float().numpy()[:, hs]
+        self.k = w.k_sel(lay.n_cols)
+        for r in range(1, 4):
+            if r <= w.dense_loops:
+                lay.dense_loop(r, self.q[r])
+            else:
+                S, _, _ = lay.select(self.k)
+                lay.sparse_loop(r, self.q[r], S)
+        self.lay = lay
+        self.p_save, self.lam_save = lay.p_tilde.copy(), lay.lam.copy()
+
+    def run_once(self) -> float:
+        """One timed loop-4 step on a single host thread (BLAS pool limited to 1)."""
+        from threadpoolctl import threadpool_limits
+
+        lay = self.lay
+        lay.p_tilde, lay.lam = self.p_save.copy(), self.lam_save.copy()
+        with threadpool_limits(limits=1):
+            t = time.perf_counter()
+            S = self.fo.select_topk(lay.p_tilde, self.k)
+            lay.sparse_loop(4, self.q[4], S)
+            dt = time.perf_counter() - t
+        return dt / self.nh
+
+
+def oracle_loop4_sample(w: synth.Workload, budget_s: float, heads=(0,)):
+    """Seconds per (layer, head) of the oracle's loop-4 step, averaged over repetitions
+    that fill about ``budget_s`` seconds; returns (seconds, repetitions)."""
+    o = OracleLoop4(w, heads)
     times = []
     t_all = time.perf_counter()
     while True:
-        lay.p_tilde, lay.lam = p_save.copy(), lam_save.copy()
-        t = time.perf_counter()
-        S = fo.select_topk(lay.p_tilde, k)
-        lay.sparse_loop(4, q[4], S)
-        times.append(time.perf_counter() - t)
+        times.append(o.run_once())
         if time.perf_counter() - t_all > budget_s and len(times) >= 2:
             break
-    return float(np.mean(times)) / len(hs), len(times)
+    return float(np.mean(times)), len(times)
 
 
 def cpu_baseline(w: synth.Workload, layers: int, budget_s: float):
@@ -418,10 +468,8 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        per_step = []
-        for _ in range(args.warmup + args.steps):
-            per_lh, _ = oracle_loop4_sample(w, 0.0)
-            per_step.append(per_lh * layers * w.heads * 1e6)
+        ora = OracleLoop4(w)
+        per_step = [ora.run_once() * layers * w.heads * 1e6 for _ in range(args.warmup + args.steps)]
         v = float(np.mean(per_step[args.warmup:]))
         line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3, "higher_is_better": False,
@@ -456,11 +504,11 @@ def main():
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": {**config, "context_at_end": r["N"],
                                                                           "k_sel": r["k_sel"]},
         "roofline": {"bound": "hbm", "kernel": "fl_decode_attn_sparse (loop 4)", "achieved": r["sp_gbs"],
-                     "peak": hbm, "unit": "GB/s", "frac": r["sp_gbs"] / hbm, "traffic": None,
+                     "peak": hbm, "unit": "GB/s", "frac": r["sp_gbs"] / hbm, "traffic": _kernel_traffic("sparse_kernel"),
                      "peak_kind": peak_kind_str(r["peak_kind"]), "bytes_per_launch": r["sp_bytes"],
                      "us_per_launch": r["sp_launch_us"]},
         "roofline_dense": {"bound": "hbm", "kernel": "fl_decode_attn_dense (loops 1-2)", "achieved": r["d_gbs"],
-                           "peak": hbm, "unit": "GB/s", "frac": r["d_gbs"] / hbm, "traffic": None,
+                           "peak": hbm, "unit": "GB/s", "frac": r["d_gbs"] / hbm, "traffic": _kernel_traffic("dense_staged_kernel"),
                            "bytes_per_launch": r["d_bytes"], "us_per_launch": r["d_launch_us"]},
         "segments_ms": r["seg"], "clocks": r["clocks"], "gpu_launches": r["launches"],
         "e2e": r["e2e"], "cpu_baseline": cpu, "setup_s": r["setup_s"],
