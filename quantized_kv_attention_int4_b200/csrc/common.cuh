@@ -391,6 +391,32 @@ __device__ __forceinline__ void load_limbs(const uint32_t* rec, int qq, uint32_t
   }
 }
 
+// ---- programmatic dependent launch ----
+// A reader lets the next kernel of its stream start as soon as all of its own CTAs are
+// running (the next reader stages and computes meanwhile), and waits for the previous
+// kernel to finish before it touches the state readers share: the split partials and
+// tickets of the workspace, and the previous loop's outputs.  Both are no-ops for a
+// kernel launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch `kernel` on `s` with programmatic stream serialization allowed.
+template <class... KArgs, class... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // log2(e) / sqrt(128): scores are kept in the base-2 domain.
 constexpr float kQScale = 1.4426950408889634f * 0.08838834764831845f;
 

@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
   const int U0 = (int)((long long)cta * U / n_cta), U1 = (int)((long long)(cta + 1) * U / n_cta);
   const int h0 = U0 / nbp, h1 = (U1 - 1) / nbp;
   const int nst = r - 1;
+  grid_dep_launch();
 
   for (int i = tid; i < 2 * kD; i += kThreads) {
     const int hh = h0 + i / kD;
@@ -587,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
   }
   if (cur_hs >= 0) flush(cur_hs);
   __syncthreads();
+  grid_dep_wait();  // the previous reader's partials and tickets are final from here
 
   // ---- CTA partials per head, then the last CTA of each head combines ----
   for (int hs = 0; hs <= h1 - h0; ++hs) {
@@ -686,8 +688,7 @@ cudaError_t launch_dense(ReaderArgs a, cudaStream_t s) {
     attr_set[dev] = true;
   }
   a.n_splits = (int)n;
-  dense_staged_kernel<<<(int)n, kThreads, kSmemTotal, s>>>(a, (int)n);
-  return cudaGetLastError();
+  return launch_pdl(dense_staged_kernel, dim3((int)n), dim3(kThreads), (size_t)kSmemTotal, s, a, (int)n);
 }
 
 }  // namespace fl

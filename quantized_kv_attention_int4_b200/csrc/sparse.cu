@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
   const int32_t* plan_g = arr<int32_t>(c, A_PLAN, a.layer) + (size_t)h * c.max_select * ps;
   const bool has_new = a.k_new != nullptr;
 
+  grid_dep_launch();
   const int k0 = (int)((long long)split * K / a.n_splits);
   const int k1 = (int)((long long)(split + 1) * K / a.n_splits);
   const int ncols = k1 - k0;
@@ -528,6 +529,7 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
     sm.msw[warp] = msum;
   }
   __syncthreads();
+  grid_dep_wait();  // the previous reader's partials, tickets and outputs are final from here
   float* part = a.part + ((size_t)h * a.n_splits + split) * kPartStride;
   if (tid < kD) {
     float Mx = -INFINITY;
@@ -607,8 +609,7 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(sparse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_splits, a.c.H);
-  sparse_kernel<<<grid, NT, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(sparse_kernel, grid, dim3(NT), smem, s, a);
 }
 
 }  // namespace fl
