@@ -26,6 +26,12 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarpsSel = kThreads / 32;
+constexpr int kDynMax = 200 * 1024;  // dynamic shared memory: keys [, selected columns]
+
+// Selected columns are kept in shared memory after the keys when both fit.
+__host__ __device__ inline bool sel_fits(int N, int K) {
+  return ((size_t)((N + 3) & ~3) + (size_t)K) * sizeof(uint32_t) <= (size_t)kDynMax;
+}
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t b = __float_as_uint(f);
@@ -59,7 +65,9 @@ __device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* wtot, int l
 }
 
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
-  extern __shared__ uint32_t keys[];
+  extern __shared__ uint32_t keys[];  // [N] keys, then [K] selected columns when they fit
+  const bool sel_smem = sel_fits(a.n_q + a.n_tail, a.k_sel);
+  int32_t* sel_s = reinterpret_cast<int32_t*>(keys + ((a.n_q + a.n_tail + 3) & ~3));
   __shared__ __align__(16) uint32_t hist[4096];
   __shared__ float offs[kOffStride];
   __shared__ uint32_t wtot[32];
@@ -78,14 +86,26 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
 
   if (tid < kOffStride) offs[tid] = arr<float>(c, A_OFFSET, layer)[(size_t)h * kOffStride + tid];
   __syncthreads();
-  for (int j = tid; j < N; j += kThreads) {
-    int t = tag[j];
+  // keys, four columns per thread per step (score rows are 16-byte and tag rows 4-byte
+  // aligned: cap is a multiple of 64); loads of several steps are in flight together
+  auto key_of = [&](float sc, int t, int j) {
     if (t < 1 || t > R) {
       record_error(c.status, FL_DEV_TAG_RANGE, j);
       t = t < 1 ? 1 : R;
     }
-    keys[j] = order_key(score[j] - offs[t]);
+    return order_key(sc - offs[t]);
+  };
+  const int N4 = N & ~3;
+#pragma unroll 4
+  for (int j = 4 * tid; j < N4; j += 4 * kThreads) {
+    const float4 sc = *reinterpret_cast<const float4*>(score + j);
+    const uint32_t tg = *reinterpret_cast<const uint32_t*>(tag + j);
+    keys[j] = key_of(sc.x, (int)(tg & 0xff), j);
+    keys[j + 1] = key_of(sc.y, (int)((tg >> 8) & 0xff), j + 1);
+    keys[j + 2] = key_of(sc.z, (int)((tg >> 16) & 0xff), j + 2);
+    keys[j + 3] = key_of(sc.w, (int)(tg >> 24), j + 3);
   }
+  for (int j = N4 + tid; j < N; j += kThreads) keys[j] = key_of(score[j], tag[j], j);
   __syncthreads();
 
   // ---- radix select of the K-th largest key ----
@@ -166,7 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     eqrun += __popc(be);
     const unsigned bs = __ballot_sync(kFull, s);
     if (s) {
-      sel[pos + __popc(bs & lt)] = j;
+      const int k = pos + __popc(bs & lt);
+      sel[k] = j;
+      if (sel_smem) sel_s[k] = j;
       mpart += ex2(key_value(u));
     }
     pos += __popc(bs);
@@ -182,8 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int ps = c.plan_stride;
   int32_t* plan = arr<int32_t>(c, A_PLAN, layer) + (size_t)h * c.max_select * ps;
   const int r = a.r;
+  __syncthreads();
+#pragma unroll 2
   for (int k = tid; k < K; k += kThreads) {
-    const int j = sel[k];
+    const int j = sel_smem ? sel_s[k] : sel[k];
     int lam = tag[j];
     lam = lam < 1 ? 1 : (lam > R ? R : lam);
     int stores = 0;
@@ -212,9 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
 
 cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s) {
   const int N = a.n_q + a.n_tail;
-  const size_t smem = (size_t)N * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(FL_MAX_SELECT_COLS * sizeof(uint32_t)));
+  const size_t smem = ((size_t)((N + 3) & ~3) + (sel_fits(N, a.k_sel) ? (size_t)a.k_sel : 0)) * sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynMax);
   if (e != cudaSuccess) return e;
   dim3 grid(a.c.H, n_layers);
   select_kernel<<<grid, kThreads, smem, s>>>(a);
