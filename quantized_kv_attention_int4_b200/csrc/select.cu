@@ -10,9 +10,10 @@
 // One CTA (1024 threads) per (layer, head), launched for a range of layers at once.
 //   keys:     log2 p~_j = score_j - offset[tag_j], mapped to an order-preserving u32
 //             and kept in shared memory (N <= FL_MAX_SELECT_COLS);
-//   select:   radix select of the K-th largest key, digits 12 + 12 + 8 bits, each
-//             pass a shared-memory histogram over the keys that still match the
-//             prefix and a block-wide scan from the top bin;
+//   select:   radix select of the K-th largest key over the bits where the keys
+//             differ (the prefix every key shares is skipped), digits of up to 12
+//             bits, each pass a shared-memory histogram over the keys that still match
+//             the prefix and a block-wide scan from the top bin;
 //   compact:  keys above the threshold plus the lowest-index ties, written in index
 //             order (per-warp ballots and a block prefix), so S is ascending;
 //   m, plan:  m = sum_S p~_j; for every j in S its tag, p~_j, the number of stores it
@@ -96,23 +97,56 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     return order_key(sc - offs[t]);
   };
   const int N4 = N & ~3;
+  uint32_t kand = 0xffffffffu, kor = 0u;  // bits common to every key
 #pragma unroll 4
   for (int j = 4 * tid; j < N4; j += 4 * kThreads) {
     const float4 sc = *reinterpret_cast<const float4*>(score + j);
     const uint32_t tg = *reinterpret_cast<const uint32_t*>(tag + j);
-    keys[j] = key_of(sc.x, (int)(tg & 0xff), j);
-    keys[j + 1] = key_of(sc.y, (int)((tg >> 8) & 0xff), j + 1);
-    keys[j + 2] = key_of(sc.z, (int)((tg >> 16) & 0xff), j + 2);
-    keys[j + 3] = key_of(sc.w, (int)(tg >> 24), j + 3);
+    const uint32_t k0 = key_of(sc.x, (int)(tg & 0xff), j), k1 = key_of(sc.y, (int)((tg >> 8) & 0xff), j + 1);
+    const uint32_t k2 = key_of(sc.z, (int)((tg >> 16) & 0xff), j + 2), k3 = key_of(sc.w, (int)(tg >> 24), j + 3);
+    keys[j] = k0;
+    keys[j + 1] = k1;
+    keys[j + 2] = k2;
+    keys[j + 3] = k3;
+    kand &= k0 & k1 & k2 & k3;
+    kor |= k0 | k1 | k2 | k3;
   }
-  for (int j = N4 + tid; j < N; j += kThreads) keys[j] = key_of(score[j], tag[j], j);
+  for (int j = N4 + tid; j < N; j += kThreads) {
+    const uint32_t k = key_of(score[j], tag[j], j);
+    keys[j] = k;
+    kand &= k;
+    kor |= k;
+  }
+  kand = __reduce_and_sync(kFull, kand);
+  kor = __reduce_or_sync(kFull, kor);
+  if (lane == 0) {
+    hist[warp] = kand;
+    hist[32 + warp] = kor;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    kand = __reduce_and_sync(kFull, hist[lane]);
+    kor = __reduce_or_sync(kFull, hist[32 + lane]);
+    if (lane == 0) {
+      hist[64] = kand;
+      hist[65] = kor;
+    }
+  }
+  __syncthreads();
+  kand = hist[64];
+  kor = hist[65];
   __syncthreads();
 
-  // ---- radix select of the K-th largest key ----
-  uint32_t prefix = 0u, pmask = 0u, krem = (uint32_t)K;
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
-    const int nbins = pass < 2 ? 4096 : 256;
+  // ---- radix select of the K-th largest key, over the bits where keys differ ----
+  const uint32_t diff = kand ^ kor;
+  int nbits = diff ? 32 - __clz(diff) : 0;  // digits cover bits [0, nbits)
+  uint32_t pmask = nbits >= 32 ? 0u : ~((1u << nbits) - 1u);
+  uint32_t prefix = kand & pmask, krem = (uint32_t)K;
+  while (nbits > 0) {
+    const int wbits = nbits < 12 ? nbits : 12;
+    const int shift = nbits - wbits;
+    nbits = shift;
+    const int nbins = 1 << wbits;
     const uint32_t dmask = (uint32_t)nbins - 1u;
     for (int i = tid; i < nbins; i += kThreads) hist[i] = 0u;
     __syncthreads();
