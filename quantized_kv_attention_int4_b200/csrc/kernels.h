@@ -44,6 +44,7 @@ cudaError_t launch_encode_residual(const EncodeResArgs& a, cudaStream_t s);
 cudaError_t launch_dense(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_dense_direct(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s);
+cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s);
 
 int dense_splits(int heads, int n_q);

@@ -603,7 +603,7 @@ int sparse_splits(int heads, int k_sel, int loops) {
   return s;
 }
 
-cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s) {
+cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s) {
   a.n_splits = sparse_splits(a.c.H, a.k_sel, a.c.R);
   const size_t smem = sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(sparse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
