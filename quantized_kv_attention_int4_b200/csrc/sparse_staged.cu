@@ -59,7 +59,6 @@ struct alignas(16) WarpCtlS {
   float2 wrow[kMaxRows][2];        // span being consumed: per row and half (wS, wU)
   float lr[kMaxRows];              // span being consumed: per-row logit parts
   float rec_c[kMaxRecs];           // span being consumed: record constants
-  int32_t row_g[kMaxRows];         // span being issued: group record of each row
   int32_t rec_g[kMaxRecs];         // span being issued: group record of each key record
   uint8_t rec_s[kMaxRecs];         // span being issued: store of each key record
 };
@@ -270,7 +269,13 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
           hd.row_rec[ri] = (uint8_t)ki;
           hd.row_pin[ri] = (uint8_t)pin;
           hd.row_store[ri] = (uint8_t)s;
-          wc.row_g[ri] = g;
+          // the row (8 pieces) and its value (scale, zero) pair, issued by the column's lane
+          const uint8_t* base = (s == 1 ? brec : rrec) + (size_t)g * kRec;
+          const uint8_t* src = base + pin * 128;
+          uint8_t* dst = rows + ri * 128;
+#pragma unroll
+          for (int pc = 0; pc < 8; ++pc) cp_async16(dst + pc * 16, src + pc * 16);
+          cp_async8(szs + ri * 8, base + kRecVsz + pin * 8);
           if (isnew) {
             wc.rec_g[ki] = g;
             wc.rec_s[ki] = (uint8_t)s;
@@ -280,17 +285,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
         recbase += __popc(nb);
       }
       __syncwarp();
-      // the span's copies, spread over the lanes: 8 pieces per row, one value (scale,
-      // zero) chunk per row, 32 pieces per record
-      for (int t = lane; t < nrows * 8; t += 32) {
-        const int ri = t >> 3, pc = t & 7;
-        const uint8_t* base = (hd.row_store[ri] == 1 ? brec : rrec) + (size_t)wc.row_g[ri] * kRec;
-        cp_async16(rows + ri * 128 + pc * 16, base + hd.row_pin[ri] * 128 + pc * 16);
-      }
-      for (int t = lane; t < nrows; t += 32) {
-        const uint8_t* base = (hd.row_store[t] == 1 ? brec : rrec) + (size_t)wc.row_g[t] * kRec;
-        cp_async8(szs + t * 8, base + kRecVsz + hd.row_pin[t] * 8);
-      }
+      // key records: 32 pieces each, spread over the lanes
       for (int k = 0; k < nrecs; ++k) {
         const uint8_t* base = (wc.rec_s[k] == 1 ? brec : rrec) + (size_t)wc.rec_g[k] * kRec;
         cp_async16(recs + k * 512 + lane * 16, base + kRecKsz + lane * 16);
