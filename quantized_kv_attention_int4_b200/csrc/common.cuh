@@ -306,6 +306,11 @@ __device__ __forceinline__ void axpy8_h(uint32_t w, unsigned short we, unsigned 
   hfma_f32(acc[7], (unsigned short)(d >> 16), wo);
 }
 
+// 2^e as an fp32 value, for -126 <= e <= 127 (built from the exponent field).
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+// The exponent e of x > 0 written as f * 2^e with f in [0.5, 1); subnormal x gives -126.
+__device__ __forceinline__ int exp_frexp(float x) { return (int)((__float_as_uint(x) >> 23) & 0xffu) - 126; }
+
 // ---- exact integer key dots (dp4a) against fixed-point query weights ----
 // A key group's weights qs_c = q_c * s_c become Q_c = rint(qs_c * 2^E) with
 // |Q_c| < 2^23 (24-bit fixed point, E per record from the largest |qs_c|), split into
@@ -329,12 +334,8 @@ __device__ __forceinline__ void record_to_limbs(uint32_t* rec, const float* q_s,
   mx = warp_max(mx);
   cz = warp_sum(cz);
   int E = 0;
-  if (mx > 0.f) {
-    int e2;
-    frexpf(mx, &e2);  // mx = f * 2^e2, f in [0.5, 1)
-    E = min(23 - e2, 126);
-  }
-  const float sc = ldexpf(1.0f, E);
+  if (mx > 0.f) E = min(23 - exp_frexp(mx), 126);
+  const float sc = pow2i(E);
   auto fix = [&](float v) {
     const int x = __float2int_rn(v * sc);
     return x > 8388607 ? 8388607 : (x < -8388607 ? -8388607 : x);

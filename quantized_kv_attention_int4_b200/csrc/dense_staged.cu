@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         const uint32_t* lim = reinterpret_cast<const uint32_t*>(sp + kRecKsz);
         uint32_t lw[24];
         load_limbs(lim, qq, lw);
-        const float sc = ldexpf(1.f, -(int)lim[kLimbE]);
+        const float sc = pow2i(-(int)lim[kLimbE]);
         const float C = __uint_as_float(lim[kLimbC]);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
           uint32_t lw[24];
           load_limbs(lim, qq, lw);
           const uint4 code = *reinterpret_cast<const uint4*>(sp + G.off_codes + ii * 128 + 16 * qq);
-          float v = limb_dot(code, lw) * ldexpf(1.f, -(int)lim[kLimbE]);
+          float v = limb_dot(code, lw) * pow2i(-(int)lim[kLimbE]);
           v += __shfl_xor_sync(kFull, v, 1);
           v += __shfl_xor_sync(kFull, v, 2);
           if (act && qq == 0) w.lg[w.tok[s][i]] += v + __uint_as_float(lim[kLimbC]);
@@ -448,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       z0 = warp_sum(z0);
       z1 = warp_sum(z1);
       int E0 = 0, E1 = 0;
-      if (mx0 > 0.f) { int e; frexpf(mx0, &e); E0 = min(24 - e, 126); }
-      if (mx1 > 0.f) { int e; frexpf(mx1, &e); E1 = min(24 - e, 126); }
-      const float sc0 = ldexpf(1.f, E0), sc1 = ldexpf(1.f, E1);
+      if (mx0 > 0.f) E0 = min(24 - exp_frexp(mx0), 126);
+      if (mx1 > 0.f) E1 = min(24 - exp_frexp(mx1), 126);
+      const float sc0 = pow2i(E0), sc1 = pow2i(E1);
 #pragma unroll
       for (int i = 0; i < 6; ++i) {
         if (32 * i >= nvr) break;
@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
                   w.wl[kb + kg][hv], a0, a1, a2);
         }
       }
-      const float isc = ldexpf(1.f, -(hv ? E1 : E0));
+      const float isc = pow2i(-(hv ? E1 : E0));
       const float zh = gv == 0 ? (hv ? z1 : z0) : 0.f;
       float val[8];
 #pragma unroll

@@ -22,9 +22,9 @@
 // group per span, and a warp keeps up to kSlots spans in flight in its ring of shared
 // memory (cp.async.wait_group parks the warp in hardware until its span has landed).
 // Per span:
-//   records -> pre-scaled fp32 query weights (in place);
-//   keys    -> one logit part per row (8 rows per pass, a lane per row quarter), then
-//              each column sums its parts in store order;
+//   records -> 24-bit fixed-point query weights q_c s_c 2^E in byte limbs (in place);
+//   keys    -> one logit part per row (8 rows per pass, a lane per row quarter, exact
+//              dp4a dots), then each column sums its parts in store order;
 //   softmax -> online, base-2, over the warp's columns; score and tag are spliced;
 //   values  -> per-row weights 128 p s_h and 128 p~ s_h (the latter for rows within
 //              the column's tag-loop prefix) accumulate two fp32 sums.
@@ -58,7 +58,6 @@ struct alignas(16) WarpCtlS {
   int32_t slot_off[kSlotsS];
   float2 wrow[kMaxRows][2];        // span being consumed: per row and half (wS, wU)
   float lr[kMaxRows];              // span being consumed: per-row logit parts
-  float rec_c[kMaxRecs];           // span being consumed: record constants
   int32_t rec_g[kMaxRecs];         // span being issued: group record of each key record
   uint8_t rec_s[kMaxRecs];         // span being issued: store of each key record
 };
@@ -307,28 +306,25 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
     const uint8_t* szs = rows + nrows * 128;
     uint8_t* recs = sp + kHdrS + nrows * 128 + ((nrows * 8 + 15) & ~15);
 
-    // records -> pre-scaled fp32 query weights, in place
-#pragma unroll 2
-    for (int k = 0; k < nrecs; ++k) {
-      const float cst = group_weights_smem(reinterpret_cast<uint32_t*>(recs + k * 512), ch.q, lane);
-      if (lane == 0) wc.rec_c[k] = cst;
-    }
+    // records -> 24-bit fixed-point query weights in byte limbs, in place
+    for (int k = 0; k < nrecs; ++k) record_to_limbs(reinterpret_cast<uint32_t*>(recs + k * 512), ch.q, lane);
     __syncwarp();
-    // one logit part per row
+    // one logit part per row: exact dp4a dot of the row quarter with its record's limbs
 #pragma unroll 2
     for (int p0 = 0; p0 < nrows; p0 += 8) {
       const int row = p0 + tr;
       const bool act = row < nrows;
       const int rid = act ? hd.row_rec[row] : 0;
+      const uint32_t* lim = reinterpret_cast<const uint32_t*>(recs + rid * 512);
       float d = 0.f;
       if (act) {
-        float qsr[32];
-        load32(reinterpret_cast<const float*>(recs + rid * 512) + 32 * qq, qsr);
-        d = dot32(*reinterpret_cast<const uint4*>(rows + row * 128 + 16 * qq), qsr);
+        uint32_t lw[24];
+        load_limbs(lim, qq, lw);
+        d = limb_dot(*reinterpret_cast<const uint4*>(rows + row * 128 + 16 * qq), lw) * pow2i(-(int)lim[kLimbE]);
       }
       d += __shfl_xor_sync(kFull, d, 1);
       d += __shfl_xor_sync(kFull, d, 2);
-      if (act && qq == 0) wc.lr[row] = d + wc.rec_c[rid];
+      if (act && qq == 0) wc.lr[row] = d + __uint_as_float(lim[kLimbC]);
     }
     __syncwarp();
     // columns: sum the parts in store order, online softmax, splice score and tag
