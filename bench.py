@@ -504,7 +504,7 @@ def main():
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": {**config, "context_at_end": r["N"],
                                                                           "k_sel": r["k_sel"]},
         "roofline": {"bound": "hbm", "kernel": "fl_decode_attn_sparse (loop 4)", "achieved": r["sp_gbs"],
-                     "peak": hbm, "unit": "GB/s", "frac": r["sp_gbs"] / hbm, "traffic": _kernel_traffic("sparse_kernel"),
+                     "peak": hbm, "unit": "GB/s", "frac": r["sp_gbs"] / hbm, "traffic": _kernel_traffic("sparse_staged_kernel"),
                      "peak_kind": peak_kind_str(r["peak_kind"]), "bytes_per_launch": r["sp_bytes"],
                      "us_per_launch": r["sp_launch_us"]},
         "roofline_dense": {"bound": "hbm", "kernel": "fl_decode_attn_dense (loops 1-2)", "achieved": r["d_gbs"],
