@@ -187,30 +187,29 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int chunk = ((((N + kWarpsSel - 1) / kWarpsSel) + 31) / 32) * 32;
   const int wbeg = warp * chunk;
   const unsigned lt = (1u << lane) - 1u;
-  uint32_t eqc = 0u;
-  for (int i = 0; i < chunk; i += 32) {
-    const int j = wbeg + i + lane;
-    eqc += __popc(__ballot_sync(kFull, j < N && keys[j] == thr));
-  }
-  if (lane == 0) wtot[warp] = eqc;
-  __syncthreads();
-  uint32_t eq_base = 0u;
-  for (int w = 0; w < warp; ++w) eq_base += wtot[w];
-  __syncthreads();
-  uint32_t selc = 0u, eqrun = eq_base;
+  // one pass counts this warp's keys above the threshold and equal to it; the number it
+  // selects follows from the equal keys of the warps before it (lowest indices first)
+  uint32_t gtc = 0u, eqc = 0u;
   for (int i = 0; i < chunk; i += 32) {
     const int j = wbeg + i + lane;
     const uint32_t u = j < N ? keys[j] : 0u;
-    const unsigned be = __ballot_sync(kFull, j < N && u == thr);
-    const bool s = (j < N && u > thr) || (j < N && u == thr && eqrun + __popc(be & lt) < krem);
-    eqrun += __popc(be);
-    selc += __popc(__ballot_sync(kFull, s));
+    gtc += __popc(__ballot_sync(kFull, j < N && u > thr));
+    eqc += __popc(__ballot_sync(kFull, j < N && u == thr));
   }
-  if (lane == 0) wtot[warp] = selc;
+  if (lane == 0) {
+    wtot[warp] = eqc;
+    hist[warp] = gtc;  // the histogram is no longer needed
+  }
   __syncthreads();
-  uint32_t pos = 0u;
-  for (int w = 0; w < warp; ++w) pos += wtot[w];
-  eqrun = eq_base;
+  uint32_t eq_base = 0u, pos = 0u;
+  for (int w = 0; w < warp; ++w) {
+    const uint32_t eb = eq_base;
+    eq_base += wtot[w];
+    const uint32_t take = krem > eb ? min(krem - eb, wtot[w]) : 0u;
+    pos += hist[w] + take;
+  }
+  __syncthreads();
+  uint32_t eqrun = eq_base;
   float mpart = 0.f;
   for (int i = 0; i < chunk; i += 32) {
     const int j = wbeg + i + lane;

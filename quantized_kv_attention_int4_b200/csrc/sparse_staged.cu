@@ -177,7 +177,9 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
   float accS[8], accU[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) accS[k] = accU[k] = 0.f;
-  float corrS = 0.f, corrU = 0.f;
+  // per-lane parts of the per-half constants of the S and U sums (summed over the warp
+  // once, at the end); Ls and msum are per-lane parts too
+  float kS0 = 0.f, kS1 = 0.f, kU0 = 0.f, kU1 = 0.f;
   const int w16 = lane & 15, par16 = lane >> 4, half = w16 >> 3;
 
   // record of column lane's row in store s (base block or residual group record)
@@ -342,19 +344,19 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
     const float Mn = fmaxf(M, mb);
     const float al = Mn == -INFINITY ? 1.f : ex2(M - Mn);
     const float p = in ? ex2(l - Mn) : 0.f;
-    Ls = Ls * al + warp_sum(p);
-    msum += warp_sum(in ? pt_c : 0.f);
+    Ls = Ls * al + p;
+    msum += in ? pt_c : 0.f;
     M = Mn;
 #pragma unroll
     for (int k = 0; k < 8; ++k) accS[k] *= al;
-    corrS *= al;
+    kS0 *= al;
+    kS1 *= al;
     if (in) {
       score[j_c] = l;
       tag[j_c] = (uint8_t)r;
     }
     // per-row value weights, lanes = rows
     {
-      float cS0 = 0.f, cS1 = 0.f, cU0 = 0.f, cU1 = 0.f;
       for (int row0 = 0; row0 < nrows; row0 += 32) {
         const int row = row0 + lane;
         const bool act = row < nrows;
@@ -370,19 +372,11 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
           const float wU0 = 128.f * (pu * z0.x), wU1 = 128.f * (pu * z1.x);
           wc.wrow[row][0] = make_float2(wS0, wU0);
           wc.wrow[row][1] = make_float2(wS1, wU1);
-          cS0 += fmaf(pc, z0.y, -wS0);
-          cS1 += fmaf(pc, z1.y, -wS1);
-          cU0 += fmaf(pu, z0.y, -wU0);
-          cU1 += fmaf(pu, z1.y, -wU1);
+          kS0 += fmaf(pc, z0.y, -wS0);
+          kS1 += fmaf(pc, z1.y, -wS1);
+          kU0 += fmaf(pu, z0.y, -wU0);
+          kU1 += fmaf(pu, z1.y, -wU1);
         }
-      }
-      cS0 = warp_sum(cS0);
-      cS1 = warp_sum(cS1);
-      cU0 = warp_sum(cU0);
-      cU1 = warp_sum(cU1);
-      if (par16 == 0) {
-        corrS += half ? cS1 : cS0;
-        corrU += half ? cU1 : cU0;
       }
     }
     __syncwarp();
@@ -434,12 +428,13 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
     const float al = Mn == -INFINITY ? 1.f : ex2(M - Mn);
     const float p = in ? ex2(l - Mn) : 0.f;
     const float pt = in ? __int_as_float(e[2]) : 0.f;
-    Ls = Ls * al + warp_sum(qq == 0 ? p : 0.f);
-    msum += warp_sum(qq == 0 ? pt : 0.f);
+    Ls = Ls * al + (qq == 0 ? p : 0.f);
+    msum += qq == 0 ? pt : 0.f;
     M = Mn;
 #pragma unroll
     for (int k = 0; k < 8; ++k) accS[k] *= al;
-    corrS *= al;
+    kS0 *= al;
+    kS1 *= al;
     if (in && qq == 0) {
       score[j] = l;
       tag[j] = (uint8_t)r;
@@ -469,6 +464,15 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
   }
 
   // ---- merge the warps: lane (w16, parity) holds channels 8*w16..8*w16+7 ----
+  Ls = warp_sum(Ls);
+  msum = warp_sum(msum);
+  kS0 = warp_sum(kS0);
+  kS1 = warp_sum(kS1);
+  kU0 = warp_sum(kU0);
+  kU1 = warp_sum(kU1);
+  // one lane of each (word, parity) pair carries the constants
+  const float corrS = par16 == 0 ? (half ? kS1 : kS0) : 0.f;
+  const float corrU = par16 == 0 ? (half ? kU1 : kU0) : 0.f;
   float outS[8], outU[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
