@@ -6,58 +6,63 @@
 // (Step 03), or the loop's BF16 tail row (flashloop 0.1.0 PyPI description,
 // "Configuration and supported scope": 64-token BF16 tail).
 //
-// Grid: one persistent CTA per SM, kWS warps each.  The units of all heads (each
-// head's 64-token blocks, then its tail unit) are numbered head-major and cut into one
-// contiguous range per CTA (at most two heads per range); warp w takes units w,
-// w + kWS, ... of its CTA's range and owns a ring of shared memory.  Ahead of use it
-// stages into the ring, for each block, one span:
+// Grid: one persistent CTA per SM of kPairs teams of two warps.  The units of all heads
+// (each head's 64-token blocks, then its tail unit) are numbered head-major and cut into
+// one contiguous range per CTA (at most two heads per range); team p takes units p,
+// p + kPairs, ... of its CTA's range and owns a ring of shared memory.  Its first warp
+// stages into the ring, ahead of use, for each block, one span:
 //   [0, 9216)   the block's base group record (one bulk copy);
 //   per residual store s of loops 2..r, if the block has rows there: the rows' code
 //               lines (128 B each, from one or two group records), then per group record
 //               its key (scale, zero) record (512 B) and the value (scale, zero) words of
 //               the rows (rounded out to an even slot so the copy is 16-byte aligned).
-// The copies of one span complete on one mbarrier (kSlots per warp, round robin).
+// The copies of one span complete on one mbarrier (kSlots per team, round robin).  The
+// two warps of a team share each block (named barrier per team): warp h takes key rows
+// 32h..32h+31 and alternate passes of residual rows, and the values of channel half h.
 //
 // Per block, all on the staged bytes:
 //   keys    every key (scale, zero) record becomes 24-bit fixed-point query weights
 //           Q_c = rint(q_c s_c 2^E) split into byte limbs; a code row is dotted with
 //           them by dp4a (exact integer sums), then scaled by 2^-E, plus sum_c q_c z_c;
-//           residual rows add their dot to the logit of their token;
-//   softmax p'_t = 2^(l_t - m_b) with m_b the block maximum; the warp's running (M, L)
-//           and output are rescaled once per block;
-//   values  row weights W = p' s_h per 64-channel half h become 24-bit fixed point
+//           each residual row's part is added to the logit of its token in store order;
+//   softmax p'_t = 2^(l_t - m_b) with m_b the block maximum (both warps, identically);
+//           the running (M, L) and output are rescaled once per block;
+//   values  row weights W = p' s_h of the warp's half h become 24-bit fixed point
 //           numbers (E_h from the block's largest weight); the code words of four rows are
 //           transposed by byte permutes into per-channel nibble quadruples and dotted
 //           by dp4a with the four rows' weight limbs; plus Z_h = sum_t p'_t z_t,h.
 // The tail unit reads its BF16 rows from global memory in fp32.
-// Warps' partials merge per CTA; the last CTA of each head (atomic ticket) combines the
+// Teams' partials merge per CTA; the last CTA of each head (atomic ticket) combines the
 // CTA partials by log-sum-exp and writes o and offset[r] = M + log2 L.
 #include "kernels.h"
 
 namespace fl {
 namespace {
 
-constexpr int kWS = 7;                           // warps per CTA
-constexpr int kThreads = kWS * 32;
-constexpr int kSlots = 4;                        // staged blocks in flight per warp
+constexpr int kPairs = 7;                        // teams of two warps per CTA
+constexpr int kThreads = kPairs * 64;
+constexpr int kSlots = 4;                        // staged blocks in flight per team
 constexpr int kStores = 2;                       // residual stores staged (loops 2, 3)
 constexpr int kMaxGroups = 16 + kStores * 16;    // 4-row weight groups of one block
 constexpr int kSmemTotal = 232448;               // opt-in shared memory per CTA
 constexpr int kHdr = 64 + 2 * kD * 4;            // flags + the CTA's two queries
 
-struct alignas(16) WarpCtl {
+struct alignas(16) TeamCtl {
   uint64_t bar[kSlots];
   int32_t slot_off[kSlots];
   int32_t slot_gs0[kSlots][kStores];
   unsigned long long slot_mk[kSlots][kStores];
-  float lg[kG];                  // logits of the block, then p'
+  float lg[kG];                  // base logits of the block (tail unit: its logits)
+  float rl[kStores][kG];         // residual logit part of each residual row
+  float pw[kG];                  // tail unit: p'
   uint8_t tok[kStores][kG];      // token of each residual row
   uint4 wl[kMaxGroups][2];       // weight limbs (bytes 0, 1, 2 of four rows) per group, half
-  float part0[2 + kD];           // (M, L, o) of the warp's first head
+  float part0[2 + kD];           // (M, L, o) of the team's first head
   int32_t has[2];
+  int32_t ok[2];                 // each warp's staged-block wait succeeded
 };
 
-constexpr int kRing = ((kSmemTotal - kHdr - kWS * (int)sizeof(WarpCtl)) / kWS) & ~15;
+constexpr int kRing = ((kSmemTotal - kHdr - kPairs * (int)sizeof(TeamCtl)) / kPairs) & ~15;
 // largest span: base record + 2 stores x (64 code rows + 2 key records + 66 value words)
 constexpr int kMaxSpan = kRec + kStores * (kG * 128 + 2 * 512 + (kG + 2) * 8);
 static_assert(kRing >= kMaxSpan, "ring must hold the largest span");
@@ -162,17 +167,23 @@ __device__ __forceinline__ uint32_t fix24(float w, float sc) {
   return q > 16777215u ? 16777215u : q;
 }
 
+__device__ __forceinline__ void pair_sync(int pair) {
+  asm volatile("bar.sync %0, 64;" ::"r"(pair + 1) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a, int n_cta) {
   extern __shared__ __align__(128) uint8_t smem[];
   int* last = reinterpret_cast<int*>(smem);
   float* q_all = reinterpret_cast<float*>(smem + 64);
-  WarpCtl* ctl = reinterpret_cast<WarpCtl*>(smem + kHdr);
-  uint8_t* rings = smem + kHdr + kWS * sizeof(WarpCtl);
+  TeamCtl* ctl = reinterpret_cast<TeamCtl*>(smem + kHdr);
+  uint8_t* rings = smem + kHdr + kPairs * sizeof(TeamCtl);
 
   const CacheView& c = a.c;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int qq = lane & 3, tr = lane >> 2;        // key mapping: row tr of 8, quarter qq
-  const int wv = lane & 15, gv = lane >> 4, hv = wv >> 3;  // value mapping: word, row parity
+  const int pair = warp >> 1, hw = warp & 1;          // team and this warp's value half
+  const int qq = lane & 3, tr = lane >> 2;             // key mapping: row tr of 8, quarter qq
+  const int w8 = lane & 7, g4 = lane >> 3;             // value mapping: word of the half, row group mod 4
+  const int wv = 8 * hw + w8;                          // code word (channels 8 wv .. 8 wv + 7)
   const int H = c.H, cap = c.cap, ncb = cap / kG, T = c.total_slots, r = a.r;
   const int nb = a.n_q / kG, nbp = nb + 1;
   const long long U = (long long)H * nbp;
@@ -186,9 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
     const int hh = h0 + i / kD;
     q_all[i] = hh <= h1 ? __uint_as_float((uint32_t)a.q[(size_t)hh * kD + (i % kD)] << 16) * kQScale : 0.f;
   }
-  WarpCtl& w = ctl[warp];
-  uint8_t* ring = rings + (size_t)warp * kRing;
-  if (lane == 0) {
+  TeamCtl& w = ctl[pair];
+  uint8_t* ring = rings + (size_t)pair * kRing;
+  if (tid == 64 * pair) {
     for (int i = 0; i < kSlots; ++i) mbar_init(&w.bar[i], 1);
     fence_mbar_init();
     w.has[0] = w.has[1] = 0;
@@ -199,16 +210,17 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
   const int32_t* first = arr<int32_t>(c, A_FIRST, a.layer);
   const uint8_t* brec_l = arr<uint8_t>(c, A_BREC, a.layer);
   const uint8_t* rrec_l = arr<uint8_t>(c, A_RREC, a.layer);
-  const int n_my = U1 - U0 > warp ? (U1 - U0 - warp + kWS - 1) / kWS : 0;
+  const int n_my = U1 - U0 > pair ? (U1 - U0 - pair + kPairs - 1) / kPairs : 0;
   const bool has_new = a.k_new != nullptr;
 
-  // metadata window: lane (k_off = lane >> 1, s = lane & 1) holds store 2+s of unit iss_k + k_off
+  // metadata window (producer warp): lane (k_off = lane >> 1, s = lane & 1) holds store 2+s
+  // of unit iss_k + k_off
   const int ms = lane & 1;
   auto load_meta = [&](int k, unsigned long long& mk, int& g0) {
     mk = 0ull;
     g0 = 0;
     if (k < n_my && ms < nst) {
-      const int u = U0 + warp + k * kWS, b = u % nbp;
+      const int u = U0 + pair + k * kPairs, b = u % nbp;
       if (b < nb) {
         const int rp = 2 + ms;
         mk = __ldg(mask + (size_t)rp * ncb + b);
@@ -216,9 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       }
     }
   };
-  unsigned long long m_mk;
-  int m_gs;
-  load_meta(lane >> 1, m_mk, m_gs);
+  unsigned long long m_mk = 0ull;
+  int m_gs = 0;
+  if (hw == 0) load_meta(lane >> 1, m_mk, m_gs);
 
   int iss_k = 0, iss_seq = 0, con_seq = 0, wpos = 0;
   bool failed = false;
@@ -227,17 +239,21 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
   float M = -INFINITY, Ls = 0.f;
   int cur_hs = -1;
 
+  // write this warp's half of the team's (M, L, o) for head slot hs
   auto flush = [&](int hs) {
     float* dst = hs == 0 ? w.part0 : reinterpret_cast<float*>(ring);
     float o8[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) o8[k] = acc[k] + __shfl_xor_sync(kFull, acc[k], 16);
+    for (int k = 0; k < 8; ++k) {
+      o8[k] = acc[k] + __shfl_xor_sync(kFull, acc[k], 8);
+      o8[k] += __shfl_xor_sync(kFull, o8[k], 16);
+    }
     const float Lw = warp_sum(Ls);
-    if (gv == 0) {
+    if (g4 == 0) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) dst[2 + 8 * wv + k] = o8[k];
     }
-    if (lane == 0) {
+    if (hw == 0 && lane == 0) {
       dst[0] = M;
       dst[1] = Lw;
       w.has[hs] = 1;
@@ -254,60 +270,62 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
   };
 
   for (int k = 0; k < n_my; ++k) {
-    // ---- stage ahead: issue spans while a slot and ring space are free ----
-    while (!failed && iss_k < n_my) {
-      const int u = U0 + warp + iss_k * kWS, b = u % nbp;
-      if (b < nb) {
-        if (iss_seq - con_seq >= kSlots) break;
-        unsigned long long mk2[kStores];
-        int gs[kStores];
-        mk2[0] = __shfl_sync(kFull, m_mk, 0);
-        mk2[1] = __shfl_sync(kFull, m_mk, 1);
-        gs[0] = __shfl_sync(kFull, m_gs, 0);
-        gs[1] = __shfl_sync(kFull, m_gs, 1);
-        StoreGeom g[kStores];
-        int pos = store_geom(mk2[0], gs[0], kRec, g[0]);
-        pos = store_geom(mk2[1], gs[1], pos, g[1]);
-        int start = -1;
-        if (iss_seq == con_seq) {
-          start = 0;
-        } else {
-          const int rp = w.slot_off[con_seq % kSlots];
-          if (wpos > rp) {
-            if (wpos + pos <= kRing) start = wpos;
-            else if (pos <= rp) start = 0;
-          } else if (wpos + pos <= rp) {
-            start = wpos;
+    pair_sync(pair);  // both warps are done with the previous unit: its span may be reused
+    // ---- producer warp: issue spans while a slot and ring space are free ----
+    if (hw == 0) {
+      while (iss_k < n_my) {
+        const int u = U0 + pair + iss_k * kPairs, b = u % nbp;
+        if (b < nb) {
+          if (iss_seq - con_seq >= kSlots) break;
+          unsigned long long mk2[kStores];
+          int gs[kStores];
+          mk2[0] = __shfl_sync(kFull, m_mk, 0);
+          mk2[1] = __shfl_sync(kFull, m_mk, 1);
+          gs[0] = __shfl_sync(kFull, m_gs, 0);
+          gs[1] = __shfl_sync(kFull, m_gs, 1);
+          StoreGeom g[kStores];
+          int pos = store_geom(mk2[0], gs[0], kRec, g[0]);
+          pos = store_geom(mk2[1], gs[1], pos, g[1]);
+          int start = -1;
+          if (iss_seq == con_seq) {
+            start = 0;
+          } else {
+            const int rp = w.slot_off[con_seq % kSlots];
+            if (wpos > rp) {
+              if (wpos + pos <= kRing) start = wpos;
+              else if (pos <= rp) start = 0;
+            } else if (wpos + pos <= rp) {
+              start = wpos;
+            }
           }
+          if (start < 0) break;
+          wpos = start + pos;
+          const int slot = iss_seq % kSlots;
+          __syncwarp();
+          if (lane == 0) {
+            w.slot_off[slot] = start;
+            w.slot_mk[slot][0] = mk2[0];
+            w.slot_mk[slot][1] = mk2[1];
+            w.slot_gs0[slot][0] = gs[0];
+            w.slot_gs0[slot][1] = gs[1];
+            const int h = u / nbp;
+            issue_span(ring + start, brec_l + ((size_t)h * ncb + b) * kRec,
+                       rrec_l + (size_t)h * (T / kG) * kRec, g, gs, pos, &w.bar[slot]);
+          }
+          ++iss_seq;
         }
-        if (start < 0) break;
-        wpos = start + pos;
-        const int slot = iss_seq % kSlots;
-        __syncwarp();
-        if (lane == 0) {
-          w.slot_off[slot] = start;
-          w.slot_mk[slot][0] = mk2[0];
-          w.slot_mk[slot][1] = mk2[1];
-          w.slot_gs0[slot][0] = gs[0];
-          w.slot_gs0[slot][1] = gs[1];
-          const int h = u / nbp;
-          issue_span(ring + start, brec_l + ((size_t)h * ncb + b) * kRec,
-                     rrec_l + (size_t)h * (T / kG) * kRec, g, gs, pos, &w.bar[slot]);
-        }
-        ++iss_seq;
+        ++iss_k;
+        // slide the metadata window by one unit
+        const unsigned lo_m = __shfl_down_sync(kFull, (unsigned)m_mk, 2);
+        const unsigned hi_m = __shfl_down_sync(kFull, (unsigned)(m_mk >> 32), 2);
+        m_gs = __shfl_down_sync(kFull, m_gs, 2);
+        m_mk = ((unsigned long long)hi_m << 32) | lo_m;
+        if (lane >= 30) load_meta(iss_k + 15, m_mk, m_gs);
       }
-      ++iss_k;
-      // slide the metadata window by one unit
-      const unsigned lo_m = __shfl_down_sync(kFull, (unsigned)m_mk, 2);
-      const unsigned hi_m = __shfl_down_sync(kFull, (unsigned)(m_mk >> 32), 2);
-      m_gs = __shfl_down_sync(kFull, m_gs, 2);
-      m_mk = ((unsigned long long)hi_m << 32) | lo_m;
-      if (lane >= 30) load_meta(iss_k + 15, m_mk, m_gs);
+      __syncwarp();
     }
-    __syncwarp();
-    if (failed) break;
 
-    const int u = U0 + warp + k * kWS, h = u / nbp, b = u % nbp, hs = h - h0;
+    const int u = U0 + pair + k * kPairs, h = u / nbp, b = u % nbp, hs = h - h0;
     if (hs != cur_hs) {
       if (cur_hs >= 0) flush(cur_hs);
       cur_hs = hs;
@@ -323,12 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
     if (b < nb) {
       // ================= staged block =================
       const int slot = con_seq % kSlots;
-      const bool ok = __any_sync(kFull, mbar_wait(&w.bar[slot], (unsigned)(con_seq / kSlots) & 1u));
-      if (!ok) {
-        if (lane == 0) record_error(c.status, FL_DEV_TIMEOUT, b);
-        failed = true;
-        break;
-      }
+      const bool okw = __any_sync(kFull, mbar_wait(&w.bar[slot], (unsigned)(con_seq / kSlots) & 1u));
+      if (lane == 0) w.ok[hw] = okw ? 1 : 0;
       uint8_t* sp = ring + w.slot_off[slot];
       StoreGeom g[kStores];
       const unsigned long long mkA = w.slot_mk[slot][0], mkB = w.slot_mk[slot][1];
@@ -336,18 +350,31 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         const int pos = store_geom(mkA, w.slot_gs0[slot][0], kRec, g[0]);
         store_geom(mkB, w.slot_gs0[slot][1], pos, g[1]);
       }
-
-      // ---- key limbs of the base record and of every residual group record ----
-      record_to_limbs(reinterpret_cast<uint32_t*>(sp + kRecKsz), qh, lane);
+      // ---- key limbs (warp 0: the base record; warp 1: residual records and token maps) ----
+      if (hw == 0) {
+        record_to_limbs(reinterpret_cast<uint32_t*>(sp + kRecKsz), qh, lane);
+      } else {
 #pragma unroll
-      for (int s = 0; s < kStores; ++s) {
-        if (g[s].na == 0) continue;
-        record_to_limbs(reinterpret_cast<uint32_t*>(sp + g[s].off_k0), qh, lane);
-        if (g[s].n1 < g[s].na) record_to_limbs(reinterpret_cast<uint32_t*>(sp + g[s].off_k1), qh, lane);
+        for (int s = 0; s < kStores; ++s) {
+          if (g[s].na == 0) continue;
+          const unsigned long long mk = s == 0 ? mkA : mkB;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int tt = lane + 32 * e;
+            if ((mk >> tt) & 1ull) w.tok[s][__popcll(mk & ((1ull << tt) - 1ull))] = (uint8_t)tt;
+          }
+          record_to_limbs(reinterpret_cast<uint32_t*>(sp + g[s].off_k0), qh, lane);
+          if (g[s].n1 < g[s].na) record_to_limbs(reinterpret_cast<uint32_t*>(sp + g[s].off_k1), qh, lane);
+        }
       }
-      __syncwarp();
+      pair_sync(pair);
+      if (!(w.ok[0] && w.ok[1])) {
+        if (hw == 0 && lane == 0) record_error(c.status, FL_DEV_TIMEOUT, b);
+        failed = true;
+        break;
+      }
 
-      // ---- base logits ----
+      // ---- base logits: rows 32 hw .. 32 hw + 31 ----
       {
         const uint32_t* lim = reinterpret_cast<const uint32_t*>(sp + kRecKsz);
         uint32_t lw[24];
@@ -355,8 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         const float sc = pow2i(-(int)lim[kLimbE]);
         const float C = __uint_as_float(lim[kLimbC]);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int t = 8 * i + tr;
+        for (int i = 0; i < 4; ++i) {
+          const int t = 32 * hw + 8 * i + tr;
           const uint4 code = *reinterpret_cast<const uint4*>(sp + t * 128 + 16 * qq);
           float v = limb_dot(code, lw) * sc;
           v += __shfl_xor_sync(kFull, v, 1);
@@ -364,20 +391,12 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
           if (qq == 0) w.lg[t] = v + C;
         }
       }
-      // ---- residual logits, added to their tokens ----
+      // ---- residual logit parts, one per residual row (passes of 8 rows, alternating warps) ----
 #pragma unroll
       for (int s = 0; s < kStores; ++s) {
         const StoreGeom& G = g[s];
         if (G.na == 0) continue;
-        const unsigned long long mk = s == 0 ? mkA : mkB;
-        __syncwarp();
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tt = lane + 32 * e;
-          if ((mk >> tt) & 1ull) w.tok[s][__popcll(mk & ((1ull << tt) - 1ull))] = (uint8_t)tt;
-        }
-        __syncwarp();
-        for (int i0 = 0; i0 < G.na; i0 += 8) {
+        for (int i0 = 8 * hw; i0 < G.na; i0 += 16) {
           const int i = i0 + tr;
           const bool act = i < G.na;
           const int ii = act ? i : G.na - 1;
@@ -388,14 +407,21 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
           float v = limb_dot(code, lw) * pow2i(-(int)lim[kLimbE]);
           v += __shfl_xor_sync(kFull, v, 1);
           v += __shfl_xor_sync(kFull, v, 2);
-          if (act && qq == 0) w.lg[w.tok[s][i]] += v + __uint_as_float(lim[kLimbC]);
+          if (act && qq == 0) w.rl[s][i] = v + __uint_as_float(lim[kLimbC]);
         }
       }
-      __syncwarp();
+      pair_sync(pair);
 
-      // ---- block softmax ----
-      const float l0 = w.lg[lane], l1 = w.lg[lane + 32];
-      if (a.keep) {
+      // ---- block softmax (both warps, identically) ----
+      float l0 = w.lg[lane], l1 = w.lg[lane + 32];
+#pragma unroll
+      for (int s = 0; s < kStores; ++s) {
+        if (g[s].na == 0) continue;
+        const unsigned long long mk = s == 0 ? mkA : mkB;
+        if ((mk >> lane) & 1ull) l0 += w.rl[s][__popcll(mk & ((1ull << lane) - 1ull))];
+        if ((mk >> (lane + 32)) & 1ull) l1 += w.rl[s][__popcll(mk & ((1ull << (lane + 32)) - 1ull))];
+      }
+      if (a.keep && hw == 0) {
         score[(size_t)b * kG + lane] = l0;
         score[(size_t)b * kG + lane + 32] = l1;
         tag[(size_t)b * kG + lane] = (uint8_t)r;
@@ -403,91 +429,74 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       }
       const float mb = warp_max(fmaxf(l0, l1));
       const float p0 = ex2(l0 - mb), p1 = ex2(l1 - mb);
-      __syncwarp();
-      w.lg[lane] = p0;
-      w.lg[lane + 32] = p1;
-      __syncwarp();
 
-      // ---- value weights: W = p' s_h as 16-bit fixed point per half ----
+      // ---- value weights of this warp's half: W = p' s as 24-bit fixed point ----
       const int pad0 = (g[0].na + 3) & ~3, pad1 = (g[1].na + 3) & ~3;
       const int nvr = kG + pad0 + pad1;
-      float W0[6], W1[6];
-      float z0 = 0.f, z1 = 0.f, mx0 = 0.f, mx1 = 0.f;
+      float Wt[6];
+      float zs = 0.f, mx = 0.f;
 #pragma unroll
       for (int i = 0; i < 6; ++i) {
-        W0[i] = W1[i] = 0.f;
+        Wt[i] = 0.f;
         if (32 * i >= nvr) break;
         const int v = lane + 32 * i;
-        float p = 0.f;
-        uint2 sz = make_uint2(0u, 0u);
-        if (v < kG) {
-          p = w.lg[v];
-          sz = *reinterpret_cast<const uint2*>(sp + kRecVsz + v * 8);
-        } else if (v < nvr) {
+        int tok = v, off = kRecVsz + v * 8;  // base rows: token v, (scale, zero) in the base record
+        bool act = v < kG;
+        if (!act && v < nvr) {
           int vv = v - kG;
           const int s = vv >= pad0 ? 1 : 0;
           if (s) vv -= pad0;
           const int na = s ? g[1].na : g[0].na, n1 = s ? g[1].n1 : g[0].n1;
           if (vv < na) {
-            p = w.lg[w.tok[s][vv]];
-            const int off = vv < n1 ? (s ? g[1].off_v0 : g[0].off_v0) + ((s ? g[1].vskip0 : g[0].vskip0) + vv) * 8
-                                    : (s ? g[1].off_v1 : g[0].off_v1) + (vv - n1) * 8;
-            sz = *reinterpret_cast<const uint2*>(sp + off);
+            act = true;
+            tok = w.tok[s][vv];
+            off = vv < n1 ? (s ? g[1].off_v0 : g[0].off_v0) + ((s ? g[1].vskip0 : g[0].vskip0) + vv) * 8
+                          : (s ? g[1].off_v1 : g[0].off_v1) + (vv - n1) * 8;
           }
         }
-        const float2 e0 = unpack_sz(sz.x), e1 = unpack_sz(sz.y);
-        W0[i] = p * e0.x;
-        W1[i] = p * e1.x;
-        z0 = fmaf(p, e0.y, z0);
-        z1 = fmaf(p, e1.y, z1);
-        mx0 = fmaxf(mx0, W0[i]);
-        mx1 = fmaxf(mx1, W1[i]);
+        // p' of the row's token sits in lane tok & 31 (p0 for tokens < 32, else p1)
+        const float pa = __shfl_sync(kFull, p0, tok & 31), pb = __shfl_sync(kFull, p1, tok & 31);
+        if (act) {
+          const float p = tok < 32 ? pa : pb;
+          const float2 e = unpack_sz(*reinterpret_cast<const uint32_t*>(sp + off + 4 * hw));
+          Wt[i] = p * e.x;
+          zs = fmaf(p, e.y, zs);
+          mx = fmaxf(mx, Wt[i]);
+        }
       }
-      mx0 = warp_max(mx0);
-      mx1 = warp_max(mx1);
-      z0 = warp_sum(z0);
-      z1 = warp_sum(z1);
-      int E0 = 0, E1 = 0;
-      if (mx0 > 0.f) E0 = min(24 - exp_frexp(mx0), 126);
-      if (mx1 > 0.f) E1 = min(24 - exp_frexp(mx1), 126);
-      const float sc0 = pow2i(E0), sc1 = pow2i(E1);
+      mx = warp_max(mx);
+      zs = warp_sum(zs);
+      const int E = mx > 0.f ? min(24 - exp_frexp(mx), 126) : 0;
+      const float scw = pow2i(E);
 #pragma unroll
       for (int i = 0; i < 6; ++i) {
         if (32 * i >= nvr) break;
         const int v = lane + 32 * i;
-        const uint32_t Q0 = fix24(W0[i], sc0), Q1 = fix24(W1[i], sc1);
-        // lane 4m gathers rows 4m..4m+3 and writes their three limb words per half
-        const uint32_t Q0b = __shfl_down_sync(kFull, Q0, 1), Q0c = __shfl_down_sync(kFull, Q0, 2),
-                       Q0d = __shfl_down_sync(kFull, Q0, 3);
-        const uint32_t Q1b = __shfl_down_sync(kFull, Q1, 1), Q1c = __shfl_down_sync(kFull, Q1, 2),
-                       Q1d = __shfl_down_sync(kFull, Q1, 3);
+        const uint32_t Q = fix24(Wt[i], scw);
+        // lane 4m gathers rows 4m..4m+3 and writes their three limb words
+        const uint32_t Qb = __shfl_down_sync(kFull, Q, 1), Qc = __shfl_down_sync(kFull, Q, 2),
+                       Qd = __shfl_down_sync(kFull, Q, 3);
         if ((lane & 3) == 0 && v < nvr) {
-          uint32_t A = __byte_perm(Q0, Q0b, 0x5140), B = __byte_perm(Q0c, Q0d, 0x5140);
-          uint32_t C = __byte_perm(Q0, Q0b, 0x7362), D = __byte_perm(Q0c, Q0d, 0x7362);
-          w.wl[v >> 2][0] = make_uint4(__byte_perm(A, B, 0x5410), __byte_perm(A, B, 0x7632),
-                                       __byte_perm(C, D, 0x5410), 0u);
-          A = __byte_perm(Q1, Q1b, 0x5140);
-          B = __byte_perm(Q1c, Q1d, 0x5140);
-          C = __byte_perm(Q1, Q1b, 0x7362);
-          D = __byte_perm(Q1c, Q1d, 0x7362);
-          w.wl[v >> 2][1] = make_uint4(__byte_perm(A, B, 0x5410), __byte_perm(A, B, 0x7632),
-                                       __byte_perm(C, D, 0x5410), 0u);
+          const uint32_t A = __byte_perm(Q, Qb, 0x5140), B = __byte_perm(Qc, Qd, 0x5140);
+          const uint32_t C = __byte_perm(Q, Qb, 0x7362), D = __byte_perm(Qc, Qd, 0x7362);
+          w.wl[v >> 2][hw] = make_uint4(__byte_perm(A, B, 0x5410), __byte_perm(A, B, 0x7632),
+                                        __byte_perm(C, D, 0x5410), 0u);
         }
       }
       __syncwarp();
 
-      // ---- values: dp4a over transposed nibbles ----
+      // ---- values of this warp's half: dp4a over transposed nibbles ----
       int a0[8], a1[8], a2[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) a0[i] = a1[i] = a2[i] = 0;
       {
         const uint8_t* vb = sp + 64 + 4 * wv;
 #pragma unroll
-        for (int kg = gv; kg < 16; kg += 2) {
+        for (int kg = g4; kg < 16; kg += 4) {
           const uint8_t* rp = vb + kg * 512;
           v_group(*reinterpret_cast<const uint32_t*>(rp), *reinterpret_cast<const uint32_t*>(rp + 128),
                   *reinterpret_cast<const uint32_t*>(rp + 256), *reinterpret_cast<const uint32_t*>(rp + 384),
-                  w.wl[kg][hv], a0, a1, a2);
+                  w.wl[kg][hw], a0, a1, a2);
         }
       }
 #pragma unroll
@@ -495,15 +504,15 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         const int ng = (s ? pad1 : pad0) >> 2;
         const int kb = 16 + (s ? (pad0 >> 2) : 0);
         const uint8_t* vb = sp + (s ? g[1].off_codes : g[0].off_codes) + 64 + 4 * wv;
-        for (int kg = gv; kg < ng; kg += 2) {
+        for (int kg = g4; kg < ng; kg += 4) {
           const uint8_t* rp = vb + kg * 512;
           v_group(*reinterpret_cast<const uint32_t*>(rp), *reinterpret_cast<const uint32_t*>(rp + 128),
                   *reinterpret_cast<const uint32_t*>(rp + 256), *reinterpret_cast<const uint32_t*>(rp + 384),
-                  w.wl[kb + kg][hv], a0, a1, a2);
+                  w.wl[kb + kg][hw], a0, a1, a2);
         }
       }
-      const float isc = pow2i(-(hv ? E1 : E0));
-      const float zh = gv == 0 ? (hv ? z1 : z0) : 0.f;
+      const float isc = pow2i(-E);
+      const float zh = g4 == 0 ? zs : 0.f;
       float val[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i)
@@ -511,7 +520,6 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
                       (i & 1) ? isc * 0.0625f : isc, zh);
       merge(mb, p0 + p1, val);
       fence_proxy_async();  // this span's generic reads and writes precede its reuse by bulk copies
-      __syncwarp();
       ++con_seq;
     } else {
       // ================= BF16 tail unit (global loads) =================
@@ -520,16 +528,15 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       uint16_t* tail_v = arr<uint16_t>(c, A_TAILV, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
       const uint16_t* kn = has_new ? a.k_new + (size_t)h * kD : nullptr;
       const uint16_t* vn = has_new ? a.v_new + (size_t)h * kD : nullptr;
-      if (has_new) {
+      if (has_new && hw == 0) {
         reinterpret_cast<uint2*>(tail_k + (size_t)(nt - 1) * kD)[lane] = reinterpret_cast<const uint2*>(kn)[lane];
         reinterpret_cast<uint2*>(tail_v + (size_t)(nt - 1) * kD)[lane] = reinterpret_cast<const uint2*>(vn)[lane];
       }
       float qsr[32];
       load32(qh + 32 * qq, qsr);
-      __syncwarp();
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = 8 * i + tr;
+      for (int i = 0; i < 4; ++i) {
+        const int t = 32 * hw + 8 * i + tr;
         const bool act = t < nt;
         float p = 0.f;
         if (act) {
@@ -540,9 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         p += __shfl_xor_sync(kFull, p, 2);
         if (qq == 0) w.lg[t] = act ? p : -INFINITY;
       }
-      __syncwarp();
+      pair_sync(pair);
       const float l0 = w.lg[lane], l1 = w.lg[lane + 32];
-      if (a.keep) {
+      if (a.keep && hw == 0) {
         if (lane < nt) {
           score[(size_t)a.n_q + lane] = l0;
           tag[(size_t)a.n_q + lane] = (uint8_t)r;
@@ -553,19 +560,20 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         }
       }
       const float mb = warp_max(fmaxf(l0, l1));
+      const float p0 = mb == -INFINITY ? 0.f : ex2(l0 - mb), p1 = mb == -INFINITY ? 0.f : ex2(l1 - mb);
+      if (hw == 0) {
+        w.pw[lane] = p0;
+        w.pw[lane + 32] = p1;
+      }
+      pair_sync(pair);
       if (mb != -INFINITY) {
-        const float p0 = ex2(l0 - mb), p1 = ex2(l1 - mb);
-        __syncwarp();
-        w.lg[lane] = p0;
-        w.lg[lane + 32] = p1;
-        __syncwarp();
         float val[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) val[i] = 0.f;
-        for (int t = gv; t < nt; t += 2) {
+        for (int t = g4; t < nt; t += 4) {
           const uint16_t* row = (has_new && t == nt - 1) ? vn : tail_v + (size_t)t * kD;
           const uint4 x = __ldg(reinterpret_cast<const uint4*>(row) + wv);
-          const float pt = w.lg[t];
+          const float pt = w.pw[t];
           val[0] = fmaf(pt, bf16_lo(x.x), val[0]);
           val[1] = fmaf(pt, bf16_hi(x.x), val[1]);
           val[2] = fmaf(pt, bf16_lo(x.y), val[2]);
@@ -577,7 +585,6 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         }
         merge(mb, p0 + p1, val);
       }
-      __syncwarp();
     }
   }
 
@@ -586,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
     for (int s = con_seq; s < iss_seq; ++s) mbar_wait(&w.bar[s % kSlots], (unsigned)(s / kSlots) & 1u);
     __syncwarp();
   }
+  pair_sync(pair);  // both warps of the team are done with the ring
   if (cur_hs >= 0) flush(cur_hs);
   __syncthreads();
   grid_dep_wait();  // the previous reader's partials and tickets are final from here
@@ -597,13 +605,13 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
     float* part = a.part + ((size_t)h * kMaxSplits + (cta - c_lo)) * kPartStride;
     if (tid < kD) {
       float Mx = -INFINITY;
-      for (int v = 0; v < kWS; ++v)
+      for (int v = 0; v < kPairs; ++v)
         if (ctl[v].has[hs]) {
           const float* src = hs == 0 ? ctl[v].part0 : reinterpret_cast<const float*>(rings + (size_t)v * kRing);
           Mx = fmaxf(Mx, src[0]);
         }
       float Lt = 0.f, ot = 0.f;
-      for (int v = 0; v < kWS; ++v)
+      for (int v = 0; v < kPairs; ++v)
         if (ctl[v].has[hs]) {
           const float* src = hs == 0 ? ctl[v].part0 : reinterpret_cast<const float*>(rings + (size_t)v * kRing);
           if (src[0] == -INFINITY) continue;
