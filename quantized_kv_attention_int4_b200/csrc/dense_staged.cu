@@ -350,10 +350,10 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         const int pos = store_geom(mkA, w.slot_gs0[slot][0], kRec, g[0]);
         store_geom(mkB, w.slot_gs0[slot][1], pos, g[1]);
       }
-      // ---- key limbs (warp 0: the base record; warp 1: residual records and token maps) ----
-      if (hw == 0) {
+      // ---- key limbs (warp 1: the base record and the token maps; warp 0, which also
+      //      staged the spans: the residual records) ----
+      if (hw == 1) {
         record_to_limbs(reinterpret_cast<uint32_t*>(sp + kRecKsz), qh, lane);
-      } else {
 #pragma unroll
         for (int s = 0; s < kStores; ++s) {
           if (g[s].na == 0) continue;
@@ -363,6 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
             const int tt = lane + 32 * e;
             if ((mk >> tt) & 1ull) w.tok[s][__popcll(mk & ((1ull << tt) - 1ull))] = (uint8_t)tt;
           }
+        }
+      } else {
+#pragma unroll
+        for (int s = 0; s < kStores; ++s) {
+          if (g[s].na == 0) continue;
           record_to_limbs(reinterpret_cast<uint32_t*>(sp + g[s].off_k0), qh, lane);
           if (g[s].n1 < g[s].na) record_to_limbs(reinterpret_cast<uint32_t*>(sp + g[s].off_k1), qh, lane);
         }
