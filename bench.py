@@ -333,7 +333,7 @@ def run_e2e(step, cache, w, layers, inputs, device):
     """The metric end to end through the C ABI: each step runs loops 1-3 untimed, then times
     the loop-4 inputs copied from pinned host memory, the loop-4 selection and sparse
     readers, and the loop-4 outputs read back to pinned host memory."""
-    res = []
+    res, parts = [], []
     H = w.heads
     for q, kn, vn in inputs:
         hq = q[4].cpu().pin_memory()
@@ -345,20 +345,24 @@ def run_e2e(step, cache, w, layers, inputs, device):
         vn[4].zero_()
         step.run(q, kn, vn, loop_first=1, loop_last=3)
         torch.cuda.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
+        a, a1, a2, b = (torch.cuda.Event(enable_timing=True) for _ in range(4))
         a.record()
         q[4].copy_(hq, non_blocking=True)
         kn[4].copy_(hk, non_blocking=True)
         vn[4].copy_(hv, non_blocking=True)
+        a1.record()
         step.run(q, kn, vn, loop_first=4, loop_last=4)
+        a2.record()
         hout.copy_(step.O[4], non_blocking=True)
         b.record()
         b.synchronize()
         res.append(a.elapsed_time(b) * 1e3)
+        parts.append((a.elapsed_time(a1) * 1e3, a1.elapsed_time(a2) * 1e3, a2.elapsed_time(b) * 1e3))
     h2d = 3 * layers * H * 128 * 2
     d2h = layers * H * 128 * 4
-    return {"value": float(np.mean(res)), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    seg = np.mean(np.array(parts), axis=0)
+    return {"value": float(np.mean(res)), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "segments_us": {"h2d": float(seg[0]), "select_and_readers": float(seg[1]), "d2h": float(seg[2])}}
 
 
 # ----------------------------------------------------------------------------

@@ -58,8 +58,7 @@ struct alignas(16) WarpCtlS {
   int32_t slot_off[kSlotsS];
   float2 wrow[kMaxRows][2];        // span being consumed: per row and half (wS, wU)
   float lr[kMaxRows];              // span being consumed: per-row logit parts
-  int32_t rec_g[kMaxRecs];         // span being issued: group record of each key record
-  uint8_t rec_s[kMaxRecs];         // span being issued: store of each key record
+  const uint8_t* rec_src[kMaxRecs];  // span being issued: source of each key record
 };
 
 struct alignas(16) CtaHdr {
@@ -277,20 +276,14 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
 #pragma unroll
           for (int pc = 0; pc < 8; ++pc) cp_async16(dst + pc * 16, src + pc * 16);
           cp_async8(szs + ri * 8, base + kRecVsz + pin * 8);
-          if (isnew) {
-            wc.rec_g[ki] = g;
-            wc.rec_s[ki] = (uint8_t)s;
-          }
+          if (isnew) wc.rec_src[ki] = base + kRecKsz;
         }
         rowbase += __popc(b);
         recbase += __popc(nb);
       }
       __syncwarp();
       // key records: 32 pieces each, spread over the lanes
-      for (int k = 0; k < nrecs; ++k) {
-        const uint8_t* base = (wc.rec_s[k] == 1 ? brec : rrec) + (size_t)wc.rec_g[k] * kRec;
-        cp_async16(recs + k * 512 + lane * 16, base + kRecKsz + lane * 16);
-      }
+      for (int k = 0; k < nrecs; ++k) cp_async16(recs + k * 512 + lane * 16, wc.rec_src[k] + lane * 16);
       asm volatile("cp.async.commit_group;" ::: "memory");
       iss_pos += ncol;
       ++iss_seq;
