@@ -649,17 +649,27 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
     const int h = h0 + hs;
     const int c_lo = cta_of((long long)h * nbp, U, n_cta);
     const int n_parts = cta_of((long long)(h + 1) * nbp - 1, U, n_cta) - c_lo + 1;
+    // the CTA partials, staged in shared memory with coalesced loads (one round trip)
+    const float* hp = a.part + (size_t)h * kMaxSplits * kPartStride;
+    const int nwords = n_parts * kPartStride;
+    const bool staged = (size_t)nwords * sizeof(float) <= (size_t)kPairs * kRing;
+    float* stp = reinterpret_cast<float*>(rings);
+    __syncthreads();  // the previous head's combine is done reading the staged partials
+    if (staged) {
+      for (int i = tid; i < nwords; i += kThreads) stp[i] = __ldcg(hp + i);
+      __syncthreads();
+    }
+    auto ld = [&](int i) { return staged ? stp[i] : __ldcg(hp + i); };
     if (tid < kD) {
-      const float* hp = a.part + (size_t)h * kMaxSplits * kPartStride;
       float Mx = -INFINITY;
-      for (int s = 0; s < n_parts; ++s) Mx = fmaxf(Mx, __ldcg(hp + (size_t)s * kPartStride));
+      for (int s = 0; s < n_parts; ++s) Mx = fmaxf(Mx, ld(s * kPartStride));
       float Lt = 0.f, ot = 0.f;
       for (int s = 0; s < n_parts; ++s) {
-        const float m_s = __ldcg(hp + (size_t)s * kPartStride);
+        const float m_s = ld(s * kPartStride);
         if (m_s == -INFINITY) continue;
         const float e = ex2(m_s - Mx);
-        Lt = fmaf(__ldcg(hp + (size_t)s * kPartStride + 1), e, Lt);
-        ot = fmaf(__ldcg(hp + (size_t)s * kPartStride + 4 + tid), e, ot);
+        Lt = fmaf(ld(s * kPartStride + 1), e, Lt);
+        ot = fmaf(ld(s * kPartStride + 4 + tid), e, ot);
       }
       a.o[(size_t)h * kD + tid] = ot / Lt;
       if (tid == 0) {

@@ -521,21 +521,30 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
   if (!ch.last_cta) return;
   __threadfence();
 
-  // ---- last CTA of the head: combine every split ----
+  // ---- last CTA of the head: combine every split (partials first staged in shared
+  //      memory with coalesced loads, so the combine waits for one round trip) ----
+  const float* hp = a.part + (size_t)h * a.n_splits * kPartStride;
+  const int nwords = a.n_splits * kPartStride;
+  const bool staged = (size_t)nwords * sizeof(float) <= (size_t)kW * kRingS;
+  float* stp = reinterpret_cast<float*>(rings);
+  if (staged) {
+    for (int i = tid; i < nwords; i += kNT) stp[i] = __ldcg(hp + i);
+    __syncthreads();
+  }
+  auto ld = [&](int i) { return staged ? stp[i] : __ldcg(hp + i); };
   if (tid < kD) {
-    const float* hp = a.part + (size_t)h * a.n_splits * kPartStride;
     float Mx = -INFINITY;
-    for (int s = 0; s < a.n_splits; ++s) Mx = fmaxf(Mx, __ldcg(hp + (size_t)s * kPartStride));
+    for (int s = 0; s < a.n_splits; ++s) Mx = fmaxf(Mx, ld(s * kPartStride));
     float Lt = 0.f, St = 0.f, Ut = 0.f, mt = 0.f;
     for (int s = 0; s < a.n_splits; ++s) {
-      const float* pp = hp + (size_t)s * kPartStride;
-      Ut += __ldcg(pp + 4 + kD + tid);
-      mt += __ldcg(pp + 2);
-      const float ms = __ldcg(pp);
+      const int pp = s * kPartStride;
+      Ut += ld(pp + 4 + kD + tid);
+      mt += ld(pp + 2);
+      const float ms = ld(pp);
       if (ms == -INFINITY) continue;
       const float e = ex2(ms - Mx);
-      Lt = fmaf(__ldcg(pp + 1), e, Lt);
-      St = fmaf(__ldcg(pp + 4 + tid), e, St);
+      Lt = fmaf(ld(pp + 1), e, Lt);
+      St = fmaf(ld(pp + 4 + tid), e, St);
     }
     const float op = a.o_prev[(size_t)h * kD + tid];
     const float u = op - Ut;
