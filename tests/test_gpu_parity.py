@@ -169,3 +169,26 @@ def test_device_errors_are_recorded_not_trapped():
     st, info = c.status()
     assert st == abi.FL_ERR_DEVICE and info[0] == 4 and info[1] == 100000
     assert torch.isfinite(o2).all()
+
+
+@pytest.mark.parametrize("name", ["tiny_h1_n256", "layer_h16_n4096"])
+def test_dense_reader_at_every_loop(name):
+    """The dense reader at loops 1..R (loops 1-3: the staged form with up to two residual
+    stores; deeper loops: the direct form) against the oracle's full attention, with the
+    kept scores reproducing the oracle's log-probabilities."""
+    w = W[name]
+    pair = Pair(w)
+    c, lay = pair.cache, pair.oracle
+    q = synth.queries(w, 0, 0, device="cuda")
+    H, N = w.heads, c.n_cols
+    for r in range(1, w.loops + 1):
+        o = torch.empty(H, 128, dtype=torch.float32, device="cuda")
+        c.dense(0, r, q[r].contiguous(), o, keep_scores=True)
+        ref = lay.dense_loop(r, f32(q[r]))
+        assert rel_err(o.cpu().numpy(), ref["o"]) < TOL, r
+        sc = c.raw("score", 0).view(torch.float32)[: H * c.dims.capacity].view(H, -1)[:, :N].cpu().numpy()
+        off = c.raw("offset", 0).view(torch.float32)[: H * 33].view(H, 33)[:, r].cpu().numpy()
+        lp = sc.astype(np.float64) - off[:, None]
+        assert np.abs(lp - np.log2(ref["p"])).max() < 1e-4, r
+    st, info = c.status()
+    assert st == abi.FL_OK, info
