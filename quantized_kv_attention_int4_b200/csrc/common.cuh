@@ -392,6 +392,55 @@ __device__ __forceinline__ void load_limbs(const uint32_t* rec, int qq, uint32_t
   }
 }
 
+// ---- exact integer value sums (dp4a) against fixed-point row weights ----
+__device__ __forceinline__ void dp4a_u(int& acc, uint32_t a, uint32_t b) {
+  asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(acc) : "r"(a), "r"(b));
+}
+
+// Four rows' code words x0..x3 (same word, channels 8w..8w+7) against the four rows'
+// weight limbs (byte 0, 1, 2 words): a0/a1/a2[c] accumulate channel 8w + c (odd
+// channels x16).
+__device__ __forceinline__ void v_group(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint4 wq,
+                                        int* a0, int* a1, int* a2) {
+  const uint32_t a_lo = __byte_perm(x0, x1, 0x5140), a_hi = __byte_perm(x0, x1, 0x7362);
+  const uint32_t b_lo = __byte_perm(x2, x3, 0x5140), b_hi = __byte_perm(x2, x3, 0x7362);
+  uint32_t T[4];
+  T[0] = __byte_perm(a_lo, b_lo, 0x5410);  // byte 0 of rows 0..3
+  T[1] = __byte_perm(a_lo, b_lo, 0x7632);  // byte 1
+  T[2] = __byte_perm(a_hi, b_hi, 0x5410);  // byte 2
+  T[3] = __byte_perm(a_hi, b_hi, 0x7632);  // byte 3
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t ev = T[b] & 0x0F0F0F0Fu, od = T[b] & 0xF0F0F0F0u;
+    dp4a_u(a0[2 * b], ev, wq.x);
+    dp4a_u(a1[2 * b], ev, wq.y);
+    dp4a_u(a2[2 * b], ev, wq.z);
+    dp4a_u(a0[2 * b + 1], od, wq.x);
+    dp4a_u(a1[2 * b + 1], od, wq.y);
+    dp4a_u(a2[2 * b + 1], od, wq.z);
+  }
+}
+
+__device__ __forceinline__ uint32_t fix24(float w, float sc) {
+  const uint32_t q = __float2uint_rn(w * sc);
+  return q > 16777215u ? 16777215u : q;
+}
+
+// Row weights w >= 0 of one 4-row group (lanes 4m..4m+3 hold rows 4m..4m+3) as 24-bit
+// fixed point at scale sc, gathered to lane 4m as three limb words (bytes 0, 1, 2 of the
+// four rows' values; the fourth word is 0).
+__device__ __forceinline__ uint4 pack_group24(float wgt, float sc) {
+  const uint32_t Q = fix24(wgt, sc);
+  const uint32_t Qb = __shfl_down_sync(kFull, Q, 1), Qc = __shfl_down_sync(kFull, Q, 2),
+                 Qd = __shfl_down_sync(kFull, Q, 3);
+  const uint32_t A = __byte_perm(Q, Qb, 0x5140), B = __byte_perm(Qc, Qd, 0x5140);
+  const uint32_t C = __byte_perm(Q, Qb, 0x7362), D = __byte_perm(Qc, Qd, 0x7362);
+  return make_uint4(__byte_perm(A, B, 0x5410), __byte_perm(A, B, 0x7632), __byte_perm(C, D, 0x5410), 0u);
+}
+
+// The exponent E of a 24-bit fixed-point scale for weights whose largest is mx (0 if none).
+__device__ __forceinline__ int fix24_exp(float mx) { return mx > 0.f ? min(24 - exp_frexp(mx), 126) : 0; }
+
 // ---- programmatic dependent launch ----
 // A reader lets the next kernel of its stream start as soon as all of its own CTAs are
 // running (the next reader stages and computes meanwhile), and waits for the previous

@@ -129,43 +129,11 @@ __device__ __forceinline__ void issue_span(uint8_t* sp, const uint8_t* brec_b, c
   }
 }
 
-__device__ __forceinline__ void dp4a_u(int& acc, uint32_t a, uint32_t b) {
-  asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(acc) : "r"(a), "r"(b));
-}
-
-// Four rows' code words x0..x3 (same word, channels 8w..8w+7) against the four rows'
-// weight limbs (byte 0, 1, 2 words): a0/a1/a2[c] accumulate channel 8w + c (odd
-// channels x16).
-__device__ __forceinline__ void v_group(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint4 wq,
-                                        int* a0, int* a1, int* a2) {
-  const uint32_t a_lo = __byte_perm(x0, x1, 0x5140), a_hi = __byte_perm(x0, x1, 0x7362);
-  const uint32_t b_lo = __byte_perm(x2, x3, 0x5140), b_hi = __byte_perm(x2, x3, 0x7362);
-  uint32_t T[4];
-  T[0] = __byte_perm(a_lo, b_lo, 0x5410);  // byte 0 of rows 0..3
-  T[1] = __byte_perm(a_lo, b_lo, 0x7632);  // byte 1
-  T[2] = __byte_perm(a_hi, b_hi, 0x5410);  // byte 2
-  T[3] = __byte_perm(a_hi, b_hi, 0x7632);  // byte 3
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const uint32_t ev = T[b] & 0x0F0F0F0Fu, od = T[b] & 0xF0F0F0F0u;
-    dp4a_u(a0[2 * b], ev, wq.x);
-    dp4a_u(a1[2 * b], ev, wq.y);
-    dp4a_u(a2[2 * b], ev, wq.z);
-    dp4a_u(a0[2 * b + 1], od, wq.x);
-    dp4a_u(a1[2 * b + 1], od, wq.y);
-    dp4a_u(a2[2 * b + 1], od, wq.z);
-  }
-}
-
 // CTA holding unit x when U units are cut into n contiguous ranges floor(cU/n).
 __device__ __forceinline__ int cta_of(long long x, long long U, int n) {
   return (int)(((x + 1) * n + U - 1) / U) - 1;
 }
 
-__device__ __forceinline__ uint32_t fix24(float w, float sc) {
-  const uint32_t q = __float2uint_rn(w * sc);
-  return q > 16777215u ? 16777215u : q;
-}
 
 __device__ __forceinline__ void pair_sync(int pair) {
   asm volatile("bar.sync %0, 64;" ::"r"(pair + 1) : "memory");
