@@ -36,12 +36,12 @@
 namespace fl {
 namespace {
 
-constexpr int kW = 4;              // warps per CTA
+constexpr int kW = 5;              // warps per CTA
 constexpr int kNT = kW * 32;
 constexpr int kCtaPerSm = 3;
 constexpr int kStoresMax = 8;      // loops served
-constexpr int kMaxRows = 64;       // rows per span
-constexpr int kMaxRecs = 12;       // key records per span
+constexpr int kMaxRows = 52;       // rows per span
+constexpr int kMaxRecs = 10;       // key records per span
 constexpr int kSlotsS = 4;         // spans in flight per warp
 constexpr int kPlanWords = 1024;   // plan words of one CTA
 constexpr int kSmemCta = 76800;    // three CTAs per SM
