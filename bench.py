@@ -145,12 +145,12 @@ def max_over_ranks(values, device):
     return [float(x) for x in t.tolist()]
 
 
-def build_cache(w: synth.Workload, layers: int, rank: int, device):
+def build_cache(w: synth.Workload, layers: int, rank: int, device, new_tokens: int = 256):
     from quantized_kv_attention_int4_b200.cache import FlashLoopCache, round_up
 
     n = w.n_ctx
     sets = synth.active_sets(w, n)
-    extra = 64 * 4 + 64
+    extra = (new_tokens + 63) // 64 * 64 + 64  # room for the decoded tokens and one tail
     cap = round_up(n + extra)
     res_cap = {r: round_up(min(cap, int((sets[r] < n).sum()) + extra + 64 * 4)) for r in range(2, w.loops + 1)}
     cache = FlashLoopCache(layers, w.heads, w.loops, cap, res_capacity=res_cap,
@@ -262,7 +262,7 @@ def run_gpu(args, rank, world):
     w = synth.WORKLOADS[args.workload]
     layers = args.layers or w.layers
     t0 = time.time()
-    cache, wr = build_cache(w, layers, rank, device)
+    cache, wr = build_cache(w, layers, rank, device, new_tokens=args.warmup + args.steps + args.e2e_steps)
     total_steps = args.warmup + args.steps
     inputs = step_inputs(wr, layers, total_steps + args.e2e_steps, device)
     step = Step(cache, wr, layers, device)

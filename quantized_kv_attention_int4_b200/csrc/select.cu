@@ -11,7 +11,7 @@
 //   keys:     log2 p~_j = score_j - offset[tag_j], mapped to an order-preserving u32
 //             and kept in shared memory (N <= FL_MAX_SELECT_COLS);
 //   select:   radix select of the K-th largest key over the bits where the keys
-//             differ (the prefix every key shares is skipped), digits of up to 12
+//             differ (the prefix every key shares is skipped), digits of up to 13
 //             bits, each pass a shared-memory histogram over the keys that still match
 //             the prefix and a block-wide scan from the top bin;
 //   compact:  keys above the threshold plus the lowest-index ties, written in index
@@ -27,7 +27,7 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarpsSel = kThreads / 32;
-constexpr int kDynMax = 200 * 1024;  // dynamic shared memory: keys [, selected columns]
+constexpr int kDynMax = 194 * 1024;  // dynamic shared memory: keys [, selected columns]
 
 // Selected columns are kept in shared memory after the keys when both fit.
 __host__ __device__ inline bool sel_fits(int N, int K) {
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   extern __shared__ uint32_t keys[];  // [N] keys, then [K] selected columns when they fit
   const bool sel_smem = sel_fits(a.n_q + a.n_tail, a.k_sel);
   int32_t* sel_s = reinterpret_cast<int32_t*>(keys + ((a.n_q + a.n_tail + 3) & ~3));
-  __shared__ __align__(16) uint32_t hist[4096];
+  __shared__ __align__(16) uint32_t hist[8192];
   __shared__ float offs[kOffStride];
   __shared__ uint32_t wtot[32];
   __shared__ uint32_t sh_digit, sh_krem;
@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   uint32_t pmask = nbits >= 32 ? 0u : ~((1u << nbits) - 1u);
   uint32_t prefix = kand & pmask, krem = (uint32_t)K;
   while (nbits > 0) {
-    const int wbits = nbits < 12 ? nbits : 12;
+    // up to 13-bit digits; two balanced passes whenever the keys differ in <= 26 bits
+    const int wbits = nbits > 26 ? 13 : (nbits > 13 ? (nbits + 1) / 2 : nbits);
     const int shift = nbits - wbits;
     nbits = shift;
     const int nbins = 1 << wbits;
