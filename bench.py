@@ -5,7 +5,7 @@ context with 4 loops (Ouro-2.6B-shaped), INT4 base + nested 25 % / 10 % residual
 + BF16 tail, synthetic seeded data.  A *step* decodes one token through every
 layer and loop in loop-major order (loop r runs all layers before loop r+1):
 
-    append / flush tail -> loop 1 dense (48) -> loop 2 dense (48, keeps scores)
+    append token -> loop 1 dense (48) -> loop 2 dense (48, keeps scores)
     -> select for loop 3 (all layers, one launch) -> loop 3 sparse (48)
     -> select for loop 4 (one launch) -> loop 4 sparse (48)
 
@@ -180,8 +180,10 @@ def step_inputs(w: synth.Workload, layers: int, steps: int, device):
 
 
 class Step:
-    """One decode step: flush the tail if full (Python bookkeeping, native encoders), then the
-    native loop-major executor over every layer and loop."""
+    """One decode step: append the token (host bookkeeping), then the native loop-major
+    executor over every layer and loop.  The step in which the tail reaches 64 rows also
+    quantises it inside its readers (fused flush); only a prompt that ends with a full tail
+    is flushed by the encode launches, at the first token."""
 
     def __init__(self, cache, w, layers, device):
         self.c, self.w, self.L = cache, w, layers
@@ -202,7 +204,7 @@ class Step:
             c.begin_token()
         seg = [ev[k] for k in EXEC_EVENTS] if ev is not None else None
         c.step(w.dense_loops, w.k_sel(c.n_cols), q, self.O, kn, vn, loop_first=loop_first,
-               loop_last=loop_last or w.loops, events=seg)
+               loop_last=loop_last or w.loops, events=seg, flush=c.n_tail == 64)
         return self.launches(flushed)
 
 

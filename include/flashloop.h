@@ -268,6 +268,39 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
                          const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new, float* o,
                          void* ws, size_t ws_bytes, void* const* events, void* stream);
 
+/* [Project] "The Method", closing paragraph (KV updates and quantisation fused into the
+ * attention kernel); Step 03; Step 01.  The 64-row tail group that a decode step
+ * quantises while it attends over it (fl_decode_step_flush). */
+typedef struct fl_flush {
+  /* active[r], r = 2..R: bit i set when tail row i (token n_q + i) enters loop r's
+   * residual store.  Must nest: active[r] is a subset of active[r-1], and every row is in
+   * the base (entries 0 and 1 are ignored). */
+  uint64_t active[FL_MAX_LOOPS + 1];
+  /* HOST int32 [layers][FL_MAX_LOOPS + 1]: slot0[l * (FL_MAX_LOOPS + 1) + r] is the first
+   * slot of loop r's residual store that layer l's group takes (a multiple of 64, with
+   * slot0 + popcount(active[r]) <= res_capacity[r]; unused when active[r] is 0). */
+  const int32_t* slot0;
+} fl_flush;
+
+/* fl_decode_step that also moves a full BF16 tail (n_tail == 64, n_q + 64 <= capacity)
+ * into the INT4 stores as the step runs, with no encode launches.  flush == NULL is
+ * exactly fl_decode_step.  Each reader of a loop r in loop_first..loop_last, dense or
+ * sparse, first attends over the tail as BF16 (the
+ * outputs are those of fl_decode_step) and then writes, for every head, store r of the
+ * 64 tail rows [n_q, n_q + 64): for r = 1 the base group record (depth 1, the block's
+ * residual mask/first entries cleared), for r >= 2 the residual record of the rows in
+ * active[r] at slot0[l][r] (mask = active[r], first = slot0 or -1, depth = r).  The bytes
+ * equal those of fl_encode_base / fl_encode_residual on the same rows after the step;
+ * the new token (tail row 63) is taken from k_new / v_new when they are given.  A step
+ * split over several calls (loop ranges) passes the same `flush` to each and must run
+ * its loops in order.  After loop R the caller's timeline moves on: n_q += 64, n_tail
+ * = 0.  Validated on the host (nesting, slot alignment and capacity per layer). */
+fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail,
+                               int32_t dense_loops, int32_t k_sel, int32_t loop_first,
+                               int32_t loop_last, const uint16_t* q, const uint16_t* k_new,
+                               const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,
+                               void* const* events, const fl_flush* flush, void* stream);
+
 /* Synchronise `stream`, copy the cache's status words to host `out[0..2]`, and return
  * FL_ERR_DEVICE if a kernel recorded an error (FL_OK otherwise).  With `clear` != 0
  * the words are zeroed afterwards. */

@@ -33,7 +33,7 @@ FL_OK, FL_ERR_INVALID, FL_ERR_UNSUPPORTED, FL_ERR_CUDA, FL_ERR_WORKSPACE, FL_ERR
 EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init", "fl_workspace_bytes",
             "fl_workspace_init", "fl_write_tail", "fl_encode_base", "fl_encode_residual",
             "fl_decode_attn_dense", "fl_select_topk", "fl_decode_attn_sparse", "fl_decode_step",
-            "fl_read_status", "fl_decode_attn_sparse_noalloc")
+            "fl_read_status", "fl_decode_attn_sparse_noalloc", "fl_decode_step_flush")
 
 
 class fl_dims(ctypes.Structure):
@@ -48,6 +48,10 @@ class fl_layout(ctypes.Structure):
                 + [("status", ctypes.c_uint64), ("layer_stride", ctypes.c_uint64 * N_ARRAYS),
                    ("plan_stride", ctypes.c_int32), ("slot_base", ctypes.c_int32 * (MAX_LOOPS + 1)),
                    ("total_slots", ctypes.c_int32)])
+
+
+class fl_flush(ctypes.Structure):
+    _fields_ = [("active", ctypes.c_uint64 * (MAX_LOOPS + 1)), ("slot0", ctypes.POINTER(ctypes.c_int32))]
 
 
 _P = ctypes.c_void_p
@@ -81,6 +85,8 @@ _c_sparse_noalloc = _sig("fl_decode_attn_sparse_noalloc", _I, _DP, _P, _I, _I, _
                          _P)
 _c_step = _sig("fl_decode_step", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t,
                 ctypes.POINTER(ctypes.c_void_p), _P)
+_c_step_flush = _sig("fl_decode_step_flush", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                      ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(fl_flush), _P)
 _c_read_status = _sig("fl_read_status", _I, _DP, _P, ctypes.POINTER(ctypes.c_int32), _I, _P)
 
 
@@ -226,11 +232,28 @@ def fl_decode_attn_sparse_noalloc(dims, cache, layer, loop, n_q, n_tail, k_sel, 
         _ptr(o_prev, torch.float32, "o_prev"), _ptr(o, torch.float32, "o"), _stream(stream)))
 
 
+def Flush(active, slot0) -> fl_flush:
+    """fl_flush from active[r] (64-bit row masks, index = loop) and slot0[l][r] (host ints)."""
+    f = fl_flush()
+    for r, m in enumerate(active):
+        f.active[r] = int(m)
+    rows = [list(x) for x in slot0]
+    arr = (ctypes.c_int32 * (len(rows) * (MAX_LOOPS + 1)))()
+    for l, row in enumerate(rows):
+        for r, v in enumerate(row):
+            arr[l * (MAX_LOOPS + 1) + r] = int(v)
+    f.slot0 = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
+    f._keep = arr  # the struct points into this array
+    return f
+
+
 def fl_decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, k_new, v_new, o, ws,
-                   events=None, stream=None):
+                   events=None, stream=None, flush=None):
     """One loop-major decode step over every layer; q/k_new/v_new BF16 and o fp32, all [R+1][L][H][128].
 
     ``events``: None or a list of 2R+1 torch.cuda.Event (enable_timing) recorded at segment boundaries.
+    ``flush``: None, or an fl_flush (see Flush): the step also quantises its full 64-row tail
+    (fl_decode_step_flush).
     """
     ev = None
     if events is not None:
@@ -242,10 +265,14 @@ def fl_decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loo
             raise ValueError(f"{name} must be contiguous [R+1][L][H][128]")
     if not o.is_contiguous():
         raise ValueError("o must be contiguous [R+1][L][H][128]")
-    _check("fl_decode_step", _c_step(
-        ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), n_q, n_tail, dense_loops, k_sel, loop_first, loop_last,
-        _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
-        _ptr(o, torch.float32, "o"), _ptr(ws, torch.uint8, "ws"), ws.numel(), ev, _stream(stream)))
+    args = (ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), n_q, n_tail, dense_loops, k_sel, loop_first,
+            loop_last, _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
+            _ptr(v_new, torch.bfloat16, "v_new"), _ptr(o, torch.float32, "o"), _ptr(ws, torch.uint8, "ws"),
+            ws.numel(), ev)
+    if flush is None:
+        _check("fl_decode_step", _c_step(*args, _stream(stream)))
+    else:
+        _check("fl_decode_step_flush", _c_step_flush(*args, ctypes.byref(flush), _stream(stream)))
 
 
 def fl_read_status(dims, cache, clear=True, stream=None):

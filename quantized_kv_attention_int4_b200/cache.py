@@ -56,6 +56,7 @@ class FlashLoopCache:
         self.n_rows = [[0] * (loops + 1) for _ in range(layers)]   # residual rows actually stored
         self.tail_depth: list[int] = []
         self._rows_cache: dict = {}
+        self._plan = None   # (n_q, fl_flush) of a flushing step split over loop ranges
 
     # ---- views into the device buffer (for tests and inspection) -----------------
     def raw(self, name: str, layer: int) -> torch.Tensor:
@@ -126,9 +127,36 @@ class FlashLoopCache:
             self.n_slots[layer][r] = slot0 + rows.numel()
             self.n_rows[layer][r] += rows.numel()
 
+    def flush_plan(self):
+        """The fl_flush that moves the current full tail into the INT4 stores inside a step.
+
+        Loop r's residual store takes the tail rows whose last active loop is >= r, at the
+        next 64-aligned slot of each layer's store (the slots fl_encode_residual would use).
+        """
+        assert self.n_tail == TAIL
+        active = [0] * (self.R + 1)
+        for r in range(2, self.R + 1):
+            active[r] = sum(1 << i for i, dep in enumerate(self.tail_depth) if dep >= r)
+        slot0 = [[0] + [0] + [round_up(self.n_slots[layer][r]) for r in range(2, self.R + 1)]
+                 for layer in range(self.L)]
+        return abi.Flush(active, slot0)
+
+    def _flushed(self, plan):
+        """Host bookkeeping once a step has written every store of the flushed tail."""
+        for layer in range(self.L):
+            for r in range(2, self.R + 1):
+                n = bin(plan.active[r]).count("1")
+                self.n_slots[layer][r] = plan.slot0[layer * (abi.MAX_LOOPS + 1) + r] + n
+                self.n_rows[layer][r] += n
+        self.n_q += TAIL
+        self.n_tail = 0
+        self.tail_depth = []
+
     def begin_token(self, layers=None):
         """Make room for the next token: flush a full tail (every layer), then add one row.
 
+        A step run with ``flush=True`` has already moved its full tail into the INT4
+        stores; otherwise the tail is flushed here with the encode entry points.
         The new row's per-loop key/value are written by the readers (k_new / v_new).
         """
         if self.n_tail == TAIL:
@@ -153,10 +181,24 @@ class FlashLoopCache:
                                   o_prev, o, self.ws, stream)
 
     def step(self, dense_loops, k_sel, q, o, k_new=None, v_new=None, loop_first=1, loop_last=None, events=None,
-             stream=None):
-        """Loops loop_first..loop_last of one decode step for every layer (native executor)."""
+             stream=None, flush=False):
+        """Loops loop_first..loop_last of one decode step for every layer (native executor).
+
+        With ``flush`` (the tail must hold 64 rows) each reader also quantises its loop's
+        store of the tail group; once loop R has run, the tail is part of the INT4 cache.
+        A step split over loop ranges keeps one plan for all of its calls.
+        """
+        loop_last = loop_last or self.R
+        plan = None
+        if flush:
+            if self._plan is None or self._plan[0] != self.n_q:
+                self._plan = (self.n_q, self.flush_plan())
+            plan = self._plan[1]
         abi.fl_decode_step(self.dims, self.buf, self.n_q, self.n_tail, dense_loops, k_sel, loop_first,
-                           loop_last or self.R, q, k_new, v_new, o, self.ws, events, stream)
+                           loop_last, q, k_new, v_new, o, self.ws, events, stream, flush=plan)
+        if plan is not None and loop_last == self.R:
+            self._plan = None
+            self._flushed(plan)
 
     def status(self, clear=True):
         return abi.fl_read_status(self.dims, self.buf, clear)

@@ -119,6 +119,13 @@ fl_status check_reader(const fl_dims* d, void* cache, int layer, int loop, int n
   return FL_OK;
 }
 
+// The fused tail flush of layer l's loop-r reader (none when flush is NULL).
+void set_flush(ReaderArgs& a, const fl_flush* flush, int l, int r) {
+  a.flush = flush ? 1 : 0;
+  a.flush_act = flush && r >= 2 ? flush->active[r] : 0ull;
+  a.flush_slot0 = flush && r >= 2 ? flush->slot0[(size_t)l * (FL_MAX_LOOPS + 1) + r] : 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -264,7 +271,7 @@ fl_status fl_decode_attn_dense(const fl_dims* dims, void* cache, int32_t layer, 
   if (st != FL_OK) return st;
   fl_layout L;
   make_layout(dims, &L);
-  ReaderArgs a;
+  ReaderArgs a{};
   a.c = make_view(dims, L, cache);
   a.layer = layer;
   a.r = loop;
@@ -317,7 +324,7 @@ fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer,
   if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
   fl_layout L;
   make_layout(dims, &L);
-  ReaderArgs a;
+  ReaderArgs a{};
   a.c = make_view(dims, L, cache);
   a.layer = layer;
   a.r = loop;
@@ -379,7 +386,7 @@ fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_
   if (cudaMemsetAsync(scratch, 0, (size_t)dims->heads * sizeof(int32_t), s) != cudaSuccess) return FL_ERR_CUDA;
   fl_layout L;
   make_layout(dims, &L);
-  ReaderArgs a;
+  ReaderArgs a{};
   a.c = make_view(dims, L, cache);
   a.layer = layer;
   a.r = loop;
@@ -402,11 +409,34 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
                          int32_t k_sel, int32_t loop_first, int32_t loop_last, const uint16_t* q,
                          const uint16_t* k_new, const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,
                          void* const* events, void* stream) {
+  return fl_decode_step_flush(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, k_new, v_new,
+                              o, ws, ws_bytes, events, nullptr, stream);
+}
+
+fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
+                               int32_t k_sel, int32_t loop_first, int32_t loop_last, const uint16_t* q,
+                               const uint16_t* k_new, const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,
+                               void* const* events, const fl_flush* flush, void* stream) {
   fl_status st = check_reader(dims, cache, 0, 1, n_q, n_tail, q, k_new, v_new, o, ws, ws_bytes);
   if (st != FL_OK) return st;
   const int R = dims->loops, L = dims->layers, H = dims->heads;
   if (dense_loops < 0 || dense_loops > R || loop_first < 1 || loop_last > R || loop_first > loop_last)
     return FL_ERR_INVALID;
+  if (flush) {
+    if (n_tail != FL_TAIL || (int64_t)n_q + FL_TAIL > dims->capacity || !flush->slot0) return FL_ERR_INVALID;
+    uint64_t prev = ~0ull;
+    for (int r = 2; r <= R; ++r) {
+      const uint64_t act = flush->active[r];
+      if (act & ~prev) return FL_ERR_INVALID;  // the active sets nest
+      prev = act;
+      if (!act) continue;
+      const int nr = __builtin_popcountll(act);
+      for (int l = 0; l < L; ++l) {
+        const int32_t s0 = flush->slot0[(size_t)l * (FL_MAX_LOOPS + 1) + r];
+        if (s0 < 0 || s0 % FL_GROUP || (int64_t)s0 + nr > dims->res_capacity[r]) return FL_ERR_INVALID;
+      }
+    }
+  }
   const int64_t N = (int64_t)n_q + n_tail;
   const bool any_sparse = loop_last > dense_loops;
   if (any_sparse) {
@@ -422,7 +452,7 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
   auto rec = [&](int i) -> bool {
     return !events || cudaEventRecord((cudaEvent_t)events[i], s) == cudaSuccess;
   };
-  ReaderArgs a;
+  ReaderArgs a{};
   a.c = make_view(dims, lay, cache);
   a.o_prev = nullptr;
   a.n_q = n_q;
@@ -431,6 +461,9 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
   a.n_splits = 1;
   a.part = static_cast<float*>(ws);
   a.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_part_bytes(dims));
+  // the step's first reader is an ordinary launch: nothing of it runs before the
+  // previous step (including its tail flush) has completed
+  bool first_launch = true;
   if (!rec(0)) return FL_ERR_CUDA;
   for (int r = loop_first; r <= loop_last; ++r) {
     a.r = r;
@@ -444,7 +477,9 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
         a.k_new = k_new ? k_new + qo : nullptr;
         a.v_new = v_new ? v_new + qo : nullptr;
         a.o = o + qo;
-        if (launch_dense(a, s) != cudaSuccess) return FL_ERR_CUDA;
+        set_flush(a, flush, l, r);
+        if (launch_dense(a, s, !first_launch) != cudaSuccess) return FL_ERR_CUDA;
+        first_launch = false;
       }
     } else {
       SelectArgs sa;
@@ -465,6 +500,7 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
         a.v_new = v_new ? v_new + qo : nullptr;
         a.o = o + qo;
         a.o_prev = o + qo - ostride_r;
+        set_flush(a, flush, l, r);
         if (launch_sparse(a, s) != cudaSuccess) return FL_ERR_CUDA;
       }
     }

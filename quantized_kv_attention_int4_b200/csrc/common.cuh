@@ -450,10 +450,12 @@ __device__ __forceinline__ int fix24_exp(float mx) { return mx > 0.f ? min(24 - 
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Launch `kernel` on `s` with programmatic stream serialization allowed.
+// Launch `kernel` on `s`; with `chain`, programmatic stream serialization is allowed
+// (the kernel may start while its predecessor finishes), otherwise it is an ordinary
+// stream-ordered launch.
 template <class... KArgs, class... Args>
-inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                              Args... args) {
+inline cudaError_t launch_pdl_if(bool chain, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t s, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -463,8 +465,14 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = chain ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <class... KArgs, class... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  return launch_pdl_if(true, kernel, grid, block, smem, s, args...);
 }
 
 // log2(e) / sqrt(128): scores are kept in the base-2 domain.

@@ -21,6 +21,7 @@
 //      128 p s and a per-half correction sum(p z - 128 p s).
 // Warps merge in shared memory, CTAs write (M, L, o) partials, and the last CTA of
 // each head (an atomic ticket, no waiting) combines them by log-sum-exp.
+#include "flush.cuh"
 #include "kernels.h"
 
 namespace fl {
@@ -28,6 +29,8 @@ namespace {
 
 constexpr int kWarps = 8;
 
+// kFlush: the step also writes this loop's store of a full tail (fused flush)
+template <bool kFlush>
 __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs a) {
   const int h = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, qq = lane & 3, tr = lane >> 2;
@@ -298,11 +301,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
   __syncthreads();
   if (tid == 0) last_cta = (atomicAdd(&a.counter[h], 1) == a.n_splits - 1);
   __syncthreads();
-  if (!last_cta) return;
-  __threadfence();
+  if (last_cta) __threadfence();
 
   // ---- last CTA of this head: log-sum-exp combine of every split ----
-  if (tid < kD) {
+  if (last_cta && tid < kD) {
     const float* hp = a.part + (size_t)h * a.n_splits * kPartStride;
     float Mx = -INFINITY;
     for (int s = 0; s < a.n_splits; ++s) Mx = fmaxf(Mx, __ldcg(hp + (size_t)s * kPartStride));
@@ -319,6 +321,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
       arr<float>(c, A_OFFSET, a.layer)[(size_t)h * kOffStride + r] = Mx + log2f(Lt);
       a.counter[h] = 0;
     }
+  }
+  if constexpr (kFlush) {  // dynamic shared memory holds the encoder's staging (launched with it)
+    extern __shared__ __align__(16) uint8_t flush_smem[];
+    flush_tail(a, blockIdx.y * gridDim.x + blockIdx.x, gridDim.x * gridDim.y,
+               *reinterpret_cast<EncodeSmem*>(flush_smem), tid, kWarps * 32);
   }
 }
 
@@ -338,7 +345,10 @@ int dense_splits(int heads, int n_q) {
 cudaError_t launch_dense_direct(ReaderArgs a, cudaStream_t s) {
   a.n_splits = dense_splits(a.c.H, a.n_q);
   dim3 grid(a.n_splits, a.c.H);
-  dense_direct_kernel<<<grid, kWarps * 32, 0, s>>>(a);
+  if (a.flush)
+    dense_direct_kernel<true><<<grid, kWarps * 32, sizeof(EncodeSmem), s>>>(a);
+  else
+    dense_direct_kernel<false><<<grid, kWarps * 32, 0, s>>>(a);
   return cudaGetLastError();
 }
 

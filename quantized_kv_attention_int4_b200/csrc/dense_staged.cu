@@ -34,6 +34,7 @@
 // The tail unit reads its BF16 rows from global memory in fp32.
 // Teams' partials merge per CTA; the last CTA of each head (atomic ticket) combines the
 // CTA partials by log-sum-exp and writes o and offset[r] = M + log2 L.
+#include "flush.cuh"
 #include "kernels.h"
 
 namespace fl {
@@ -139,6 +140,8 @@ __device__ __forceinline__ void pair_sync(int pair) {
   asm volatile("bar.sync %0, 64;" ::"r"(pair + 1) : "memory");
 }
 
+// kFlush: the step also writes this loop's store of a full tail (fused flush)
+template <bool kFlush>
 __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a, int n_cta) {
   extern __shared__ __align__(128) uint8_t smem[];
   int* last = reinterpret_cast<int*>(smem);
@@ -646,6 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       }
     }
   }
+  if constexpr (kFlush) {
+    __syncthreads();  // the combines above are done with the staged partials
+    flush_tail(a, cta, n_cta, *reinterpret_cast<EncodeSmem*>(rings), tid, kThreads);
+  }
 }
 
 int num_sms() {
@@ -663,7 +670,7 @@ int num_sms() {
 
 }  // namespace
 
-cudaError_t launch_dense(ReaderArgs a, cudaStream_t s) {
+cudaError_t launch_dense(ReaderArgs a, cudaStream_t s, bool chain) {
   const int sms = num_sms();
   const long long U = (long long)a.c.H * (a.n_q / kG + 1);
   long long n = sms < U ? sms : U;
@@ -673,13 +680,15 @@ cudaError_t launch_dense(ReaderArgs a, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(dense_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
-    if (e != cudaSuccess) return e;
+    for (auto k : {dense_staged_kernel<false>, dense_staged_kernel<true>}) {
+      const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+      if (e != cudaSuccess) return e;
+    }
     attr_set[dev] = true;
   }
   a.n_splits = (int)n;
-  return launch_pdl(dense_staged_kernel, dim3((int)n), dim3(kThreads), (size_t)kSmemTotal, s, a, (int)n);
+  return launch_pdl_if(chain, a.flush ? dense_staged_kernel<true> : dense_staged_kernel<false>, dim3((int)n),
+                       dim3(kThreads), (size_t)kSmemTotal, s, a, (int)n);
 }
 
 }  // namespace fl

@@ -32,6 +32,11 @@ struct ReaderArgs {
   float* o;
   float* part;
   int32_t* counter;
+  // fused tail flush (flush != 0): after attending, write store r of the 64 tail rows
+  // [n_q, n_q + 64); a residual store takes the rows set in flush_act into the 64-slot
+  // group that starts at residual slot flush_slot0
+  int flush, flush_slot0;
+  unsigned long long flush_act;
 };
 
 struct SelectArgs {
@@ -41,7 +46,9 @@ struct SelectArgs {
 
 cudaError_t launch_encode_base(const EncodeBaseArgs& a, cudaStream_t s);
 cudaError_t launch_encode_residual(const EncodeResArgs& a, cudaStream_t s);
-cudaError_t launch_dense(ReaderArgs a, cudaStream_t s);
+// chain = false: an ordinary stream-ordered launch (no programmatic overlap with the
+// preceding kernel)
+cudaError_t launch_dense(ReaderArgs a, cudaStream_t s, bool chain = true);
 cudaError_t launch_dense_direct(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s);

@@ -28,6 +28,7 @@
 // BF16 tail columns are handled last from global memory.  Warps merge in shared memory,
 // CTAs write (M, L, m, sum p v, sum p~ v) partials, and the last CTA of each head
 // combines them (atomic ticket, no waiting).
+#include "flush.cuh"
 #include "kernels.h"
 
 namespace fl {
@@ -191,6 +192,8 @@ __device__ void issue_stage(Stage& sg, int lane) {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
+// kFlush: the step also writes this loop's store of a full tail (fused flush)
+template <bool kFlush>
 __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
@@ -557,34 +560,40 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
   __syncthreads();
   if (tid == 0) sm.last_cta = (atomicAdd(&a.counter[h], 1) == a.n_splits - 1);
   __syncthreads();
-  if (!sm.last_cta) return;
-  __threadfence();
+  if (sm.last_cta) {
+    __threadfence();
 
-  // ---- last CTA of the head: combine every split ----
-  if (tid < kD) {
-    const float* hp = a.part + (size_t)h * a.n_splits * kPartStride;
-    float Mx = -INFINITY;
-    for (int s = 0; s < a.n_splits; ++s) Mx = fmaxf(Mx, __ldcg(hp + (size_t)s * kPartStride));
-    float Lt = 0.f, St = 0.f, Ut = 0.f, mt = 0.f;
-    for (int s = 0; s < a.n_splits; ++s) {
-      const float* pp = hp + (size_t)s * kPartStride;
-      Ut += __ldcg(pp + 4 + kD + tid);
-      mt += __ldcg(pp + 2);
-      const float ms = __ldcg(pp);
-      if (ms == -INFINITY) continue;
-      const float e = ex2(ms - Mx);
-      Lt = fmaf(__ldcg(pp + 1), e, Lt);
-      St = fmaf(__ldcg(pp + 4 + tid), e, St);
+    // ---- last CTA of the head: combine every split ----
+    if (tid < kD) {
+      const float* hp = a.part + (size_t)h * a.n_splits * kPartStride;
+      float Mx = -INFINITY;
+      for (int s = 0; s < a.n_splits; ++s) Mx = fmaxf(Mx, __ldcg(hp + (size_t)s * kPartStride));
+      float Lt = 0.f, St = 0.f, Ut = 0.f, mt = 0.f;
+      for (int s = 0; s < a.n_splits; ++s) {
+        const float* pp = hp + (size_t)s * kPartStride;
+        Ut += __ldcg(pp + 4 + kD + tid);
+        mt += __ldcg(pp + 2);
+        const float ms = __ldcg(pp);
+        if (ms == -INFINITY) continue;
+        const float e = ex2(ms - Mx);
+        Lt = fmaf(__ldcg(pp + 1), e, Lt);
+        St = fmaf(__ldcg(pp + 4 + tid), e, St);
+      }
+      const float op = a.o_prev[(size_t)h * kD + tid];
+      const float u = op - Ut;
+      a.o[(size_t)h * kD + tid] = Lt > 0.f ? fmaf(mt, St / Lt, u) : u;
+      arr<float>(c, A_UNSEL, a.layer)[(size_t)h * kD + tid] = u;
+      if (tid == 0) {
+        arr<float>(c, A_MASS, a.layer)[h] = mt;
+        arr<float>(c, A_OFFSET, a.layer)[(size_t)h * kOffStride + r] = Mx + log2f(Lt) - log2f(mt);
+        a.counter[h] = 0;
+      }
     }
-    const float op = a.o_prev[(size_t)h * kD + tid];
-    const float u = op - Ut;
-    a.o[(size_t)h * kD + tid] = Lt > 0.f ? fmaf(mt, St / Lt, u) : u;
-    arr<float>(c, A_UNSEL, a.layer)[(size_t)h * kD + tid] = u;
-    if (tid == 0) {
-      arr<float>(c, A_MASS, a.layer)[h] = mt;
-      arr<float>(c, A_OFFSET, a.layer)[(size_t)h * kOffStride + r] = Mx + log2f(Lt) - log2f(mt);
-      a.counter[h] = 0;
-    }
+  }
+  if constexpr (kFlush) {
+    __syncthreads();  // the combine is done with shared memory
+    flush_tail(a, blockIdx.y * gridDim.x + blockIdx.x, gridDim.x * gridDim.y, *reinterpret_cast<EncodeSmem*>(smem_raw),
+               tid, NT);
   }
 }
 
@@ -605,11 +614,12 @@ int sparse_splits(int heads, int k_sel, int loops) {
 
 cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s) {
   a.n_splits = sparse_splits(a.c.H, a.k_sel, a.c.R);
-  const size_t smem = sizeof(Smem);
-  cudaError_t e = cudaFuncSetAttribute(sparse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = a.flush && sizeof(EncodeSmem) > sizeof(Smem) ? sizeof(EncodeSmem) : sizeof(Smem);
+  auto kern = a.flush ? sparse_kernel<true> : sparse_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_splits, a.c.H);
-  return launch_pdl(sparse_kernel, grid, dim3(NT), smem, s, a);
+  return launch_pdl(kern, grid, dim3(NT), smem, s, a);
 }
 
 }  // namespace fl

@@ -31,6 +31,7 @@
 // BF16 tail columns are handled last from global memory.  Warps merge in shared memory,
 // CTAs write (M, L, m, sum p v, sum p~ v) partials, and the last CTA of each head
 // combines them (atomic ticket, no waiting).
+#include "flush.cuh"
 #include "kernels.h"
 
 namespace fl {
@@ -99,6 +100,8 @@ __device__ __forceinline__ int scan_incl(int v, int lane) {
   return v;
 }
 
+// kFlush: the step also writes this loop's store of a full tail (fused flush)
+template <bool kFlush>
 __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& ch = *reinterpret_cast<CtaHdr*>(smem);
@@ -518,43 +521,49 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
   __syncthreads();
   if (tid == 0) ch.last_cta = (atomicAdd(&a.counter[h], 1) == a.n_splits - 1);
   __syncthreads();
-  if (!ch.last_cta) return;
-  __threadfence();
+  if (ch.last_cta) {
+    __threadfence();
 
-  // ---- last CTA of the head: combine every split (partials first staged in shared
-  //      memory with coalesced loads, so the combine waits for one round trip) ----
-  const float* hp = a.part + (size_t)h * a.n_splits * kPartStride;
-  const int nwords = a.n_splits * kPartStride;
-  const bool staged = (size_t)nwords * sizeof(float) <= (size_t)kW * kRingS;
-  float* stp = reinterpret_cast<float*>(rings);
-  if (staged) {
-    for (int i = tid; i < nwords; i += kNT) stp[i] = __ldcg(hp + i);
-    __syncthreads();
+    // ---- last CTA of the head: combine every split (partials first staged in shared
+    //      memory with coalesced loads, so the combine waits for one round trip) ----
+    const float* hp = a.part + (size_t)h * a.n_splits * kPartStride;
+    const int nwords = a.n_splits * kPartStride;
+    const bool staged = (size_t)nwords * sizeof(float) <= (size_t)kW * kRingS;
+    float* stp = reinterpret_cast<float*>(rings);
+    if (staged) {
+      for (int i = tid; i < nwords; i += kNT) stp[i] = __ldcg(hp + i);
+      __syncthreads();
+    }
+    auto ld = [&](int i) { return staged ? stp[i] : __ldcg(hp + i); };
+    if (tid < kD) {
+      float Mx = -INFINITY;
+      for (int s = 0; s < a.n_splits; ++s) Mx = fmaxf(Mx, ld(s * kPartStride));
+      float Lt = 0.f, St = 0.f, Ut = 0.f, mt = 0.f;
+      for (int s = 0; s < a.n_splits; ++s) {
+        const int pp = s * kPartStride;
+        Ut += ld(pp + 4 + kD + tid);
+        mt += ld(pp + 2);
+        const float ms = ld(pp);
+        if (ms == -INFINITY) continue;
+        const float e = ex2(ms - Mx);
+        Lt = fmaf(ld(pp + 1), e, Lt);
+        St = fmaf(ld(pp + 4 + tid), e, St);
+      }
+      const float op = a.o_prev[(size_t)h * kD + tid];
+      const float u = op - Ut;
+      a.o[(size_t)h * kD + tid] = Lt > 0.f ? fmaf(mt, St / Lt, u) : u;
+      arr<float>(c, A_UNSEL, a.layer)[(size_t)h * kD + tid] = u;
+      if (tid == 0) {
+        arr<float>(c, A_MASS, a.layer)[h] = mt;
+        arr<float>(c, A_OFFSET, a.layer)[(size_t)h * kOffStride + r] = Mx + log2f(Lt) - log2f(mt);
+        a.counter[h] = 0;
+      }
+    }
   }
-  auto ld = [&](int i) { return staged ? stp[i] : __ldcg(hp + i); };
-  if (tid < kD) {
-    float Mx = -INFINITY;
-    for (int s = 0; s < a.n_splits; ++s) Mx = fmaxf(Mx, ld(s * kPartStride));
-    float Lt = 0.f, St = 0.f, Ut = 0.f, mt = 0.f;
-    for (int s = 0; s < a.n_splits; ++s) {
-      const int pp = s * kPartStride;
-      Ut += ld(pp + 4 + kD + tid);
-      mt += ld(pp + 2);
-      const float ms = ld(pp);
-      if (ms == -INFINITY) continue;
-      const float e = ex2(ms - Mx);
-      Lt = fmaf(ld(pp + 1), e, Lt);
-      St = fmaf(ld(pp + 4 + tid), e, St);
-    }
-    const float op = a.o_prev[(size_t)h * kD + tid];
-    const float u = op - Ut;
-    a.o[(size_t)h * kD + tid] = Lt > 0.f ? fmaf(mt, St / Lt, u) : u;
-    arr<float>(c, A_UNSEL, a.layer)[(size_t)h * kD + tid] = u;
-    if (tid == 0) {
-      arr<float>(c, A_MASS, a.layer)[h] = mt;
-      arr<float>(c, A_OFFSET, a.layer)[(size_t)h * kOffStride + r] = Mx + log2f(Lt) - log2f(mt);
-      a.counter[h] = 0;
-    }
+  if constexpr (kFlush) {
+    __syncthreads();  // the combine is done with shared memory
+    flush_tail(a, blockIdx.y * gridDim.x + blockIdx.x, gridDim.x * gridDim.y, *reinterpret_cast<EncodeSmem*>(smem),
+               tid, kNT);
   }
 }
 
@@ -585,15 +594,18 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s) {
   const int n = staged_splits(a.c.H, a.k_sel, ps, sms > 0 ? sms : 148);
   if (a.r > kStoresMax || sms == 0 || n > kMaxSplits) return launch_sparse_direct(a, s);
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(sparse_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCta);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(sparse_staged_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
+    for (auto k : {sparse_staged_kernel<false>, sparse_staged_kernel<true>}) {
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCta);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return e;
+    }
     attr_set[dev] = true;
   }
   a.n_splits = n;
   dim3 grid(n, a.c.H);
-  return launch_pdl(sparse_staged_kernel, grid, dim3(kNT), (size_t)kSmemCta, s, a);
+  return launch_pdl(a.flush ? sparse_staged_kernel<true> : sparse_staged_kernel<false>, grid, dim3(kNT),
+                    (size_t)kSmemCta, s, a);
 }
 
 }  // namespace fl

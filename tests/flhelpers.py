@@ -117,42 +117,65 @@ class Pair:
         del d
 
     # -- decode --------------------------------------------------------------------
+    def _note_flush(self):
+        """The residual slots a flush of the current full tail takes (for compare_encoding)."""
+        for r in range(2, self.w.loops + 1):
+            slot0 = round_up(self.cache.n_slots[0][r])
+            self.calls[r].append((slot0, sum(1 for dep in self.cache.tail_depth if dep >= r)))
+
     def begin_token(self, step: int):
         """Append decode token ``step`` (flushing a full tail first) on both sides."""
         w, hs = self.w, self.heads
         if self.cache.n_tail == 64:
-            for r in range(2, w.loops + 1):
-                slot0 = round_up(self.cache.n_slots[0][r])
-                self.calls[r].append((slot0, sum(1 for dep in self.cache.tail_depth if dep >= r)))
+            self._note_flush()
         self.cache.begin_token()
         tok = synth.decode_token(w, self.layer, step, device="cuda")
         self.oracle.append_token([None] + [f32(tok["k"][r][hs]) for r in range(1, w.loops + 1)],
                                  [None] + [f32(tok["v"][r][hs]) for r in range(1, w.loops + 1)])
         return tok
 
-    def run_loops(self, q, tok=None, k_sel=None, loops=None, check=True):
-        """Every loop of one decode step on the GPU and in the oracle; returns per-loop errors."""
+    def run_loops(self, q, tok=None, k_sel=None, loops=None, check=True, fused=False):
+        """Every loop of one decode step on the GPU and in the oracle; returns per-loop errors.
+
+        With ``fused`` the GPU side runs each loop through the step executor, and a full
+        tail is flushed by the step's own readers (fl_decode_step_flush)."""
         w, hs, c, lay = self.w, self.heads, self.cache, self.oracle
         H = w.heads
         N = c.n_cols
         k_sel = w.k_sel(N) if k_sel is None else k_sel
         errs = {}
         o_prev = None
+        flush = fused and c.n_tail == 64
+        if fused:
+            if flush:
+                self._note_flush()
+            R = w.loops
+            Q = q[:, None].contiguous()
+            O = torch.zeros(R + 1, 1, H, 128, dtype=torch.float32, device="cuda")
+            zero = torch.zeros(H, 128, dtype=torch.bfloat16, device="cuda")
+            KN = torch.stack([zero] + [tok["k"][r] for r in range(1, R + 1)])[:, None].contiguous() if tok else None
+            VN = torch.stack([zero] + [tok["v"][r] for r in range(1, R + 1)])[:, None].contiguous() if tok else None
         for r in range(1, (loops or w.loops) + 1):
             o = torch.empty(H, 128, dtype=torch.float32, device="cuda")
             kn = tok["k"][r] if tok else None
             vn = tok["v"][r] if tok else None
             qr = q[r].contiguous()
+            if fused:
+                c.step(w.dense_loops, k_sel, Q, O, KN, VN, loop_first=r, loop_last=r, flush=flush)
+                o = O[r, 0]
             if r <= w.dense_loops:
-                c.dense(0, r, qr, o, kn, vn, keep_scores=True)
+                if not fused:
+                    c.dense(0, r, qr, o, kn, vn, keep_scores=True)
                 ref = lay.dense_loop(r, f32(q[r][hs]))
                 errs[r] = rel_err(o.cpu().numpy()[hs], ref["o"])
             else:
-                c.select(0, 1, r, k_sel)
+                if not fused:
+                    c.select(0, 1, r, k_sel)
                 S, _, _ = selection(c, 0, k_sel)
                 if check:
                     check_topk_valid(S[hs], lay.p_tilde, k_sel)
-                c.sparse(0, r, k_sel, qr, o_prev, o, kn, vn)
+                if not fused:
+                    c.sparse(0, r, k_sel, qr, o_prev, o, kn, vn)
                 _, m, u = selection(c, 0, k_sel)
                 ref = lay.sparse_loop(r, f32(q[r][hs]), S[hs])
                 errs[(r, "m")] = float(np.max(np.abs(m[hs] - ref["m"]) / ref["m"]))
