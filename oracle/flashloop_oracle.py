@@ -27,6 +27,9 @@ Readings where the pages are silent (each listed again in the design notes):
 * residual key groups are 64 consecutive compact rows ("slots") of one encode
   call, per channel; a call's last group may be partial;
 * the BF16 tail holds the most recent 1..64 columns of every loop;
+* token-sparse updates rank the tokens of A_{r-1} by the squared relative L2 change
+  ||h^(r-1) - h^(r-2)||^2 / ||h^(r-2)||^2 of their hidden state over loop r-1, in
+  fp64, ties to the lower token;
 * sparse loop r re-selects from the spliced distribution of loop r-1, ties go
   to the smaller column index, and its output is
   o_r = u + m * softmax_S(q K_S^T / sqrt(d)) V_S with m the selected mass and u
@@ -227,6 +230,59 @@ def attention_sparse(q, Kc, Vc, S, m, u):
     pi = softmax(lS)
     o = np.asarray(u, F64) + np.asarray(m, F64)[:, None] * np.einsum("hk,hkd->hd", pi, VS)
     return o, pi, lS
+
+
+# ----------------------------------------------------------------------------
+# Cross-loop token-sparse updates  ([Project] "The Method", Step 01: only the
+# tokens that stay active are updated; [Guide] section 3 "Cross-loop token-sparse
+# updates": after the dense early loops each loop ranks the previously updated
+# tokens by normalized hidden-state change, keeps a top-k subset, and later
+# selections are restricted to earlier active sets, so the sets nest)
+# ----------------------------------------------------------------------------
+def token_change(h_prev, h_cur) -> np.ndarray:
+    """Squared normalized hidden-state change of each token row, fp64:
+
+        key_j = ||h_cur[j] - h_prev[j]||^2 / ||h_prev[j]||^2
+
+    (delta_j^2; ranking by it is ranking by delta_j).  BF16 inputs widen exactly to
+    fp64.  A row whose previous state is all zero has key +inf when it changed and 0
+    when it did not.
+    """
+    hp = np.asarray(h_prev, F64)
+    hc = np.asarray(h_cur, F64)
+    num = np.sum((hc - hp) ** 2, axis=-1)
+    den = np.sum(hp ** 2, axis=-1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        key = num / den
+    return np.where((den == 0) & (num == 0), 0.0, key)
+
+
+def select_active(h_prev, h_cur, prev_rows, k: int) -> np.ndarray:
+    """A_r from A_{r-1}: the k tokens of ``prev_rows`` (those updated in loop r-1)
+    whose hidden state changed most in loop r-1, measured by ``token_change`` of
+    their states entering (h_prev = h^(r-2)) and leaving (h_cur = h^(r-1)) that
+    loop; ties go to the lower token; returned in ascending token order (int64).
+    """
+    prev_rows = np.asarray(prev_rows, np.int64)
+    assert 0 <= k <= prev_rows.size
+    key = token_change(np.asarray(h_prev)[prev_rows], np.asarray(h_cur)[prev_rows])
+    order = np.lexsort((prev_rows, -key))
+    return np.sort(prev_rows[order[:k]])
+
+
+def nested_active_sets(h, n_active) -> list:
+    """A_1 .. A_R from hidden states h[0..R-1] (h[0] enters loop 1, h[r] leaves loop r)
+    and the per-loop sizes n_active[r]: A_1 is every token; a loop whose size is not
+    smaller than its predecessor's keeps that set; otherwise A_r = select_active(
+    h[r-2], h[r-1], A_{r-1}, n_active[r]).  Entry 0 of the result is None.
+    """
+    n = np.asarray(h[0]).shape[0]
+    sets = [None, np.arange(n, dtype=np.int64)]
+    for r in range(2, len(n_active)):
+        prev = sets[r - 1]
+        k = min(int(n_active[r]), prev.size)
+        sets.append(prev.copy() if k == prev.size else select_active(h[r - 2], h[r - 1], prev, k))
+    return sets
 
 
 # ----------------------------------------------------------------------------

@@ -13,6 +13,7 @@ from .gen import (  # noqa: F401
     depth_of,
     prefill_layer,
     decode_token,
+    hidden_states,
     queries,
     split_prefill,
 )

@@ -178,6 +178,27 @@ def decode_token(w: Workload, layer: int, step: int, device="cpu") -> dict:
     return {"k": k, "v": v}
 
 
+def hidden_states(w: Workload, n_tokens: int, d_model: int, device="cpu", loops=None) -> list:
+    """Hidden states for the token selector: h[0..R-1], BF16 [n_tokens][d_model].
+
+    h[0] enters loop 1 and h[r] leaves loop r: h[0] = bf16(N(0,1)) and
+    h[r] = bf16(h[r-1] + c_r g_{r,j} N(0,1)) with c_1 = 1, c_r = sigma_r for r >= 2 and
+    a per-token magnitude g_{r,j} = exp(N(0,1)), so a few tokens move much more than the
+    rest.  Every row is drawn as if its token were updated in every loop; a selector
+    reads only the rows of the tokens it ranks.
+    """
+    R = w.loops if loops is None else loops
+    g = _generator(device, "hidden", w.seed, n_tokens, d_model)
+    h = [_bf16_normal((n_tokens, d_model), g, device)]
+    for r in range(1, R):
+        c = 1.0 if r == 1 else float(w.sigma[r])
+        mag = torch.exp(torch.randn(n_tokens, generator=g, device=device, dtype=torch.float32))
+        noise = torch.randn((n_tokens, d_model), generator=g, device=device, dtype=torch.float32)
+        h.append((h[-1].float() + (c * mag)[:, None] * noise).to(torch.bfloat16))
+        del noise
+    return h
+
+
 def queries(w: Workload, layer: int, step: int, device="cpu") -> torch.Tensor:
     """BF16 queries [R + 1][H][128] (row 0 unused) for one decode step of one layer."""
     g = _generator(device, "query", w.layer_seed(layer), step)

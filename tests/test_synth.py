@@ -54,3 +54,13 @@ def test_prefill_changes_only_active_rows():
         assert bool(same[~act].all()) and not bool(same[act].all())
     q = synth.queries(w, 0, 3)
     assert q.shape == (5, 1, 128) and not q[0].any()
+
+
+def test_hidden_states_are_seeded_bf16_and_move_each_loop():
+    w = synth.WORKLOADS["tiny_h1_n256"]
+    a = synth.hidden_states(w, 50, 32)
+    b = synth.hidden_states(w, 50, 32)
+    assert len(a) == w.loops and all(t.dtype == torch.bfloat16 and t.shape == (50, 32) for t in a)
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    for r in range(1, w.loops):
+        assert not torch.equal(a[r], a[r - 1])
