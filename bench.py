@@ -325,10 +325,57 @@ def run_gpu(args, rank, world):
     d_gbs = d_bytes / (d_launch_us * 1e-6) / 1e9
 
     e2e = run_e2e(step, cache, wr, layers, inputs[total_steps:], device) if args.e2e_steps else None
+    del inputs, step, cache
+    tokens = run_token_select(wr, device, hbm) if args.token_select else None
     return dict(metric_us=metric_us, step_ms=step_ms, seg=mean, clocks=clocks, launches=launches / args.steps,
                 sp_bytes=sp_bytes, sp_launch_us=sp_launch_us, sp_gbs=sp_gbs, d_bytes=d_bytes,
                 d_launch_us=d_launch_us, d_gbs=d_gbs, hbm=hbm, peak_kind=peak_kind, N=N, k_sel=k_sel,
-                layers=layers, setup_s=setup_s, e2e=e2e, w=wr)
+                layers=layers, setup_s=setup_s, e2e=e2e, w=wr, tokens=tokens)
+
+
+def run_token_select(w, device, hbm, reps=5):
+    """The token-sparse update selector (fl_select_active) on the workload's prompt with a
+    hidden state of H x 128 = 2048 BF16 per token: the loop-3 ranking (A_3, 25 %, from
+    every token) and the loop-4 ranking (A_4, 10 %, from A_3).  CUDA events on the launch
+    stream, L2 flushed before each timed call; the change kernel alone is the k = 0 call
+    (keys only), whose bytes are both hidden-state rows of every candidate."""
+    from quantized_kv_attention_int4_b200 import abi
+    from quantized_kv_attention_int4_b200.tokens import nested_active_sets
+
+    n, d = w.n_ctx, w.heads * 128
+    h = synth.hidden_states(w, n, d, device=device)
+    sizes = [0] + [w.n_active(r, n) for r in range(1, w.loops + 1)]
+    sets = nested_active_sets(h, sizes)
+    keys = torch.empty(n, dtype=torch.float64, device=device)
+    out3 = torch.empty(sizes[3], dtype=torch.int32, device=device)
+    out4 = torch.empty(sizes[4], dtype=torch.int32, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    calls = {
+        "change": lambda: abi.fl_select_active(h[1], h[2], sets[2], 0, None, keys),
+        "a3": lambda: abi.fl_select_active(h[1], h[2], sets[2], sizes[3], out3, keys),
+        "a4": lambda: abi.fl_select_active(h[2], h[3], out3, sizes[4], out4, keys),
+    }
+    times = {k: [] for k in calls}
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for rep in range(reps + 1):
+        for name, fn in calls.items():
+            flush.zero_()
+            ev[0].record()
+            fn()
+            ev[1].record()
+            torch.cuda.synchronize()
+            if rep:
+                times[name].append(ev[0].elapsed_time(ev[1]) * 1e3)
+    assert torch.equal(out3, sets[3]) and torch.equal(out4, sets[4])
+    t = {k: float(np.mean(v)) for k, v in times.items()}
+    nbytes = n * d * 2 * 2 + n * (4 + 8)
+    gbs = nbytes / (t["change"] * 1e-6) / 1e9
+    del h, flush
+    return {"bound": "hbm", "kernel": f"token_change_kernel (loop-3 ranking over {n} tokens x {d})",
+            "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+            "traffic": _kernel_traffic("token_change_kernel"), "bytes_per_launch": nbytes,
+            "us_per_launch": t["change"], "a3_us": t["a3"], "a4_us": t["a4"],
+            "select_us_a3": t["a3"] - t["change"]}
 
 
 def run_e2e(step, cache, w, layers, inputs, device):
@@ -457,6 +504,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-token-select", dest="token_select", action="store_false",
+                    help="skip the token-sparse update selector measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -516,6 +565,7 @@ def main():
         "roofline_dense": {"bound": "hbm", "kernel": "fl_decode_attn_dense (loops 1-2)", "achieved": r["d_gbs"],
                            "peak": hbm, "unit": "GB/s", "frac": r["d_gbs"] / hbm, "traffic": _kernel_traffic("dense_staged_kernel"),
                            "bytes_per_launch": r["d_bytes"], "us_per_launch": r["d_launch_us"]},
+        "roofline_token_select": r["tokens"],
         "segments_ms": r["seg"], "clocks": r["clocks"], "gpu_launches": r["launches"],
         "e2e": r["e2e"], "cpu_baseline": cpu, "setup_s": r["setup_s"],
     }

@@ -301,6 +301,31 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
                                const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,
                                void* const* events, const fl_flush* flush, void* stream);
 
+/* [Project] Step 01; [Guide] section 3 (cross-loop token-sparse updates: after the dense
+ * early loops each loop ranks the tokens updated in the previous loop by normalized
+ * hidden-state change and keeps a top-k subset, so the active sets nest).  A_r from
+ * A_{r-1}: for the n_rows candidate tokens `rows` (device int32, strictly ascending:
+ * A_{r-1}) compute
+ *     keys[i] = ||h_cur[j] - h_prev[j]||^2 / ||h_prev[j]||^2,   j = rows[i]
+ * (fp64 sums of the exactly widened BF16 values; 0 when both norms are 0, +inf when only
+ * the previous state is 0), and write the k candidates with the largest key -- ties to
+ * the lower token -- to rows_out in ascending token order (A_r, ready to be the `rows` of
+ * fl_encode_residual).  Ranking by the squared ratio is ranking by the ratio.
+ *   h_prev: the state entering loop r-1 (h^(r-2)); h_cur: the state leaving it (h^(r-1));
+ *           BF16 [n_tokens][d_model], rows `row_stride` elements apart; 16-byte aligned,
+ *           d_model and row_stride multiples of 8, d_model <= row_stride.
+ *   keys: device fp64 [n_rows], caller-owned: receives every candidate's key (it is also
+ *         the selector's scratch).  rows_out: device int32 [k].  0 <= k <= n_rows.
+ *   status: NULL or device int32[3] (first error code, detail, count) receiving
+ *           FL_DEV_ROWS_RANGE for a candidate outside [0, n_tokens) -- its key is NaN and
+ *           it ranks below every valid one -- or FL_DEV_ROWS_ORDER for a candidate not
+ *           above its predecessor (still ranked).
+ * Two launches on `stream` (per-token change, HBM-bound; one-CTA radix select); nothing
+ * is allocated. */
+fl_status fl_select_active(const uint16_t* h_prev, const uint16_t* h_cur, int32_t n_tokens,
+                           int32_t d_model, int64_t row_stride, const int32_t* rows, int32_t n_rows,
+                           int32_t k, int32_t* rows_out, double* keys, int32_t* status, void* stream);
+
 /* Synchronise `stream`, copy the cache's status words to host `out[0..2]`, and return
  * FL_ERR_DEVICE if a kernel recorded an error (FL_OK otherwise).  With `clear` != 0
  * the words are zeroed afterwards. */

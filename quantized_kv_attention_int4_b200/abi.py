@@ -30,10 +30,12 @@ ARRAY_NAMES = ("brec", "rrec", "mask", "first", "depth", "tail_k", "tail_v", "sc
 GROUP_RECORD = 9216
 
 FL_OK, FL_ERR_INVALID, FL_ERR_UNSUPPORTED, FL_ERR_CUDA, FL_ERR_WORKSPACE, FL_ERR_DEVICE = 0, -1, -2, -3, -4, -6
+# device error codes recorded in status words (include/flashloop.h)
+FL_DEV_ROWS_ORDER, FL_DEV_ROWS_RANGE, FL_DEV_NOT_NESTED, FL_DEV_SEL_RANGE, FL_DEV_TAG_RANGE, FL_DEV_TIMEOUT = 1, 2, 3, 4, 5, 6
 EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init", "fl_workspace_bytes",
             "fl_workspace_init", "fl_write_tail", "fl_encode_base", "fl_encode_residual",
             "fl_decode_attn_dense", "fl_select_topk", "fl_decode_attn_sparse", "fl_decode_step",
-            "fl_read_status", "fl_decode_attn_sparse_noalloc", "fl_decode_step_flush")
+            "fl_read_status", "fl_decode_attn_sparse_noalloc", "fl_decode_step_flush", "fl_select_active")
 
 
 class fl_dims(ctypes.Structure):
@@ -87,6 +89,7 @@ _c_step = _sig("fl_decode_step", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P
                 ctypes.POINTER(ctypes.c_void_p), _P)
 _c_step_flush = _sig("fl_decode_step_flush", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(fl_flush), _P)
+_c_select_active = _sig("fl_select_active", _I, _P, _P, _I, _I, _L, _P, _I, _I, _P, _P, _P, _P)
 _c_read_status = _sig("fl_read_status", _I, _DP, _P, ctypes.POINTER(ctypes.c_int32), _I, _P)
 
 
@@ -273,6 +276,26 @@ def fl_decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loo
         _check("fl_decode_step", _c_step(*args, _stream(stream)))
     else:
         _check("fl_decode_step_flush", _c_step_flush(*args, ctypes.byref(flush), _stream(stream)))
+
+
+def fl_select_active(h_prev, h_cur, rows, k, rows_out, keys, status=None, stream=None):
+    """A_r from A_{r-1}: the k tokens of ``rows`` (int32, ascending) whose hidden state
+    changed most between h_prev and h_cur (BF16 [n_tokens][d], unit-stride rows), written
+    ascending to rows_out (int32 [>= k]); keys (fp64 [>= len(rows)]) receives every
+    candidate's squared relative change."""
+    for t, name in ((h_prev, "h_prev"), (h_cur, "h_cur")):
+        if t.dim() != 2 or t.stride(1) != 1:
+            raise ValueError(f"{name} must be [n_tokens][d] with unit-stride rows")
+    if h_prev.shape != h_cur.shape or h_prev.stride() != h_cur.stride():
+        raise ValueError("h_prev and h_cur must have the same shape and strides")
+    n = rows.numel()
+    if keys.numel() < n or (k > 0 and rows_out.numel() < k):
+        raise ValueError("keys must hold len(rows) entries and rows_out k entries")
+    _check("fl_select_active", _c_select_active(
+        _ptr(h_prev, torch.bfloat16, "h_prev"), _ptr(h_cur, torch.bfloat16, "h_cur"), h_prev.shape[0],
+        h_prev.shape[1], h_prev.stride(0), _ptr(rows, torch.int32, "rows"), n, k,
+        _ptr(rows_out, torch.int32, "rows_out"), _ptr(keys, torch.float64, "keys"),
+        _ptr(status, torch.int32, "status"), _stream(stream)))
 
 
 def fl_read_status(dims, cache, clear=True, stream=None):

@@ -509,6 +509,30 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
   return FL_OK;
 }
 
+fl_status fl_select_active(const uint16_t* h_prev, const uint16_t* h_cur, int32_t n_tokens, int32_t d_model,
+                           int64_t row_stride, const int32_t* rows, int32_t n_rows, int32_t k, int32_t* rows_out,
+                           double* keys, int32_t* status, void* stream) {
+  if (n_tokens < 1 || d_model < 8 || d_model % 8 || row_stride < d_model || row_stride % 8) return FL_ERR_INVALID;
+  if (n_rows < 0 || n_rows > n_tokens || k < 0 || k > n_rows) return FL_ERR_INVALID;
+  if (n_rows > 0 && (!h_prev || !h_cur || !rows || !keys || !aligned16(h_prev) || !aligned16(h_cur)))
+    return FL_ERR_INVALID;
+  if (k > 0 && !rows_out) return FL_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(keys) % 8 || reinterpret_cast<uintptr_t>(status) % 4) return FL_ERR_INVALID;
+  TokenArgs a;
+  a.h_prev = h_prev;
+  a.h_cur = h_cur;
+  a.row_stride = row_stride;
+  a.d_model = d_model;
+  a.n_tokens = n_tokens;
+  a.rows = rows;
+  a.n_rows = n_rows;
+  a.k = k;
+  a.rows_out = rows_out;
+  a.keys = keys;
+  a.status = status;
+  return cuda_status(launch_token_select(a, (cudaStream_t)stream));
+}
+
 fl_status fl_read_status(const fl_dims* dims, void* cache, int32_t* out, int32_t clear, void* stream) {
   fl_layout L;
   fl_status st = make_layout(dims, &L);

@@ -44,6 +44,19 @@ struct SelectArgs {
   int layer0, r, n_q, n_tail, k_sel;
 };
 
+struct TokenArgs {
+  const uint16_t* h_prev;   // BF16 [n_tokens][row_stride]: state entering the ranked loop
+  const uint16_t* h_cur;    // BF16 [n_tokens][row_stride]: state leaving it
+  int64_t row_stride;
+  int32_t d_model, n_tokens;
+  const int32_t* rows;      // candidates, ascending
+  int64_t n_rows;
+  int32_t k;
+  int32_t* rows_out;        // [k]
+  double* keys;             // [n_rows]
+  int32_t* status;          // optional device int32[3]
+};
+
 cudaError_t launch_encode_base(const EncodeBaseArgs& a, cudaStream_t s);
 cudaError_t launch_encode_residual(const EncodeResArgs& a, cudaStream_t s);
 // chain = false: an ordinary stream-ordered launch (no programmatic overlap with the
@@ -53,6 +66,7 @@ cudaError_t launch_dense_direct(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s);
+cudaError_t launch_token_select(const TokenArgs& a, cudaStream_t s);
 
 int dense_splits(int heads, int n_q);
 int sparse_splits(int heads, int k_sel, int loops);
