@@ -286,6 +286,35 @@ def nested_active_sets(h, n_active) -> list:
 
 
 # ----------------------------------------------------------------------------
+# Sparse prefill attention  ([Project] "The Method", Step 01: in a token-sparse
+# loop only the active tokens are recomputed; the paragraph after Step 03: the
+# selected tokens are gathered into compact buffers so that the work stays a regular
+# GEMM)
+# ----------------------------------------------------------------------------
+def prefill_attention(q_act, pos, K, V) -> np.ndarray:
+    """Causal attention of the active tokens of one loop, fp64.
+
+    q_act [H][n_act][D]: the queries of the active tokens (compact, in token order);
+    pos [n_act]: their token positions (ascending); K, V [H][N][D]: every token's key
+    and value in this loop (an active token's new ones, an inactive token's reused
+    from the previous loop).  Row i attends over the keys 0..pos[i] with scale
+    1/sqrt(D); returns o [H][n_act][D].
+    """
+    q = np.asarray(q_act, F64)
+    K = np.asarray(K, F64)
+    V = np.asarray(V, F64)
+    pos = np.asarray(pos, np.int64)
+    H, n, D = q.shape
+    o = np.zeros((H, n, D), F64)
+    for i in range(n):
+        j = int(pos[i]) + 1
+        l = np.einsum("hd,hnd->hn", q[:, i], K[:, :j]) / np.sqrt(D)
+        p = softmax(l)
+        o[:, i] = np.einsum("hn,hnd->hd", p, V[:, :j])
+    return o
+
+
+# ----------------------------------------------------------------------------
 # One layer's cross-loop cache and decode state
 # ----------------------------------------------------------------------------
 class OracleLayer:
