@@ -326,6 +326,27 @@ fl_status fl_select_active(const uint16_t* h_prev, const uint16_t* h_cur, int32_
                            int32_t d_model, int64_t row_stride, const int32_t* rows, int32_t n_rows,
                            int32_t k, int32_t* rows_out, double* keys, int32_t* status, void* stream);
 
+/* [Project] "The Method", Step 01 (only the active tokens are recomputed in a
+ * token-sparse loop) and the closing paragraph (selected tokens gathered into compact
+ * buffers so the work stays a regular GEMM).  Sparse prefill attention of one loop: the
+ * n_act active tokens' queries attend causally over every token's key and value,
+ *     o[h][i] = softmax_{j <= pos[i]}(q[h][i] . k[h][j] / sqrt(128)) v[h][j],
+ * on the tensor cores (BF16 operands, fp32 accumulation; the probabilities are rounded
+ * to BF16 for the value product and the row sum uses the rounded values).
+ *   q: BF16 [heads][n_act][128] (compact, in token order; head stride q_head_stride
+ *      elements); pos: device int32 [n_act], strictly ascending, in [0, n_tokens);
+ *   k, v: BF16 [heads][n_tokens][128] (head stride kv_head_stride): each token's key and
+ *      value in this loop (an inactive token's reused from the previous loop);
+ *   o: fp32 [heads][n_act][128] (head stride o_head_stride), written for every row.
+ * Rows are 128 elements apart; pointers 16-byte aligned; head strides multiples of 8.
+ * status: NULL or device int32[3] receiving FL_DEV_ROWS_RANGE / FL_DEV_ROWS_ORDER for a
+ * bad position (that row attends over nothing and is left unwritten) or FL_DEV_TIMEOUT
+ * (a bounded wait for the tensor cores ran out).  One launch; nothing is allocated. */
+fl_status fl_prefill_attn_sparse(const uint16_t* q, const int32_t* pos, int32_t n_act, const uint16_t* k,
+                                 const uint16_t* v, int32_t n_tokens, int32_t heads, int64_t q_head_stride,
+                                 int64_t kv_head_stride, float* o, int64_t o_head_stride, int32_t* status,
+                                 void* stream);
+
 /* Synchronise `stream`, copy the cache's status words to host `out[0..2]`, and return
  * FL_ERR_DEVICE if a kernel recorded an error (FL_OK otherwise).  With `clear` != 0
  * the words are zeroed afterwards. */

@@ -35,7 +35,8 @@ FL_DEV_ROWS_ORDER, FL_DEV_ROWS_RANGE, FL_DEV_NOT_NESTED, FL_DEV_SEL_RANGE, FL_DE
 EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init", "fl_workspace_bytes",
             "fl_workspace_init", "fl_write_tail", "fl_encode_base", "fl_encode_residual",
             "fl_decode_attn_dense", "fl_select_topk", "fl_decode_attn_sparse", "fl_decode_step",
-            "fl_read_status", "fl_decode_attn_sparse_noalloc", "fl_decode_step_flush", "fl_select_active")
+            "fl_read_status", "fl_decode_attn_sparse_noalloc", "fl_decode_step_flush", "fl_select_active",
+            "fl_prefill_attn_sparse")
 
 
 class fl_dims(ctypes.Structure):
@@ -90,6 +91,7 @@ _c_step = _sig("fl_decode_step", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P
 _c_step_flush = _sig("fl_decode_step_flush", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                       ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(fl_flush), _P)
 _c_select_active = _sig("fl_select_active", _I, _P, _P, _I, _I, _L, _P, _I, _I, _P, _P, _P, _P)
+_c_prefill = _sig("fl_prefill_attn_sparse", _I, _P, _P, _I, _P, _P, _I, _I, _L, _L, _P, _L, _P, _P)
 _c_read_status = _sig("fl_read_status", _I, _DP, _P, ctypes.POINTER(ctypes.c_int32), _I, _P)
 
 
@@ -296,6 +298,23 @@ def fl_select_active(h_prev, h_cur, rows, k, rows_out, keys, status=None, stream
         h_prev.shape[1], h_prev.stride(0), _ptr(rows, torch.int32, "rows"), n, k,
         _ptr(rows_out, torch.int32, "rows_out"), _ptr(keys, torch.float64, "keys"),
         _ptr(status, torch.int32, "status"), _stream(stream)))
+
+
+def fl_prefill_attn_sparse(q, pos, k, v, o, status=None, stream=None):
+    """Causal attention of the active tokens: q BF16 [H][n_act][128] (compact), pos int32
+    [n_act] (ascending token positions), k, v BF16 [H][N][128], o fp32 [H][n_act][128]."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        if t.dim() != 3 or t.shape[2] != HEAD_DIM or t.stride(2) != 1 or t.stride(1) != HEAD_DIM:
+            raise ValueError(f"{name} must be [H][n][128] with contiguous rows")
+    H, n_act = q.shape[0], q.shape[1]
+    if k.shape != v.shape or k.stride() != v.stride() or k.shape[0] != H or o.shape[:2] != q.shape[:2]:
+        raise ValueError("q, k, v, o shapes do not agree")
+    if pos.numel() != n_act:
+        raise ValueError("pos must hold one position per query row")
+    _check("fl_prefill_attn_sparse", _c_prefill(
+        _ptr(q, torch.bfloat16, "q"), _ptr(pos, torch.int32, "pos"), n_act, _ptr(k, torch.bfloat16, "k"),
+        _ptr(v, torch.bfloat16, "v"), k.shape[1], H, q.stride(0), k.stride(0), _ptr(o, torch.float32, "o"),
+        o.stride(0), _ptr(status, torch.int32, "status"), _stream(stream)))
 
 
 def fl_read_status(dims, cache, clear=True, stream=None):

@@ -533,6 +533,36 @@ fl_status fl_select_active(const uint16_t* h_prev, const uint16_t* h_cur, int32_
   return cuda_status(launch_token_select(a, (cudaStream_t)stream));
 }
 
+fl_status fl_prefill_attn_sparse(const uint16_t* q, const int32_t* pos, int32_t n_act, const uint16_t* k,
+                                 const uint16_t* v, int32_t n_tokens, int32_t heads, int64_t q_head_stride,
+                                 int64_t kv_head_stride, float* o, int64_t o_head_stride, int32_t* status,
+                                 void* stream) {
+  if (n_act < 0 || n_tokens < 1 || heads < 1 || n_act > n_tokens) return FL_ERR_INVALID;
+  if (n_act == 0) return FL_OK;
+  if (!q || !pos || !k || !v || !o) return FL_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FL_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(pos) % 4 || reinterpret_cast<uintptr_t>(status) % 4) return FL_ERR_INVALID;
+  if (q_head_stride % 8 || kv_head_stride % 8 || o_head_stride % 4) return FL_ERR_INVALID;
+  if (heads > 1 && (q_head_stride < (int64_t)n_act * FL_HEAD_DIM || kv_head_stride < (int64_t)n_tokens * FL_HEAD_DIM ||
+                    o_head_stride < (int64_t)n_act * FL_HEAD_DIM))
+    return FL_ERR_INVALID;
+  if ((int64_t)heads > 65535) return FL_ERR_UNSUPPORTED;
+  PrefillArgs a;
+  a.q = q;
+  a.pos = pos;
+  a.n_act = n_act;
+  a.n_tokens = n_tokens;
+  a.heads = heads;
+  a.k = k;
+  a.v = v;
+  a.q_head_stride = q_head_stride;
+  a.kv_head_stride = kv_head_stride;
+  a.o_head_stride = o_head_stride;
+  a.o = o;
+  a.status = status;
+  return cuda_status(launch_prefill_attn(a, (cudaStream_t)stream));
+}
+
 fl_status fl_read_status(const fl_dims* dims, void* cache, int32_t* out, int32_t clear, void* stream) {
   fl_layout L;
   fl_status st = make_layout(dims, &L);

@@ -57,6 +57,17 @@ struct TokenArgs {
   int32_t* status;          // optional device int32[3]
 };
 
+struct PrefillArgs {
+  const uint16_t* q;        // BF16 [heads][n_act][128]: the active tokens' queries
+  const int32_t* pos;       // [n_act] their token positions, ascending
+  int32_t n_act, n_tokens, heads;
+  const uint16_t* k;        // BF16 [heads][n_tokens][128]
+  const uint16_t* v;
+  int64_t q_head_stride, kv_head_stride, o_head_stride;
+  float* o;                 // fp32 [heads][n_act][128]
+  int32_t* status;          // optional device int32[3]
+};
+
 cudaError_t launch_encode_base(const EncodeBaseArgs& a, cudaStream_t s);
 cudaError_t launch_encode_residual(const EncodeResArgs& a, cudaStream_t s);
 // chain = false: an ordinary stream-ordered launch (no programmatic overlap with the
@@ -67,6 +78,7 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s);
 cudaError_t launch_token_select(const TokenArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_attn(const PrefillArgs& a, cudaStream_t s);
 
 int dense_splits(int heads, int n_q);
 int sparse_splits(int heads, int k_sel, int loops);
