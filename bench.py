@@ -327,10 +327,11 @@ def run_gpu(args, rank, world):
     e2e = run_e2e(step, cache, wr, layers, inputs[total_steps:], device) if args.e2e_steps else None
     del inputs, step, cache
     tokens = run_token_select(wr, device, hbm) if args.token_select else None
+    prefill = run_prefill(wr, device) if args.prefill else None
     return dict(metric_us=metric_us, step_ms=step_ms, seg=mean, clocks=clocks, launches=launches / args.steps,
                 sp_bytes=sp_bytes, sp_launch_us=sp_launch_us, sp_gbs=sp_gbs, d_bytes=d_bytes,
                 d_launch_us=d_launch_us, d_gbs=d_gbs, hbm=hbm, peak_kind=peak_kind, N=N, k_sel=k_sel,
-                layers=layers, setup_s=setup_s, e2e=e2e, w=wr, tokens=tokens)
+                layers=layers, setup_s=setup_s, e2e=e2e, w=wr, tokens=tokens, prefill=prefill)
 
 
 def run_token_select(w, device, hbm, reps=5):
@@ -376,6 +377,49 @@ def run_token_select(w, device, hbm, reps=5):
             "traffic": _kernel_traffic("token_change_kernel"), "bytes_per_launch": nbytes,
             "us_per_launch": t["change"], "a3_us": t["a3"], "a4_us": t["a4"],
             "select_us_a3": t["a3"] - t["change"]}
+
+
+def _tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "of measured"
+    except Exception:
+        return 1590.0, "of fallback"
+
+
+def run_prefill(w, device, reps=5):
+    """Sparse prefill attention (fl_prefill_attn_sparse) on the workload's prompt: the loop-3
+    active tokens (25 %) of every head attend causally over all tokens, BF16 K/V of
+    H x N x 128.  Algorithmic FLOPs = 4 x 128 x (pos_i + 1) per active query and head (QK^T
+    and PV, two per multiply-add, masked keys not counted); CUDA events on the launch stream
+    after warm-up, inputs (2 x 134 MB of K/V) larger than L2."""
+    from quantized_kv_attention_int4_b200 import abi
+
+    n, H = w.n_ctx, w.heads
+    pos = synth.active_sets(w, n)[3].to(torch.int32)
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    k = torch.randn(H, n, 128, generator=g, device=device).to(torch.bfloat16)
+    v = torch.randn(H, n, 128, generator=g, device=device).to(torch.bfloat16)
+    q = torch.randn(H, pos.numel(), 128, generator=g, device=device).to(torch.bfloat16)
+    o = torch.empty(H, pos.numel(), 128, dtype=torch.float32, device=device)
+    pos_d = pos.to(device)
+    flops = 4.0 * 128 * H * float((pos.to(torch.float64) + 1).sum())
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ts = []
+    for rep in range(reps + 2):
+        ev[0].record()
+        abi.fl_prefill_attn_sparse(q, pos_d, k, v, o)
+        ev[1].record()
+        torch.cuda.synchronize()
+        if rep >= 2:
+            ts.append(ev[0].elapsed_time(ev[1]) * 1e3)
+    us = float(np.mean(ts))
+    tf = flops / (us * 1e-6) / 1e12
+    peak, kind = _tensor_peak()
+    del q, k, v, o
+    return {"bound": "tensor", "kernel": f"prefill_attn_kernel (tcgen05; {pos.numel()} of {n} tokens active, {H} heads)",
+            "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak, "peak_kind": kind,
+            "traffic": None, "flops_per_launch": flops, "us_per_launch": us}
 
 
 def run_e2e(step, cache, w, layers, inputs, device):
@@ -506,6 +550,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-token-select", dest="token_select", action="store_false",
                     help="skip the token-sparse update selector measurement")
+    ap.add_argument("--no-prefill", dest="prefill", action="store_false",
+                    help="skip the sparse prefill attention measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -566,6 +612,7 @@ def main():
                            "peak": hbm, "unit": "GB/s", "frac": r["d_gbs"] / hbm, "traffic": _kernel_traffic("dense_staged_kernel"),
                            "bytes_per_launch": r["d_bytes"], "us_per_launch": r["d_launch_us"]},
         "roofline_token_select": r["tokens"],
+        "roofline_prefill": r["prefill"],
         "segments_ms": r["seg"], "clocks": r["clocks"], "gpu_launches": r["launches"],
         "e2e": r["e2e"], "cpu_baseline": cpu, "setup_s": r["setup_s"],
     }

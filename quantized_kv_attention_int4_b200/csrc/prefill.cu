@@ -7,15 +7,19 @@
 // token's key and value of the loop:
 //     o_i = softmax_{j <= pos_i}(q_i k_j^T / sqrt(128)) v_j.
 //
-// One CTA of 4 warps per (128 active queries, head).  The query tile stays in shared
-// memory; key/value tiles of 128 tokens stream through it (cp.async, zero-filled past
-// the end).  Per key tile one thread issues S = Q K^T as 8 tcgen05.mma (M = N = 128,
-// K = 16, BF16 operands from 128-byte-swizzled shared memory, fp32 accumulator in
-// TMEM); warp w reads TMEM lanes 32w..32w+31, so thread t owns query row t: it masks,
-// runs the online softmax in the base-2 domain, writes P (BF16) back to shared memory
-// in the operand layout and rescales its row of the output accumulator in TMEM; then
-// O += P V as 8 more tcgen05.mma (V read MN-major).  Completion of each group of MMAs
-// is signalled by tcgen05.commit on an mbarrier; every wait is bounded.
+// One CTA of 8 warps per (128 active queries, head).  The query tile stays in shared
+// memory; key tiles of 128 tokens stream through three buffers (fetched two tiles
+// ahead) and value tiles through two (one tile ahead), by cp.async, zero-filled past the
+// end.  One thread issues S = Q K^T as 8
+// tcgen05.mma (M = N = 128, K = 16, BF16 operands from 128-byte-swizzled shared memory,
+// fp32 accumulators in TMEM) one tile ahead, into alternating TMEM buffers, so the
+// tensor cores compute the next scores while the warps run this tile's softmax.  Warp w
+// reads TMEM lanes 32 (w % 4) ..: thread t of warp w owns query row 32 (w % 4) + t and
+// the 64 columns of half w / 4 -- it masks, runs the online softmax in the base-2 domain,
+// writes its half of P (BF16) to shared memory in the operand layout and rescales its
+// half of the output accumulator row in TMEM; then O += P V as 8 more tcgen05.mma (V
+// read MN-major).  Each group of MMAs signals an mbarrier through tcgen05.commit; every
+// wait is bounded.
 #include "kernels.h"
 
 namespace fl {
@@ -23,18 +27,19 @@ namespace {
 
 constexpr int kPT = 128;                      // queries per tile = keys per tile = head dim
 constexpr int kTileB = kPT * kPT * 2;         // one 128 x 128 BF16 tile
-constexpr int kPrefillThreads = 128;
-constexpr int kTmemCols = 256;                // S: columns 0..127, O: 128..255
+constexpr int kPrefillThreads = 256;          // 8 warps: TMEM lane group w % 4, column half w / 4
+constexpr int kTmemCols = 512;                // S buffers: columns 0..127, 128..255; O: 256..383
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kPT >> 3) << 17) | ((kPT >> 4) << 24);
 constexpr uint32_t kIdescPV = kIdescS | (1u << 16);  // B (V) read MN-major
 
 struct PrefillCtl {
-  uint64_t bar_s, bar_o;
+  uint64_t bar_s[2], bar_o;
   uint32_t tmem;
-  int32_t pad;
-  int32_t qpos[kPT];
+  int32_t pmax;
+  float rmax[2][kPT];  // per column half: this tile's row maxima (exchanged within a row pair)
 };
-constexpr int kPrefillSmem = 4 * kTileB + (int)sizeof(PrefillCtl) + 1024;  // + alignment slack
+// the control block, then 1024-byte-aligned tiles: Q, K[3], V[2], P
+constexpr int kPrefillSmem = (int)sizeof(PrefillCtl) + 1023 + 7 * kTileB;
 
 // Byte offset of 16-byte chunk c (0..15) of row r in a 128 x 128 BF16 tile: two 64-column
 // blocks of 128 rows x 128 bytes (16 KB apart); within each 1024-byte group of 8 rows the
@@ -95,15 +100,23 @@ __device__ __forceinline__ void cp16_zfill(uint32_t dst, const void* src, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
 }
 
-// rows [row0, row0 + 128) of a BF16 [n][128] matrix into a swizzled tile (zero past n)
+// rows [row0, row0 + 128) of a BF16 [n][128] matrix into a swizzled tile (zero past n):
+// thread t copies chunk t % 16 of rows t / 16 + 16 i (rows 16 apart keep their swizzle
+// phase, so the shared-memory offset steps by 16 x 128 bytes)
 __device__ __forceinline__ void load_tile(uint32_t tile, const uint16_t* src, int row0, int n, int tid) {
-#pragma unroll 4
-  for (int it = 0; it < 16; ++it) {
-    const int r = it * 8 + (tid >> 4), c = tid & 15;
-    const bool ok = row0 + r < n;
-    cp16_zfill(tile + sw128(r, c), src + (size_t)(ok ? row0 + r : 0) * kD + c * 8, ok);
+  constexpr int kRowsPer = kPrefillThreads / 16;
+  const int r0 = tid >> 4, c = tid & 15;
+  const uint32_t d0 = tile + sw128(r0, c);
+  const uint16_t* s0 = src + (size_t)(row0 + r0) * kD + c * 8;
+#pragma unroll
+  for (int it = 0; it < kPT / kRowsPer; ++it) {
+    const bool ok = row0 + r0 + kRowsPer * it < n;
+    cp16_zfill(d0 + (uint32_t)(it * kRowsPer * 128), ok ? s0 + (size_t)it * kRowsPer * kD : src, ok);
   }
 }
+
+// barrier of the two warps (w, w + 4) that share TMEM lanes 32 w ..
+__device__ __forceinline__ void pair_bar(int grp) { asm volatile("bar.sync %0, 64;" ::"r"(grp + 1) : "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
@@ -112,34 +125,39 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(PrefillArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  PrefillCtl& ctl = *reinterpret_cast<PrefillCtl*>(smem_raw);
   const uint32_t raw = smem_addr(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;               // 1024-byte aligned tiles
+  const uint32_t base = (raw + (uint32_t)sizeof(PrefillCtl) + 1023u) & ~1023u;  // 1024-byte aligned tiles
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t sQ = base, sK = base + kTileB, sV = base + 2 * kTileB, sP = base + 3 * kTileB;
-  uint8_t* gP = gbase + 3 * kTileB;
-  PrefillCtl& ctl = *reinterpret_cast<PrefillCtl*>(gbase + 4 * kTileB);
+  const uint32_t sQ = base;
+  auto sK = [&](int t) { return base + (uint32_t)(1 + t % 3) * kTileB; };  // K(t): buffer t % 3
+  auto sV = [&](int t) { return base + (uint32_t)(4 + (t & 1)) * kTileB; };  // V(t): buffer t % 2
+  const uint32_t sP = base + 6u * kTileB;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = warp & 3, hf = warp >> 2;
+  const int row = 32 * grp + lane;  // this thread's query row = its TMEM lane
   const int h = blockIdx.y, i0 = blockIdx.x * kPT;
   const uint16_t* qh = a.q + (size_t)h * a.q_head_stride;
   const uint16_t* kh = a.k + (size_t)h * a.kv_head_stride;
   const uint16_t* vh = a.v + (size_t)h * a.kv_head_stride;
 
-  // this thread's query row and its position (-1: padding row or a bad position)
+  // the row's position (-1: a padding row or a bad position)
   int qp = -1;
-  if (i0 + tid < a.n_act) {
-    qp = __ldg(a.pos + i0 + tid);
-    const bool bad_order = i0 + tid > 0 && __ldg(a.pos + i0 + tid - 1) >= qp;
-    if (qp < 0 || qp >= a.n_tokens || bad_order) {
-      if (a.status) record_error(a.status, bad_order ? FL_DEV_ROWS_ORDER : FL_DEV_ROWS_RANGE, qp);
-      if (qp < 0 || qp >= a.n_tokens) qp = -1;
-    }
+  if (i0 + row < a.n_act) {
+    qp = __ldg(a.pos + i0 + row);
+    const bool bad_order = i0 + row > 0 && __ldg(a.pos + i0 + row - 1) >= qp;
+    const bool bad_range = qp < 0 || qp >= a.n_tokens;
+    if ((bad_order || bad_range) && hf == 0 && a.status)
+      record_error(a.status, bad_range ? FL_DEV_ROWS_RANGE : FL_DEV_ROWS_ORDER, qp);
+    if (bad_range) qp = -1;
   }
-  ctl.qpos[tid] = qp;
   if (tid == 0) {
-    mbar_init(&ctl.bar_s, 1);
+    mbar_init(&ctl.bar_s[0], 1);
+    mbar_init(&ctl.bar_s[1], 1);
     mbar_init(&ctl.bar_o, 1);
     fence_mbar_init();
+    ctl.pmax = -1;
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&ctl.tmem)),
@@ -147,96 +165,147 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  load_tile(sQ, qh, i0, a.n_act, tid);
-  asm volatile("cp.async.commit_group;" ::: "memory");
+  __syncthreads();
+  {
+    int m = qp;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+    if (lane == 0) atomicMax(&ctl.pmax, m);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl.tmem;
-  const uint32_t tS = tmem, tO = tmem + kPT;
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;     // this warp's TMEM lanes
-
-  int pmax = -1;  // the tile's last real position decides how many key tiles it needs
-  for (int r = 0; r < kPT; ++r) pmax = max(pmax, ctl.qpos[r]);
-  const int n_kt = pmax < 0 ? 0 : pmax / kPT + 1;
+  const uint32_t tO = tmem + 2 * kPT;
+  auto tS = [&](int b) { return tmem + (uint32_t)(b * kPT); };
+  const uint32_t lane_off = (uint32_t)(32 * grp) << 16;  // this warp's TMEM lanes
+  const int pmax = ctl.pmax;
+  const int n_kt = pmax < 0 ? 0 : pmax / kPT + 1;  // key tiles up to the tile's last position
   const float kScale = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
 
-  float m_run = -INFINITY, l_run = 0.f;
-  unsigned ph_s = 0, ph_o = 0;
-  bool ok = true;
-  uint64_t* pend = nullptr;  // the barrier whose commit is still outstanding after a failed wait
-  unsigned pend_ph = 0;
-  for (int t = 0; t < n_kt; ++t) {
-    const int j0 = t * kPT;
-    load_tile(sK, kh, j0, a.n_tokens, tid);
-    load_tile(sV, vh, j0, a.n_tokens, tid);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    fence_proxy_async();  // this thread's shared-memory writes, before the tensor cores read them
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+  // S(t) is the (t / 2)-th commit on bar_s[t % 2] and PV(t) the t-th on bar_o; these count
+  // the tiles issued and waited for (the same in every thread)
+  int s_iss = 0, s_wait = 0, o_iss = 0, o_wait = 0;
+  auto issue_s = [&](int t) {  // S(t) = Q K(t)^T into S buffer t & 1
+    const int b = t & 1;
     if (tid == 0) {
 #pragma unroll
       for (int s = 0; s < kPT / 16; ++s) {
         const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
-        mma_bf16(tS, desc_k(sQ + off), desc_k(sK + off), kIdescS, s > 0 ? 1u : 0u);
+        mma_bf16(tS(b), desc_k(sQ + off), desc_k(sK(t) + off), kIdescS, s > 0 ? 1u : 0u);
       }
-      mma_commit(&ctl.bar_s);
+      mma_commit(&ctl.bar_s[b]);
     }
-    ok = __syncthreads_and(mbar_wait(&ctl.bar_s, ph_s));
-    if (!ok) {
-      pend = &ctl.bar_s;
-      pend_ph = ph_s;
-      break;
-    }
-    ph_s ^= 1u;
+    s_iss = t + 1;
+  };
+
+  bool ok = true;
+  // cp.async groups, committed by every thread in the same order (empty ones included):
+  // prologue {Q, K(0), V(0)}, {K(1)}; then per tile t: {K(t+2)} in step A, {V(t+1)} in D
+  if (n_kt > 0) {
+    load_tile(sQ, qh, i0, a.n_act, tid);
+    load_tile(sK(0), kh, 0, a.n_tokens, tid);
+    load_tile(sV(0), vh, 0, a.n_tokens, tid);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (n_kt > 1) load_tile(sK(1), kh, kPT, a.n_tokens, tid);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  float m_run = -INFINITY, l_half = 0.f;
+  for (int t = 0; t < n_kt; ++t) {
+    const int b = t & 1, j0 = t * kPT;
+    // (A) K(t+1) has landed (V(t) may still be in flight): S(t+1) goes to the tensor cores
+    //     ahead of this tile's softmax, and K(t+2) is fetched into the buffer S(t-1) used
+    if (t == 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+    else asm volatile("cp.async.wait_group 1;" ::: "memory");
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) issue_s(0);
+    if (t + 1 < n_kt) issue_s(t + 1);
+    if (t + 2 < n_kt) load_tile(sK(t + 2), kh, j0 + 2 * kPT, a.n_tokens, tid);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    // (B) S(t) is complete
+    ok = __syncthreads_and(mbar_wait(&ctl.bar_s[b], (unsigned)((t >> 1) & 1)));
+    if (!ok) break;
+    s_wait = t + 1;
     tc_fence_after();
 
-    // row max of this tile's visible keys (scores in the base-2 domain)
+    // (C) softmax of this row's own 64 columns (in registers); the row maximum is
+    //     exchanged with the partner half.  Lazy rescaling: the running maximum is kept
+    //     unless this tile exceeds it by more than 8 (weights then stay below 2^8, and O
+    //     and l share the scale, so o = O / l is unchanged).
+    float sv[64];
+    tmem_ld32(tS(b) + lane_off + 64 * hf, sv);
+    tmem_ld32(tS(b) + lane_off + 64 * hf + 32, sv + 32);
+    const int c_own = j0 + 64 * hf;
+    const bool full = c_own + 63 <= qp;  // every own column visible (no mask needed)
     float mx = -INFINITY;
-    float sv[32];
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      tmem_ld32(tS + lane_off + 32 * c, sv);
+    if (full) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (j0 + 32 * c + i <= qp) mx = fmaxf(mx, sv[i] * kScale);
+      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        if (c_own + i <= qp) mx = fmaxf(mx, sv[i]);
     }
-    const float m_new = fmaxf(m_run, mx);
-    const float alpha = m_new == -INFINITY ? 1.f : ex2(m_run - m_new);
-    // P = 2^(s - m_new) on visible keys, rounded to BF16; the row sum uses the rounded values
+    ctl.rmax[hf][row] = mx;
+    pair_bar(grp);
+    mx = fmaxf(mx, ctl.rmax[1 - hf][row]);
+    const float m_tile = mx * kScale;
+    float alpha = 1.f;
+    if (m_tile > m_run + 8.f) {  // also the first visible tile (m_run = -inf): alpha = 0
+      alpha = ex2(m_run - m_tile);
+      m_run = m_tile;
+    }
     float lsum = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      tmem_ld32(tS + lane_off + 32 * c, sv);
-      uint32_t w[16];
+    uint32_t pw[32];
+    if (full) {
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float p0 = (j0 + 32 * c + i <= qp) ? ex2(sv[i] * kScale - m_new) : 0.f;
-        const float p1 = (j0 + 32 * c + i + 1 <= qp) ? ex2(sv[i + 1] * kScale - m_new) : 0.f;
-        w[i >> 1] = pack_bf16(p0, p1);
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[i >> 1]);
-        lsum += __low2float(b) + __high2float(b);
+      for (int e = 0; e < 32; ++e) {
+        pw[e] = pack_bf16(ex2(fmaf(sv[2 * e], kScale, -m_run)), ex2(fmaf(sv[2 * e + 1], kScale, -m_run)));
+        lsum += __uint_as_float(pw[e] << 16) + __uint_as_float(pw[e] & 0xffff0000u);
       }
+    } else {
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
-        *reinterpret_cast<uint4*>(gP + sw128(tid, 4 * c + q4)) =
-            make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-    }
-    l_run = l_run * alpha + lsum;
-    m_run = m_new;
-    if (t > 0 && __any_sync(kFull, alpha != 1.f)) {  // rescale the warp's rows of the output accumulator
-      float ov[32];
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tO + lane_off + 32 * c, ov);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-        tmem_st32(tO + lane_off + 32 * c, ov);
+      for (int e = 0; e < 32; ++e) {
+        const int i = 2 * e;
+        const float p0 = (c_own + i <= qp) ? ex2(fmaf(sv[i], kScale, -m_run)) : 0.f;
+        const float p1 = (c_own + i + 1 <= qp) ? ex2(fmaf(sv[i + 1], kScale, -m_run)) : 0.f;
+        pw[e] = pack_bf16(p0, p1);
+        lsum += __uint_as_float(pw[e] << 16) + __uint_as_float(pw[e] & 0xffff0000u);
       }
     }
-    fence_proxy_async();  // P, written by this thread, before the tensor cores read it
+    l_half = fmaf(l_half, alpha, lsum);
+
+    // (D) PV(t-1) is complete: P may be overwritten, the output accumulator rescaled and
+    //     V buffer (t+1) % 2 refilled
+    if (t > 0) {
+      ok = __syncthreads_and(mbar_wait(&ctl.bar_o, (unsigned)(o_wait & 1)));
+      if (!ok) break;
+      ++o_wait;
+      tc_fence_after();
+      if (__any_sync(kFull, alpha != 1.f)) {
+        float ov[32];
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(tO + lane_off + 64 * hf + 32 * c, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          tmem_st32(tO + lane_off + 64 * hf + 32 * c, ov);
+        }
+      }
+    }
+#pragma unroll
+    for (int q8 = 0; q8 < 8; ++q8)  // 16-byte chunk 8 hf + q8 of the row
+      *reinterpret_cast<uint4*>(gbase + 6 * kTileB + sw128(row, 8 * hf + q8)) =
+          make_uint4(pw[4 * q8], pw[4 * q8 + 1], pw[4 * q8 + 2], pw[4 * q8 + 3]);
+    if (t + 1 < n_kt) load_tile(sV(t + 1), vh, j0 + kPT, a.n_tokens, tid);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    // (E) V(t) has landed (the two newest groups may still be in flight); P(t) and the
+    //     rescaled O are in place: O += P(t) V(t)
+    asm volatile("cp.async.wait_group 2;" ::: "memory");
+    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -244,32 +313,37 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
 #pragma unroll
       for (int s = 0; s < kPT / 16; ++s) {
         const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
-        mma_bf16(tO, desc_k(sP + off), desc_mn(sV + (uint32_t)s * 2048u), kIdescPV, (t > 0 || s > 0) ? 1u : 0u);
+        mma_bf16(tO, desc_k(sP + off), desc_mn(sV(t) + (uint32_t)s * 2048u), kIdescPV, (t > 0 || s > 0) ? 1u : 0u);
       }
       mma_commit(&ctl.bar_o);
     }
-    ok = __syncthreads_and(mbar_wait(&ctl.bar_o, ph_o));
-    if (!ok) {
-      pend = &ctl.bar_o;
-      pend_ph = ph_o;
-      break;
-    }
-    ph_o ^= 1u;
+    ++o_iss;
+  }
+  if (ok && o_iss > o_wait) {
+    ok = __syncthreads_and(mbar_wait(&ctl.bar_o, (unsigned)(o_wait & 1)));
+    if (ok) ++o_wait;
     tc_fence_after();
   }
 
   if (!ok) {
     if (tid == 0 && a.status) record_error(a.status, FL_DEV_TIMEOUT, i0);
-    // a last bounded wait for the outstanding MMAs before TMEM is released
-    mbar_wait(pend, pend_ph);
+    // last bounded waits for every outstanding group of MMAs before TMEM is released
+    for (; s_wait < s_iss; ++s_wait) mbar_wait(&ctl.bar_s[s_wait & 1], (unsigned)((s_wait >> 1) & 1));
+    for (; o_wait < o_iss; ++o_wait) mbar_wait(&ctl.bar_o, (unsigned)(o_wait & 1));
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
   } else if (n_kt > 0) {
-    // o = O / l for this thread's row (every lane reads TMEM; padding rows store nothing)
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    float* orow = a.o + (size_t)h * a.o_head_stride + (size_t)(i0 + tid) * kD;
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    // row sum = both halves' sums (exchanged through the now idle P buffer)
+    float* lx = reinterpret_cast<float*>(gbase + 6 * kTileB);
+    lx[hf * kPT + row] = l_half;
+    __syncthreads();
+    const float l = lx[row] + lx[kPT + row];
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float* orow = a.o + (size_t)h * a.o_head_stride + (size_t)(i0 + row) * kD + 64 * hf;
     float ov[32];
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      tmem_ld32(tO + lane_off + 32 * c, ov);
+    for (int c = 0; c < 2; ++c) {
+      tmem_ld32(tO + lane_off + 64 * hf + 32 * c, ov);
       if (qp >= 0) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
