@@ -211,6 +211,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
   float m_run = -INFINITY, l_half = 0.f;
+  uint8_t* p_row = gbase + 6 * kTileB + hf * 16384 + row * 128;  // this thread's half-row of P
   for (int t = 0; t < n_kt; ++t) {
     const int b = t & 1, j0 = t * kPT;
     // (A) K(t+1) has landed (V(t) may still be in flight): S(t+1) goes to the tensor cores
@@ -240,15 +241,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     tmem_ld32(tS(b) + lane_off + 64 * hf + 32, sv + 32);
     const int c_own = j0 + 64 * hf;
     const bool full = c_own + 63 <= qp;  // every own column visible (no mask needed)
-    float mx = -INFINITY;
+    float mx8[8];  // eight independent partial maxima (short dependency chains)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
     if (full) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+      for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
     } else {
 #pragma unroll
       for (int i = 0; i < 64; ++i)
-        if (c_own + i <= qp) mx = fmaxf(mx, sv[i]);
+        if (c_own + i <= qp) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
     }
+    float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
     ctl.rmax[hf][row] = mx;
     pair_bar(grp);
     mx = fmaxf(mx, ctl.rmax[1 - hf][row]);
@@ -258,13 +263,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
       alpha = ex2(m_run - m_tile);
       m_run = m_tile;
     }
-    float lsum = 0.f;
+    // weights (fp32 row sum in four partial sums; P rounded to BF16 for the tensor cores)
+    float ls4[4] = {0.f, 0.f, 0.f, 0.f};
     uint32_t pw[32];
     if (full) {
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        pw[e] = pack_bf16(ex2(fmaf(sv[2 * e], kScale, -m_run)), ex2(fmaf(sv[2 * e + 1], kScale, -m_run)));
-        lsum += __uint_as_float(pw[e] << 16) + __uint_as_float(pw[e] & 0xffff0000u);
+        const float p0 = ex2(fmaf(sv[2 * e], kScale, -m_run)), p1 = ex2(fmaf(sv[2 * e + 1], kScale, -m_run));
+        pw[e] = pack_bf16(p0, p1);
+        ls4[e & 3] += p0 + p1;
       }
     } else {
 #pragma unroll
@@ -273,10 +280,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
         const float p0 = (c_own + i <= qp) ? ex2(fmaf(sv[i], kScale, -m_run)) : 0.f;
         const float p1 = (c_own + i + 1 <= qp) ? ex2(fmaf(sv[i + 1], kScale, -m_run)) : 0.f;
         pw[e] = pack_bf16(p0, p1);
-        lsum += __uint_as_float(pw[e] << 16) + __uint_as_float(pw[e] & 0xffff0000u);
+        ls4[e & 3] += p0 + p1;
       }
     }
-    l_half = fmaf(l_half, alpha, lsum);
+    l_half = fmaf(l_half, alpha, (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
 
     // (D) PV(t-1) is complete: P may be overwritten, the output accumulator rescaled and
     //     V buffer (t+1) % 2 refilled
@@ -297,8 +304,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
       }
     }
 #pragma unroll
-    for (int q8 = 0; q8 < 8; ++q8)  // 16-byte chunk 8 hf + q8 of the row
-      *reinterpret_cast<uint4*>(gbase + 6 * kTileB + sw128(row, 8 * hf + q8)) =
+    for (int q8 = 0; q8 < 8; ++q8)  // 16-byte chunk 8 hf + q8 of the row (see sw128)
+      *reinterpret_cast<uint4*>(p_row + ((q8 ^ (row & 7)) << 4)) =
           make_uint4(pw[4 * q8], pw[4 * q8 + 1], pw[4 * q8 + 2], pw[4 * q8 + 3]);
     if (t + 1 < n_kt) load_tile(sV(t + 1), vh, j0 + kPT, a.n_tokens, tid);
     asm volatile("cp.async.commit_group;" ::: "memory");

@@ -4,9 +4,9 @@ oracle.
 FlashLoop project page, "The Method", Step 01 (only the active tokens are recomputed)
 and the paragraph after Step 03 (selected tokens gathered into compact buffers so the
 work stays a regular GEMM).  Tolerance, from the arithmetic: the kernel rounds each
-probability to BF16 (relative error <= 2^-9) before the value product and normalises
-by the sum of the rounded values, so |o - o_ref| <= 2^-9 * sum_j p_j |v_j| <= 2^-9 max|v|
-per head, plus fp32 accumulation; the test allows 2^-8 max|v|.
+probability to BF16 (relative error <= 2^-9) before the value product and normalises by
+the fp32 sum of the unrounded ones, so |o - o_ref| <= 2^-9 * sum_j p_j |v_j| / sum_j p_j
+<= 2^-9 max|v| per head, plus fp32 accumulation; the test allows 2^-8 max|v|.
 """
 import numpy as np
 import pytest
