@@ -226,9 +226,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     if (t + 1 < n_kt) issue_s(t + 1);
     if (t + 2 < n_kt) load_tile(sK(t + 2), kh, j0 + 2 * kPT, a.n_tokens, tid);
     asm volatile("cp.async.commit_group;" ::: "memory");
-    // (B) S(t) is complete
-    ok = __syncthreads_and(mbar_wait(&ctl.bar_s[b], (unsigned)((t >> 1) & 1)));
-    if (!ok) break;
+    // (B) S(t) is complete (each thread waits for itself; a failed wait is agreed on at (E))
+    bool okw = mbar_wait(&ctl.bar_s[b], (unsigned)((t >> 1) & 1));
     s_wait = t + 1;
     tc_fence_after();
 
@@ -288,8 +287,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     // (D) PV(t-1) is complete: P may be overwritten, the output accumulator rescaled and
     //     V buffer (t+1) % 2 refilled
     if (t > 0) {
-      ok = __syncthreads_and(mbar_wait(&ctl.bar_o, (unsigned)(o_wait & 1)));
-      if (!ok) break;
+      okw = mbar_wait(&ctl.bar_o, (unsigned)(o_wait & 1)) && okw;
       ++o_wait;
       tc_fence_after();
       if (__any_sync(kFull, alpha != 1.f)) {
@@ -314,8 +312,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     asm volatile("cp.async.wait_group 2;" ::: "memory");
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    ok = !__syncthreads_or(!okw);
     tc_fence_after();
+    if (!ok) {  // a wait ran out: leave with S(t) or PV(t-1) possibly outstanding
+      s_wait = t;
+      if (t > 0) o_wait = t - 1;
+      break;
+    }
     if (tid == 0) {
 #pragma unroll
       for (int s = 0; s < kPT / 16; ++s) {
