@@ -7,19 +7,19 @@
 // token's key and value of the loop:
 //     o_i = softmax_{j <= pos_i}(q_i k_j^T / sqrt(128)) v_j.
 //
-// One CTA of 8 warps per (128 active queries, head).  The query tile stays in shared
-// memory; key tiles of 128 tokens stream through three buffers (fetched two tiles
-// ahead) and value tiles through two (one tile ahead), by cp.async, zero-filled past the
-// end.  One thread issues S = Q K^T as 8
-// tcgen05.mma (M = N = 128, K = 16, BF16 operands from 128-byte-swizzled shared memory,
-// fp32 accumulators in TMEM) one tile ahead, into alternating TMEM buffers, so the
-// tensor cores compute the next scores while the warps run this tile's softmax.  Warp w
-// reads TMEM lanes 32 (w % 4) ..: thread t of warp w owns query row 32 (w % 4) + t and
-// the 64 columns of half w / 4 -- it masks, runs the online softmax in the base-2 domain,
-// writes its half of P (BF16) to shared memory in the operand layout and rescales its
-// half of the output accumulator row in TMEM; then O += P V as 8 more tcgen05.mma (V
-// read MN-major).  Each group of MMAs signals an mbarrier through tcgen05.commit; every
-// wait is bounded.
+// One CTA of 8 softmax warps and one MMA warp per (128 active queries, head).  The query
+// tile stays in shared memory; key tiles of 128 tokens stream through three buffers
+// (fetched two tiles ahead) and value tiles through two (one tile ahead), by cp.async
+// issued by the softmax warps, zero-filled past the end.  The MMA warp issues S = Q K^T
+// (8 tcgen05.mma of M = N = 128, K = 16; BF16 operands from 128-byte-swizzled shared
+// memory; fp32 accumulators in TMEM) one tile ahead into alternating TMEM buffers, and
+// O += P V once P is written (V read MN-major).  Softmax warp w reads TMEM lanes
+// 32 (w % 4) ..: its thread t owns query row 32 (w % 4) + t and the 64 columns of half
+// w / 4 -- it masks, runs the online softmax in the base-2 domain, writes its half of P
+// (BF16) to shared memory in the operand layout and rescales its half of the output row
+// in TMEM.  The two sides hand over through mbarriers only (softmax threads arrive when
+// their copies and P are in place; tcgen05.commit signals finished MMAs), so no CTA-wide
+// barrier sits in the loop; every wait is bounded.
 #include "kernels.h"
 
 namespace fl {
@@ -27,16 +27,20 @@ namespace {
 
 constexpr int kPT = 128;                      // queries per tile = keys per tile = head dim
 constexpr int kTileB = kPT * kPT * 2;         // one 128 x 128 BF16 tile
-constexpr int kPrefillThreads = 256;          // 8 warps: TMEM lane group w % 4, column half w / 4
+constexpr int kSoftmaxThreads = 256;          // 8 softmax warps: TMEM lane group w % 4, column half w / 4
+constexpr int kPrefillThreads = kSoftmaxThreads + 32;  // + one warp that issues the MMAs
 constexpr int kTmemCols = 512;                // S buffers: columns 0..127, 128..255; O: 256..383
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kPT >> 3) << 17) | ((kPT >> 4) << 24);
 constexpr uint32_t kIdescPV = kIdescS | (1u << 16);  // B (V) read MN-major
 
 struct PrefillCtl {
-  uint64_t bar_s[2], bar_o;
+  uint64_t bar_s[2], bar_o;      // tensor cores -> softmax warps (tcgen05.commit)
+  uint64_t bar_a[2], bar_e[2];   // softmax warps -> MMA warp, one arrival per softmax thread
   uint32_t tmem;
   int32_t pmax;
-  float rmax[2][kPT];  // per column half: this tile's row maxima (exchanged within a row pair)
+  int32_t failed;                // a bounded wait ran out somewhere
+  int32_t pad;
+  float rmax[2][kPT];            // per column half: this tile's row maxima
 };
 // the control block, then 1024-byte-aligned tiles: Q, K[3], V[2], P
 constexpr int kPrefillSmem = (int)sizeof(PrefillCtl) + 1023 + 7 * kTileB;
@@ -104,7 +108,7 @@ __device__ __forceinline__ void cp16_zfill(uint32_t dst, const void* src, bool v
 // thread t copies chunk t % 16 of rows t / 16 + 16 i (rows 16 apart keep their swizzle
 // phase, so the shared-memory offset steps by 16 x 128 bytes)
 __device__ __forceinline__ void load_tile(uint32_t tile, const uint16_t* src, int row0, int n, int tid) {
-  constexpr int kRowsPer = kPrefillThreads / 16;
+  constexpr int kRowsPer = kSoftmaxThreads / 16;
   const int r0 = tid >> 4, c = tid & 15;
   const uint32_t d0 = tile + sw128(r0, c);
   const uint16_t* s0 = src + (size_t)(row0 + r0) * kD + c * 8;
@@ -117,6 +121,11 @@ __device__ __forceinline__ void load_tile(uint32_t tile, const uint16_t* src, in
 
 // barrier of the two warps (w, w + 4) that share TMEM lanes 32 w ..
 __device__ __forceinline__ void pair_bar(int grp) { asm volatile("bar.sync %0, 64;" ::"r"(grp + 1) : "memory"); }
+// barrier of the eight softmax warps
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 5, %0;" ::"n"(kSoftmaxThreads) : "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_addr(bar)) : "memory");
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
@@ -135,8 +144,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
   const uint32_t sP = base + 6u * kTileB;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int grp = warp & 3, hf = warp >> 2;
-  const int row = 32 * grp + lane;  // this thread's query row = its TMEM lane
+  const bool mma_warp = warp == kSoftmaxThreads / 32;
+  const int grp = warp & 3, hf = (warp >> 2) & 1;
+  const int row = 32 * grp + lane;  // a softmax thread's query row = its TMEM lane
   const int h = blockIdx.y, i0 = blockIdx.x * kPT;
   const uint16_t* qh = a.q + (size_t)h * a.q_head_stride;
   const uint16_t* kh = a.k + (size_t)h * a.kv_head_stride;
@@ -144,7 +154,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
 
   // the row's position (-1: a padding row or a bad position)
   int qp = -1;
-  if (i0 + row < a.n_act) {
+  if (!mma_warp && i0 + row < a.n_act) {
     qp = __ldg(a.pos + i0 + row);
     const bool bad_order = i0 + row > 0 && __ldg(a.pos + i0 + row - 1) >= qp;
     const bool bad_range = qp < 0 || qp >= a.n_tokens;
@@ -156,8 +166,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     mbar_init(&ctl.bar_s[0], 1);
     mbar_init(&ctl.bar_s[1], 1);
     mbar_init(&ctl.bar_o, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl.bar_a[i], kSoftmaxThreads);
+      mbar_init(&ctl.bar_e[i], kSoftmaxThreads);
+    }
     fence_mbar_init();
     ctl.pmax = -1;
+    ctl.failed = 0;
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&ctl.tmem)),
@@ -178,175 +193,171 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
   const uint32_t tmem = ctl.tmem;
   const uint32_t tO = tmem + 2 * kPT;
   auto tS = [&](int b) { return tmem + (uint32_t)(b * kPT); };
-  const uint32_t lane_off = (uint32_t)(32 * grp) << 16;  // this warp's TMEM lanes
   const int pmax = ctl.pmax;
   const int n_kt = pmax < 0 ? 0 : pmax / kPT + 1;  // key tiles up to the tile's last position
-  const float kScale = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
 
-  // S(t) is the (t / 2)-th commit on bar_s[t % 2] and PV(t) the t-th on bar_o; these count
-  // the tiles issued and waited for (the same in every thread)
-  int s_iss = 0, s_wait = 0, o_iss = 0, o_wait = 0;
-  auto issue_s = [&](int t) {  // S(t) = Q K(t)^T into S buffer t & 1
-    const int b = t & 1;
-    if (tid == 0) {
-#pragma unroll
-      for (int s = 0; s < kPT / 16; ++s) {
-        const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
-        mma_bf16(tS(b), desc_k(sQ + off), desc_k(sK(t) + off), kIdescS, s > 0 ? 1u : 0u);
-      }
-      mma_commit(&ctl.bar_s[b]);
+  // A wait that ran out marks the CTA failed; later waits are then skipped (every barrier
+  // and arrival still happens, so nothing can block), and the results are not used.
+  bool failed = false;
+  auto wait = [&](uint64_t* bar, unsigned parity) {
+    if (failed) return;
+    if (!mbar_wait(bar, parity)) {
+      failed = true;
+      ctl.failed = 1;
     }
-    s_iss = t + 1;
   };
 
-  bool ok = true;
-  // cp.async groups, committed by every thread in the same order (empty ones included):
-  // prologue {Q, K(0), V(0)}, {K(1)}; then per tile t: {K(t+2)} in step A, {V(t+1)} in D
-  if (n_kt > 0) {
+  if (mma_warp) {
+    // ---- MMA warp: lane 0 issues; S(t+1) as soon as its key tile is in place, PV(t) once
+    //      the softmax warps have written P(t) ----
+    for (int t = 0; t < n_kt; ++t) {
+      const int b = t & 1;
+      wait(&ctl.bar_a[b], (unsigned)((t >> 1) & 1));
+      tc_fence_after();
+      if (lane == 0 && !failed) {
+        for (int u = t == 0 ? 0 : t + 1; u <= t + 1 && u < n_kt; ++u) {
+#pragma unroll
+          for (int s = 0; s < kPT / 16; ++s) {
+            const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
+            mma_bf16(tS(u & 1), desc_k(sQ + off), desc_k(sK(u) + off), kIdescS, s > 0 ? 1u : 0u);
+          }
+          mma_commit(&ctl.bar_s[u & 1]);
+        }
+      }
+      __syncwarp();
+      wait(&ctl.bar_e[b], (unsigned)((t >> 1) & 1));
+      tc_fence_after();
+      if (lane == 0 && !failed) {
+#pragma unroll
+        for (int s = 0; s < kPT / 16; ++s) {
+          const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
+          mma_bf16(tO, desc_k(sP + off), desc_mn(sV(t) + (uint32_t)s * 2048u), kIdescPV,
+                   (t > 0 || s > 0) ? 1u : 0u);
+        }
+        mma_commit(&ctl.bar_o);
+      }
+      __syncwarp();
+    }
+  } else if (n_kt > 0) {
+    // ---- softmax warps ----
+    const uint32_t lane_off = (uint32_t)(32 * grp) << 16;  // this warp's TMEM lanes
+    const float kScale = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    uint8_t* p_row = gbase + 6 * kTileB + hf * 16384 + row * 128;   // this thread's half-row of P
+    // cp.async groups (committed in the same order by every softmax thread, empty ones
+    // included): {Q, K(0), V(0)}, {K(1)}; then per tile t: {K(t+2)} in (A), {V(t+1)} in (D)
     load_tile(sQ, qh, i0, a.n_act, tid);
     load_tile(sK(0), kh, 0, a.n_tokens, tid);
     load_tile(sV(0), vh, 0, a.n_tokens, tid);
     asm volatile("cp.async.commit_group;" ::: "memory");
     if (n_kt > 1) load_tile(sK(1), kh, kPT, a.n_tokens, tid);
     asm volatile("cp.async.commit_group;" ::: "memory");
-  }
-  float m_run = -INFINITY, l_half = 0.f;
-  uint8_t* p_row = gbase + 6 * kTileB + hf * 16384 + row * 128;  // this thread's half-row of P
-  for (int t = 0; t < n_kt; ++t) {
-    const int b = t & 1, j0 = t * kPT;
-    // (A) K(t+1) has landed (V(t) may still be in flight): S(t+1) goes to the tensor cores
-    //     ahead of this tile's softmax, and K(t+2) is fetched into the buffer S(t-1) used
-    if (t == 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
-    else asm volatile("cp.async.wait_group 1;" ::: "memory");
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (t == 0) issue_s(0);
-    if (t + 1 < n_kt) issue_s(t + 1);
-    if (t + 2 < n_kt) load_tile(sK(t + 2), kh, j0 + 2 * kPT, a.n_tokens, tid);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    // (B) S(t) is complete (each thread waits for itself; a failed wait is agreed on at (E))
-    bool okw = mbar_wait(&ctl.bar_s[b], (unsigned)((t >> 1) & 1));
-    s_wait = t + 1;
-    tc_fence_after();
-
-    // (C) softmax of this row's own 64 columns (in registers); the row maximum is
-    //     exchanged with the partner half.  Lazy rescaling: the running maximum is kept
-    //     unless this tile exceeds it by more than 8 (weights then stay below 2^8, and O
-    //     and l share the scale, so o = O / l is unchanged).
-    float sv[64];
-    tmem_ld32(tS(b) + lane_off + 64 * hf, sv);
-    tmem_ld32(tS(b) + lane_off + 64 * hf + 32, sv + 32);
-    const int c_own = j0 + 64 * hf;
-    const bool full = c_own + 63 <= qp;  // every own column visible (no mask needed)
-    float mx8[8];  // eight independent partial maxima (short dependency chains)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
-    if (full) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 64; ++i)
-        if (c_own + i <= qp) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-    }
-    float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-    ctl.rmax[hf][row] = mx;
-    pair_bar(grp);
-    mx = fmaxf(mx, ctl.rmax[1 - hf][row]);
-    const float m_tile = mx * kScale;
-    float alpha = 1.f;
-    if (m_tile > m_run + 8.f) {  // also the first visible tile (m_run = -inf): alpha = 0
-      alpha = ex2(m_run - m_tile);
-      m_run = m_tile;
-    }
-    // weights (fp32 row sum in four partial sums; P rounded to BF16 for the tensor cores)
-    float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t pw[32];
-    if (full) {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float p0 = ex2(fmaf(sv[2 * e], kScale, -m_run)), p1 = ex2(fmaf(sv[2 * e + 1], kScale, -m_run));
-        pw[e] = pack_bf16(p0, p1);
-        ls4[e & 3] += p0 + p1;
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int i = 2 * e;
-        const float p0 = (c_own + i <= qp) ? ex2(fmaf(sv[i], kScale, -m_run)) : 0.f;
-        const float p1 = (c_own + i + 1 <= qp) ? ex2(fmaf(sv[i + 1], kScale, -m_run)) : 0.f;
-        pw[e] = pack_bf16(p0, p1);
-        ls4[e & 3] += p0 + p1;
-      }
-    }
-    l_half = fmaf(l_half, alpha, (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
-
-    // (D) PV(t-1) is complete: P may be overwritten, the output accumulator rescaled and
-    //     V buffer (t+1) % 2 refilled
-    if (t > 0) {
-      okw = mbar_wait(&ctl.bar_o, (unsigned)(o_wait & 1)) && okw;
-      ++o_wait;
+    float m_run = -INFINITY, l_half = 0.f;
+    for (int t = 0; t < n_kt; ++t) {
+      const int b = t & 1, j0 = t * kPT;
+      // (A) this thread's part of K(t+1) (at t = 0 also Q, K(0)) has landed and S(t-1)
+      //     is consumed: tell the MMA warp; fetch K(t+2) into the buffer S(t-1) used
+      if (t == 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+      else asm volatile("cp.async.wait_group 1;" ::: "memory");
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(&ctl.bar_a[b]);
+      if (t + 2 < n_kt) load_tile(sK(t + 2), kh, j0 + 2 * kPT, a.n_tokens, tid);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      // (B) S(t) is complete
+      wait(&ctl.bar_s[b], (unsigned)((t >> 1) & 1));
       tc_fence_after();
-      if (__any_sync(kFull, alpha != 1.f)) {
-        float ov[32];
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld32(tO + lane_off + 64 * hf + 32 * c, ov);
+
+      // (C) softmax of this row's own 64 columns (in registers); the row maximum is
+      //     exchanged with the partner half.  Lazy rescaling: the running maximum is kept
+      //     unless this tile exceeds it by more than 8 (weights then stay below 2^8, and O
+      //     and l share the scale, so o = O / l is unchanged).
+      float sv[64];
+      tmem_ld32(tS(b) + lane_off + 64 * hf, sv);
+      tmem_ld32(tS(b) + lane_off + 64 * hf + 32, sv + 32);
+      const int c_own = j0 + 64 * hf;
+      const bool full = c_own + 63 <= qp;  // every own column visible (no mask needed)
+      float mx8[8];  // eight independent partial maxima (short dependency chains)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          tmem_st32(tO + lane_off + 64 * hf + 32 * c, ov);
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (c_own + i <= qp) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+      }
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      ctl.rmax[hf][row] = mx;
+      pair_bar(grp);
+      mx = fmaxf(mx, ctl.rmax[1 - hf][row]);
+      const float m_tile = mx * kScale;
+      float alpha = 1.f;
+      if (m_tile > m_run + 8.f) {  // also the first visible tile (m_run = -inf): alpha = 0
+        alpha = ex2(m_run - m_tile);
+        m_run = m_tile;
+      }
+      // weights (fp32 row sum in four partial sums; P rounded to BF16 for the tensor cores)
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pw[32];
+      if (full) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = ex2(fmaf(sv[2 * e], kScale, -m_run)), p1 = ex2(fmaf(sv[2 * e + 1], kScale, -m_run));
+          pw[e] = pack_bf16(p0, p1);
+          ls4[e & 3] += p0 + p1;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int i = 2 * e;
+          const float p0 = (c_own + i <= qp) ? ex2(fmaf(sv[i], kScale, -m_run)) : 0.f;
+          const float p1 = (c_own + i + 1 <= qp) ? ex2(fmaf(sv[i + 1], kScale, -m_run)) : 0.f;
+          pw[e] = pack_bf16(p0, p1);
+          ls4[e & 3] += p0 + p1;
         }
       }
-    }
-#pragma unroll
-    for (int q8 = 0; q8 < 8; ++q8)  // 16-byte chunk 8 hf + q8 of the row (see sw128)
-      *reinterpret_cast<uint4*>(p_row + ((q8 ^ (row & 7)) << 4)) =
-          make_uint4(pw[4 * q8], pw[4 * q8 + 1], pw[4 * q8 + 2], pw[4 * q8 + 3]);
-    if (t + 1 < n_kt) load_tile(sV(t + 1), vh, j0 + kPT, a.n_tokens, tid);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    // (E) V(t) has landed (the two newest groups may still be in flight); P(t) and the
-    //     rescaled O are in place: O += P(t) V(t)
-    asm volatile("cp.async.wait_group 2;" ::: "memory");
-    fence_proxy_async();
-    tc_fence_before();
-    ok = !__syncthreads_or(!okw);
-    tc_fence_after();
-    if (!ok) {  // a wait ran out: leave with S(t) or PV(t-1) possibly outstanding
-      s_wait = t;
-      if (t > 0) o_wait = t - 1;
-      break;
-    }
-    if (tid == 0) {
-#pragma unroll
-      for (int s = 0; s < kPT / 16; ++s) {
-        const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
-        mma_bf16(tO, desc_k(sP + off), desc_mn(sV(t) + (uint32_t)s * 2048u), kIdescPV, (t > 0 || s > 0) ? 1u : 0u);
-      }
-      mma_commit(&ctl.bar_o);
-    }
-    ++o_iss;
-  }
-  if (ok && o_iss > o_wait) {
-    ok = __syncthreads_and(mbar_wait(&ctl.bar_o, (unsigned)(o_wait & 1)));
-    if (ok) ++o_wait;
-    tc_fence_after();
-  }
+      l_half = fmaf(l_half, alpha, (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
 
-  if (!ok) {
-    if (tid == 0 && a.status) record_error(a.status, FL_DEV_TIMEOUT, i0);
-    // last bounded waits for every outstanding group of MMAs before TMEM is released
-    for (; s_wait < s_iss; ++s_wait) mbar_wait(&ctl.bar_s[s_wait & 1], (unsigned)((s_wait >> 1) & 1));
-    for (; o_wait < o_iss; ++o_wait) mbar_wait(&ctl.bar_o, (unsigned)(o_wait & 1));
+      // (D) PV(t-1) is complete: P may be overwritten, the output accumulator rescaled and
+      //     V buffer (t+1) % 2 refilled
+      if (t > 0) {
+        wait(&ctl.bar_o, (unsigned)((t - 1) & 1));
+        tc_fence_after();
+        if (__any_sync(kFull, alpha != 1.f)) {
+          float ov[32];
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld32(tO + lane_off + 64 * hf + 32 * c, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            tmem_st32(tO + lane_off + 64 * hf + 32 * c, ov);
+          }
+        }
+      }
+#pragma unroll
+      for (int q8 = 0; q8 < 8; ++q8)  // 16-byte chunk 8 hf + q8 of the row (see sw128)
+        *reinterpret_cast<uint4*>(p_row + ((q8 ^ (row & 7)) << 4)) =
+            make_uint4(pw[4 * q8], pw[4 * q8 + 1], pw[4 * q8 + 2], pw[4 * q8 + 3]);
+      if (t + 1 < n_kt) load_tile(sV(t + 1), vh, j0 + kPT, a.n_tokens, tid);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      // (E) V(t) has landed (the two newest groups may still be in flight), P(t) and the
+      //     rescaled O are in place: the MMA warp may issue O += P(t) V(t)
+      asm volatile("cp.async.wait_group 2;" ::: "memory");
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(&ctl.bar_e[b]);
+    }
+    // the last PV, then o = O / l for this thread's half-row; the halves' row sums meet in
+    // the idle P buffer
+    wait(&ctl.bar_o, (unsigned)((n_kt - 1) & 1));
+    tc_fence_after();
     asm volatile("cp.async.wait_group 0;" ::: "memory");
-  } else if (n_kt > 0) {
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    // row sum = both halves' sums (exchanged through the now idle P buffer)
     float* lx = reinterpret_cast<float*>(gbase + 6 * kTileB);
+    softmax_bar();  // every softmax warp is done reading P
     lx[hf * kPT + row] = l_half;
-    __syncthreads();
+    softmax_bar();
     const float l = lx[row] + lx[kPT + row];
     const float inv = l > 0.f ? 1.f / l : 0.f;
     float* orow = a.o + (size_t)h * a.o_head_stride + (size_t)(i0 + row) * kD + 64 * hf;
@@ -354,7 +365,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       tmem_ld32(tO + lane_off + 64 * hf + 32 * c, ov);
-      if (qp >= 0) {
+      if (qp >= 0 && !ctl.failed) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
           *reinterpret_cast<float4*>(orow + 32 * c + i) =
@@ -364,6 +375,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
   }
   tc_fence_before();
   __syncthreads();
+  if (ctl.failed) {
+    // a wait ran out: record it, and give any MMA still in flight time to finish before
+    // TMEM is released
+    if (tid == 0) {
+      if (a.status) record_error(a.status, FL_DEV_TIMEOUT, i0);
+      const uint64_t t0 = global_ns();
+      while (global_ns() - t0 < 2000000ull) __nanosleep(1000);
+    }
+    __syncthreads();
+  }
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
