@@ -9,17 +9,22 @@
 //
 // One CTA of 8 softmax warps and one MMA warp per (128 active queries, head).  The query
 // tile stays in shared memory; key tiles of 128 tokens stream through three buffers
-// (fetched two tiles ahead) and value tiles through two (one tile ahead), by cp.async
-// issued by the softmax warps, zero-filled past the end.  The MMA warp issues S = Q K^T
+// and value tiles through two, copied by a load warp with tensor maps (TMA: 64 x 128
+// boxes in the 128-byte swizzle the MMA descriptors name, zeros past the end) as soon as
+// the tensor cores release a buffer.  The MMA warp issues S = Q K^T
 // (8 tcgen05.mma of M = N = 128, K = 16; BF16 operands from 128-byte-swizzled shared
 // memory; fp32 accumulators in TMEM) one tile ahead into alternating TMEM buffers, and
 // O += P V once P is written (V read MN-major).  Softmax warp w reads TMEM lanes
 // 32 (w % 4) ..: its thread t owns query row 32 (w % 4) + t and the 64 columns of half
 // w / 4 -- it masks, runs the online softmax in the base-2 domain, writes its half of P
 // (BF16) to shared memory in the operand layout and rescales its half of the output row
-// in TMEM.  The two sides hand over through mbarriers only (softmax threads arrive when
-// their copies and P are in place; tcgen05.commit signals finished MMAs), so no CTA-wide
-// barrier sits in the loop; every wait is bounded.
+// in TMEM.  The warps hand over through mbarriers only (copies count transaction bytes,
+// softmax threads arrive when a score buffer is consumed and when P is in place,
+// tcgen05.commit signals finished MMAs), so no CTA-wide barrier sits in the loop; every
+// wait is bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kernels.h"
 
 namespace fl {
@@ -28,7 +33,9 @@ namespace {
 constexpr int kPT = 128;                      // queries per tile = keys per tile = head dim
 constexpr int kTileB = kPT * kPT * 2;         // one 128 x 128 BF16 tile
 constexpr int kSoftmaxThreads = 256;          // 8 softmax warps: TMEM lane group w % 4, column half w / 4
-constexpr int kPrefillThreads = kSoftmaxThreads + 32;  // + one warp that issues the MMAs
+constexpr int kMmaWarp = kSoftmaxThreads / 32;  // issues the MMAs
+constexpr int kLoadWarp = kMmaWarp + 1;         // issues the tensor-map copies
+constexpr int kPrefillThreads = kSoftmaxThreads + 64;
 constexpr int kTmemCols = 512;                // S buffers: columns 0..127, 128..255; O: 256..383
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kPT >> 3) << 17) | ((kPT >> 4) << 24);
 constexpr uint32_t kIdescPV = kIdescS | (1u << 16);  // B (V) read MN-major
@@ -36,6 +43,8 @@ constexpr uint32_t kIdescPV = kIdescS | (1u << 16);  // B (V) read MN-major
 struct PrefillCtl {
   uint64_t bar_s[2], bar_o;      // tensor cores -> softmax warps (tcgen05.commit)
   uint64_t bar_a[2], bar_e[2];   // softmax warps -> MMA warp, one arrival per softmax thread
+  uint64_t qfull, kfull[3], vfull[2];  // copies landed (transaction bytes)
+  uint64_t kempty[3], vempty[2];       // tensor cores done with a K / V buffer (tcgen05.commit)
   uint32_t tmem;
   int32_t pmax;
   int32_t failed;                // a bounded wait ran out somewhere
@@ -45,12 +54,10 @@ struct PrefillCtl {
 // the control block, then 1024-byte-aligned tiles: Q, K[3], V[2], P
 constexpr int kPrefillSmem = (int)sizeof(PrefillCtl) + 1023 + 7 * kTileB;
 
-// Byte offset of 16-byte chunk c (0..15) of row r in a 128 x 128 BF16 tile: two 64-column
-// blocks of 128 rows x 128 bytes (16 KB apart); within each 1024-byte group of 8 rows the
-// chunk index is XOR-ed with (row mod 8) -- the 128-byte swizzle the descriptors name.
-__device__ __forceinline__ uint32_t sw128(int r, int c) {
-  return (uint32_t)((c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
+// Operand tiles (128 x 128 BF16): two 64-column blocks of 128 rows x 128 bytes, 16 KB
+// apart; within each 1024-byte group of 8 rows the 16-byte chunk index is XOR-ed with
+// (row mod 8) -- the 128-byte swizzle that the tensor-map copies write and the
+// descriptors below name.
 
 // Shared-memory matrix descriptors (tcgen05): start address >> 4 in bits 0..13, leading
 // byte offset >> 4 in bits 16..29, stride byte offset >> 4 in bits 32..45, version 1 in
@@ -100,23 +107,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp16_zfill(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
+// A 128-row x 64-column BF16 box of a [heads][rows][128] tensor (tensor map `map`: 128-byte
+// swizzle, zeros past the rows) into shared memory at dst (1024-byte aligned); completion
+// is counted in transaction bytes on `bar`.
+__device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, int col, int row, int head, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row), "r"(head), "r"(smem_addr(bar))
+      : "memory");
 }
-
-// rows [row0, row0 + 128) of a BF16 [n][128] matrix into a swizzled tile (zero past n):
-// thread t copies chunk t % 16 of rows t / 16 + 16 i (rows 16 apart keep their swizzle
-// phase, so the shared-memory offset steps by 16 x 128 bytes)
-__device__ __forceinline__ void load_tile(uint32_t tile, const uint16_t* src, int row0, int n, int tid) {
-  constexpr int kRowsPer = kSoftmaxThreads / 16;
-  const int r0 = tid >> 4, c = tid & 15;
-  const uint32_t d0 = tile + sw128(r0, c);
-  const uint16_t* s0 = src + (size_t)(row0 + r0) * kD + c * 8;
-#pragma unroll
-  for (int it = 0; it < kPT / kRowsPer; ++it) {
-    const bool ok = row0 + r0 + kRowsPer * it < n;
-    cp16_zfill(d0 + (uint32_t)(it * kRowsPer * 128), ok ? s0 + (size_t)it * kRowsPer * kD : src, ok);
-  }
+// a whole 128 x 128 tile: its two 64-column blocks, 16 KB apart
+__device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row, int head, uint64_t* bar) {
+  mbar_expect_tx(bar, kTileB);
+  tma_box(dst, map, 0, row, head, bar);
+  tma_box(dst + 16384u, map, 64, row, head, bar);
 }
 
 // barrier of the two warps (w, w + 4) that share TMEM lanes 32 w ..
@@ -132,7 +136,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-__global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    prefill_attn_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   PrefillCtl& ctl = *reinterpret_cast<PrefillCtl*>(smem_raw);
   const uint32_t raw = smem_addr(smem_raw);
@@ -144,17 +150,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
   const uint32_t sP = base + 6u * kTileB;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool mma_warp = warp == kSoftmaxThreads / 32;
+  const bool softmax_warp = warp < kMmaWarp;
   const int grp = warp & 3, hf = (warp >> 2) & 1;
   const int row = 32 * grp + lane;  // a softmax thread's query row = its TMEM lane
   const int h = blockIdx.y, i0 = blockIdx.x * kPT;
-  const uint16_t* qh = a.q + (size_t)h * a.q_head_stride;
-  const uint16_t* kh = a.k + (size_t)h * a.kv_head_stride;
-  const uint16_t* vh = a.v + (size_t)h * a.kv_head_stride;
 
   // the row's position (-1: a padding row or a bad position)
   int qp = -1;
-  if (!mma_warp && i0 + row < a.n_act) {
+  if (softmax_warp && i0 + row < a.n_act) {
     qp = __ldg(a.pos + i0 + row);
     const bool bad_order = i0 + row > 0 && __ldg(a.pos + i0 + row - 1) >= qp;
     const bool bad_range = qp < 0 || qp >= a.n_tokens;
@@ -169,7 +172,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.bar_a[i], kSoftmaxThreads);
       mbar_init(&ctl.bar_e[i], kSoftmaxThreads);
+      mbar_init(&ctl.vfull[i], 1);
+      mbar_init(&ctl.vempty[i], 1);
     }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&ctl.kfull[i], 1);
+      mbar_init(&ctl.kempty[i], 1);
+    }
+    mbar_init(&ctl.qfull, 1);
     fence_mbar_init();
     ctl.pmax = -1;
     ctl.failed = 0;
@@ -207,25 +217,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     }
   };
 
-  if (mma_warp) {
-    // ---- MMA warp: lane 0 issues; S(t+1) as soon as its key tile is in place, PV(t) once
-    //      the softmax warps have written P(t) ----
+  if (warp == kMmaWarp) {
+    // ---- MMA warp: lane 0 issues; S(t+1) once its key tile has landed and S buffer
+    //      (t+1) % 2 is consumed, PV(t) once P(t) is written and V(t) has landed ----
     for (int t = 0; t < n_kt; ++t) {
       const int b = t & 1;
       wait(&ctl.bar_a[b], (unsigned)((t >> 1) & 1));
-      tc_fence_after();
-      if (lane == 0 && !failed) {
-        for (int u = t == 0 ? 0 : t + 1; u <= t + 1 && u < n_kt; ++u) {
+      if (t == 0) wait(&ctl.qfull, 0u);
+      for (int u = t == 0 ? 0 : t + 1; u <= t + 1 && u < n_kt; ++u) {
+        wait(&ctl.kfull[u % 3], (unsigned)((u / 3) & 1));
+        tc_fence_after();
+        if (lane == 0 && !failed) {
 #pragma unroll
           for (int s = 0; s < kPT / 16; ++s) {
             const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
             mma_bf16(tS(u & 1), desc_k(sQ + off), desc_k(sK(u) + off), kIdescS, s > 0 ? 1u : 0u);
           }
           mma_commit(&ctl.bar_s[u & 1]);
+          mma_commit(&ctl.kempty[u % 3]);
         }
+        __syncwarp();
       }
-      __syncwarp();
       wait(&ctl.bar_e[b], (unsigned)((t >> 1) & 1));
+      wait(&ctl.vfull[b], (unsigned)((t >> 1) & 1));
       tc_fence_after();
       if (lane == 0 && !failed) {
 #pragma unroll
@@ -235,38 +249,37 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
                    (t > 0 || s > 0) ? 1u : 0u);
         }
         mma_commit(&ctl.bar_o);
+        mma_commit(&ctl.vempty[b]);
       }
       __syncwarp();
     }
+  } else if (warp == kLoadWarp) {
+    // ---- load warp: lane 0 copies Q once, then K(t) into buffer t % 3 and V(t) into
+    //      buffer t % 2 as soon as the tensor cores are done with the tile they held ----
+    if (lane == 0 && n_kt > 0) {
+      tma_tile(sQ, &tm_q, i0, h, &ctl.qfull);
+      for (int t = 0; t < n_kt; ++t) {
+        if (t >= 3) wait(&ctl.kempty[t % 3], (unsigned)(((t - 3) / 3) & 1));
+        if (!failed) tma_tile(sK(t), &tm_k, t * kPT, h, &ctl.kfull[t % 3]);
+        if (t >= 2) wait(&ctl.vempty[t & 1], (unsigned)(((t - 2) >> 1) & 1));
+        if (!failed) tma_tile(sV(t), &tm_v, t * kPT, h, &ctl.vfull[t & 1]);
+      }
+    }
+    __syncwarp();
   } else if (n_kt > 0) {
     // ---- softmax warps ----
     const uint32_t lane_off = (uint32_t)(32 * grp) << 16;  // this warp's TMEM lanes
     const float kScale = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
     uint8_t* p_row = gbase + 6 * kTileB + hf * 16384 + row * 128;   // this thread's half-row of P
-    // cp.async groups (committed in the same order by every softmax thread, empty ones
-    // included): {Q, K(0), V(0)}, {K(1)}; then per tile t: {K(t+2)} in (A), {V(t+1)} in (D)
-    load_tile(sQ, qh, i0, a.n_act, tid);
-    load_tile(sK(0), kh, 0, a.n_tokens, tid);
-    load_tile(sV(0), vh, 0, a.n_tokens, tid);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    if (n_kt > 1) load_tile(sK(1), kh, kPT, a.n_tokens, tid);
-    asm volatile("cp.async.commit_group;" ::: "memory");
     float m_run = -INFINITY, l_half = 0.f;
     for (int t = 0; t < n_kt; ++t) {
       const int b = t & 1, j0 = t * kPT;
-      // (A) this thread's part of K(t+1) (at t = 0 also Q, K(0)) has landed and S(t-1)
-      //     is consumed: tell the MMA warp; fetch K(t+2) into the buffer S(t-1) used
-      if (t == 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
-      else asm volatile("cp.async.wait_group 1;" ::: "memory");
-      fence_proxy_async();
+      // (A) S(t-1) is consumed: S buffer (t+1) % 2 may be overwritten
       tc_fence_before();
       mbar_arrive(&ctl.bar_a[b]);
-      if (t + 2 < n_kt) load_tile(sK(t + 2), kh, j0 + 2 * kPT, a.n_tokens, tid);
-      asm volatile("cp.async.commit_group;" ::: "memory");
       // (B) S(t) is complete
       wait(&ctl.bar_s[b], (unsigned)((t >> 1) & 1));
       tc_fence_after();
-
       // (C) softmax of this row's own 64 columns (in registers); the row maximum is
       //     exchanged with the partner half.  Lazy rescaling: the running maximum is kept
       //     unless this tile exceeds it by more than 8 (weights then stay below 2^8, and O
@@ -320,8 +333,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
       }
       l_half = fmaf(l_half, alpha, (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
 
-      // (D) PV(t-1) is complete: P may be overwritten, the output accumulator rescaled and
-      //     V buffer (t+1) % 2 refilled
+      // (D) PV(t-1) is complete: P may be overwritten and the output accumulator rescaled
       if (t > 0) {
         wait(&ctl.bar_o, (unsigned)((t - 1) & 1));
         tc_fence_after();
@@ -337,14 +349,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
         }
       }
 #pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8)  // 16-byte chunk 8 hf + q8 of the row (see sw128)
+      for (int q8 = 0; q8 < 8; ++q8)  // 16-byte chunk 8 hf + q8 of the row, swizzled
         *reinterpret_cast<uint4*>(p_row + ((q8 ^ (row & 7)) << 4)) =
             make_uint4(pw[4 * q8], pw[4 * q8 + 1], pw[4 * q8 + 2], pw[4 * q8 + 3]);
-      if (t + 1 < n_kt) load_tile(sV(t + 1), vh, j0 + kPT, a.n_tokens, tid);
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      // (E) V(t) has landed (the two newest groups may still be in flight), P(t) and the
-      //     rescaled O are in place: the MMA warp may issue O += P(t) V(t)
-      asm volatile("cp.async.wait_group 2;" ::: "memory");
+      // (E) P(t) and the rescaled O are in place: the MMA warp may issue O += P(t) V(t)
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&ctl.bar_e[b]);
@@ -353,7 +361,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
     // the idle P buffer
     wait(&ctl.bar_o, (unsigned)((n_kt - 1) & 1));
     tc_fence_after();
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
     float* lx = reinterpret_cast<float*>(gbase + 6 * kTileB);
     softmax_bar();  // every softmax warp is done reading P
     lx[hf * kPT + row] = l_half;
@@ -393,8 +400,46 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_attn_kernel(Prefil
 
 }  // namespace
 
+namespace {
+
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [heads][rows][128] BF16 (row stride 256 bytes, head stride head_stride elements) as a 3-D
+// tensor map read in 64 x 128 boxes with the 128-byte swizzle; rows past `rows` read as 0
+bool make_map(CUtensorMap* m, const uint16_t* base, int rows, int heads, int64_t head_stride) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  if (heads == 1 || head_stride < (int64_t)rows * kD) head_stride = (int64_t)rows * kD;  // unused with one head
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)head_stride * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)kPT, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_prefill_attn(const PrefillArgs& a, cudaStream_t s) {
   if (a.n_act == 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, a.n_act, a.heads, a.q_head_stride) || !make_map(&mk, a.k, a.n_tokens, a.heads, a.kv_head_stride) ||
+      !make_map(&mv, a.v, a.n_tokens, a.heads, a.kv_head_stride))
+    return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
@@ -405,7 +450,7 @@ cudaError_t launch_prefill_attn(const PrefillArgs& a, cudaStream_t s) {
     attr_set[dev] = true;
   }
   dim3 grid((a.n_act + kPT - 1) / kPT, a.heads);
-  prefill_attn_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(a);
+  prefill_attn_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(a, mq, mk, mv);
   return cudaGetLastError();
 }
 
