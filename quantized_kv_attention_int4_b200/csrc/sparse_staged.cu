@@ -60,6 +60,7 @@ struct alignas(16) WarpCtlS {
   float2 wrow[kMaxRows][2];        // span being consumed: per row and half (wS, wU)
   float lr[kMaxRows];              // span being consumed: per-row logit parts
   const uint8_t* rec_src[kMaxRecs];  // span being issued: source of each key record
+  const uint8_t* row_src[kMaxRows];  // span being issued: source of each row
 };
 
 struct alignas(16) CtaHdr {
@@ -272,12 +273,10 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
           hd.row_rec[ri] = (uint8_t)ki;
           hd.row_pin[ri] = (uint8_t)pin;
           hd.row_store[ri] = (uint8_t)s;
-          // the row (8 pieces) and its value (scale, zero) pair, issued by the column's lane
+          // the row's source (copied below by eight lanes at a time) and its value (scale,
+          // zero) pair, issued by the column's lane
           const uint8_t* base = (s == 1 ? brec : rrec) + (size_t)g * kRec;
-          const uint8_t* src = base + pin * 128;
-          uint8_t* dst = rows + ri * 128;
-#pragma unroll
-          for (int pc = 0; pc < 8; ++pc) cp_async16(dst + pc * 16, src + pc * 16);
+          wc.row_src[ri] = base + pin * 128;
           cp_async8(szs + ri * 8, base + kRecVsz + pin * 8);
           if (isnew) wc.rec_src[ki] = base + kRecKsz;
         }
@@ -285,6 +284,10 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
         recbase += __popc(nb);
       }
       __syncwarp();
+      // rows: eight lanes per 128-byte row, four rows per copy instruction (contiguous
+      // pieces, so each instruction touches four lines rather than 32)
+      for (int ri = lane >> 3; ri < nrows; ri += 4)
+        cp_async16(rows + ri * 128 + (lane & 7) * 16, wc.row_src[ri] + (lane & 7) * 16);
       // key records: 32 pieces each, spread over the lanes
       for (int k = 0; k < nrecs; ++k) cp_async16(recs + k * 512 + lane * 16, wc.rec_src[k] + lane * 16);
       asm volatile("cp.async.commit_group;" ::: "memory");
