@@ -249,15 +249,21 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       const int dep = depth[j];
       stores = dep < r ? dep : r;
     }
-    int32_t* e = plan + (size_t)k * ps;
-    e[0] = j;
-    e[1] = lam | (stores << 8);
-    e[2] = __float_as_int(ex2(key_value(keys[j])));
+    // the entry's words, stored 16 bytes at a time (ps is a multiple of 4; unused words 0)
     const int b = j >> 6, jt = j & 63;
-    for (int rp = 2; rp <= stores; ++rp) {
+    uint4* e = reinterpret_cast<uint4*>(plan + (size_t)k * ps);
+    const int w2 = __float_as_int(ex2(key_value(keys[j])));
+    auto word = [&](int i) -> int {
+      if (i == 0) return j;
+      if (i == 1) return lam | (stores << 8);
+      if (i == 2) return w2;
+      const int rp = i - 1;
+      if (rp > stores) return 0;
       const unsigned long long mk = mask[(size_t)rp * ncb + b];
-      e[1 + rp] = c.slot_base[rp] + first[(size_t)rp * ncb + b] + __popcll(mk & ((1ull << jt) - 1ull));
-    }
+      return c.slot_base[rp] + first[(size_t)rp * ncb + b] + __popcll(mk & ((1ull << jt) - 1ull));
+    };
+    for (int q4 = 0; q4 < ps; q4 += 4)
+      e[q4 >> 2] = make_uint4((uint32_t)word(q4), (uint32_t)word(q4 + 1), (uint32_t)word(q4 + 2), (uint32_t)word(q4 + 3));
   }
   if (tid == 0) {
     float m = 0.f;
