@@ -26,6 +26,13 @@ Readings where the pages are silent (each listed again in the design notes):
   rounding fma(code, s, z);
 * residual key groups are 64 consecutive compact rows ("slots") of one encode
   call, per channel; a call's last group may be partial;
+* codec variants (the ablations named in [Guide] section 4, the "Per-loop KIVI4"
+  row and the 2-bit row of Figure 5, and the [Project] "Experiments" caption of
+  Figure 5, right: residual precision varied): "per-loop KIVI4" stores each loop
+  r >= 2 as INT4 codes of the full state X^(r) of its active rows (grouped like the
+  residual stores), and a token's loop-r state is then that one store, the one of
+  loop min(r, depth); "INT2 residuals" keeps the INT4 base and quantises the
+  residuals with 2-bit codes, s = fp16((max - min) / 3);
 * the BF16 tail holds the most recent 1..64 columns of every loop;
 * token-sparse updates rank the tokens of A_{r-1} by the squared relative L2 change
   ||h^(r-1) - h^(r-2)||^2 / ||h^(r-2)||^2 of their hidden state over loop r-1, in
@@ -50,6 +57,12 @@ HEAD_DIM = 128
 GROUP = 64
 TAIL = 64
 LEVELS = 15  # 4-bit codes 0..15
+LEVELS2 = 3  # 2-bit codes 0..3
+
+# Codecs of the loop r >= 2 stores (the base is always 4-bit):
+RESIDUAL_INT4 = 0  # X^(r) - X_hat^(r-1), 4-bit (the method)
+FULL_INT4 = 1      # X^(r) itself, 4-bit ("per-loop KIVI4")
+RESIDUAL_INT2 = 2  # X^(r) - X_hat^(r-1), 2-bit
 
 
 # ----------------------------------------------------------------------------
@@ -61,24 +74,24 @@ def half_rn(x) -> np.ndarray:
     return np.asarray(x, dtype=F32).astype(F16)
 
 
-def quantize(x, axis: int = -1):
-    """Quantise every group laid out along ``axis`` to 4-bit codes.
+def quantize(x, axis: int = -1, levels: int = LEVELS):
+    """Quantise every group laid out along ``axis`` to codes 0 .. levels (15: 4-bit).
 
     Returns (codes uint8 with x's shape, scale fp16, zero fp16) where scale and
     zero have ``axis`` removed.  Arithmetic is fp32 with one rounding per
-    operation: s = fp16((max - min) / 15), z = fp16(min),
-    code = clamp(rint((x - z) / s), 0, 15), and 0 when s is zero.
+    operation: s = fp16((max - min) / levels), z = fp16(min),
+    code = clamp(rint((x - z) / s), 0, levels), and 0 when s is zero.
     """
     x = np.moveaxis(np.asarray(x, dtype=F32), axis, -1)
     mn = x.min(axis=-1)
     mx = x.max(axis=-1)
-    s = half_rn(np.subtract(mx, mn, dtype=F32) / F32(LEVELS))
+    s = half_rn(np.subtract(mx, mn, dtype=F32) / F32(levels))
     z = half_rn(mn)
     sf = s.astype(F32)[..., None]
     zf = z.astype(F32)[..., None]
     with np.errstate(divide="ignore", invalid="ignore"):
         t = np.subtract(x, zf, dtype=F32) / sf
-    codes = np.clip(np.rint(t), 0, LEVELS)
+    codes = np.clip(np.rint(t), 0, levels)
     codes = np.where(sf == 0, F32(0), codes)
     return np.moveaxis(codes.astype(np.uint8), -1, axis), s, z
 
@@ -123,13 +136,13 @@ def decode_base(enc: dict):
     return kh, vh
 
 
-def encode_residual(EK, EV) -> dict:
+def encode_residual(EK, EV, levels: int = LEVELS) -> dict:
     """Quantise the residual rows of one encode call, given in slot order.
 
     EK, EV: fp32 [H][n][128].  Keys: one group per (64 consecutive slots,
     channel); the last group holds only the rows present.  Values: one group per
     (row, 64-channel half).  Returns kc/vc uint8 [H][n][128], ks/kz fp16
-    [H][ceil(n/64)][128], vs/vz fp16 [H][n][2].
+    [H][ceil(n/64)][128], vs/vz fp16 [H][n][2].  ``levels`` 3 gives 2-bit codes.
     """
     EK = np.asarray(EK, F32)
     EV = np.asarray(EV, F32)
@@ -140,8 +153,8 @@ def encode_residual(EK, EV) -> dict:
     kz = np.zeros((H, ng, D), F16)
     for g in range(ng):
         sl = slice(g * GROUP, min(n, (g + 1) * GROUP))
-        kc[:, sl], ks[:, g], kz[:, g] = quantize(EK[:, sl, :], axis=1)
-    vc, vs, vz = quantize(EV.reshape(H, n, 2, D // 2), axis=3)
+        kc[:, sl], ks[:, g], kz[:, g] = quantize(EK[:, sl, :], axis=1, levels=levels)
+    vc, vs, vz = quantize(EV.reshape(H, n, 2, D // 2), axis=3, levels=levels)
     return dict(kc=kc, ks=ks, kz=kz, vc=vc.reshape(H, n, D), vs=vs, vz=vz)
 
 
@@ -325,8 +338,9 @@ class OracleLayer:
     loop, and the attention state (p_tilde, lam) the sparse loops need.
     """
 
-    def __init__(self, heads: int, loops: int, capacity: int):
-        self.H, self.R, self.cap = heads, loops, capacity
+    def __init__(self, heads: int, loops: int, capacity: int, codec: int = RESIDUAL_INT4):
+        assert codec in (RESIDUAL_INT4, FULL_INT4, RESIDUAL_INT2)
+        self.H, self.R, self.cap, self.codec = heads, loops, capacity, codec
         D = HEAD_DIM
         self.n_q = 0
         self.n_tail = 0
@@ -365,24 +379,30 @@ class OracleLayer:
         return enc
 
     def encode_residual(self, r: int, rows, Kr, Vr):
-        """Loop-r residuals of the active ``rows`` (ascending token ids) of one call.
+        """Loop-r store of the active ``rows`` (ascending token ids) of one call.
 
         Kr, Vr: fp32 [H][n][128], the loop-r keys/values of those rows.  The
-        residual is taken against the reconstructed state of loop r-1.
+        residual is taken against the reconstructed state of loop r-1 and added back
+        onto it; with the per-loop KIVI4 codec the store holds the state itself and
+        replaces the earlier reconstruction.
         """
         rows = np.asarray(rows, np.int64)
         assert 2 <= r <= self.R
         if rows.size:
             assert np.all(np.diff(rows) > 0) and rows[-1] < self.n_q
             assert np.all(self.depth[rows] >= r - 1), "active sets must nest"
-        prev_k = self.khat[r - 1][:, rows]
-        prev_v = self.vhat[r - 1][:, rows]
-        EK = np.subtract(np.asarray(Kr, F32), prev_k, dtype=F32)
-        EV = np.subtract(np.asarray(Vr, F32), prev_v, dtype=F32)
-        enc = encode_residual(EK, EV)
-        dk, dv = decode_residual(enc)
-        newk = np.add(prev_k, dk, dtype=F32)
-        newv = np.add(prev_v, dv, dtype=F32)
+        if self.codec == FULL_INT4:
+            enc = encode_residual(np.asarray(Kr, F32), np.asarray(Vr, F32))
+            newk, newv = decode_residual(enc)
+        else:
+            prev_k = self.khat[r - 1][:, rows]
+            prev_v = self.vhat[r - 1][:, rows]
+            EK = np.subtract(np.asarray(Kr, F32), prev_k, dtype=F32)
+            EV = np.subtract(np.asarray(Vr, F32), prev_v, dtype=F32)
+            enc = encode_residual(EK, EV, LEVELS2 if self.codec == RESIDUAL_INT2 else LEVELS)
+            dk, dv = decode_residual(enc)
+            newk = np.add(prev_k, dk, dtype=F32)
+            newv = np.add(prev_v, dv, dtype=F32)
         for rr in range(r, self.R + 1):
             self.khat[rr][:, rows] = newk
             self.vhat[rr][:, rows] = newv
