@@ -18,7 +18,10 @@
  *   [Guide]   flozi.net "FlashLoop: store changes between repeated passes", section 3:
  *             per-channel (post-RoPE) key groups, per-token value groups, residuals of
  *             active tokens only; sparse loops are a rank-K correction of the previous
- *             loop's output.
+ *             loop's output.  Section 4: the "Per-loop KIVI4" ablation (full KV states
+ *             quantised per loop instead of residuals) and the 2-bit residual row of
+ *             Figure 5; the project page's "Experiments" caption of Figure 5 (residual
+ *             precision varied).
  *
  * Conventions for every entry point
  *   - All data pointers are DEVICE pointers owned by the caller.  The library never
@@ -43,6 +46,20 @@
  *   slots of one encode call, channel) in a residual store; value groups are
  *   (token or slot, 64-channel half).
  *
+ * Codecs of the loop r >= 2 stores (fl_dims.codec; the base is always the 4-bit
+ * quantiser of loop-1 K/V):
+ *   FL_CODEC_RESIDUAL_INT4  the method: store r holds E = X^(r) - X_hat^(r-1) of the
+ *                           rows active in loop r, 4-bit; a token's loop-r state is the
+ *                           base plus its stores 2 .. min(r, depth), added in loop order.
+ *   FL_CODEC_FULL_INT4      per-loop KIVI4: store r holds X^(r) itself, 4-bit, same
+ *                           groups; a token's loop-r state is its store min(r, depth)
+ *                           alone (the base when that is 1).
+ *   FL_CODEC_RESIDUAL_INT2  residuals as in the method with 2-bit codes:
+ *                           s = fp16_rn(fp32_rn(max - min) / 3), code = clamp(.., 0, 3),
+ *                           in 5120-byte residual records (below).
+ *   The variants are served by the direct readers and the encode entry points; the
+ *   fused tail flush (fl_decode_step_flush) takes FL_CODEC_RESIDUAL_INT4 only.
+ *
  * Packed cache layout (one buffer of fl_cache_layout().total_bytes; every array
  * starts on a 256-byte boundary; L layers, H heads, C = capacity, T = total slots,
  * R loops; "sz" = a (scale, zero) fp16 pair stored as scale in the low half of a
@@ -54,8 +71,17 @@
  *                         2b+1 (high nibble)
  *     bytes [8192, 8704)  64 x 2 value sz: row i, half h (channels 64h..64h+63)
  *     bytes [8704, 9216)  128 key sz: one per channel of the group
+ *   With FL_CODEC_RESIDUAL_INT2 the residual records are 5120 bytes:
+ *     bytes [0, 4096)     64 rows x 64 B: row i = 32 B of key codes then 32 B of value
+ *                         codes; 32-bit word w of a part holds channels 16w .. 16w+15:
+ *                         channel 16w+k (k < 8) in bits 4k..4k+1 and channel 16w+8+k in
+ *                         bits 4k+2..4k+3 (so word & 0x33333333 and (word >> 2) &
+ *                         0x33333333 are the two 8-channel words of the 4-bit layout)
+ *     bytes [4096, 4608)  64 x 2 value sz
+ *     bytes [4608, 5120)  128 key sz
  *   brec   u8  [L][H][C/64][9216]  base group records (loop 1), block b = tokens 64b..64b+63
- *   rrec   u8  [L][H][T/64][9216]  residual group records of every loop; loop r owns slots
+ *   rrec   u8  [L][H][T/64][RB]    residual group records of every loop (RB = 9216, or 5120
+ *                                   with 2-bit codes); loop r owns slots
  *                                   [slot_base[r], slot_base[r] + res_capacity[r])
  *   mask   u64 [L][R+1][C/64]      bit t of mask[r][b]: token 64b+t has a loop-r residual
  *   first  i32 [L][R+1][C/64]      slot (within loop r's store) of block b's first loop-r row;
@@ -112,6 +138,12 @@ typedef enum fl_status {
 #define FL_DEV_TAG_RANGE 5    /* a column's loop tag outside [1, R] */
 #define FL_DEV_TIMEOUT 6      /* a bounded wait for staged data ran out (the kernel returned early) */
 #define FL_GROUP_RECORD 9216  /* bytes of one group record */
+#define FL_GROUP_RECORD_INT2 5120  /* bytes of one 2-bit residual group record */
+
+/* fl_dims.codec: what the loop r >= 2 stores hold (see the codec notes above). */
+#define FL_CODEC_RESIDUAL_INT4 0
+#define FL_CODEC_FULL_INT4 1
+#define FL_CODEC_RESIDUAL_INT2 2
 
 typedef struct fl_dims {
   int32_t layers;      /* L >= 1 */
@@ -122,6 +154,7 @@ typedef struct fl_dims {
   int32_t capacity;    /* max columns N = quantised + tail; a positive multiple of 64 */
   int32_t max_select;  /* capacity of the selected-column list per (layer, head), >= 1 */
   int32_t res_capacity[FL_MAX_LOOPS + 1]; /* slots of loop r's residual store, r = 2..R, multiples of 64 */
+  int32_t codec;       /* FL_CODEC_*: 0 (zero-initialised) is the method's INT4 residuals */
 } fl_dims;
 
 typedef struct fl_layout {

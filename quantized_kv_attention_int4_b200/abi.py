@@ -28,6 +28,9 @@ N_ARRAYS = 14
 ARRAY_NAMES = ("brec", "rrec", "mask", "first", "depth", "tail_k", "tail_v", "score", "tag", "offset", "sel",
                "mass", "unsel", "plan")
 GROUP_RECORD = 9216
+GROUP_RECORD_INT2 = 5120
+# codecs of the loop r >= 2 stores (fl_dims.codec)
+FL_CODEC_RESIDUAL_INT4, FL_CODEC_FULL_INT4, FL_CODEC_RESIDUAL_INT2 = 0, 1, 2
 
 FL_OK, FL_ERR_INVALID, FL_ERR_UNSUPPORTED, FL_ERR_CUDA, FL_ERR_WORKSPACE, FL_ERR_DEVICE = 0, -1, -2, -3, -4, -6
 # device error codes recorded in status words (include/flashloop.h)
@@ -42,7 +45,8 @@ EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init"
 class fl_dims(ctypes.Structure):
     _fields_ = [("layers", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("group", ctypes.c_int32), ("loops", ctypes.c_int32), ("capacity", ctypes.c_int32),
-                ("max_select", ctypes.c_int32), ("res_capacity", ctypes.c_int32 * (MAX_LOOPS + 1))]
+                ("max_select", ctypes.c_int32), ("res_capacity", ctypes.c_int32 * (MAX_LOOPS + 1)),
+                ("codec", ctypes.c_int32)]
 
 
 class fl_layout(ctypes.Structure):
@@ -106,11 +110,12 @@ def _check(where: str, st: int):
         raise FlashLoopError(where, st)
 
 
-def Dims(layers: int, heads: int, loops: int, capacity: int, max_select: int, res_capacity) -> fl_dims:
+def Dims(layers: int, heads: int, loops: int, capacity: int, max_select: int, res_capacity,
+         codec: int = FL_CODEC_RESIDUAL_INT4) -> fl_dims:
     """fl_dims with head_dim 128 / group 64; res_capacity[r] for r = 2..loops (mapping or list)."""
     d = fl_dims()
     d.layers, d.heads, d.head_dim, d.group = layers, heads, HEAD_DIM, GROUP
-    d.loops, d.capacity, d.max_select = loops, capacity, max_select
+    d.loops, d.capacity, d.max_select, d.codec = loops, capacity, max_select, codec
     items = res_capacity.items() if isinstance(res_capacity, dict) else enumerate(res_capacity)
     for r, v in items:
         d.res_capacity[r] = int(v)

@@ -36,15 +36,15 @@ def split_prefill(n_cols: int) -> tuple[int, int]:
 
 class FlashLoopCache:
     def __init__(self, layers: int, heads: int, loops: int, capacity: int, res_capacity=None,
-                 max_select: int | None = None, device="cuda"):
+                 max_select: int | None = None, device="cuda", codec: int = abi.FL_CODEC_RESIDUAL_INT4):
         capacity = round_up(capacity)
         if res_capacity is None:
             res_capacity = {r: capacity for r in range(2, loops + 1)}
         if max_select is None:
             max_select = capacity
-        self.L, self.H, self.R, self.capacity = layers, heads, loops, capacity
+        self.L, self.H, self.R, self.capacity, self.codec = layers, heads, loops, capacity, codec
         self.device = torch.device(device)
-        self.dims = abi.Dims(layers, heads, loops, capacity, max_select, res_capacity)
+        self.dims = abi.Dims(layers, heads, loops, capacity, max_select, res_capacity, codec)
         self.layout = abi.fl_cache_layout(self.dims)
         self.buf = torch.empty(self.layout.total_bytes, dtype=torch.uint8, device=self.device)
         abi.fl_cache_init(self.dims, self.buf)

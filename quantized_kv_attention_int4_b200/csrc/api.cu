@@ -18,6 +18,8 @@ fl_status check_dims(const fl_dims* d) {
   if (d->layers < 1 || d->heads < 1 || d->loops < 1 || d->loops > FL_MAX_LOOPS) return FL_ERR_INVALID;
   if (d->capacity < FL_GROUP || d->capacity % FL_GROUP != 0) return FL_ERR_INVALID;
   if (d->max_select < 1) return FL_ERR_INVALID;
+  if (d->codec != FL_CODEC_RESIDUAL_INT4 && d->codec != FL_CODEC_FULL_INT4 && d->codec != FL_CODEC_RESIDUAL_INT2)
+    return FL_ERR_UNSUPPORTED;
   for (int r = 2; r <= d->loops; ++r)
     if (d->res_capacity[r] < 0 || d->res_capacity[r] % FL_GROUP != 0) return FL_ERR_INVALID;
   return FL_OK;
@@ -36,7 +38,8 @@ void layer_sizes(const fl_dims* d, uint64_t* sz, int32_t* slot_base, int32_t* to
   }
   *total_slots = (int32_t)T;
   sz[A_BREC] = H * (C / 64) * (uint64_t)FL_GROUP_RECORD;
-  sz[A_RREC] = H * (T / 64) * (uint64_t)FL_GROUP_RECORD;
+  const uint64_t rrec_bytes = d->codec == FL_CODEC_RESIDUAL_INT2 ? FL_GROUP_RECORD_INT2 : FL_GROUP_RECORD;
+  sz[A_RREC] = H * (T / 64) * rrec_bytes;
   sz[A_MASK] = (R + 1) * (C / 64) * 8;
   sz[A_FIRST] = (R + 1) * (C / 64) * 4;
   sz[A_DEPTH] = C;
@@ -92,6 +95,7 @@ CacheView make_view(const fl_dims* d, const fl_layout& L, void* cache) {
   v.total_slots = L.total_slots;
   v.max_select = d->max_select;
   v.plan_stride = L.plan_stride;
+  v.codec = d->codec;
   return v;
 }
 
@@ -423,6 +427,7 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
   if (dense_loops < 0 || dense_loops > R || loop_first < 1 || loop_last > R || loop_first > loop_last)
     return FL_ERR_INVALID;
   if (flush) {
+    if (dims->codec != FL_CODEC_RESIDUAL_INT4) return FL_ERR_UNSUPPORTED;  // the fused flush writes 4-bit residuals
     if (n_tail != FL_TAIL || (int64_t)n_q + FL_TAIL > dims->capacity || !flush->slot0) return FL_ERR_INVALID;
     uint64_t prev = ~0ull;
     for (int r = 2; r <= R; ++r) {

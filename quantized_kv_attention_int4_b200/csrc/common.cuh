@@ -32,6 +32,40 @@ constexpr int kRec = FL_GROUP_RECORD;
 constexpr int kRecVsz = 8192;
 constexpr int kRecKsz = 8704;
 
+// Byte geometry of a group record with kBits-bit codes: 4 (the base, and the residual
+// stores of the 4-bit codecs) or 2 (2-bit residual stores: 64-byte rows of 32 B key
+// codes and 32 B value codes, the value and key (scale, zero) words after them).
+template <int kBits>
+struct Rec {
+  static constexpr int kBytes = kBits == 4 ? FL_GROUP_RECORD : FL_GROUP_RECORD_INT2;
+  static constexpr int kRow = kBits == 4 ? 128 : 64;  // bytes of one row
+  static constexpr int kHalf = kRow / 2;              // offset of the value codes in a row
+  static constexpr int kVsz = kG * kRow;
+  static constexpr int kKsz = kVsz + kG * 8;
+  static constexpr float kLevels = kBits == 4 ? 15.0f : 3.0f;
+  static constexpr int kMaxCode = kBits == 4 ? 15 : 3;
+};
+static_assert(Rec<4>::kVsz == kRecVsz && Rec<4>::kKsz == kRecKsz, "4-bit record geometry");
+static_assert(Rec<2>::kKsz + 512 == FL_GROUP_RECORD_INT2, "2-bit record geometry");
+
+// What the loop r >= 2 stores of a codec hold (FL_CODEC_*): full states or residuals,
+// and their code width.
+template <int kCodec>
+struct CodecT {
+  static constexpr bool kFullState = kCodec == FL_CODEC_FULL_INT4;
+  static constexpr int kResBits = kCodec == FL_CODEC_RESIDUAL_INT2 ? 2 : 4;
+};
+
+// A 2-bit record word holds channels 16w .. 16w + 15: channel 16w + k (k < 8) in bits
+// 4k .. 4k + 1 and 16w + 8 + k in bits 4k + 2 .. 4k + 3.  Masking gives the 4-bit
+// layout's 8-channel words (channel k in nibble k) with codes 0 .. 3.
+constexpr uint32_t kInt2Mask = 0x33333333u;
+__device__ __forceinline__ uint32_t int2_word(uint32_t w, int upper) { return (w >> (2 * upper)) & kInt2Mask; }
+// 32 consecutive channels of 2-bit codes (8 bytes) as the 16-byte 4-bit layout.
+__device__ __forceinline__ uint4 int2_to_nib(uint2 x) {
+  return make_uint4(x.x & kInt2Mask, (x.x >> 2) & kInt2Mask, x.y & kInt2Mask, (x.y >> 2) & kInt2Mask);
+}
+
 // Device view of one cache buffer: base pointer, array offsets and per-layer strides.
 struct CacheView {
   uint8_t* base;
@@ -40,6 +74,7 @@ struct CacheView {
   int32_t slot_base[FL_MAX_LOOPS + 1];
   int32_t* status;
   int32_t H, R, cap, total_slots, max_select, plan_stride;
+  int32_t codec;  // FL_CODEC_*
 };
 
 template <class T>

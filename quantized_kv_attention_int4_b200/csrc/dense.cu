@@ -21,6 +21,14 @@
 //      128 p s and a per-half correction sum(p z - 128 p s).
 // Warps merge in shared memory, CTAs write (M, L, o) partials, and the last CTA of
 // each head (an atomic ticket, no waiting) combines them by log-sum-exp.
+//
+// Codec variants (flozi guide, section 4: the "Per-loop KIVI4" row and the 2-bit row
+// of Figure 5): with 2-bit residual stores each row quarter is loaded as 8 bytes and
+// widened to the 4-bit layout (codes 0..3), the arithmetic is unchanged; with
+// full-state stores a token's loop-r key/value is its store min(r, depth) alone, so
+// each store contributes only the rows of tokens whose last store it is, and their
+// logits are assigned rather than added (the base is skipped when every token of the
+// block has a later store).
 #include "flush.cuh"
 #include "kernels.h"
 
@@ -29,18 +37,30 @@ namespace {
 
 constexpr int kWarps = 8;
 
-// kFlush: the step also writes this loop's store of a full tail (fused flush)
-template <bool kFlush>
+// kFlush: the step also writes this loop's store of a full tail (fused flush);
+// kCodec: FL_CODEC_* of the loop r >= 2 stores
+template <bool kFlush, int kCodec>
 __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs a) {
+  using CT = CodecT<kCodec>;
+  using RB = Rec<CT::kResBits>;
   const int h = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, qq = lane & 3, tr = lane >> 2;
   const CacheView& c = a.c;
   const int H = c.H, cap = c.cap, ncb = cap / kG, T = c.total_slots, r = a.r;
 
   const uint8_t* brec = arr<uint8_t>(c, A_BREC, a.layer) + (size_t)h * ncb * kRec;
-  const uint8_t* rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * kRec;
+  const uint8_t* rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * RB::kBytes;
   // residual slot gs: row (gs & 63) of group record (gs >> 6)
-  auto rrow = [&](int gs) { return rrec + (size_t)(gs >> 6) * kRec + (size_t)(gs & 63) * 128; };
+  auto rrow = [&](int gs) { return rrec + (size_t)(gs >> 6) * RB::kBytes + (size_t)(gs & 63) * RB::kRow; };
+  // quarter qq of a residual row's key / value codes in the 4-bit layout
+  auto res_key = [&](const uint8_t* row) -> uint4 {
+    if constexpr (CT::kResBits == 4) return __ldg(reinterpret_cast<const uint4*>(row) + qq);
+    else return int2_to_nib(__ldg(reinterpret_cast<const uint2*>(row) + qq));
+  };
+  auto res_val = [&](const uint8_t* row) -> uint4 {
+    if constexpr (CT::kResBits == 4) return __ldg(reinterpret_cast<const uint4*>(row + RB::kHalf) + qq);
+    else return int2_to_nib(__ldg(reinterpret_cast<const uint2*>(row + RB::kHalf) + qq));
+  };
   const unsigned long long* mask = arr<unsigned long long>(c, A_MASK, a.layer);
   const int32_t* first = arr<int32_t>(c, A_FIRST, a.layer);
   uint16_t* tail_k = arr<uint16_t>(c, A_TAILK, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
@@ -77,27 +97,34 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
     float qsr[32];
     if (u < nb) {
       const int b = u;
+      // full-state stores: tokens whose key/value is the base (no store of loops 2..r)
+      const unsigned long long need_b = (CT::kFullState && r >= 2) ? ~mask[(size_t)2 * ncb + b] : ~0ull;
       // ---- keys: base ----
-      __syncwarp();
-      const uint8_t* rec = brec + (size_t)b * kRec;
-      float cb = group_weights(reinterpret_cast<const uint32_t*>(rec + kRecKsz), q_s, qsw, lane);
-      __syncwarp();
-      load32(qsw + 32 * qq, qsr);
-      const uint4* kc = reinterpret_cast<const uint4*>(rec);
-      uint4 w[8];
+      if (need_b) {
+        __syncwarp();
+        const uint8_t* rec = brec + (size_t)b * kRec;
+        float cb = group_weights(reinterpret_cast<const uint32_t*>(rec + kRecKsz), q_s, qsw, lane);
+        __syncwarp();
+        load32(qsw + 32 * qq, qsr);
+        const uint4* kc = reinterpret_cast<const uint4*>(rec);
+        uint4 w[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] = __ldg(kc + (8 * i + tr) * 8 + qq);
+        for (int i = 0; i < 8; ++i) w[i] = __ldg(kc + (8 * i + tr) * 8 + qq);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float p = dot32(w[i], qsr);
-        p += __shfl_xor_sync(kFull, p, 1);
-        p += __shfl_xor_sync(kFull, p, 2);
-        if (qq == 0) lgw[8 * i + tr] = p + cb;
+        for (int i = 0; i < 8; ++i) {
+          float p = dot32(w[i], qsr);
+          p += __shfl_xor_sync(kFull, p, 1);
+          p += __shfl_xor_sync(kFull, p, 2);
+          if (qq == 0) lgw[8 * i + tr] = p + cb;
+        }
       }
-      // ---- keys: residual loops 2..r ----
+      // ---- keys: stores of loops 2..r ----
       for (int rp = 2; rp <= r; ++rp) {
         const unsigned long long mk = mask[(size_t)rp * ncb + b];
-        if (mk == 0ull) continue;
+        // full-state: only the tokens whose last store in loop r is this one
+        const unsigned long long need =
+            CT::kFullState && rp < r ? mk & ~mask[(size_t)(rp + 1) * ncb + b] : mk;
+        if (need == 0ull) continue;
         const int na = __popcll(mk);
         const int gs0 = c.slot_base[rp] + first[(size_t)rp * ncb + b];
         __syncwarp();
@@ -109,18 +136,21 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
           const int row_end = min(na, ((grp + 1) << 6) - gs0);
           __syncwarp();
           const float cg = group_weights(
-              reinterpret_cast<const uint32_t*>(rrec + (size_t)grp * kRec + kRecKsz), q_s, qsw, lane);
+              reinterpret_cast<const uint32_t*>(rrec + (size_t)grp * RB::kBytes + RB::kKsz), q_s, qsw, lane);
           __syncwarp();
           load32(qsw + 32 * qq, qsr);
           for (int i0 = row; i0 < row_end; i0 += 8) {
             const int rw = i0 + tr;
-            const bool act = rw < row_end;
+            const bool act = rw < row_end && (!CT::kFullState || ((need >> tokw[rw]) & 1ull));
             uint4 x = make_uint4(0u, 0u, 0u, 0u);
-            if (act) x = __ldg(reinterpret_cast<const uint4*>(rrow(gs0 + rw)) + qq);
+            if (act) x = res_key(rrow(gs0 + rw));
             float p = dot32(x, qsr);
             p += __shfl_xor_sync(kFull, p, 1);
             p += __shfl_xor_sync(kFull, p, 2);
-            if (act && qq == 0) lgw[tokw[rw]] += p + cg;
+            if (act && qq == 0) {
+              if constexpr (CT::kFullState) lgw[tokw[rw]] = p + cg;
+              else lgw[tokw[rw]] += p + cg;
+            }
           }
           row = row_end;
         }
@@ -150,7 +180,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
       lgw[lane + 32] = p1;
       __syncwarp();
       // ---- values: base ----
-      {
+      if (need_b) {
         const uint8_t* rec = brec + (size_t)b * kRec;
         const uint4* vc = reinterpret_cast<const uint4*>(rec);
         const uint32_t* vs = reinterpret_cast<const uint32_t*>(rec + kRecVsz);
@@ -163,17 +193,19 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float p = lgw[8 * i + tr];
+          const float p = ((need_b >> (8 * i + tr)) & 1ull) ? lgw[8 * i + tr] : 0.f;
           const float2 sz = unpack_sz(sw[i]);
           const float P = 128.f * (p * sz.x);
           corr += fmaf(p, sz.y, -P);
           axpy32(vw[i], P, acc);
         }
       }
-      // ---- values: residual loops ----
+      // ---- values: stores of loops 2..r ----
       for (int rp = 2; rp <= r; ++rp) {
         const unsigned long long mk = mask[(size_t)rp * ncb + b];
-        if (mk == 0ull) continue;
+        const unsigned long long need =
+            CT::kFullState && rp < r ? mk & ~mask[(size_t)(rp + 1) * ncb + b] : mk;
+        if (need == 0ull) continue;
         const int na = __popcll(mk);
         const int gs0 = c.slot_base[rp] + first[(size_t)rp * ncb + b];
         __syncwarp();
@@ -182,11 +214,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
         __syncwarp();
         for (int i0 = 0; i0 < na; i0 += 8) {
           const int rw = i0 + tr;
-          if (rw < na) {
+          if (rw < na && (!CT::kFullState || ((need >> tokw[rw]) & 1ull))) {
             const int gs = gs0 + rw;
-            const uint4 x = __ldg(reinterpret_cast<const uint4*>(rrow(gs)) + 4 + qq);
+            const uint4 x = res_val(rrow(gs));
             const float2 sz = unpack_sz(__ldg(reinterpret_cast<const uint32_t*>(
-                rrec + (size_t)(gs >> 6) * kRec + kRecVsz) + (gs & 63) * 2 + (qq >> 1)));
+                rrec + (size_t)(gs >> 6) * RB::kBytes + RB::kVsz) + (gs & 63) * 2 + (qq >> 1)));
             const float p = lgw[tokw[rw]];
             const float P = 128.f * (p * sz.x);
             corr += fmaf(p, sz.y, -P);
@@ -345,10 +377,14 @@ int dense_splits(int heads, int n_q) {
 cudaError_t launch_dense_direct(ReaderArgs a, cudaStream_t s) {
   a.n_splits = dense_splits(a.c.H, a.n_q);
   dim3 grid(a.n_splits, a.c.H);
-  if (a.flush)
-    dense_direct_kernel<true><<<grid, kWarps * 32, sizeof(EncodeSmem), s>>>(a);
+  if (a.c.codec == FL_CODEC_FULL_INT4)
+    dense_direct_kernel<false, FL_CODEC_FULL_INT4><<<grid, kWarps * 32, 0, s>>>(a);
+  else if (a.c.codec == FL_CODEC_RESIDUAL_INT2)
+    dense_direct_kernel<false, FL_CODEC_RESIDUAL_INT2><<<grid, kWarps * 32, 0, s>>>(a);
+  else if (a.flush)
+    dense_direct_kernel<true, FL_CODEC_RESIDUAL_INT4><<<grid, kWarps * 32, sizeof(EncodeSmem), s>>>(a);
   else
-    dense_direct_kernel<false><<<grid, kWarps * 32, 0, s>>>(a);
+    dense_direct_kernel<false, FL_CODEC_RESIDUAL_INT4><<<grid, kWarps * 32, 0, s>>>(a);
   return cudaGetLastError();
 }
 

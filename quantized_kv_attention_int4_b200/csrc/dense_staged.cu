@@ -675,7 +675,8 @@ cudaError_t launch_dense(ReaderArgs a, cudaStream_t s, bool chain) {
   const long long U = (long long)a.c.H * (a.n_q / kG + 1);
   long long n = sms < U ? sms : U;
   if (n < a.c.H) n = a.c.H;  // every CTA range then touches at most two heads
-  if (a.r > 3 || sms == 0 || n > kMaxSplits) return launch_dense_direct(a, s);
+  // the codec variants are served by the direct reader
+  if (a.c.codec != FL_CODEC_RESIDUAL_INT4 || a.r > 3 || sms == 0 || n > kMaxSplits) return launch_dense_direct(a, s);
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);

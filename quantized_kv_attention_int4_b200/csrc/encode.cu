@@ -1,10 +1,13 @@
-// Base (loop 1) and residual (loop r >= 2) INT4 encoders.
+// Base (loop 1) and residual (loop r >= 2) encoders.
 //
 // FlashLoop project page, "The Method", Step 03: loop-1 K/V are quantised as the
 // base; each later loop stores only its residual against the reconstructed state of
 // the preceding loop.  flozi guide "FlashLoop: store changes between repeated
 // passes", section 3: group-wise asymmetric 4-bit, group 64, keys per channel,
-// values per token, residuals for active tokens only.
+// values per token, residuals for active tokens only.  Section 4 of the same guide
+// (the "Per-loop KIVI4" row, and the 2-bit row of Figure 5) gives the two codec
+// variants of the loop r >= 2 stores: the full state X^(r) in 4 bits, or the residual
+// in 2 bits.
 //
 // Every arithmetic step of the quantiser is one IEEE fp32 operation with explicit
 // round-to-nearest intrinsics so that codes, scales and zero points are exact
@@ -57,7 +60,10 @@ __global__ void __launch_bounds__(256) encode_base_kernel(EncodeBaseArgs a) {
   }
 }
 
+template <int kCodec>
 __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
+  using CT = CodecT<kCodec>;
+  constexpr int kRB = CT::kResBits;
   const int g = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   const CacheView& c = a.c;
   const int cap = c.cap, ncb = cap / kG, T = c.total_slots, r = a.r;
@@ -92,14 +98,14 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
 
   const int gslot0 = c.slot_base[r] + a.slot0 + i0;  // a multiple of 64
   const uint8_t* brec = arr<uint8_t>(c, A_BREC, a.layer) + (size_t)h * ncb * kRec;
-  uint8_t* rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * kRec;
-  uint8_t* orec = rrec + (size_t)(gslot0 >> 6) * kRec;  // this CTA's output group record
+  uint8_t* rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * Rec<kRB>::kBytes;
+  uint8_t* orec = rrec + (size_t)(gslot0 >> 6) * Rec<kRB>::kBytes;  // this CTA's output group record
 
   for (int part = 0; part < 2; ++part) {
     const bool is_v = part == 1;
     const uint16_t* src = is_v ? a.v : a.k;
 
-    // residual E = X^(r) - X_hat^(r-1) for 8 channels per item
+    // residual E = X^(r) - X_hat^(r-1) (the full-state codec: X^(r) itself), 8 channels per item
     for (int item = tid; item < kG * 16; item += 256) {
       const int tt = item >> 4, c8 = (item & 15) * 8;
       const int j = tok[tt];
@@ -111,17 +117,23 @@ __global__ void __launch_bounds__(256) encode_residual_kernel(EncodeResArgs a) {
       const size_t row = a.compact ? (size_t)(i0 + tt) : (size_t)(j - a.row0);
       float x[8];
       bf16x8(ldg_u4(src + (size_t)h * a.head_stride + row * kD + c8), x);
-      float xh[8];
-      recon8<false>(c, brec, rrec, mask, first, j, r, is_v, c8, xh);
+      if constexpr (CT::kFullState) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) xs[tt][c8 + e] = __fsub_rn(x[e], xh[e]);
+        for (int e = 0; e < 8; ++e) xs[tt][c8 + e] = x[e];
+      } else {
+        float xh[8];
+        recon8<false, kRB>(c, brec, rrec, mask, first, j, r, is_v, c8, xh);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xs[tt][c8 + e] = __fsub_rn(x[e], xh[e]);
+      }
     }
     __syncthreads();
 
-    if (is_v) value_params(sm, orec, 0, kG, nr, tid, 256);
-    else key_params(sm, orec, 0, kD, nr, tid, 256);
+    if (is_v) value_params<kRB>(sm, orec, 0, kG, nr, tid, 256);
+    else key_params<kRB>(sm, orec, 0, kD, nr, tid, 256);
     __syncthreads();
-    group_codes(sm, orec, is_v, 0, kG, 0, kD / 8, nr, tid, 256);
+    if constexpr (kRB == 4) group_codes(sm, orec, is_v, 0, kG, 0, kD / 8, nr, tid, 256);
+    else group_codes2(sm, orec, is_v, nr, tid, 256);
     __syncthreads();
   }
 
@@ -149,7 +161,12 @@ cudaError_t launch_encode_base(const EncodeBaseArgs& a, cudaStream_t s) {
 cudaError_t launch_encode_residual(const EncodeResArgs& a, cudaStream_t s) {
   if (a.n_rows == 0) return cudaSuccess;
   dim3 grid((a.n_rows + kG - 1) / kG, a.c.H);
-  encode_residual_kernel<<<grid, 256, 0, s>>>(a);
+  if (a.c.codec == FL_CODEC_FULL_INT4)
+    encode_residual_kernel<FL_CODEC_FULL_INT4><<<grid, 256, 0, s>>>(a);
+  else if (a.c.codec == FL_CODEC_RESIDUAL_INT2)
+    encode_residual_kernel<FL_CODEC_RESIDUAL_INT2><<<grid, 256, 0, s>>>(a);
+  else
+    encode_residual_kernel<FL_CODEC_RESIDUAL_INT4><<<grid, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -1,11 +1,13 @@
-// INT4 group quantiser shared by the encode kernels and the readers' fused tail flush.
+// Group quantiser shared by the encode kernels and the readers' fused tail flush.
 //
 // flozi guide "FlashLoop: store changes between repeated passes", section 3:
 // group-wise asymmetric 4-bit codes, group 64, keys grouped per channel, values per
-// token.  Every arithmetic step is one IEEE fp32 operation with an explicit
-// round-to-nearest intrinsic, so codes, scales and zero points are exact functions of
-// the inputs (the contract in include/flashloop.h): s = fp16_rn((max - min) / 15),
-// z = fp16_rn(min), code = clamp(rint_even((x - z) / s), 0, 15), x_hat = fma(code, s, z).
+// token; section 4 and the 2-bit row of its Figure 5: 2-bit residual codes.  Every
+// arithmetic step is one IEEE fp32 operation with an explicit round-to-nearest
+// intrinsic, so codes, scales and zero points are exact functions of the inputs (the
+// contract in include/flashloop.h): s = fp16_rn((max - min) / L), z = fp16_rn(min),
+// code = clamp(rint_even((x - z) / s), 0, L), x_hat = fma(code, s, z), with L = 15
+// for 4-bit codes and 3 for 2-bit codes.
 #pragma once
 
 #include "common.cuh"
@@ -17,15 +19,17 @@ __device__ __forceinline__ uint32_t pack_sz(__half s, __half z) {
 }
 
 // One group's scale and zero from its exact min and max.
+template <int kBits = 4>
 __device__ __forceinline__ void group_sz(float mn, float mx, __half& hs, __half& hz) {
-  hs = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+  hs = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), Rec<kBits>::kLevels));
   hz = __float2half_rn(mn);
 }
 
+template <int kBits = 4>
 __device__ __forceinline__ uint32_t quant(float x, float s, float z) {
   if (s == 0.0f) return 0u;
   int q = __float2int_rn(__fdiv_rn(__fsub_rn(x, z), s));  // round half to even
-  q = q < 0 ? 0 : (q > 15 ? 15 : q);
+  q = q < 0 ? 0 : (q > Rec<kBits>::kMaxCode ? Rec<kBits>::kMaxCode : q);
   return (uint32_t)q;
 }
 
@@ -53,18 +57,26 @@ __device__ __forceinline__ T ld_rec(const T* p) {
   else return *p;
 }
 
-// Dequantised channels c8 .. c8 + 7 (c8 a multiple of 8) of row `row` of group record g:
-// keys use the record's per-channel (scale, zero) words, values the row's half.
-template <bool kL2>
+// Dequantised channels c8 .. c8 + 7 (c8 a multiple of 8) of row `row` of group record g
+// (kBits-bit codes): keys use the record's per-channel (scale, zero) words, values the
+// row's half.
+template <bool kL2, int kBits = 4>
 __device__ __forceinline__ void deq8(const uint8_t* g, int row, bool is_v, int c8, float* out) {
-  const uint32_t cw =
-      ld_rec<kL2>(reinterpret_cast<const unsigned int*>(g + (size_t)row * 128 + (is_v ? 64 : 0) + c8 / 2));
+  using RB = Rec<kBits>;
+  uint32_t cw;
+  if constexpr (kBits == 4) {
+    cw = ld_rec<kL2>(reinterpret_cast<const unsigned int*>(g + (size_t)row * RB::kRow + (is_v ? RB::kHalf : 0) + c8 / 2));
+  } else {
+    cw = int2_word(ld_rec<kL2>(reinterpret_cast<const unsigned int*>(g + (size_t)row * RB::kRow + (is_v ? RB::kHalf : 0) +
+                                                                     (c8 >> 4) * 4)),
+                   (c8 >> 3) & 1);
+  }
   if (is_v) {
-    const float2 sz = unpack_sz(ld_rec<kL2>(reinterpret_cast<const unsigned int*>(g + kRecVsz) + row * 2 + (c8 >> 6)));
+    const float2 sz = unpack_sz(ld_rec<kL2>(reinterpret_cast<const unsigned int*>(g + RB::kVsz) + row * 2 + (c8 >> 6)));
 #pragma unroll
     for (int e = 0; e < 8; ++e) out[e] = deq((cw >> (4 * e)) & 15u, sz);
   } else {
-    const uint4* ks = reinterpret_cast<const uint4*>(g + kRecKsz + (size_t)c8 * 4);
+    const uint4* ks = reinterpret_cast<const uint4*>(g + RB::kKsz + (size_t)c8 * 4);
     const uint4 lo = ld_rec<kL2>(ks), hi = ld_rec<kL2>(ks + 1);
     const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
@@ -75,8 +87,8 @@ __device__ __forceinline__ void deq8(const uint8_t* g, int row, bool is_v, int c
 // X_hat^(r-1) of channels c8 .. c8 + 7 of token j (keys, or values when is_v): the base
 // record's dequantised row plus the residual stores 2 .. r - 1 that hold j, added in
 // loop order (FlashLoop project page, "The Method", Step 03).  brec / rrec are the
-// head's base and residual record arrays.
-template <bool kL2>
+// head's base and residual record arrays; the residual records have kResBits-bit codes.
+template <bool kL2, int kResBits = 4>
 __device__ __forceinline__ void recon8(const CacheView& c, const uint8_t* brec, const uint8_t* rrec,
                                        const unsigned long long* mask, const int32_t* first, int j, int r,
                                        bool is_v, int c8, float* xh) {
@@ -86,7 +98,7 @@ __device__ __forceinline__ void recon8(const CacheView& c, const uint8_t* brec, 
     const unsigned long long mk = ld_rec<kL2>(mask + (size_t)rp * ncb + b);
     const int gs = c.slot_base[rp] + ld_rec<kL2>(first + (size_t)rp * ncb + b) + __popcll(mk & ((1ull << jt) - 1ull));
     float d[8];
-    deq8<kL2>(rrec + (size_t)(gs >> 6) * kRec, gs & 63, is_v, c8, d);
+    deq8<kL2, kResBits>(rrec + (size_t)(gs >> 6) * Rec<kResBits>::kBytes, gs & 63, is_v, c8, d);
 #pragma unroll
     for (int e = 0; e < 8; ++e) xh[e] = __fadd_rn(xh[e], d[e]);
   }
@@ -105,8 +117,9 @@ struct EncodeSmem {
 
 // Key groups of channels [ch0, ch0 + nch): scale/zero over xs rows 0 .. nr - 1, written
 // to the record's per-channel words and to shared memory.  Block-strided over tid / nt.
+template <int kBits = 4>
 __device__ __forceinline__ void key_params(EncodeSmem& sm, uint8_t* rec, int ch0, int nch, int nr, int tid, int nt) {
-  uint32_t* ks = reinterpret_cast<uint32_t*>(rec + kRecKsz);
+  uint32_t* ks = reinterpret_cast<uint32_t*>(rec + Rec<kBits>::kKsz);
   for (int i = tid; i < nch; i += nt) {
     const int ch = ch0 + i;
     float mn = sm.xs[0][ch], mx = mn;
@@ -115,7 +128,7 @@ __device__ __forceinline__ void key_params(EncodeSmem& sm, uint8_t* rec, int ch0
       mx = fmaxf(mx, sm.xs[rr][ch]);
     }
     __half hs, hz;
-    group_sz(mn, mx, hs, hz);
+    group_sz<kBits>(mn, mx, hs, hz);
     sm.sk[ch] = __half2float(hs);
     sm.zk[ch] = __half2float(hz);
     ks[ch] = pack_sz(hs, hz);
@@ -124,9 +137,10 @@ __device__ __forceinline__ void key_params(EncodeSmem& sm, uint8_t* rec, int ch0
 
 // Value groups of rows [t0, t0 + nt_rows), one per (row, 64-channel half); rows >= nr
 // (absent slots) get zero words.
+template <int kBits = 4>
 __device__ __forceinline__ void value_params(EncodeSmem& sm, uint8_t* rec, int t0, int n_rows, int nr, int tid,
                                              int nt) {
-  uint32_t* vs = reinterpret_cast<uint32_t*>(rec + kRecVsz);
+  uint32_t* vs = reinterpret_cast<uint32_t*>(rec + Rec<kBits>::kVsz);
   for (int i = tid; i < 2 * n_rows; i += nt) {
     const int tt = t0 + (i >> 1), hf = i & 1;
     float sval = 0.f, zval = 0.f;
@@ -138,7 +152,7 @@ __device__ __forceinline__ void value_params(EncodeSmem& sm, uint8_t* rec, int t
         mx = fmaxf(mx, sm.xs[tt][64 * hf + ch]);
       }
       __half hs, hz;
-      group_sz(mn, mx, hs, hz);
+      group_sz<kBits>(mn, mx, hs, hz);
       sval = __half2float(hs);
       zval = __half2float(hz);
       packed = pack_sz(hs, hz);
@@ -168,6 +182,26 @@ __device__ __forceinline__ void group_codes(const EncodeSmem& sm, uint8_t* rec, 
       }
     }
     words[(size_t)t * 32 + w] = word;
+  }
+}
+
+// 2-bit code words of every row of one part (the layout in include/flashloop.h: word w
+// of a row's part holds channels 16w .. 16w + 15); rows >= nr get zero words.
+__device__ __forceinline__ void group_codes2(const EncodeSmem& sm, uint8_t* rec, bool is_v, int nr, int tid, int nt) {
+  uint32_t* words = reinterpret_cast<uint32_t*>(rec + (is_v ? Rec<2>::kHalf : 0));
+  for (int i = tid; i < kG * 8; i += nt) {
+    const int t = i >> 3, w = i & 7;
+    uint32_t word = 0u;
+    if (t < nr) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int ch = 16 * w + k;
+        const float s = is_v ? sm.sv[t][ch >> 6] : sm.sk[ch];
+        const float z = is_v ? sm.zv[t][ch >> 6] : sm.zk[ch];
+        word |= quant<2>(sm.xs[t][ch], s, z) << (k < 8 ? 4 * k : 4 * (k - 8) + 2);
+      }
+    }
+    words[(size_t)t * (Rec<2>::kRow / 4) + w] = word;
   }
 }
 

@@ -28,6 +28,13 @@
 // BF16 tail columns are handled last from global memory.  Warps merge in shared memory,
 // CTAs write (M, L, m, sum p v, sum p~ v) partials, and the last CTA of each head
 // combines them (atomic ticket, no waiting).
+//
+// Codec variants (flozi guide, section 4: the "Per-loop KIVI4" row and the 2-bit row
+// of Figure 5): 2-bit residual rows are staged as 32-byte halves and read through the
+// 4-bit layout (codes 0..3); with full-state stores a column's loop-r key/value is its
+// store st = min(r, depth) alone and its value at its tag loop the store
+// min(tag, st), so a key stage of store s holds the columns with st == s and a value
+// stage the columns for which s is one of those two stores.
 #include "flush.cuh"
 #include "kernels.h"
 
@@ -114,11 +121,21 @@ __device__ void setup_chunk(ChunkTab& t, const Smem& sm, int start, int end, int
 
 __device__ __forceinline__ unsigned below(int c) { return c >= 32 ? 0xffffffffu : ((1u << c) - 1u); }
 
+// Does a column with `st` stores and tag `lam` read a row of store s in a key (kind 0)
+// or value (kind 1) stage?
+template <int kCodec>
+__device__ __forceinline__ bool uses_row(int kind, int s, int st, int lam) {
+  if constexpr (CodecT<kCodec>::kFullState) return s == st || (kind == 1 && s == min(lam, st));
+  else return st >= s;
+}
+
 // lanes = columns: lay out the stage of store `s` that starts at chunk column `c0`;
 // returns the first column after it (32 when the store is done).
+template <int kCodec>
 __device__ int form_stage(Stage& sg, const ChunkTab& t, const Smem& sm, const Ctx& cx, int kind, int tab, int s,
                           int c0, int lane) {
-  const bool act = lane < t.ncol && t.st[lane] >= s && lane >= c0;
+  using RB = Rec<CodecT<kCodec>::kResBits>;
+  const bool act = lane < t.ncol && uses_row<kCodec>(kind, s, t.st[lane], t.lam[lane]) && lane >= c0;
   const unsigned bal = __ballot_sync(kFull, act);
   int grp = 0, pos = 0;
   if (act) {
@@ -131,7 +148,8 @@ __device__ int form_stage(Stage& sg, const ChunkTab& t, const Smem& sm, const Ct
       pos = slot & 63;
     }
   }
-  const uint8_t* recb = (s == 1 ? cx.brec : cx.rrec) + (size_t)grp * kRec;
+  const uint8_t* recb = s == 1 ? cx.brec + (size_t)grp * kRec : cx.rrec + (size_t)grp * RB::kBytes;
+  const int row_bytes = s == 1 ? 128 : RB::kRow;
   const unsigned lt = below(lane);
   const int row = __popc(bal & lt);
   int c_to = 32, nrec = 0;
@@ -148,18 +166,19 @@ __device__ int form_stage(Stage& sg, const ChunkTab& t, const Smem& sm, const Ct
     if (over) c_to = __ffs(over) - 1;
     nrec = __popc(nb & below(c_to));
     if (act && lane < c_to) {
-      sg.row_src[row] = recb + (size_t)pos * 128;
+      sg.row_src[row] = recb + (size_t)pos * row_bytes;
       sg.row_rec[row] = (uint8_t)(upto - 1);
-      if (isnew) sg.rec_src[upto - 1] = recb + kRecKsz;
+      if (isnew) sg.rec_src[upto - 1] = recb + (s == 1 ? kRecKsz : RB::kKsz);
     }
   } else if (act) {
-    sg.row_src[row] = recb + (size_t)pos * 128 + 64;
-    sg.sz_src[row] = recb + kRecVsz + (size_t)(pos & ~1) * 8;
+    sg.row_src[row] = recb + (size_t)pos * row_bytes + row_bytes / 2;
+    sg.sz_src[row] = recb + (s == 1 ? kRecVsz : RB::kVsz) + (size_t)(pos & ~1) * 8;
     sg.row_par[row] = (uint8_t)(pos & 1);
   }
   if (act && lane < c_to) sg.row_col[row] = (uint8_t)lane;
   const int nrow = __popc(bal & below(c_to));
-  const unsigned uball = __ballot_sync(kFull, act && s <= t.lam[lane]);
+  const bool uses_u = CodecT<kCodec>::kFullState ? s == min(t.lam[lane], t.st[lane]) : s <= t.lam[lane];
+  const unsigned uball = __ballot_sync(kFull, act && uses_u);
   if (lane == 0) {
     sg.kind = kind;
     sg.tab = tab;
@@ -178,12 +197,18 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 }
 
 // Every lane issues its share of the stage's 16-byte asynchronous copies (one commit
-// group per stage): 4 chunks per staged row, 32 chunks per key record, and one value
-// (scale, zero) pair per row.
+// group per stage): 4 chunks per staged row (2 for a 2-bit row), 32 chunks per key
+// record, and one value (scale, zero) pair per row.
+template <int kCodec>
 __device__ void issue_stage(Stage& sg, int lane) {
   const int nrow = sg.nrow, nrec = sg.nrec, kind = sg.kind;
-  for (int t = lane; t < 4 * nrow; t += 32)
-    cp_async16(&sg.code[t >> 2][16 * (t & 3)], sg.row_src[t >> 2] + 16 * (t & 3));
+  if (CodecT<kCodec>::kResBits == 2 && sg.store >= 2) {
+    for (int t = lane; t < 2 * nrow; t += 32)
+      cp_async16(&sg.code[t >> 1][16 * (t & 1)], sg.row_src[t >> 1] + 16 * (t & 1));
+  } else {
+    for (int t = lane; t < 4 * nrow; t += 32)
+      cp_async16(&sg.code[t >> 2][16 * (t & 3)], sg.row_src[t >> 2] + 16 * (t & 3));
+  }
   if (kind == 0) {
     for (int k = 0; k < nrec; ++k) cp_async16(&sg.rec[k][4 * lane], sg.rec_src[k] + 16 * lane);
   } else if (lane < nrow) {
@@ -192,9 +217,11 @@ __device__ void issue_stage(Stage& sg, int lane) {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// kFlush: the step also writes this loop's store of a full tail (fused flush)
-template <bool kFlush>
+// kFlush: the step also writes this loop's store of a full tail (fused flush);
+// kCodec: FL_CODEC_* of the loop r >= 2 stores
+template <bool kFlush, int kCodec>
 __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
+  using CT = CodecT<kCodec>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int h = blockIdx.y, split = blockIdx.x;
@@ -205,7 +232,7 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
 
   Ctx cx;
   cx.brec = arr<uint8_t>(c, A_BREC, a.layer) + (size_t)h * ncb * kRec;
-  cx.rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * kRec;
+  cx.rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * Rec<CT::kResBits>::kBytes;
   cx.ps = ps;
   cx.r = r;
   uint16_t* tail_k = arr<uint16_t>(c, A_TAILK, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
@@ -279,7 +306,7 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
     while (true) {
       const ChunkTab& t = wm.t[p.tab];
       if (p.store <= t.smax && p.col < 32) {
-        const bool act = lane < t.ncol && t.st[lane] >= p.store && lane >= p.col;
+        const bool act = lane < t.ncol && uses_row<kCodec>(p.phase, p.store, t.st[lane], t.lam[lane]) && lane >= p.col;
         const unsigned bal = __ballot_sync(kFull, act);
         if (bal) {
           p.col = __ffs(bal) - 1;
@@ -311,8 +338,8 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
   if (wtail > wk0) {
     setup_chunk(wm.t[0], sm, wk0, wtail, ps, lane);
     if (settle(pos)) {
-      pos.col = form_stage(wm.s[0], wm.t[pos.tab], sm, cx, pos.phase, pos.tab, pos.store, pos.col, lane);
-      issue_stage(wm.s[0], lane);
+      pos.col = form_stage<kCodec>(wm.s[0], wm.t[pos.tab], sm, cx, pos.phase, pos.tab, pos.store, pos.col, lane);
+      issue_stage<kCodec>(wm.s[0], lane);
       pending = true;
     }
   }
@@ -321,8 +348,8 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
     Stage& nx = wm.s[cur ^ 1];
     bool more = settle(pos);
     if (more) {
-      pos.col = form_stage(nx, wm.t[pos.tab], sm, cx, pos.phase, pos.tab, pos.store, pos.col, lane);
-      issue_stage(nx, lane);
+      pos.col = form_stage<kCodec>(nx, wm.t[pos.tab], sm, cx, pos.phase, pos.tab, pos.store, pos.col, lane);
+      issue_stage<kCodec>(nx, lane);
       asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
       asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -346,7 +373,10 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
           const int rid = sg.row_rec[row];
           float qsr[32];
           load32(reinterpret_cast<const float*>(sg.rec[rid]) + 32 * qq, qsr);
-          d = dot32(*reinterpret_cast<const uint4*>(&sg.code[row][16 * qq]), qsr);
+          const uint4 x = (CT::kResBits == 2 && sg.store >= 2)
+                              ? int2_to_nib(*reinterpret_cast<const uint2*>(&sg.code[row][8 * qq]))
+                              : *reinterpret_cast<const uint4*>(&sg.code[row][16 * qq]);
+          d = dot32(x, qsr);
           if (qq == 0) d += sg.rec_c[rid];
         }
         d += __shfl_xor_sync(kFull, d, 1);
@@ -387,8 +417,13 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
           const uint32_t* pr = &sg.rec[0][4 * lane + 2 * sg.row_par[lane]];
           const float2 z0 = unpack_sz(pr[0]), z1 = unpack_sz(pr[1]);
           const int ci = sg.row_col[lane];
-          const float p = t.p[ci];
-          const float pu = sg.store <= t.lam[ci] ? t.pu[ci] : 0.f;
+          float p = t.p[ci], pu;
+          if constexpr (CT::kFullState) {
+            p = sg.store == t.st[ci] ? p : 0.f;
+            pu = sg.store == min(t.lam[ci], t.st[ci]) ? t.pu[ci] : 0.f;
+          } else {
+            pu = sg.store <= t.lam[ci] ? t.pu[ci] : 0.f;
+          }
           const float wS0 = 128.f * (p * z0.x), wS1 = 128.f * (p * z1.x);
           const float wU0 = 128.f * (pu * z0.x), wU1 = 128.f * (pu * z1.x);
           wrow[2 * lane] = make_float4(wS0, wU0, 0.f, 0.f);
@@ -408,9 +443,11 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
         }
       }
       __syncwarp();
+      const bool packed = CT::kResBits == 2 && sg.store >= 2;  // 2-bit codes in the first 32 bytes
       if (sg.use_u) {
         for (int row = par16; row < sg.nrow; row += 2) {
-          const uint32_t x = *reinterpret_cast<const uint32_t*>(&sg.code[row][4 * w16]);
+          const uint32_t x = packed ? int2_word(*reinterpret_cast<const uint32_t*>(&sg.code[row][4 * (w16 >> 1)]), w16 & 1)
+                                    : *reinterpret_cast<const uint32_t*>(&sg.code[row][4 * w16]);
           const float2 wgt = *reinterpret_cast<const float2*>(&wrow[2 * row + half]);
           const float x0 = nib16(x << 16), x1 = nib16(x << 12), x2 = nib16(x << 8), x3 = nib16(x << 4);
           const float x4 = nib16(x), x5 = nib16(x >> 4), x6 = nib16(x >> 8), x7 = nib16(x >> 12);
@@ -433,7 +470,8 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
         }
       } else {
         for (int row = par16; row < sg.nrow; row += 2) {
-          const uint32_t x = *reinterpret_cast<const uint32_t*>(&sg.code[row][4 * w16]);
+          const uint32_t x = packed ? int2_word(*reinterpret_cast<const uint32_t*>(&sg.code[row][4 * (w16 >> 1)]), w16 & 1)
+                                    : *reinterpret_cast<const uint32_t*>(&sg.code[row][4 * w16]);
           const float ws = wrow[2 * row + half].x;
           accS[0] = fmaf(ws, nib16(x << 16), accS[0]);
           accS[1] = fmaf(ws, nib16(x << 12), accS[1]);
@@ -614,8 +652,12 @@ int sparse_splits(int heads, int k_sel, int loops) {
 
 cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s) {
   a.n_splits = sparse_splits(a.c.H, a.k_sel, a.c.R);
-  const size_t smem = a.flush && sizeof(EncodeSmem) > sizeof(Smem) ? sizeof(EncodeSmem) : sizeof(Smem);
-  auto kern = a.flush ? sparse_kernel<true> : sparse_kernel<false>;
+  const bool flush = a.flush && a.c.codec == FL_CODEC_RESIDUAL_INT4;
+  const size_t smem = flush && sizeof(EncodeSmem) > sizeof(Smem) ? sizeof(EncodeSmem) : sizeof(Smem);
+  auto kern = a.c.codec == FL_CODEC_FULL_INT4       ? sparse_kernel<false, FL_CODEC_FULL_INT4>
+              : a.c.codec == FL_CODEC_RESIDUAL_INT2 ? sparse_kernel<false, FL_CODEC_RESIDUAL_INT2>
+              : flush                               ? sparse_kernel<true, FL_CODEC_RESIDUAL_INT4>
+                                                    : sparse_kernel<false, FL_CODEC_RESIDUAL_INT4>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_splits, a.c.H);

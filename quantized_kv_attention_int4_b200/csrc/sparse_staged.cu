@@ -595,7 +595,9 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s) {
   sms = (dev >= 0 && dev < 64) ? sms_cached[dev] : 0;
   const int ps = a.c.plan_stride;
   const int n = staged_splits(a.c.H, a.k_sel, ps, sms > 0 ? sms : 148);
-  if (a.r > kStoresMax || sms == 0 || n > kMaxSplits) return launch_sparse_direct(a, s);
+  // the codec variants are served by the direct reader
+  if (a.c.codec != FL_CODEC_RESIDUAL_INT4 || a.r > kStoresMax || sms == 0 || n > kMaxSplits)
+    return launch_sparse_direct(a, s);
   if (!attr_set[dev]) {
     for (auto k : {sparse_staged_kernel<false>, sparse_staged_kernel<true>}) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCta);

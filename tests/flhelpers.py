@@ -41,6 +41,29 @@ def _split_records(raw: np.ndarray, H: int, G: int):
     return kc, vc, ksz, vsz
 
 
+def crumbs(words: np.ndarray) -> np.ndarray:
+    """[..., 8] uint32 words of 2-bit codes -> [..., 128] codes.
+
+    Word w holds channels 16w .. 16w+15: channel 16w+k (k < 8) in bits 4k..4k+1 and
+    channel 16w+8+k in bits 4k+2..4k+3 (include/flashloop.h, 2-bit residual records)."""
+    out = np.empty(words.shape[:-1] + (words.shape[-1], 16), np.uint8)
+    for k in range(8):
+        out[..., k] = (words >> (4 * k)) & 3
+        out[..., 8 + k] = (words >> (4 * k + 2)) & 3
+    return out.reshape(words.shape[:-1] + (words.shape[-1] * 16,))
+
+
+def _split_records2(raw: np.ndarray, H: int, G: int):
+    """2-bit residual records [H][G][5120] -> the same logical arrays as _split_records."""
+    rec = raw[: H * G * 5120].reshape(H, G, 5120)
+    rows = np.ascontiguousarray(rec[:, :, :4096]).reshape(H, G * 64, 64)
+    kc = crumbs(np.ascontiguousarray(rows[..., :32]).view(np.uint32))
+    vc = crumbs(np.ascontiguousarray(rows[..., 32:]).view(np.uint32))
+    vsz = np.ascontiguousarray(rec[:, :, 4096:4608]).view(np.uint32).reshape(H, G * 64, 2)
+    ksz = np.ascontiguousarray(rec[:, :, 4608:]).view(np.uint32).reshape(H, G, 128)
+    return kc, vc, ksz, vsz
+
+
 class Unpacked:
     """Logical views of one layer of a FlashLoopCache (CPU copies)."""
 
@@ -51,7 +74,8 @@ class Unpacked:
         self.kc, self.vc, ksz, vsz = _split_records(g("brec"), H, C // 64)
         self.ks, self.kz = split_sz(ksz)
         self.vs, self.vz = split_sz(vsz)
-        self.rkc, self.rvc, rksz, rvsz = _split_records(g("rrec"), H, T // 64)
+        split = _split_records2 if cache.codec == abi.FL_CODEC_RESIDUAL_INT2 else _split_records
+        self.rkc, self.rvc, rksz, rvsz = split(g("rrec"), H, T // 64)
         self.rks, self.rkz = split_sz(rksz)
         self.rvs, self.rvz = split_sz(rvsz)
         self.mask = g("mask").view(np.uint64)[: (R + 1) * (C // 64)].reshape(R + 1, C // 64)
@@ -92,19 +116,20 @@ def check_topk_valid(S, p_tilde, k):
 class Pair:
     """A one-layer GPU cache and its oracle, built from the same synthetic prompt."""
 
-    def __init__(self, w: synth.Workload, heads=None, extra_tokens: int = 0, layer: int = 0, data=None):
+    def __init__(self, w: synth.Workload, heads=None, extra_tokens: int = 0, layer: int = 0, data=None,
+                 codec: int = abi.FL_CODEC_RESIDUAL_INT4):
         self.w = w
         self.layer = layer
         n = w.n_ctx
         self.heads = list(range(w.heads)) if heads is None else list(heads)
         cap = round_up(n + extra_tokens + 64)
-        self.cache = FlashLoopCache(1, w.heads, w.loops, cap, max_select=cap)
+        self.cache = FlashLoopCache(1, w.heads, w.loops, cap, max_select=cap, codec=codec)
         d = synth.prefill_layer(w, layer, device="cuda") if data is None else data
         self.sets = d["sets"]
         n_q, n_tail, tail_depth = self.cache.prefill_layer(0, d["K"], d["V"], self.sets)
         self.cache.set_timeline(n_q, n_tail, tail_depth)
         hs = self.heads
-        self.oracle = fo.OracleLayer(len(hs), w.loops, cap)
+        self.oracle = fo.OracleLayer(len(hs), w.loops, cap, codec=codec)
         lay = self.oracle
         lay.encode_base(0, f32(d["K"][1][hs, :n_q]), f32(d["V"][1][hs, :n_q]))
         self.calls = {r: [] for r in range(2, w.loops + 1)}

@@ -152,3 +152,19 @@ def test_noalloc_sparse_validation():
                    max_select=128)
     code = abi._c_sparse_noalloc(ctypes.byref(big), p, 0, 3, 960, 1, 10, p, None, None, p, p, None)
     assert code == abi.FL_ERR_UNSUPPORTED
+
+
+def test_int2_records_take_5120_bytes_and_codecs_are_checked():
+    dims = dict(layers=2, heads=3, loops=4, capacity=1024, max_select=128, res_capacity={2: 1024, 3: 512, 4: 256})
+    L4 = abi.fl_cache_layout(abi.Dims(**dims))
+    L2 = abi.fl_cache_layout(abi.Dims(**dims, codec=abi.FL_CODEC_RESIDUAL_INT2))
+    T = 1024 + 512 + 256
+    assert L4.total_slots == L2.total_slots == T
+    rrec = abi.ARRAY_NAMES.index("rrec")
+    assert L4.layer_stride[rrec] == 3 * (T // 64) * 9216
+    assert L2.layer_stride[rrec] == 3 * (T // 64) * 5120
+    assert L2.total_bytes < L4.total_bytes
+    bad = abi.Dims(**dims, codec=3)
+    with pytest.raises(abi.FlashLoopError) as e:
+        abi.fl_cache_layout(bad)
+    assert e.value.status == abi.FL_ERR_UNSUPPORTED
