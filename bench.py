@@ -145,7 +145,7 @@ def max_over_ranks(values, device):
     return [float(x) for x in t.tolist()]
 
 
-def build_cache(w: synth.Workload, layers: int, rank: int, device, new_tokens: int = 256):
+def build_cache(w: synth.Workload, layers: int, rank: int, device, new_tokens: int = 256, codec: int = 0):
     from quantized_kv_attention_int4_b200.cache import FlashLoopCache, round_up
 
     n = w.n_ctx
@@ -154,7 +154,7 @@ def build_cache(w: synth.Workload, layers: int, rank: int, device, new_tokens: i
     cap = round_up(n + extra)
     res_cap = {r: round_up(min(cap, int((sets[r] < n).sum()) + extra + 64 * 4)) for r in range(2, w.loops + 1)}
     cache = FlashLoopCache(layers, w.heads, w.loops, cap, res_capacity=res_cap,
-                           max_select=w.k_sel(cap), device=device)
+                           max_select=w.k_sel(cap), device=device, codec=codec)
     wr = replica_workload(w, rank)
     info = None
     for layer in range(layers):
@@ -248,6 +248,42 @@ def sparse_bytes_from_state(cache, w, layers, loop, k_sel):
     return total / layers
 
 
+def sparse_bytes_from_plan(cache, layers, k_sel):
+    """Algorithmic bytes of one sparse-reader launch from the gather plans now in the cache,
+    for the cache's codec: the rows, key groups and tag-loop value rows each selected
+    column needs (the plan holds each column's tag, store count and residual slots)."""
+    from quantized_kv_attention_int4_b200 import abi
+
+    H, n_q, ms, ps = cache.H, cache.n_q, cache.dims.max_select, cache.layout.plan_stride
+    full = cache.codec == abi.FL_CODEC_FULL_INT4
+    total = 0
+    for l in range(layers):
+        plan = cache.raw("plan", l).view(torch.int32)[: H * ms * ps].view(H, ms, ps)[:, :k_sel].cpu().numpy()
+        cols_quant = cols_tail = res_rows = value_rows = groups = 0
+        for h in range(H):
+            e = plan[h]
+            j, st, lam = e[:, 0], (e[:, 1] >> 8) & 0xFF, e[:, 1] & 0xFF
+            q = j < n_q
+            cols_quant += int(q.sum())
+            cols_tail += int((~q).sum())
+            j, st, lam, e = j[q], st[q], lam[q], e[q]
+            if full:
+                # one row of store st (keys and values), and the value half of store min(tag, st)
+                value_rows += int((np.minimum(lam, st) != st).sum())
+                keys = set((j[st == 1] // 64).tolist())
+                for s in range(2, int(st.max(initial=1)) + 1):
+                    keys |= set((e[st == s, 1 + s].astype(np.int64) // 64 + (1 << 40)).tolist())
+                groups += len(keys)
+            else:
+                res_rows += int(np.maximum(st - 1, 0).sum())
+                groups += len(np.unique(j // 64))
+                for s in range(2, int(st.max(initial=1)) + 1):
+                    groups += len(np.unique(e[st >= s, 1 + s] // 64))
+        code_row = bytemodel.CODE_ROW2 if cache.codec == abi.FL_CODEC_RESIDUAL_INT2 else bytemodel.CODE_ROW
+        total += bytemodel.sparse_bytes(H, cols_quant, res_rows, groups, cols_tail, code_row, value_rows)
+    return total / layers
+
+
 def dense_bytes_avg(cache, w, layers, loop):
     H = cache.H
     tot = 0
@@ -327,11 +363,68 @@ def run_gpu(args, rank, world):
     e2e = run_e2e(step, cache, wr, layers, inputs[total_steps:], device) if args.e2e_steps else None
     del inputs, step, cache
     tokens = run_token_select(wr, device, hbm) if args.token_select else None
+    codecs = run_codecs(w, device, hbm, layers=args.codec_layers) if args.codecs else None
     prefill = run_prefill(wr, device) if args.prefill else None
     return dict(metric_us=metric_us, step_ms=step_ms, seg=mean, clocks=clocks, launches=launches / args.steps,
                 sp_bytes=sp_bytes, sp_launch_us=sp_launch_us, sp_gbs=sp_gbs, d_bytes=d_bytes,
                 d_launch_us=d_launch_us, d_gbs=d_gbs, hbm=hbm, peak_kind=peak_kind, N=N, k_sel=k_sel,
-                layers=layers, setup_s=setup_s, e2e=e2e, w=wr, tokens=tokens, prefill=prefill)
+                layers=layers, setup_s=setup_s, e2e=e2e, w=wr, tokens=tokens, prefill=prefill, codecs=codecs)
+
+
+def run_codecs(w, device, hbm, layers=4, warmup=3, steps=5):
+    """The codec variants of the loop r >= 2 stores (per-loop KIVI4 full state, INT2
+    residuals; flozi guide, section 4) on the workload's per-layer sizes, `layers`
+    layers: the step executor without tail flushes (the variants have none fused),
+    CUDA events around the dense loops and the loop-4 selection and sparse loop.
+    Both variants run on the direct readers."""
+    from quantized_kv_attention_int4_b200 import abi
+
+    out = {}
+    for codec, name in ((abi.FL_CODEC_FULL_INT4, "full_int4"), (abi.FL_CODEC_RESIDUAL_INT2, "residual_int2")):
+        cache, wr = build_cache(w, layers, 0, device, new_tokens=warmup + steps, codec=codec)
+        inputs = step_inputs(wr, layers, warmup + steps, device)
+        O = torch.zeros(wr.loops + 1, layers, wr.heads, 128, dtype=torch.float32, device=device)
+        evs = [{k: torch.cuda.Event(enable_timing=True) for k in EXEC_EVENTS} for _ in range(steps)]
+        for s in range(warmup + steps):
+            cache.begin_token()           # the prompt's full tail is flushed by the encoders at the first token
+            seg = [evs[s - warmup][k] for k in EXEC_EVENTS] if s >= warmup else None
+            q, kn, vn = inputs[s]
+            cache.step(wr.dense_loops, wr.k_sel(cache.n_cols), q, O, kn, vn, events=seg)
+        torch.cuda.synchronize()
+        st, info = cache.status()
+        if st != 0:
+            raise RuntimeError(f"device error in the {name} codec measurement: {info}")
+        ms = lambda a, b: float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
+        dense_ms = ms("flushed", "loop2")
+        sel_ms, sp_ms = ms("loop3", "select4"), ms("select4", "loop4")
+        k_sel = wr.k_sel(cache.n_cols)
+        sp_bytes = sparse_bytes_from_plan(cache, layers, k_sel)
+        sp_us = sp_ms * 1e3 / layers
+        d_bytes = 0.0
+        for loop in (1, 2):
+            for l in range(layers):
+                if codec == abi.FL_CODEC_FULL_INT4:
+                    rows, rb = 0, bytemodel.ROW_BYTES
+                else:
+                    rows, rb = sum(cache.n_rows[l][rp] for rp in range(2, loop + 1)), bytemodel.ROW_BYTES2
+                d_bytes += bytemodel.dense_bytes(cache.H, cache.n_q, cache.n_tail, rows, loop == wr.dense_loops, rb)
+        d_bytes /= 2 * layers
+        d_us = dense_ms * 1e3 / (2 * layers)
+        rrec = cache.layout.layer_stride[abi.ARRAY_NAMES.index("rrec")]
+        out[name] = {
+            "kernels": "dense_direct_kernel (loops 1-2), sparse_kernel (loop 4)",
+            "sparse_us_per_launch": sp_us, "sparse_bytes_per_launch": sp_bytes,
+            "sparse_gbs": sp_bytes / (sp_us * 1e-6) / 1e9, "sparse_frac": sp_bytes / (sp_us * 1e-6) / 1e9 / hbm,
+            "select4_us": sel_ms * 1e3,
+            "dense_us_per_launch": d_us, "dense_bytes_per_launch": d_bytes,
+            "dense_gbs": d_bytes / (d_us * 1e-6) / 1e9, "dense_frac": d_bytes / (d_us * 1e-6) / 1e9 / hbm,
+            "residual_store_bytes_per_layer": int(rrec), "layers": layers, "steps": steps,
+            "sparse_traffic": _kernel_traffic("sparse_kernel_" + name),
+            "dense_traffic": _kernel_traffic("dense_direct_kernel_" + name),
+        }
+        del cache, inputs, O
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_token_select(w, device, hbm, reps=5):
@@ -552,6 +645,9 @@ def main():
                     help="skip the token-sparse update selector measurement")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false",
                     help="skip the sparse prefill attention measurement")
+    ap.add_argument("--no-codecs", dest="codecs", action="store_false",
+                    help="skip the codec variant (full-state INT4, INT2 residual) measurement")
+    ap.add_argument("--codec-layers", type=int, default=4, help="layers of each codec variant's cache")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -613,6 +709,7 @@ def main():
                            "bytes_per_launch": r["d_bytes"], "us_per_launch": r["d_launch_us"]},
         "roofline_token_select": r["tokens"],
         "roofline_prefill": r["prefill"],
+        "codec_variants": r["codecs"],
         "segments_ms": r["seg"], "clocks": r["clocks"], "gpu_launches": r["launches"],
         "e2e": r["e2e"], "cpu_baseline": cpu, "setup_s": r["setup_s"],
     }

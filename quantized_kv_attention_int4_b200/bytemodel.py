@@ -24,6 +24,9 @@ VSZ_ROW = 8                       # two (scale, zero) fp16 pairs per value row
 KSZ_GROUP = HEAD_DIM * 4          # (scale, zero) fp16 pair per channel per key group
 ROW_BYTES = 2 * CODE_ROW + VSZ_ROW + KSZ_GROUP // GROUP   # 144
 TAIL_ROW = 2 * HEAD_DIM * 2       # K + V in BF16
+# a 2-bit residual row (FL_CODEC_RESIDUAL_INT2): 32 + 32 B of codes, the same scales
+CODE_ROW2 = HEAD_DIM // 4
+ROW_BYTES2 = 2 * CODE_ROW2 + VSZ_ROW + KSZ_GROUP // GROUP  # 80
 
 
 def bf16_bytes_per_token_loop(layers: int, heads: int, head_dim: int = HEAD_DIM) -> int:
@@ -49,31 +52,38 @@ def bf16_tail_extra(bf16_total: float, context: int, tail: int = 64) -> float:
 # ----------------------------------------------------------------------------
 # Algorithmic bytes per launch (one layer, all heads)
 # ----------------------------------------------------------------------------
-def dense_bytes(heads: int, n_q: int, n_tail: int, res_rows: int, keep_scores: bool) -> int:
+def dense_bytes(heads: int, n_q: int, n_tail: int, res_rows: int, keep_scores: bool,
+                res_row_bytes: int = ROW_BYTES) -> int:
     """One dense-reader launch of loop r.
 
     n_q quantised columns read their base rows, ``res_rows`` is the number of
-    residual rows of loops 2..r that belong to those columns, the tail rows are
-    BF16.  Plus q (BF16), o (fp32), and with ``keep_scores`` the per-column
-    log-score (fp32) and loop tag (u8) written for the selector.
+    residual rows of loops 2..r that belong to those columns (``res_row_bytes``
+    each), the tail rows are BF16.  Plus q (BF16), o (fp32), and with
+    ``keep_scores`` the per-column log-score (fp32) and loop tag (u8) written for
+    the selector.  With full-state stores every quantised column reads one row
+    (its last store): pass res_rows = 0.
     """
-    per_head = (n_q + res_rows) * ROW_BYTES + n_tail * TAIL_ROW + HEAD_DIM * 2 + HEAD_DIM * 4
+    per_head = n_q * ROW_BYTES + res_rows * res_row_bytes + n_tail * TAIL_ROW + HEAD_DIM * 2 + HEAD_DIM * 4
     if keep_scores:
         per_head += (n_q + n_tail) * 5
     return heads * per_head
 
 
-def sparse_bytes(heads: int, cols_quant: int, res_rows: int, key_groups: int, cols_tail: int) -> int:
+def sparse_bytes(heads: int, cols_quant: int, res_rows: int, key_groups: int, cols_tail: int,
+                 res_code_row: int = CODE_ROW, value_rows: int = 0) -> int:
     """One sparse-reader launch, summed over heads.
 
     ``cols_quant``: selected quantised columns (over all heads); ``res_rows``:
-    residual rows those columns carry up to this loop; ``key_groups``: distinct
-    (store, key group) pairs the selected rows touch (512 B of key scales each);
-    ``cols_tail``: selected tail columns.  Each selected column also reads its
-    index (4 B), writes its new log-score and loop tag (5 B); per head q, m, u
-    and o are read or written.
+    residual rows those columns carry up to this loop (``res_code_row`` bytes of
+    key and of value codes each); ``key_groups``: distinct (store, key group)
+    pairs the selected rows touch (512 B of key scales each); ``cols_tail``:
+    selected tail columns; ``value_rows``: rows read for their value half only
+    (full-state stores: a column's value at its tag loop when that is another
+    store).  Each selected column also reads its index (4 B), writes its new
+    log-score and loop tag (5 B); per head q, m, u and o are read or written.
     """
     row = 2 * CODE_ROW + VSZ_ROW
     cols = cols_quant + cols_tail
-    return ((cols_quant + res_rows) * row + key_groups * KSZ_GROUP + cols_tail * TAIL_ROW
+    return (cols_quant * row + res_rows * (2 * res_code_row + VSZ_ROW) + value_rows * (CODE_ROW + VSZ_ROW)
+            + key_groups * KSZ_GROUP + cols_tail * TAIL_ROW
             + cols * (4 + 5) + heads * (HEAD_DIM * 2 + 4 + HEAD_DIM * 4 * 2))
