@@ -562,7 +562,7 @@ class OracleLoop4:
     from the same state and returns its seconds per (layer, head).
     """
 
-    def __init__(self, w: synth.Workload, heads=(0,)):
+    def __init__(self, w: synth.Workload, heads=(0,), codec: int = 0):
         from oracle import flashloop_oracle as fo
 
         self.fo = fo
@@ -573,7 +573,7 @@ class OracleLoop4:
         hs = list(heads)
         self.nh = len(hs)
         f = lambda t: t.float().numpy()
-        lay = fo.OracleLayer(len(hs), w.loops, n + 64)
+        lay = fo.OracleLayer(len(hs), w.loops, n + 64, codec=codec)
         lay.encode_base(0, f(d["K"][1][hs, :n_q]), f(d["V"][1][hs, :n_q]))
         for r in range(2, w.loops + 1):
             rows = sets[r][sets[r] < n_q].numpy()
@@ -618,6 +618,61 @@ def oracle_loop4_sample(w: synth.Workload, budget_s: float, heads=(0,)):
         if time.perf_counter() - t_all > budget_s and len(times) >= 2:
             break
     return float(np.mean(times)), len(times)
+
+
+def oracle_beside(w: synth.Workload, layers: int, codec_layers: int, budget_s: float, rows=None):
+    """The oracle timed beside the rows measured outside the decode steps, on one host thread,
+    each on a bounded sample of the GPU leg's workload (seeded CPU inputs of the same shapes
+    and distributions): the token-sparse update selector (loop-3 ranking, every token), the
+    sparse prefill attention (the 64 latest active queries of one head, scaled by FLOPs) and
+    the loop-4 step of each codec variant (one (layer, head), scaled like cpu_baseline)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import flashloop_oracle as fo
+
+    out = {}
+    n, d = w.n_ctx, w.heads * 128
+    ns = n // 8                          # a bounded sample: an eighth of the tokens, scaled by 8
+    rng = np.random.default_rng(w.seed)
+    h1 = rng.standard_normal((ns, d), dtype=np.float32)
+    h2 = (h1 + rng.standard_normal((ns, d), dtype=np.float32) * np.exp(rng.standard_normal((ns, 1)))).astype(np.float32)
+    k3 = w.n_active(3, ns)
+    with threadpool_limits(limits=1):
+        fo.select_active(h1, h2, np.arange(ns), k3)          # untimed: first-touch of the buffers
+        t = time.perf_counter()
+        fo.select_active(h1, h2, np.arange(ns), k3)
+        dt = time.perf_counter() - t
+    out["token_select"] = {"value": dt * (n / ns) * 1e6, "unit": "us per loop-3 ranking", "cores": 1,
+                           "kind": "oracle",
+                           "sample": f"oracle select_active over {ns} of {n} tokens x {d} (fp64), scaled by {n // ns}"}
+    del h1, h2
+    pos = synth.active_sets(w, n)[3].numpy()
+    sample = pos[-64:]
+    K = rng.standard_normal((1, n, 128), dtype=np.float32)
+    V = rng.standard_normal((1, n, 128), dtype=np.float32)
+    q = rng.standard_normal((1, sample.size, 128), dtype=np.float32)
+    with threadpool_limits(limits=1):
+        fo.prefill_attention(q[:, :4], sample[:4], K, V)      # untimed: first-touch of the buffers
+        t = time.perf_counter()
+        fo.prefill_attention(q, sample, K, V)
+        dt = time.perf_counter() - t
+    scale = w.heads * float((pos.astype(np.float64) + 1).sum()) / float((sample.astype(np.float64) + 1).sum())
+    out["prefill"] = {"value": dt * scale * 1e6, "unit": "us per call", "cores": 1, "kind": "oracle",
+                      "sample": f"oracle prefill_attention for the 64 latest of {pos.size} active queries of 1 of "
+                                f"{w.heads} heads (fp64), scaled by FLOPs x{scale:.0f}"}
+    del K, V, q
+    for codec, name in ((fo.FULL_INT4, "full_int4"), (fo.RESIDUAL_INT2, "residual_int2")):
+        o = OracleLoop4(w, codec=codec)
+        times = []
+        t_all = time.perf_counter()
+        while not times or (time.perf_counter() - t_all < budget_s and len(times) < 50):
+            times.append(o.run_once())
+        out[name] = {"value": float(np.mean(times)) * codec_layers * w.heads * 1e6, "unit": "us per loop-4 step",
+                     "cores": 1, "kind": "oracle",
+                     "sample": f"oracle loop-4 selection + sparse attention, {name} stores, 1 of {codec_layers}x"
+                               f"{w.heads} (layer, head) pairs at N={n}, {len(times)} reps, scaled by "
+                               f"{codec_layers * w.heads}"}
+        del o
+    return out
 
 
 def cpu_baseline(w: synth.Workload, layers: int, budget_s: float):
@@ -694,6 +749,14 @@ def main():
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         cpu = cpu_baseline(w, layers, args.cpu_budget)
+        beside = oracle_beside(w, layers, args.codec_layers, 3.0)
+        if r["tokens"]:
+            r["tokens"]["cpu_baseline"] = beside["token_select"]
+        if r["prefill"]:
+            r["prefill"]["cpu_baseline"] = beside["prefill"]
+        if r["codecs"]:
+            for name, v in r["codecs"].items():
+                v["cpu_baseline"] = beside[name]
     hbm = r["hbm"]
     line = {
         "metric": METRIC, "value": r["metric_us"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
