@@ -31,6 +31,14 @@
 // BF16 tail columns are handled last from global memory.  Warps merge in shared memory,
 // CTAs write (M, L, m, sum p v, sum p~ v) partials, and the last CTA of each head
 // combines them (atomic ticket, no waiting).
+//
+// Codec variants (flozi guide, section 4: the "Per-loop KIVI4" row and the 2-bit row
+// of Figure 5).  2-bit residual rows are 64 bytes (32 B key codes, 32 B value codes):
+// they are staged in the first half of their 128-byte row slot and read through the
+// 4-bit layout (codes 0..3).  With full-state stores a column's loop-r key and value
+// are its store st = min(r, depth) alone and its tag-loop value the store min(tag, st):
+// a span holds each column's row of store st and, when the tag-loop store differs, that
+// store's row for its value half only (no key record, no key dot).
 #include "flush.cuh"
 #include "kernels.h"
 
@@ -101,9 +109,16 @@ __device__ __forceinline__ int scan_incl(int v, int lane) {
   return v;
 }
 
-// kFlush: the step also writes this loop's store of a full tail (fused flush)
-template <bool kFlush>
+constexpr uint8_t kValueOnly = 0xff;  // row_rec of a row staged for its value half only
+
+// kFlush: the step also writes this loop's store of a full tail (fused flush);
+// kCodec: FL_CODEC_* of the loop r >= 2 stores
+template <bool kFlush, int kCodec>
 __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArgs a) {
+  using CT = CodecT<kCodec>;
+  using RB = Rec<CT::kResBits>;
+  constexpr bool kFullS = CT::kFullState;
+  constexpr bool kPk = CT::kResBits == 2;
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& ch = *reinterpret_cast<CtaHdr*>(smem);
   int32_t* plan_s = reinterpret_cast<int32_t*>(smem + sizeof(CtaHdr));
@@ -119,7 +134,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
   const unsigned lt = lanes_below(lane);
 
   const uint8_t* brec = arr<uint8_t>(c, A_BREC, a.layer) + (size_t)h * ncb * kRec;
-  const uint8_t* rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * kRec;
+  const uint8_t* rrec = arr<uint8_t>(c, A_RREC, a.layer) + (size_t)h * (T / kG) * RB::kBytes;
   uint16_t* tail_k = arr<uint16_t>(c, A_TAILK, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
   uint16_t* tail_v = arr<uint16_t>(c, A_TAILV, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
   const uint16_t* tail_v_all = arr<uint16_t>(c, A_TAILV, a.layer);
@@ -198,22 +213,26 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
       const bool in = cpos < wtail;
       const int32_t* e = plan_s + (size_t)(in ? cpos : iss_pos) * ps;
       const int st = in ? (e[1] >> 8) & 0xff : 0;
+      // full-state: the store of the column's tag-loop value (== st: no extra row)
+      const int sv = kFullS ? min(e[1] & 0xff, st) : 0;
       if (!formed) {
         int smax = st;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) smax = max(smax, __shfl_xor_sync(kFull, smax, o));
         int nrec_c = 0;
         for (int s = 1; s <= smax; ++s) {
-          const bool act = st >= s;
+          const bool act = kFullS ? st == s : st >= s;  // rows with a key part
           const int g = act ? rec_of(e, s) : -1;
           const unsigned pb = __ballot_sync(kFull, act) & lt;
           const int gp = __shfl_sync(kFull, g, pb ? 31 - __clz(pb) : lane);
           if (act && (pb == 0u || gp != g)) ++nrec_c;
         }
-        const int rows_i = scan_incl(st, lane), recs_i = scan_incl(nrec_c, lane);
+        const int nrow_c = kFullS ? (st > 0) + (sv != st) : st;
+        const int rows_i = scan_incl(nrow_c, lane), recs_i = scan_incl(nrec_c, lane);
         const unsigned over = __ballot_sync(kFull, in && (rows_i > kMaxRows || recs_i > kMaxRecs));
         f_ncol = min(32, wtail - iss_pos);
         if (over) f_ncol = __ffs(over) - 1;  // >= 1: one column has at most 8 rows and 8 records
+        static_assert(kMaxRows >= kStoresMax && kMaxRecs >= kStoresMax, "a column fits one span");
         f_nrows = __shfl_sync(kFull, rows_i, f_ncol - 1);
         f_nrecs = __shfl_sync(kFull, recs_i, f_ncol - 1);
         f_smax = smax;
@@ -254,31 +273,40 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
       }
       int rowbase = 0, recbase = 0;
       for (int s = 1; s <= smax; ++s) {
-        const bool act = mine && st >= s;
+        const bool kact = mine && (kFullS ? st == s : st >= s);  // key and value parts
+        const bool act = kact || (kFullS && mine && s == sv);     // ... or the value part alone
         const int g = act ? rec_of(e, s) : -1;
         const unsigned b = __ballot_sync(kFull, act);
-        const unsigned pb = b & lt;
+        unsigned pb = b & lt;
+        if constexpr (kFullS) pb = __ballot_sync(kFull, kact) & lt;
         const int gp = __shfl_sync(kFull, g, pb ? 31 - __clz(pb) : lane);
-        const bool isnew = act && (pb == 0u || gp != g);
+        const bool isnew = kact && (pb == 0u || gp != g);
         const unsigned nb = __ballot_sync(kFull, isnew);
         if (lane == 0 && s <= kStoresMax) {
           hd.bal[s - 1] = b;
           hd.rowbase[s - 1] = rowbase;
         }
         if (act) {
-          const int ri = rowbase + __popc(pb);
+          const int ri = rowbase + (kFullS ? __popc(b & lt) : __popc(pb));
           const int ki = recbase + __popc(nb & (lt | (1u << lane))) - 1;
           const int pin = s == 1 ? (e[0] & 63) : (e[1 + s] & 63);
           hd.row_col[ri] = (uint8_t)lane;
-          hd.row_rec[ri] = (uint8_t)ki;
+          hd.row_rec[ri] = kact ? (uint8_t)ki : kValueOnly;
           hd.row_pin[ri] = (uint8_t)pin;
           hd.row_store[ri] = (uint8_t)s;
           // the row's source (copied below by eight lanes at a time) and its value (scale,
           // zero) pair, issued by the column's lane
-          const uint8_t* base = (s == 1 ? brec : rrec) + (size_t)g * kRec;
-          wc.row_src[ri] = base + pin * 128;
-          cp_async8(szs + ri * 8, base + kRecVsz + pin * 8);
-          if (isnew) wc.rec_src[ki] = base + kRecKsz;
+          if constexpr (kPk) {
+            const uint8_t* base = s == 1 ? brec + (size_t)g * kRec : rrec + (size_t)g * RB::kBytes;
+            wc.row_src[ri] = base + pin * (s == 1 ? 128 : RB::kRow);
+            cp_async8(szs + ri * 8, base + (s == 1 ? kRecVsz : RB::kVsz) + pin * 8);
+            if (isnew) wc.rec_src[ki] = base + (s == 1 ? kRecKsz : RB::kKsz);
+          } else {
+            const uint8_t* base = (s == 1 ? brec : rrec) + (size_t)g * kRec;
+            wc.row_src[ri] = base + pin * 128;
+            cp_async8(szs + ri * 8, base + kRecVsz + pin * 8);
+            if (isnew) wc.rec_src[ki] = base + kRecKsz;
+          }
         }
         rowbase += __popc(b);
         recbase += __popc(nb);
@@ -286,8 +314,16 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
       __syncwarp();
       // rows: eight lanes per 128-byte row, four rows per copy instruction (contiguous
       // pieces, so each instruction touches four lines rather than 32)
-      for (int ri = lane >> 3; ri < nrows; ri += 4)
+      for (int ri = lane >> 3; ri < nrows; ri += 4) {
+        // 2-bit rows are 64 bytes; a value-only row needs its value half (bytes 64..127)
+        if constexpr (kPk) {
+          if ((lane & 7) >= 4 && hd.row_store[ri] >= 2) continue;
+        }
+        if constexpr (kFullS) {
+          if ((lane & 7) < 4 && hd.row_rec[ri] == kValueOnly) continue;
+        }
         cp_async16(rows + ri * 128 + (lane & 7) * 16, wc.row_src[ri] + (lane & 7) * 16);
+      }
       // key records: 32 pieces each, spread over the lanes
       for (int k = 0; k < nrecs; ++k) cp_async16(recs + k * 512 + lane * 16, wc.rec_src[k] + lane * 16);
       asm volatile("cp.async.commit_group;" ::: "memory");
@@ -314,14 +350,25 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
 #pragma unroll 2
     for (int p0 = 0; p0 < nrows; p0 += 8) {
       const int row = p0 + tr;
-      const bool act = row < nrows;
-      const int rid = act ? hd.row_rec[row] : 0;
+      bool act = row < nrows;
+      int rid = act ? hd.row_rec[row] : 0;
+      if constexpr (kFullS) {
+        act = act && rid != kValueOnly;
+        rid = act ? rid : 0;
+      }
       const uint32_t* lim = reinterpret_cast<const uint32_t*>(recs + rid * 512);
       float d = 0.f;
       if (act) {
         uint32_t lw[24];
         load_limbs(lim, qq, lw);
-        d = limb_dot(*reinterpret_cast<const uint4*>(rows + row * 128 + 16 * qq), lw) * pow2i(-(int)lim[kLimbE]);
+        if constexpr (kPk) {
+          const uint4 code = hd.row_store[row] >= 2
+                                 ? int2_to_nib(*reinterpret_cast<const uint2*>(rows + row * 128 + 8 * qq))
+                                 : *reinterpret_cast<const uint4*>(rows + row * 128 + 16 * qq);
+          d = limb_dot(code, lw) * pow2i(-(int)lim[kLimbE]);
+        } else {
+          d = limb_dot(*reinterpret_cast<const uint4*>(rows + row * 128 + 16 * qq), lw) * pow2i(-(int)lim[kLimbE]);
+        }
       }
       d += __shfl_xor_sync(kFull, d, 1);
       d += __shfl_xor_sync(kFull, d, 2);
@@ -335,8 +382,12 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
     const int lam_c = ls_c & 0xff;
     const float pt_c = lane < ncol ? __int_as_float(ec[2]) : 0.f;
     float l = 0.f;
-    for (int s = 1; s <= smax; ++s)
-      if (st_c >= s) l += wc.lr[hd.rowbase[s - 1] + __popc(hd.bal[s - 1] & lt)];
+    if constexpr (kFullS) {
+      if (st_c > 0) l = wc.lr[hd.rowbase[st_c - 1] + __popc(hd.bal[st_c - 1] & lt)];
+    } else {
+      for (int s = 1; s <= smax; ++s)
+        if (st_c >= s) l += wc.lr[hd.rowbase[s - 1] + __popc(hd.bal[s - 1] & lt)];
+    }
     const bool in = st_c > 0;
     l = in ? l : -INFINITY;
     const float mb = warp_max(l);
@@ -360,13 +411,22 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
         const int row = row0 + lane;
         const bool act = row < nrows;
         const int cc = act ? hd.row_col[row] : 0;
-        const float pc = __shfl_sync(kFull, p, cc);
+        float pc = __shfl_sync(kFull, p, cc);
         const float ptc = __shfl_sync(kFull, pt_c, cc);
         const int lamc = __shfl_sync(kFull, lam_c, cc);
+        int stc = 0;
+        if constexpr (kFullS) stc = __shfl_sync(kFull, st_c, cc);
         if (act) {
           const uint32_t* pr = reinterpret_cast<const uint32_t*>(szs + row * 8);
           const float2 z0 = unpack_sz(pr[0]), z1 = unpack_sz(pr[1]);
-          const float pu = hd.row_store[row] <= lamc ? ptc : 0.f;
+          float pu;
+          if constexpr (kFullS) {
+            const int rs = hd.row_store[row];
+            pc = rs == stc ? pc : 0.f;               // the loop-r value: store st
+            pu = rs == min(lamc, stc) ? ptc : 0.f;   // the tag-loop value: store min(tag, st)
+          } else {
+            pu = hd.row_store[row] <= lamc ? ptc : 0.f;  // the tag loop's rows: a prefix of the stores
+          }
           const float wS0 = 128.f * (pc * z0.x), wS1 = 128.f * (pc * z1.x);
           const float wU0 = 128.f * (pu * z0.x), wU1 = 128.f * (pu * z1.x);
           wc.wrow[row][0] = make_float2(wS0, wU0);
@@ -381,7 +441,14 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
     __syncwarp();
 #pragma unroll 4
     for (int row = par16; row < nrows; row += 2) {
-      const uint32_t x = *reinterpret_cast<const uint32_t*>(rows + row * 128 + 64 + 4 * w16);
+      uint32_t x;
+      if constexpr (kPk) {
+        x = hd.row_store[row] >= 2
+                ? int2_word(*reinterpret_cast<const uint32_t*>(rows + row * 128 + 32 + 4 * (w16 >> 1)), w16 & 1)
+                : *reinterpret_cast<const uint32_t*>(rows + row * 128 + 64 + 4 * w16);
+      } else {
+        x = *reinterpret_cast<const uint32_t*>(rows + row * 128 + 64 + 4 * w16);
+      }
       const float2 wgt = wc.wrow[row][half];
       const float x0 = nib16(x << 16), x1 = nib16(x << 12), x2 = nib16(x << 8), x3 = nib16(x << 4);
       const float x4 = nib16(x), x5 = nib16(x >> 4), x6 = nib16(x >> 8), x7 = nib16(x >> 12);
@@ -595,11 +662,10 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s) {
   sms = (dev >= 0 && dev < 64) ? sms_cached[dev] : 0;
   const int ps = a.c.plan_stride;
   const int n = staged_splits(a.c.H, a.k_sel, ps, sms > 0 ? sms : 148);
-  // the codec variants are served by the direct reader
-  if (a.c.codec != FL_CODEC_RESIDUAL_INT4 || a.r > kStoresMax || sms == 0 || n > kMaxSplits)
-    return launch_sparse_direct(a, s);
+  if (a.r > kStoresMax || sms == 0 || n > kMaxSplits) return launch_sparse_direct(a, s);
   if (!attr_set[dev]) {
-    for (auto k : {sparse_staged_kernel<false>, sparse_staged_kernel<true>}) {
+    for (auto k : {sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>, sparse_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>,
+                   sparse_staged_kernel<false, FL_CODEC_FULL_INT4>, sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>}) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCta);
       if (e != cudaSuccess) return e;
       e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -609,8 +675,11 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s) {
   }
   a.n_splits = n;
   dim3 grid(n, a.c.H);
-  return launch_pdl(a.flush ? sparse_staged_kernel<true> : sparse_staged_kernel<false>, grid, dim3(kNT),
-                    (size_t)kSmemCta, s, a);
+  auto kern = a.c.codec == FL_CODEC_FULL_INT4       ? sparse_staged_kernel<false, FL_CODEC_FULL_INT4>
+              : a.c.codec == FL_CODEC_RESIDUAL_INT2 ? sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>
+              : a.flush                             ? sparse_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>
+                                                    : sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>;
+  return launch_pdl(kern, grid, dim3(kNT), (size_t)kSmemCta, s, a);
 }
 
 }  // namespace fl
