@@ -108,10 +108,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
   return v;
 }
+// Warp maximum in one redux.sync: floats map to signed integers in the same order
+// (non-negative ones keep their bits, negative ones flip their magnitude bits), so the
+// integer maximum is the image of the float maximum (inputs are never NaN).
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-  return v;
+  const int b = __float_as_int(v);
+  const int m = __reduce_max_sync(kFull, b >= 0 ? b : b ^ 0x7fffffff);
+  return __int_as_float(m >= 0 ? m : m ^ 0x7fffffff);
 }
 
 // (scale, zero) fp16 pair packed in a 32-bit word (scale in the low half).
