@@ -130,29 +130,46 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
         __syncwarp();
         for (int tt = lane; tt < kG; tt += 32)
           if ((mk >> tt) & 1ull) tokw[__popcll(mk & ((1ull << tt) - 1ull))] = (uint8_t)tt;
+        __syncwarp();
         int row = 0;
-        while (row < na) {
+        while (row < na) {  // the block's rows of one group record at a time (at most two)
           const int grp = (gs0 + row) >> 6;
           const int row_end = min(na, ((grp + 1) << 6) - gs0);
-          __syncwarp();
+          // rows of the piece in flight four passes (32 rows) at a time; the first four are
+          // issued before the weights are built
+          constexpr int kB = 4;
+          uint4 x[kB];
+          auto issue = [&](int r0) {
+#pragma unroll
+            for (int i = 0; i < kB; ++i) {
+              const int rw = r0 + 8 * i + tr;
+              const bool act = rw < row_end && (!CT::kFullState || ((need >> tokw[rw]) & 1ull));
+              x[i] = act ? res_key(rrow(gs0 + rw)) : make_uint4(0u, 0u, 0u, 0u);
+            }
+          };
+          issue(row);
           const float cg = group_weights(
               reinterpret_cast<const uint32_t*>(rrec + (size_t)grp * RB::kBytes + RB::kKsz), q_s, qsw, lane);
           __syncwarp();
           load32(qsw + 32 * qq, qsr);
-          for (int i0 = row; i0 < row_end; i0 += 8) {
-            const int rw = i0 + tr;
-            const bool act = rw < row_end && (!CT::kFullState || ((need >> tokw[rw]) & 1ull));
-            uint4 x = make_uint4(0u, 0u, 0u, 0u);
-            if (act) x = res_key(rrow(gs0 + rw));
-            float p = dot32(x, qsr);
-            p += __shfl_xor_sync(kFull, p, 1);
-            p += __shfl_xor_sync(kFull, p, 2);
-            if (act && qq == 0) {
-              if constexpr (CT::kFullState) lgw[tokw[rw]] = p + cg;
-              else lgw[tokw[rw]] += p + cg;
+          for (int r0 = row; r0 < row_end; r0 += 8 * kB) {
+            if (r0 != row) issue(r0);
+#pragma unroll
+            for (int i = 0; i < kB; ++i) {
+              if (r0 + 8 * i >= row_end) break;
+              const int rw = r0 + 8 * i + tr;
+              const bool act = rw < row_end && (!CT::kFullState || ((need >> tokw[rw]) & 1ull));
+              float p = dot32(x[i], qsr);
+              p += __shfl_xor_sync(kFull, p, 1);
+              p += __shfl_xor_sync(kFull, p, 2);
+              if (act && qq == 0) {
+                if constexpr (CT::kFullState) lgw[tokw[rw]] = p + cg;
+                else lgw[tokw[rw]] += p + cg;
+              }
             }
           }
           row = row_end;
+          __syncwarp();  // the piece's weights are used up before the next piece's are built
         }
       }
       __syncwarp();
@@ -212,17 +229,29 @@ __global__ void __launch_bounds__(kWarps * 32, 2) dense_direct_kernel(ReaderArgs
         for (int tt = lane; tt < kG; tt += 32)
           if ((mk >> tt) & 1ull) tokw[__popcll(mk & ((1ull << tt) - 1ull))] = (uint8_t)tt;
         __syncwarp();
-        for (int i0 = 0; i0 < na; i0 += 8) {
-          const int rw = i0 + tr;
+        // all of the store's rows of the block (at most 64, 8 a pass) in flight together
+        uint4 x[8];
+        uint32_t sw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rw = 8 * i + tr;
+          const bool act = rw < na && (!CT::kFullState || ((need >> tokw[rw]) & 1ull));
+          const int gs = gs0 + rw;
+          x[i] = act ? res_val(rrow(gs)) : make_uint4(0u, 0u, 0u, 0u);
+          sw[i] = act ? __ldg(reinterpret_cast<const uint32_t*>(rrec + (size_t)(gs >> 6) * RB::kBytes + RB::kVsz) +
+                              (gs & 63) * 2 + (qq >> 1))
+                      : 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rw = 8 * i + tr;
+          if (8 * i >= na) break;
           if (rw < na && (!CT::kFullState || ((need >> tokw[rw]) & 1ull))) {
-            const int gs = gs0 + rw;
-            const uint4 x = res_val(rrow(gs));
-            const float2 sz = unpack_sz(__ldg(reinterpret_cast<const uint32_t*>(
-                rrec + (size_t)(gs >> 6) * RB::kBytes + RB::kVsz) + (gs & 63) * 2 + (qq >> 1)));
+            const float2 sz = unpack_sz(sw[i]);
             const float p = lgw[tokw[rw]];
             const float P = 128.f * (p * sz.x);
             corr += fmaf(p, sz.y, -P);
-            axpy32(x, P, acc);
+            axpy32(x[i], P, acc);
           }
         }
       }

@@ -108,9 +108,7 @@ __device__ void setup_chunk(ChunkTab& t, const Smem& sm, int start, int end, int
   t.pt[lane] = pt;
   t.l[lane] = 0.f;
   t.ploc[lane] = c;
-  int mx = st;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFull, mx, o));
+  const int mx = __reduce_max_sync(kFull, st);
   if (lane == 0) {
     t.start = start;
     t.ncol = min(CHUNK, max(0, end - start));

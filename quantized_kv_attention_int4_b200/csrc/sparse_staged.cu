@@ -216,9 +216,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
       // full-state: the store of the column's tag-loop value (== st: no extra row)
       const int sv = kFullS ? min(e[1] & 0xff, st) : 0;
       if (!formed) {
-        int smax = st;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) smax = max(smax, __shfl_xor_sync(kFull, smax, o));
+        const int smax = __reduce_max_sync(kFull, st);
         int nrec_c = 0;
         for (int s = 1; s <= smax; ++s) {
           const bool act = kFullS ? st == s : st >= s;  // rows with a key part
