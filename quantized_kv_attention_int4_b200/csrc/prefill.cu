@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       ctl.rmax[hf][row] = mx;
       pair_bar(grp);
       mx = fmaxf(mx, ctl.rmax[1 - hf][row]);
+      pair_bar(grp);  // both halves have read the maxima before either writes the next tile's
       const float m_tile = mx * kScale;
       float alpha = 1.f;
       if (m_tile > m_run + 8.f) {  // also the first visible tile (m_run = -inf): alpha = 0
