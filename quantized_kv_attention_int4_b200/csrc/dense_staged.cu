@@ -34,6 +34,13 @@
 // The tail unit reads its BF16 rows from global memory in fp32.
 // Teams' partials merge per CTA; the last CTA of each head (atomic ticket) combines the
 // CTA partials by log-sum-exp and writes o and offset[r] = M + log2 L.
+//
+// Codec variants (flozi guide, section 4: the "Per-loop KIVI4" row and the 2-bit row of
+// Figure 5): 2-bit residual rows are staged as 64-byte lines and read through the 4-bit
+// layout (codes 0..3); with full-state stores a token's key and value are those of its
+// last store min(r, depth) alone: the block's base is not staged when every token has a
+// loop-2 row, a residual row's logit replaces (not adds to) its token's, and base or
+// residual rows of tokens that have a later store get zero value weight.
 #include "flush.cuh"
 #include "kernels.h"
 
@@ -71,12 +78,13 @@ static_assert(kRing >= kMaxSpan, "ring must hold the largest span");
 // Geometry of one block's rows in one residual store, as staged in the span.
 struct StoreGeom {
   int na, n1;          // rows, rows in the first group record
-  int off_codes;       // code rows 0..na-1, 128 B each (rows past na read padding)
+  int off_codes;       // code rows 0..na-1, kRow B each (rows past na read padding)
   int off_k0, off_k1;  // key (scale, zero) records, turned into limbs in place
   int off_v0, off_v1;  // value (scale, zero) words: row i of piece p at off_vp + (vskip_p + i) * 8
   int vskip0;
 };
 
+template <int kRow>
 __device__ __forceinline__ int store_geom(unsigned long long mk, int gs0, int pos, StoreGeom& g) {
   g.na = __popcll(mk);
   g.n1 = 0;
@@ -86,7 +94,7 @@ __device__ __forceinline__ int store_geom(unsigned long long mk, int gs0, int po
   const int s0 = gs0 & 63;
   g.n1 = min(g.na, kG - s0);
   g.off_codes = pos;
-  pos += g.na * 128;
+  pos += g.na * kRow;
   g.off_k0 = pos;
   pos += 512;
   g.off_v0 = pos;
@@ -104,28 +112,30 @@ __device__ __forceinline__ int store_geom(unsigned long long mk, int gs0, int po
   return pos;
 }
 
-// Bulk copies of one span (lane 0 only); `bytes` is the span size.
+// Bulk copies of one span (lane 0 only); `bytes` is the span size; the base record is
+// staged when `base` (the residual stores' records have RB's geometry).
+template <class RB>
 __device__ __forceinline__ void issue_span(uint8_t* sp, const uint8_t* brec_b, const uint8_t* rrec,
-                                           const StoreGeom* g, const int* gs0, int bytes, uint64_t* bar) {
+                                           const StoreGeom* g, const int* gs0, int bytes, bool base, uint64_t* bar) {
   fence_proxy_async();
   mbar_expect_tx(bar, (unsigned)bytes);
-  bulk_g2s(sp, brec_b, kRec, bar);
+  if (base) bulk_g2s(sp, brec_b, kRec, bar);
 #pragma unroll
   for (int s = 0; s < kStores; ++s) {
     const StoreGeom& G = g[s];
     if (G.na == 0) continue;
     const int s0 = gs0[s] & 63;
-    const uint8_t* R0 = rrec + (size_t)(gs0[s] >> 6) * kRec;
-    bulk_g2s(sp + G.off_codes, R0 + s0 * 128, G.n1 * 128, bar);
-    bulk_g2s(sp + G.off_k0, R0 + kRecKsz, 512, bar);
+    const uint8_t* R0 = rrec + (size_t)(gs0[s] >> 6) * RB::kBytes;
+    bulk_g2s(sp + G.off_codes, R0 + s0 * RB::kRow, G.n1 * RB::kRow, bar);
+    bulk_g2s(sp + G.off_k0, R0 + RB::kKsz, 512, bar);
     const int a0 = s0 & ~1, a1 = (s0 + G.n1 + 1) & ~1;
-    bulk_g2s(sp + G.off_v0, R0 + kRecVsz + a0 * 8, (a1 - a0) * 8, bar);
+    bulk_g2s(sp + G.off_v0, R0 + RB::kVsz + a0 * 8, (a1 - a0) * 8, bar);
     if (G.n1 < G.na) {
       const int n2 = G.na - G.n1;
-      const uint8_t* R1 = R0 + kRec;
-      bulk_g2s(sp + G.off_codes + G.n1 * 128, R1, n2 * 128, bar);
-      bulk_g2s(sp + G.off_k1, R1 + kRecKsz, 512, bar);
-      bulk_g2s(sp + G.off_v1, R1 + kRecVsz, ((n2 + 1) & ~1) * 8, bar);
+      const uint8_t* R1 = R0 + RB::kBytes;
+      bulk_g2s(sp + G.off_codes + G.n1 * RB::kRow, R1, n2 * RB::kRow, bar);
+      bulk_g2s(sp + G.off_k1, R1 + RB::kKsz, 512, bar);
+      bulk_g2s(sp + G.off_v1, R1 + RB::kVsz, ((n2 + 1) & ~1) * 8, bar);
     }
   }
 }
@@ -140,9 +150,14 @@ __device__ __forceinline__ void pair_sync(int pair) {
   asm volatile("bar.sync %0, 64;" ::"r"(pair + 1) : "memory");
 }
 
-// kFlush: the step also writes this loop's store of a full tail (fused flush)
-template <bool kFlush>
+// kFlush: the step also writes this loop's store of a full tail (fused flush);
+// kCodec: FL_CODEC_* of the loop r >= 2 stores
+template <bool kFlush, int kCodec>
 __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a, int n_cta) {
+  using CT = CodecT<kCodec>;
+  using RB = Rec<CT::kResBits>;
+  constexpr bool kFullS = CT::kFullState;
+  constexpr bool kPk = CT::kResBits == 2;
   extern __shared__ __align__(128) uint8_t smem[];
   int* last = reinterpret_cast<int*>(smem);
   float* q_all = reinterpret_cast<float*>(smem + 64);
@@ -255,8 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
           gs[0] = __shfl_sync(kFull, m_gs, 0);
           gs[1] = __shfl_sync(kFull, m_gs, 1);
           StoreGeom g[kStores];
-          int pos = store_geom(mk2[0], gs[0], kRec, g[0]);
-          pos = store_geom(mk2[1], gs[1], pos, g[1]);
+          // full-state stores: no base when every token of the block has a loop-2 row
+          const bool base = !kFullS || nst == 0 || mk2[0] != ~0ull;
+          int pos = store_geom<RB::kRow>(mk2[0], gs[0], base ? kRec : 0, g[0]);
+          pos = store_geom<RB::kRow>(mk2[1], gs[1], pos, g[1]);
           int start = -1;
           if (iss_seq == con_seq) {
             start = 0;
@@ -280,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
             w.slot_gs0[slot][0] = gs[0];
             w.slot_gs0[slot][1] = gs[1];
             const int h = u / nbp;
-            issue_span(ring + start, brec_l + ((size_t)h * ncb + b) * kRec,
-                       rrec_l + (size_t)h * (T / kG) * kRec, g, gs, pos, &w.bar[slot]);
+            issue_span<RB>(ring + start, brec_l + ((size_t)h * ncb + b) * kRec,
+                           rrec_l + (size_t)h * (T / kG) * RB::kBytes, g, gs, pos, base, &w.bar[slot]);
           }
           ++iss_seq;
         }
@@ -317,14 +334,19 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       uint8_t* sp = ring + w.slot_off[slot];
       StoreGeom g[kStores];
       const unsigned long long mkA = w.slot_mk[slot][0], mkB = w.slot_mk[slot][1];
+      const bool base = !kFullS || nst == 0 || mkA != ~0ull;  // as the producer decided
       {
-        const int pos = store_geom(mkA, w.slot_gs0[slot][0], kRec, g[0]);
-        store_geom(mkB, w.slot_gs0[slot][1], pos, g[1]);
+        const int pos = store_geom<RB::kRow>(mkA, w.slot_gs0[slot][0], base ? kRec : 0, g[0]);
+        store_geom<RB::kRow>(mkB, w.slot_gs0[slot][1], pos, g[1]);
       }
+      // full-state: the tokens whose last store in loop r is the base / staged store s
+      const unsigned long long need_b = kFullS && nst >= 1 ? ~mkA : ~0ull;
+      const unsigned long long need0 = kFullS && nst >= 2 ? mkA & ~mkB : mkA;
+      const unsigned long long need1 = mkB;
       // ---- key limbs (warp 1: the base record and the token maps; warp 0, which also
       //      staged the spans: the residual records) ----
       if (hw == 1) {
-        record_to_limbs(reinterpret_cast<uint32_t*>(sp + kRecKsz), qh, lane);
+        if (base) record_to_limbs(reinterpret_cast<uint32_t*>(sp + kRecKsz), qh, lane);
 #pragma unroll
         for (int s = 0; s < kStores; ++s) {
           if (g[s].na == 0) continue;
@@ -351,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       }
 
       // ---- base logits: rows 32 hw .. 32 hw + 31 ----
-      {
+      if (base) {
         const uint32_t* lim = reinterpret_cast<const uint32_t*>(sp + kRecKsz);
         uint32_t lw[24];
         load_limbs(lim, qq, lw);
@@ -379,7 +401,9 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
           const uint32_t* lim = reinterpret_cast<const uint32_t*>(sp + (ii < G.n1 ? G.off_k0 : G.off_k1));
           uint32_t lw[24];
           load_limbs(lim, qq, lw);
-          const uint4 code = *reinterpret_cast<const uint4*>(sp + G.off_codes + ii * 128 + 16 * qq);
+          uint4 code;
+          if constexpr (kPk) code = int2_to_nib(*reinterpret_cast<const uint2*>(sp + G.off_codes + ii * 64 + 8 * qq));
+          else code = *reinterpret_cast<const uint4*>(sp + G.off_codes + ii * 128 + 16 * qq);
           float v = limb_dot(code, lw) * pow2i(-(int)lim[kLimbE]);
           v += __shfl_xor_sync(kFull, v, 1);
           v += __shfl_xor_sync(kFull, v, 2);
@@ -389,13 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       pair_sync(pair);
 
       // ---- block softmax (both warps, identically) ----
-      float l0 = w.lg[lane], l1 = w.lg[lane + 32];
+      float l0 = base ? w.lg[lane] : 0.f, l1 = base ? w.lg[lane + 32] : 0.f;
 #pragma unroll
       for (int s = 0; s < kStores; ++s) {
         if (g[s].na == 0) continue;
         const unsigned long long mk = s == 0 ? mkA : mkB;
-        if ((mk >> lane) & 1ull) l0 += w.rl[s][__popcll(mk & ((1ull << lane) - 1ull))];
-        if ((mk >> (lane + 32)) & 1ull) l1 += w.rl[s][__popcll(mk & ((1ull << (lane + 32)) - 1ull))];
+        if constexpr (kFullS) {  // the logit of the token's last store
+          const unsigned long long nd = s == 0 ? need0 : need1;
+          if ((nd >> lane) & 1ull) l0 = w.rl[s][__popcll(mk & ((1ull << lane) - 1ull))];
+          if ((nd >> (lane + 32)) & 1ull) l1 = w.rl[s][__popcll(mk & ((1ull << (lane + 32)) - 1ull))];
+        } else {
+          if ((mk >> lane) & 1ull) l0 += w.rl[s][__popcll(mk & ((1ull << lane) - 1ull))];
+          if ((mk >> (lane + 32)) & 1ull) l1 += w.rl[s][__popcll(mk & ((1ull << (lane + 32)) - 1ull))];
+        }
       }
       if (a.keep && hw == 0) {
         score[(size_t)b * kG + lane] = l0;
@@ -418,7 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
         const int v = lane + 32 * i;
         int tok = v, off = kRecVsz + v * 8;  // base rows: token v, (scale, zero) in the base record
         bool act = v < kG;
-        if (!act && v < nvr) {
+        if constexpr (kFullS) act = act && base && ((need_b >> v) & 1ull);
+        if (v >= kG && v < nvr) {
           int vv = v - kG;
           const int s = vv >= pad0 ? 1 : 0;
           if (s) vv -= pad0;
@@ -428,6 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
             tok = w.tok[s][vv];
             off = vv < n1 ? (s ? g[1].off_v0 : g[0].off_v0) + ((s ? g[1].vskip0 : g[0].vskip0) + vv) * 8
                           : (s ? g[1].off_v1 : g[0].off_v1) + (vv - n1) * 8;
+            if constexpr (kFullS) act = (((s ? need1 : need0) >> tok) & 1ull) != 0;  // its last store
           }
         }
         // p' of the row's token sits in lane tok & 31 (p0 for tokens < 32, else p1)
@@ -465,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       int a0[8], a1[8], a2[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) a0[i] = a1[i] = a2[i] = 0;
-      {
+      if (base) {
         const uint8_t* vb = sp + 64 + 4 * wv;
 #pragma unroll
         for (int kg = g4; kg < 16; kg += 4) {
@@ -479,12 +511,24 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
       for (int s = 0; s < kStores; ++s) {
         const int ng = (s ? pad1 : pad0) >> 2;
         const int kb = 16 + (s ? (pad0 >> 2) : 0);
-        const uint8_t* vb = sp + (s ? g[1].off_codes : g[0].off_codes) + 64 + 4 * wv;
-        for (int kg = g4; kg < ng; kg += 4) {
-          const uint8_t* rp = vb + kg * 512;
-          v_group(*reinterpret_cast<const uint32_t*>(rp), *reinterpret_cast<const uint32_t*>(rp + 128),
-                  *reinterpret_cast<const uint32_t*>(rp + 256), *reinterpret_cast<const uint32_t*>(rp + 384),
-                  w.wl[kb + kg][hw], a0, a1, a2);
+        if constexpr (kPk) {  // 64-byte rows: value word wv / 2, its half wv % 2
+          const uint8_t* vb = sp + (s ? g[1].off_codes : g[0].off_codes) + 32 + 4 * (wv >> 1);
+          const int up = wv & 1;
+          for (int kg = g4; kg < ng; kg += 4) {
+            const uint8_t* rp = vb + kg * 256;
+            v_group(int2_word(*reinterpret_cast<const uint32_t*>(rp), up),
+                    int2_word(*reinterpret_cast<const uint32_t*>(rp + 64), up),
+                    int2_word(*reinterpret_cast<const uint32_t*>(rp + 128), up),
+                    int2_word(*reinterpret_cast<const uint32_t*>(rp + 192), up), w.wl[kb + kg][hw], a0, a1, a2);
+          }
+        } else {
+          const uint8_t* vb = sp + (s ? g[1].off_codes : g[0].off_codes) + 64 + 4 * wv;
+          for (int kg = g4; kg < ng; kg += 4) {
+            const uint8_t* rp = vb + kg * 512;
+            v_group(*reinterpret_cast<const uint32_t*>(rp), *reinterpret_cast<const uint32_t*>(rp + 128),
+                    *reinterpret_cast<const uint32_t*>(rp + 256), *reinterpret_cast<const uint32_t*>(rp + 384),
+                    w.wl[kb + kg][hw], a0, a1, a2);
+          }
         }
       }
       const float isc = pow2i(-E);
@@ -675,21 +719,24 @@ cudaError_t launch_dense(ReaderArgs a, cudaStream_t s, bool chain) {
   const long long U = (long long)a.c.H * (a.n_q / kG + 1);
   long long n = sms < U ? sms : U;
   if (n < a.c.H) n = a.c.H;  // every CTA range then touches at most two heads
-  // the codec variants are served by the direct reader
-  if (a.c.codec != FL_CODEC_RESIDUAL_INT4 || a.r > 3 || sms == 0 || n > kMaxSplits) return launch_dense_direct(a, s);
+  if (a.r > 3 || sms == 0 || n > kMaxSplits) return launch_dense_direct(a, s);
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    for (auto k : {dense_staged_kernel<false>, dense_staged_kernel<true>}) {
+    for (auto k : {dense_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>, dense_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>,
+                   dense_staged_kernel<false, FL_CODEC_FULL_INT4>, dense_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>}) {
       const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
       if (e != cudaSuccess) return e;
     }
     attr_set[dev] = true;
   }
   a.n_splits = (int)n;
-  return launch_pdl_if(chain, a.flush ? dense_staged_kernel<true> : dense_staged_kernel<false>, dim3((int)n),
-                       dim3(kThreads), (size_t)kSmemTotal, s, a, (int)n);
+  auto kern = a.c.codec == FL_CODEC_FULL_INT4       ? dense_staged_kernel<false, FL_CODEC_FULL_INT4>
+              : a.c.codec == FL_CODEC_RESIDUAL_INT2 ? dense_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>
+              : a.flush                             ? dense_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>
+                                                    : dense_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>;
+  return launch_pdl_if(chain, kern, dim3((int)n), dim3(kThreads), (size_t)kSmemTotal, s, a, (int)n);
 }
 
 }  // namespace fl
