@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
         hd.nrecs = nrecs;
         hd.smax = smax;
       }
-      int rowbase = 0, recbase = 0;
+      int rowbase = 0, recbase = 0, nbase = 0;  // nbase: rows of the base (store 1), first in the span
       for (int s = 1; s <= smax; ++s) {
         const bool kact = mine && (kFullS ? st == s : st >= s);  // key and value parts
         const bool act = kact || (kFullS && mine && s == sv);     // ... or the value part alone
@@ -308,6 +308,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
         }
         rowbase += __popc(b);
         recbase += __popc(nb);
+        if (s == 1) nbase = rowbase;
       }
       __syncwarp();
       // rows: eight lanes per 128-byte row, four rows per copy instruction (contiguous
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
       for (int ri = lane >> 3; ri < nrows; ri += 4) {
         // 2-bit rows are 64 bytes; a value-only row needs its value half (bytes 64..127)
         if constexpr (kPk) {
-          if ((lane & 7) >= 4 && hd.row_store[ri] >= 2) continue;
+          if ((lane & 7) >= 4 && ri >= nbase) continue;
         }
         if constexpr (kFullS) {
           if ((lane & 7) < 4 && hd.row_rec[ri] == kValueOnly) continue;
@@ -340,6 +341,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
     const uint8_t* rows = sp + kHdrS;
     const uint8_t* szs = rows + nrows * 128;
     uint8_t* recs = sp + kHdrS + nrows * 128 + ((nrows * 8 + 15) & ~15);
+    const int nbase = smax >= 2 ? hd.rowbase[1] : nrows;  // rows of the base come first
 
     // records -> 24-bit fixed-point query weights in byte limbs, in place
     for (int k = 0; k < nrecs; ++k) record_to_limbs(reinterpret_cast<uint32_t*>(recs + k * 512), ch.q, lane);
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
         uint32_t lw[24];
         load_limbs(lim, qq, lw);
         if constexpr (kPk) {
-          const uint4 code = hd.row_store[row] >= 2
+          const uint4 code = row >= nbase
                                  ? int2_to_nib(*reinterpret_cast<const uint2*>(rows + row * 128 + 8 * qq))
                                  : *reinterpret_cast<const uint4*>(rows + row * 128 + 16 * qq);
           d = limb_dot(code, lw) * pow2i(-(int)lim[kLimbE]);
@@ -441,7 +443,7 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
     for (int row = par16; row < nrows; row += 2) {
       uint32_t x;
       if constexpr (kPk) {
-        x = hd.row_store[row] >= 2
+        x = row >= nbase
                 ? int2_word(*reinterpret_cast<const uint32_t*>(rows + row * 128 + 32 + 4 * (w16 >> 1)), w16 & 1)
                 : *reinterpret_cast<const uint32_t*>(rows + row * 128 + 64 + 4 * w16);
       } else {
