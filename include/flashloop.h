@@ -57,8 +57,8 @@
  *   FL_CODEC_RESIDUAL_INT2  residuals as in the method with 2-bit codes:
  *                           s = fp16_rn(fp32_rn(max - min) / 3), code = clamp(.., 0, 3),
  *                           in 5120-byte residual records (below).
- *   The variants are served by the direct readers and the encode entry points; the
- *   fused tail flush (fl_decode_step_flush) takes FL_CODEC_RESIDUAL_INT4 only.
+ *   Every reader and encode entry point serves all three codecs; the fused tail flush
+ *   (fl_decode_step_flush) writes FL_CODEC_RESIDUAL_INT4 stores only.
  *
  * Packed cache layout (one buffer of fl_cache_layout().total_bytes; every array
  * starts on a 256-byte boundary; L layers, H heads, C = capacity, T = total slots,
