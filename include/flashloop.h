@@ -214,7 +214,10 @@ fl_status fl_encode_base(const fl_dims* dims, void* cache, int32_t layer, int32_
  * then rebuilt).  Rows go to slots [slot0, slot0 + n_rows) of the loop's store; slot0
  * is a multiple of 64 and slot0 + n_rows <= res_capacity[loop].  Inputs are BF16
  * [H][.][128]: with `compact` = 1 row i of k/v is token rows[i]; with `compact` = 0
- * it is token row0 + i.  n_rows may be 0 (clears the blocks' metadata only). */
+ * it is token row0 + i.  n_rows may be 0 (clears the blocks' metadata only).
+ * Codecs (fl_dims.codec): FL_CODEC_FULL_INT4 stores X^(loop) itself instead of the
+ * residual; FL_CODEC_RESIDUAL_INT2 quantises the residual to 2-bit codes in the 5120-byte
+ * records. */
 fl_status fl_encode_residual(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,
                              int32_t row0, int32_t n_span, int32_t slot0,
                              const int32_t* rows, int32_t n_rows,
