@@ -168,3 +168,23 @@ def test_int2_records_take_5120_bytes_and_codecs_are_checked():
     with pytest.raises(abi.FlashLoopError) as e:
         abi.fl_cache_layout(bad)
     assert e.value.status == abi.FL_ERR_UNSUPPORTED
+
+
+def test_fused_flush_plans_are_validated_before_launch():
+    """fl_decode_step_flush refuses the codec variants (the fused flush writes 4-bit
+    residual stores only) and plans whose active sets do not nest or whose slots are not
+    64-aligned, before any launch."""
+    good = [0, 0, 0b111, 0b011, 0b001]
+    slots = [[0, 0, 64, 0, 0], [0, 0, 128, 0, 0]]          # two layers
+    for codec, plan, st in [
+        (abi.FL_CODEC_FULL_INT4, abi.Flush(good, slots), abi.FL_ERR_UNSUPPORTED),
+        (abi.FL_CODEC_RESIDUAL_INT2, abi.Flush(good, slots), abi.FL_ERR_UNSUPPORTED),
+        (abi.FL_CODEC_RESIDUAL_INT4, abi.Flush([0, 0, 0b01, 0b11, 0], slots), abi.FL_ERR_INVALID),
+        (abi.FL_CODEC_RESIDUAL_INT4, abi.Flush(good, [[0, 0, 32, 0, 0]] * 2), abi.FL_ERR_INVALID),
+        (abi.FL_CODEC_RESIDUAL_INT4, abi.Flush(good, [[0, 0, 1024, 0, 0]] * 2), abi.FL_ERR_INVALID),
+    ]:
+        d = _dims(codec=codec)
+        ws = abi.fl_workspace_bytes(d)
+        got = abi._c_step_flush(ctypes.byref(d), FAKE, 64, 64, 2, 10, 1, 4, FAKE, None, None, FAKE, FAKE, ws,
+                                None, ctypes.byref(plan), None)
+        assert got == st, (codec, got)
