@@ -112,7 +112,8 @@ def _check(where: str, st: int):
 
 def Dims(layers: int, heads: int, loops: int, capacity: int, max_select: int, res_capacity,
          codec: int = FL_CODEC_RESIDUAL_INT4) -> fl_dims:
-    """fl_dims with head_dim 128 / group 64; res_capacity[r] for r = 2..loops (mapping or list)."""
+    """fl_dims with head_dim 128 / group 64; res_capacity[r] for r = 2..loops (mapping or list);
+    codec: FL_CODEC_* of the loop r >= 2 stores (the method's 4-bit residuals by default)."""
     d = fl_dims()
     d.layers, d.heads, d.head_dim, d.group = layers, heads, HEAD_DIM, GROUP
     d.loops, d.capacity, d.max_select, d.codec = loops, capacity, max_select, codec

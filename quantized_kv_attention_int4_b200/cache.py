@@ -12,6 +12,11 @@ that advance through the same token timeline:
   description, "Configuration and supported scope": 64-token BF16 tail; FlashLoop
   project page, "The Method", Step 03: residuals for active tokens only).
 
+``codec`` selects what the loop r >= 2 stores hold (``abi.FL_CODEC_*``): the method's
+4-bit residuals, per-loop 4-bit full states, or 2-bit residuals.  The fused tail flush
+(``step(..., flush=True)``) serves the first only; ``begin_token`` flushes any codec
+through the encode entry points.
+
 Every device operation goes through the ``abi`` wrappers.
 """
 from __future__ import annotations
