@@ -25,7 +25,13 @@
  *
  * Conventions for every entry point
  *   - All data pointers are DEVICE pointers owned by the caller.  The library never
- *     allocates, frees or keeps device memory, and keeps no global mutable state.
+ *     allocates or frees device memory.  Its only process-wide state is (a) per-device
+ *     caches filled on a device's first call (its SM count, the kernels' shared-memory
+ *     attributes, the address of the array below), each guarded so that host threads
+ *     making their first call at once neither race nor repeat it, and (b) the one static
+ *     device array of fl_decode_attn_sparse_noalloc (FL_NOALLOC_SCRATCH_BYTES per device
+ *     that loads the library).  The caches do not survive cudaDeviceReset or a context
+ *     teardown: reload the library after one.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
  *     enqueues work on it and returns; calls on one cache must be stream-ordered.
  *   - BF16 tensors are passed as uint16_t bit patterns.
@@ -185,8 +191,20 @@ fl_status fl_cache_layout(const fl_dims* dims, fl_layout* out);
 /* Zero the whole cache buffer (`cache` has fl_cache_layout().total_bytes) on `stream`. */
 fl_status fl_cache_init(const fl_dims* dims, void* cache, void* stream);
 
-/* Workspace the readers need for split-K partials and their completion counters. */
+/* Workspace the readers need for split-K partials and their completion counters: room for
+ * every dense launch and for every sparse launch with k_sel <= max_select (a sparse CTA
+ * holds at most 1024 / plan_stride selected columns, so large k_sel at many loops takes
+ * more than the usual 256 partials per head). */
 size_t fl_workspace_bytes(const fl_dims* dims);
+
+/* Host-only (no CUDA call): the number of split-K partitions per head the sparse reader
+ * of loop `loop` (2..R) uses for k_sel (1..max_select) selected columns on a device with
+ * `sm_count` SMs, into *splits; *capacity (may be NULL) receives the partials per head
+ * a workspace of fl_workspace_bytes(dims) holds.  *splits <= *capacity for every valid
+ * k_sel, and every CTA's share of the gather plan fits its shared-memory copy.
+ * FL_ERR_INVALID for out-of-range arguments. */
+fl_status fl_sparse_splits(const fl_dims* dims, int32_t loop, int32_t k_sel, int32_t sm_count, int32_t* splits,
+                           int32_t* capacity);
 
 /* Zero the workspace counters; required once before the first reader call. */
 fl_status fl_workspace_init(const fl_dims* dims, void* ws, size_t ws_bytes, void* stream);
@@ -278,7 +296,10 @@ fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer,
  *     process on that device: calls that can overlap (different streams, threads)
  *     race on it and must be serialised by the caller.
  *   - FL_ERR_UNSUPPORTED when the scratch would exceed FL_NOALLOC_SCRATCH_BYTES (many
- *     heads or a large k_sel); use fl_decode_attn_sparse with a workspace then.
+ *     heads or a large k_sel); use fl_decode_attn_sparse with a workspace then.  The
+ *     scratch is sized from the split count this very call launches with
+ *     (fl_sparse_splits with the device's SM count).
+ *   - The cached address does not survive cudaDeviceReset or a context teardown.
  * The FlashLoop pages have no counterpart: this is a deployment convenience of this
  * library, not a step of the method. */
 fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_t layer, int32_t loop,

@@ -39,7 +39,7 @@ EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init"
             "fl_workspace_init", "fl_write_tail", "fl_encode_base", "fl_encode_residual",
             "fl_decode_attn_dense", "fl_select_topk", "fl_decode_attn_sparse", "fl_decode_step",
             "fl_read_status", "fl_decode_attn_sparse_noalloc", "fl_decode_step_flush", "fl_select_active",
-            "fl_prefill_attn_sparse")
+            "fl_prefill_attn_sparse", "fl_sparse_splits")
 
 
 class fl_dims(ctypes.Structure):
@@ -97,6 +97,8 @@ _c_step_flush = _sig("fl_decode_step_flush", _I, _DP, _P, _I, _I, _I, _I, _I, _I
 _c_select_active = _sig("fl_select_active", _I, _P, _P, _I, _I, _L, _P, _I, _I, _P, _P, _P, _P)
 _c_prefill = _sig("fl_prefill_attn_sparse", _I, _P, _P, _I, _P, _P, _I, _I, _L, _L, _P, _L, _P, _P)
 _c_read_status = _sig("fl_read_status", _I, _DP, _P, ctypes.POINTER(ctypes.c_int32), _I, _P)
+_c_sparse_splits = _sig("fl_sparse_splits", _I, _DP, _I, _I, _I, ctypes.POINTER(ctypes.c_int32),
+                        ctypes.POINTER(ctypes.c_int32))
 
 
 class FlashLoopError(RuntimeError):
@@ -172,6 +174,14 @@ def fl_cache_init(dims, cache, stream=None):
 def fl_workspace_bytes(dims) -> int:
     return int(_c_workspace_bytes(ctypes.byref(dims)))
 
+
+def fl_sparse_splits(dims: fl_dims, loop: int, k_sel: int, sm_count: int):
+    """(splits, capacity): split-K partitions per head of the loop-`loop` sparse reader over
+    k_sel columns on a device with sm_count SMs, and the partials per head a workspace holds."""
+    n, cap = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("fl_sparse_splits", _c_sparse_splits(ctypes.byref(dims), loop, k_sel, sm_count, ctypes.byref(n),
+                                                ctypes.byref(cap)))
+    return n.value, cap.value
 
 def fl_workspace_init(dims, ws, stream=None):
     _check("fl_workspace_init", _c_workspace_init(ctypes.byref(dims), _ptr(ws, torch.uint8, "ws"),

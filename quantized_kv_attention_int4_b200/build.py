@@ -8,6 +8,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -42,11 +43,18 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
               "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
     if ptxas_verbose:
         common += ["-Xptxas", "-v"]
+    cmds = []
     for src in SOURCES:
         obj = os.path.join(obj_dir, src.replace(".cu", ".o"))
-        cmd = common + ["-c", os.path.join(CSRC, src), "-o", obj]
-        subprocess.run(cmd, check=True)
+        cmds.append(common + ["-c", os.path.join(CSRC, src), "-o", obj])
         objs.append(obj)
+    # translation units compile independently: one nvcc per unit, in parallel
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as pool:
+        for res in pool.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds):
+            sys.stdout.write(res.stdout)
+            sys.stderr.write(res.stderr)
+            if res.returncode != 0:
+                raise subprocess.CalledProcessError(res.returncode, res.args, res.stdout, res.stderr)
     tmp = LIB_PATH + ".tmp"
     subprocess.run([nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp], check=True)
     os.replace(tmp, LIB_PATH)

@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/flashloop.h: layout arithmetic, argument
 // validation and kernel launches.  Nothing here allocates device memory.
+#include <atomic>
 #include <cstring>
 
 #include "kernels.h"
@@ -104,7 +105,14 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 fl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FL_OK : FL_ERR_CUDA; }
 
 uint64_t ws_part_bytes(const fl_dims* d) {
-  return (uint64_t)d->heads * kMaxSplits * kPartStride * sizeof(float);
+  return (uint64_t)d->heads * workspace_splits(d->loops, d->max_select) * kPartStride * sizeof(float);
+}
+
+// The split count a sparse launch will use fits the workspace's partials (it always does
+// for k_sel <= max_select; checked before any launch all the same).
+fl_status check_sparse_splits(const fl_dims* d, int loop, int k_sel) {
+  const int n = sparse_launch_splits(d->heads, d->loops, loop, k_sel, device_sms());
+  return n <= workspace_splits(d->loops, d->max_select) ? FL_OK : FL_ERR_UNSUPPORTED;
 }
 
 fl_status check_reader(const fl_dims* d, void* cache, int layer, int loop, int n_q, int n_tail,
@@ -131,6 +139,23 @@ void set_flush(ReaderArgs& a, const fl_flush* flush, int l, int r) {
 }
 
 }  // namespace
+
+namespace fl {
+namespace {
+std::atomic<int> g_sms[kMaxDevices];
+}  // namespace
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int n = g_sms[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    g_sms[dev].store(n, std::memory_order_relaxed);  // the same value from every thread
+  }
+  return n;
+}
+}  // namespace fl
 
 extern "C" {
 
@@ -291,7 +316,9 @@ fl_status fl_decode_attn_dense(const fl_dims* dims, void* cache, int32_t layer, 
   a.o = o;
   a.part = static_cast<float*>(ws);
   a.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_part_bytes(dims));
-  return cuda_status(launch_dense(a, (cudaStream_t)stream));
+  // a standalone call is an ordinary stream-ordered launch: nothing of it may overlap the
+  // caller's preceding kernel (which may be a reader of the same layer)
+  return cuda_status(launch_dense(a, (cudaStream_t)stream, false));
 }
 
 fl_status fl_select_topk(const fl_dims* dims, void* cache, int32_t layer0, int32_t n_layers, int32_t loop,
@@ -326,6 +353,8 @@ fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer,
   if (!o_prev || loop < 2) return FL_ERR_INVALID;
   const int64_t N = (int64_t)n_q + n_tail;
   if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
+  st = check_sparse_splits(dims, loop, k_sel);
+  if (st != FL_OK) return st;
   fl_layout L;
   make_layout(dims, &L);
   ReaderArgs a{};
@@ -344,7 +373,8 @@ fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer,
   a.o = o;
   a.part = static_cast<float*>(ws);
   a.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_part_bytes(dims));
-  return cuda_status(launch_sparse(a, (cudaStream_t)stream));
+  // unchained, like the standalone dense reader
+  return cuda_status(launch_sparse(a, (cudaStream_t)stream, false));
 }
 
 // ---- sparse reader with library-owned scratch (for callers that cannot allocate) ----
@@ -354,7 +384,7 @@ fl_status fl_decode_attn_sparse(const fl_dims* dims, void* cache, int32_t layer,
 }  // extern "C"
 namespace {
 __device__ __align__(256) uint8_t g_noalloc_scratch[FL_NOALLOC_SCRATCH_BYTES];
-void* g_noalloc_ptr[64] = {nullptr};
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
 }  // namespace
 extern "C" {
 
@@ -373,19 +403,27 @@ fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_
   if (!aligned16(q) || !aligned16(o) || (k_new && (!aligned16(k_new) || !aligned16(v_new))))
     return FL_ERR_INVALID;
   if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
-  // scratch: per-head tickets (must start at zero), then the split partials
-  const int n_splits = sparse_splits(dims->heads, k_sel, dims->loops);
+  // scratch: per-head tickets (must start at zero), then the split partials of exactly the
+  // split count the launch below uses; a size that no device could fit is refused before
+  // any CUDA call (at least ceil(k_sel / columns per CTA) splits per head)
   const uint64_t ticket_bytes = ((uint64_t)dims->heads * sizeof(int32_t) + 255) / 256 * 256;
-  const uint64_t need = ticket_bytes + (uint64_t)dims->heads * n_splits * kPartStride * sizeof(float);
-  if (need > FL_NOALLOC_SCRATCH_BYTES) return FL_ERR_UNSUPPORTED;
+  const auto scratch_bytes = [&](int splits) {
+    return ticket_bytes + (uint64_t)dims->heads * splits * kPartStride * sizeof(float);
+  };
+  const int cols = sparse_cta_columns(dims->loops);
+  if (scratch_bytes((k_sel + cols - 1) / cols) > FL_NOALLOC_SCRATCH_BYTES) return FL_ERR_UNSUPPORTED;
+  const int sms = device_sms();
+  if (sms <= 0) return FL_ERR_CUDA;
+  if (scratch_bytes(sparse_launch_splits(dims->heads, dims->loops, loop, k_sel, sms)) > FL_NOALLOC_SCRATCH_BYTES)
+    return FL_ERR_UNSUPPORTED;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FL_ERR_CUDA;
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return FL_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FL_ERR_CUDA;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FL_ERR_CUDA;
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);  // the same address from every thread
   }
-  uint8_t* scratch = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
+  uint8_t* scratch = static_cast<uint8_t*>(p);
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(scratch, 0, (size_t)dims->heads * sizeof(int32_t), s) != cudaSuccess) return FL_ERR_CUDA;
   fl_layout L;
@@ -406,7 +444,18 @@ fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_
   a.o = o;
   a.counter = reinterpret_cast<int32_t*>(scratch);
   a.part = reinterpret_cast<float*>(scratch + ticket_bytes);
-  return cuda_status(launch_sparse(a, s));
+  return cuda_status(launch_sparse(a, s, false));
+}
+
+fl_status fl_sparse_splits(const fl_dims* dims, int32_t loop, int32_t k_sel, int32_t sm_count, int32_t* splits,
+                           int32_t* capacity) {
+  fl_status st = check_dims(dims);
+  if (st != FL_OK) return st;
+  if (!splits || loop < 2 || loop > dims->loops || k_sel < 1 || k_sel > dims->max_select || sm_count < 1)
+    return FL_ERR_INVALID;
+  *splits = sparse_launch_splits(dims->heads, dims->loops, loop, k_sel, sm_count);
+  if (capacity) *capacity = workspace_splits(dims->loops, dims->max_select);
+  return FL_OK;
 }
 
 fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
@@ -448,6 +497,10 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
     if (N > FL_MAX_SELECT_COLS) return FL_ERR_UNSUPPORTED;
     if (k_sel < 1 || k_sel > N || k_sel > dims->max_select) return FL_ERR_INVALID;
     if (loop_first == 1 && dense_loops == 0) return FL_ERR_INVALID;  // a sparse loop needs a predecessor
+    for (int r = loop_first > dense_loops + 1 ? loop_first : dense_loops + 1; r <= loop_last; ++r) {
+      st = check_sparse_splits(dims, r, k_sel);
+      if (st != FL_OK) return st;
+    }
   }
   fl_layout lay;
   make_layout(dims, &lay);

@@ -699,38 +699,26 @@ __global__ void __launch_bounds__(kThreads, 1) dense_staged_kernel(ReaderArgs a,
   }
 }
 
-int num_sms() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < 0 || dev >= 64) return 0;
-  if (cached[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
+std::atomic<bool> g_attr_done[kMaxDevices];
+std::mutex g_attr_mu;
 
 }  // namespace
 
 cudaError_t launch_dense(ReaderArgs a, cudaStream_t s, bool chain) {
-  const int sms = num_sms();
+  const int sms = device_sms();
   const long long U = (long long)a.c.H * (a.n_q / kG + 1);
   long long n = sms < U ? sms : U;
   if (n < a.c.H) n = a.c.H;  // every CTA range then touches at most two heads
   if (a.r > 3 || sms == 0 || n > kMaxSplits) return launch_dense_direct(a, s);
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  const cudaError_t e = once_per_device(g_attr_done, g_attr_mu, [](int) {
     for (auto k : {dense_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>, dense_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>,
                    dense_staged_kernel<false, FL_CODEC_FULL_INT4>, dense_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>}) {
       const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
       if (e != cudaSuccess) return e;
     }
-    attr_set[dev] = true;
-  }
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
   a.n_splits = (int)n;
   auto kern = a.c.codec == FL_CODEC_FULL_INT4       ? dense_staged_kernel<false, FL_CODEC_FULL_INT4>
               : a.c.codec == FL_CODEC_RESIDUAL_INT2 ? dense_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>

@@ -1,6 +1,9 @@
 // Internal launcher declarations shared by the CUDA translation units.
 #pragma once
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 
 namespace fl {
@@ -74,13 +77,47 @@ cudaError_t launch_encode_residual(const EncodeResArgs& a, cudaStream_t s);
 // preceding kernel)
 cudaError_t launch_dense(ReaderArgs a, cudaStream_t s, bool chain = true);
 cudaError_t launch_dense_direct(ReaderArgs a, cudaStream_t s);
-cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s);
-cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s);
+// a.n_splits is set by the launcher (sparse_launch_splits); it must fit the partials buffer
+cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s, bool chain = true);
+cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s, bool chain = true);
 cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s);
 cudaError_t launch_token_select(const TokenArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_attn(const PrefillArgs& a, cudaStream_t s);
 
 int dense_splits(int heads, int n_q);
-int sparse_splits(int heads, int k_sel, int loops);
+
+// Number of devices the per-device caches below cover.
+constexpr int kMaxDevices = 64;
+
+// SM count of the current device, looked up once per device (safe when several host
+// threads make their first call at the same time); 0 when it cannot be read.
+int device_sms();
+
+// Runs fn(dev) once per device (device = the current one), under a lock, so host threads
+// that make their first call at the same time neither race nor repeat it; a failed set-up
+// is retried by the next call.
+template <class F>
+cudaError_t once_per_device(std::atomic<bool>* done, std::mutex& mu, F&& fn) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+  const cudaError_t e = fn(dev);
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
+// Plan entries (selected columns) one sparse-reader CTA holds in shared memory.
+int sparse_cta_columns(int loops);
+// Split-K partitions per head that launch_sparse uses for a loop-r reader over k_sel
+// columns on a device with `sms` SMs: never fewer than ceil(k_sel / sparse_cta_columns).
+int sparse_launch_splits(int heads, int loops, int r, int k_sel, int sms);
+// Split-K partials per head that a workspace for these dims holds: enough for every
+// dense launch and for every sparse launch with k_sel <= max_select.
+int workspace_splits(int loops, int max_select);
+// The direct sparse reader's split count and per-CTA plan capacity (sparse.cu).
+int direct_splits(int heads, int k_sel, int loops, int sms);
+int direct_cta_columns(int loops);
 
 }  // namespace fl

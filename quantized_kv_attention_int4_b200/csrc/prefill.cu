@@ -404,19 +404,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 namespace {
 
 // cuTensorMapEncodeTiled, fetched once from the driver through the runtime
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime (a function-
+// local static: initialised once even when several host threads arrive together)
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
+
+std::atomic<bool> g_attr_done[kMaxDevices];
+std::mutex g_attr_mu;
 
 // [heads][rows][128] BF16 (row stride 256 bytes, head stride head_stride elements) as a 3-D
 // tensor map read in 64 x 128 boxes with the 128-byte swizzle; rows past `rows` read as 0
@@ -441,15 +444,10 @@ cudaError_t launch_prefill_attn(const PrefillArgs& a, cudaStream_t s) {
   if (!make_map(&mq, a.q, a.n_act, a.heads, a.q_head_stride) || !make_map(&mk, a.k, a.n_tokens, a.heads, a.kv_head_stride) ||
       !make_map(&mv, a.v, a.n_tokens, a.heads, a.kv_head_stride))
     return cudaErrorInvalidValue;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  const cudaError_t e = once_per_device(g_attr_done, g_attr_mu, [](int) {
+    return cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid((a.n_act + kPT - 1) / kPT, a.heads);
   prefill_attn_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(a, mq, mk, mv);
   return cudaGetLastError();

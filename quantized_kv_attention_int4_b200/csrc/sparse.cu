@@ -635,21 +635,26 @@ __global__ void __launch_bounds__(NT, 3) sparse_kernel(ReaderArgs a) {
 
 }  // namespace
 
-int sparse_splits(int heads, int k_sel, int loops) {
+// Splits of the direct reader: about one wave at 3 CTAs per SM and >= ~16 columns per
+// CTA, but never fewer than the plan needs (a CTA holds at most PLANW / plan_stride
+// columns), so no CTA's share of the plan overruns its shared-memory copy.
+int direct_splits(int heads, int k_sel, int loops, int sms) {
   const int ps = (loops + 2 + 3) / 4 * 4;
   const int cmax = PLANW / ps;                    // plan entries a CTA can hold
   const int need = (k_sel + cmax - 1) / cmax;
-  const int by_sms = (148 * 3) / heads;           // one wave at 3 CTAs per SM
+  const int by_sms = (sms * 3) / heads;           // one wave at 3 CTAs per SM
   const int by_work = (k_sel + 15) / 16;          // at least ~16 columns per CTA
   int s = by_sms < by_work ? by_sms : by_work;
+  if (s > kMaxSplits) s = kMaxSplits;
   if (s < need) s = need;
   if (s < 1) s = 1;
-  if (s > kMaxSplits) s = kMaxSplits;
   return s;
 }
 
-cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s) {
-  a.n_splits = sparse_splits(a.c.H, a.k_sel, a.c.R);
+int direct_cta_columns(int loops) { return PLANW / ((loops + 2 + 3) / 4 * 4); }
+
+cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s, bool chain) {
+  a.n_splits = direct_splits(a.c.H, a.k_sel, a.c.R, device_sms() > 0 ? device_sms() : 148);
   const bool flush = a.flush && a.c.codec == FL_CODEC_RESIDUAL_INT4;
   const size_t smem = flush && sizeof(EncodeSmem) > sizeof(Smem) ? sizeof(EncodeSmem) : sizeof(Smem);
   auto kern = a.c.codec == FL_CODEC_FULL_INT4       ? sparse_kernel<false, FL_CODEC_FULL_INT4>
@@ -659,7 +664,7 @@ cudaError_t launch_sparse_direct(ReaderArgs a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_splits, a.c.H);
-  return launch_pdl(kern, grid, dim3(NT), smem, s, a);
+  return launch_pdl_if(chain, kern, grid, dim3(NT), smem, s, a);
 }
 
 }  // namespace fl

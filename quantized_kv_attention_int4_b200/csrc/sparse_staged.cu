@@ -637,6 +637,9 @@ __global__ void __launch_bounds__(kNT, kCtaPerSm) sparse_staged_kernel(ReaderArg
   }
 }
 
+// Splits of the staged reader: one wave at kCtaPerSm CTAs per SM and >= ~32 columns per
+// CTA, but never fewer than the plan needs (a CTA holds at most kPlanWords / plan_stride
+// columns in shared memory).
 int staged_splits(int heads, int k_sel, int ps, int sms) {
   const int per = kPlanWords / ps;                                 // plan entries a CTA can hold
   const int need = (k_sel + per - 1) / per;
@@ -648,22 +651,36 @@ int staged_splits(int heads, int k_sel, int ps, int sms) {
   return s;
 }
 
+std::atomic<bool> g_attr_done[kMaxDevices];
+std::mutex g_attr_mu;
+
 }  // namespace
 
-cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s) {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  static int sms_cached[64] = {0};
-  static bool attr_set[64] = {false};
-  if (dev >= 0 && dev < 64 && sms_cached[dev] == 0) {
-    if (cudaDeviceGetAttribute(&sms_cached[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms_cached[dev] = 0;
+int sparse_cta_columns(int loops) {
+  const int ps = (loops + 2 + 3) / 4 * 4;
+  const int staged = kPlanWords / ps, direct = direct_cta_columns(loops);
+  return staged < direct ? staged : direct;
+}
+
+int sparse_launch_splits(int heads, int loops, int r, int k_sel, int sms) {
+  if (r <= kStoresMax && sms > 0) {
+    const int n = staged_splits(heads, k_sel, (loops + 2 + 3) / 4 * 4, sms);
+    if (n <= kMaxSplits) return n;
   }
-  sms = (dev >= 0 && dev < 64) ? sms_cached[dev] : 0;
-  const int ps = a.c.plan_stride;
-  const int n = staged_splits(a.c.H, a.k_sel, ps, sms > 0 ? sms : 148);
-  if (a.r > kStoresMax || sms == 0 || n > kMaxSplits) return launch_sparse_direct(a, s);
-  if (!attr_set[dev]) {
+  return direct_splits(heads, k_sel, loops, sms > 0 ? sms : 148);
+}
+
+int workspace_splits(int loops, int max_select) {
+  const int cols = sparse_cta_columns(loops);
+  const int need = (max_select + cols - 1) / cols;
+  return need > kMaxSplits ? need : kMaxSplits;
+}
+
+cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s, bool chain) {
+  const int sms = device_sms();
+  const int n = sparse_launch_splits(a.c.H, a.c.R, a.r, a.k_sel, sms);
+  if (a.r > kStoresMax || sms == 0 || n > kMaxSplits) return launch_sparse_direct(a, s, chain);
+  const cudaError_t e = once_per_device(g_attr_done, g_attr_mu, [](int) {
     for (auto k : {sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>, sparse_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>,
                    sparse_staged_kernel<false, FL_CODEC_FULL_INT4>, sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>}) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCta);
@@ -671,15 +688,16 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s) {
       e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
       if (e != cudaSuccess) return e;
     }
-    attr_set[dev] = true;
-  }
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
   a.n_splits = n;
   dim3 grid(n, a.c.H);
   auto kern = a.c.codec == FL_CODEC_FULL_INT4       ? sparse_staged_kernel<false, FL_CODEC_FULL_INT4>
               : a.c.codec == FL_CODEC_RESIDUAL_INT2 ? sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>
               : a.flush                             ? sparse_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>
                                                     : sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>;
-  return launch_pdl(kern, grid, dim3(kNT), (size_t)kSmemCta, s, a);
+  return launch_pdl_if(chain, kern, grid, dim3(kNT), (size_t)kSmemCta, s, a);
 }
 
 }  // namespace fl

@@ -25,3 +25,14 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Report the largest elementwise relative errors the parity tests saw."""
+    mod = sys.modules.get("flhelpers")
+    if mod is None or not getattr(mod, "ELEMENTWISE", None):
+        return
+    ELEMENTWISE, ELEM_FLOOR = mod.ELEMENTWISE, mod.ELEM_FLOOR
+    terminalreporter.write_sep("-", f"elementwise relative error (floor {ELEM_FLOOR:g} x ||ref||_inf per head)")
+    for label in sorted(ELEMENTWISE):
+        terminalreporter.write_line(f"{label}: {ELEMENTWISE[label]:.3e}")

@@ -19,7 +19,7 @@ def _declared():
 
 def test_every_declared_symbol_is_exported():
     names = _declared()
-    assert len(names) == 18
+    assert len(names) == 19
     for n in names:
         assert hasattr(abi.lib, n), n
     assert set(names) == set(abi.EXPORTED)
@@ -188,3 +188,33 @@ def test_fused_flush_plans_are_validated_before_launch():
         got = abi._c_step_flush(ctypes.byref(d), FAKE, 64, 64, 2, 10, 1, 4, FAKE, None, None, FAKE, FAKE, ws,
                                 None, ctypes.byref(plan), None)
         assert got == st, (codec, got)
+
+
+@pytest.mark.parametrize("loops", [4, 8, 9, 32])
+def test_sparse_split_counts_fit_the_plan_copy_and_the_workspace(loops):
+    """For every k_sel the sparse reader accepts, its split count leaves each CTA a share
+    of the gather plan that fits the CTA's 1024-word shared-memory copy, and the workspace
+    of fl_workspace_bytes holds that many partials per head -- including the deep 32-loop
+    cache with every column selected (K_sel = N = 8192, 36-word plan entries), where 256
+    splits would not do."""
+    cap = 8192 + 128
+    d = abi.Dims(layers=1, heads=16, loops=loops, capacity=cap, max_select=cap,
+                 res_capacity={r: cap for r in range(2, loops + 1)})
+    L = abi.fl_cache_layout(d)
+    per_cta = 1024 // L.plan_stride
+    base_ws = abi.fl_workspace_bytes(d)
+    for sms in (1, 148, 160, 1024):
+        for loop in sorted({2, 3, min(8, loops), loops}):
+            for k_sel in (1, 7, 31, 820, 3277, 7168, 7169, 8192, cap):
+                n, capacity = abi.fl_sparse_splits(d, loop, k_sel, sms)
+                assert 1 <= n <= capacity, (sms, loop, k_sel, n, capacity)
+                assert -(-k_sel // n) <= per_cta, (sms, loop, k_sel, n)
+                # the workspace holds `capacity` partials of 260 floats per head, then the tickets
+                assert base_ws >= 16 * capacity * 260 * 4 + 16 * 4
+    if loops == 32:
+        n, capacity = abi.fl_sparse_splits(d, 32, 8192, 148)
+        assert n > 256 and capacity >= n
+    with pytest.raises(abi.FlashLoopError):
+        abi.fl_sparse_splits(d, 1, 10, 148)          # loop 1 is never sparse
+    with pytest.raises(abi.FlashLoopError):
+        abi.fl_sparse_splits(d, 2, cap + 1, 148)     # above max_select
