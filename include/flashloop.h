@@ -388,8 +388,9 @@ fl_status fl_select_active(const uint16_t* h_prev, const uint16_t* h_cur, int32_
  * buffers so the work stays a regular GEMM).  Sparse prefill attention of one loop: the
  * n_act active tokens' queries attend causally over every token's key and value,
  *     o[h][i] = softmax_{j <= pos[i]}(q[h][i] . k[h][j] / sqrt(128)) v[h][j],
- * on the tensor cores (BF16 operands, fp32 accumulation; the probabilities are rounded
- * to BF16 for the value product, the row sum is taken in fp32).
+ * on the tensor cores (BF16 operands, fp32 accumulation; the probabilities reach the
+ * value product as two BF16 terms P_hi + P_lo, about 16 significant bits, and the row sum
+ * is taken in fp32).
  *   q: BF16 [heads][n_act][128] (compact, in token order; head stride q_head_stride
  *      elements); pos: device int32 [n_act], strictly ascending, in [0, n_tokens);
  *   k, v: BF16 [heads][n_tokens][128] (head stride kv_head_stride): each token's key and

@@ -8,16 +8,18 @@
 //     o_i = softmax_{j <= pos_i}(q_i k_j^T / sqrt(128)) v_j.
 //
 // One CTA of 8 softmax warps and one MMA warp per (128 active queries, head).  The query
-// tile stays in shared memory; key tiles of 128 tokens stream through three buffers
-// and value tiles through two, copied by a load warp with tensor maps (TMA: 64 x 128
-// boxes in the 128-byte swizzle the MMA descriptors name, zeros past the end) as soon as
-// the tensor cores release a buffer.  The MMA warp issues S = Q K^T
-// (8 tcgen05.mma of M = N = 128, K = 16; BF16 operands from 128-byte-swizzled shared
-// memory; fp32 accumulators in TMEM) one tile ahead into alternating TMEM buffers, and
-// O += P V once P is written (V read MN-major).  Softmax warp w reads TMEM lanes
+// tile stays in shared memory; key tiles of 128 tokens and value tiles stream through two
+// buffers each, copied by a load warp with tensor maps (TMA: 64 x 128 boxes in the
+// 128-byte swizzle the MMA descriptors name, zeros past the end) as soon as the tensor
+// cores release a buffer.  The MMA warp issues S = Q K^T (8 tcgen05.mma of M = N = 128,
+// K = 16; BF16 operands from 128-byte-swizzled shared memory; fp32 accumulators in TMEM)
+// one tile ahead into alternating TMEM buffers, and O += P V once P is written (V read
+// MN-major).  P reaches the tensor cores as two BF16 tiles, P = P_hi + P_lo with
+// P_hi = bf16(p) and P_lo = bf16(p - P_hi), so the value product carries p to about 16
+// significant bits rather than BF16's 8 (16 MMAs per value tile instead of 8).  Softmax warp w reads TMEM lanes
 // 32 (w % 4) ..: its thread t owns query row 32 (w % 4) + t and the 64 columns of half
-// w / 4 -- it masks, runs the online softmax in the base-2 domain, writes its half of P
-// (BF16) to shared memory in the operand layout and rescales its half of the output row
+// w / 4 -- it masks, runs the online softmax in the base-2 domain, writes its half of
+// P_hi and P_lo to shared memory in the operand layout and rescales its half of the output row
 // in TMEM.  The warps hand over through mbarriers only (copies count transaction bytes,
 // softmax threads arrive when a score buffer is consumed and when P is in place,
 // tcgen05.commit signals finished MMAs), so no CTA-wide barrier sits in the loop; every
@@ -43,8 +45,8 @@ constexpr uint32_t kIdescPV = kIdescS | (1u << 16);  // B (V) read MN-major
 struct PrefillCtl {
   uint64_t bar_s[2], bar_o;      // tensor cores -> softmax warps (tcgen05.commit)
   uint64_t bar_a[2], bar_e[2];   // softmax warps -> MMA warp, one arrival per softmax thread
-  uint64_t qfull, kfull[3], vfull[2];  // copies landed (transaction bytes)
-  uint64_t kempty[3], vempty[2];       // tensor cores done with a K / V buffer (tcgen05.commit)
+  uint64_t qfull, kfull[2], vfull[2];  // copies landed (transaction bytes)
+  uint64_t kempty[2], vempty[2];       // tensor cores done with a K / V buffer (tcgen05.commit)
   uint32_t tmem;
   int32_t pmax;
   int32_t failed;                // a bounded wait ran out somewhere
@@ -145,9 +147,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t base = (raw + (uint32_t)sizeof(PrefillCtl) + 1023u) & ~1023u;  // 1024-byte aligned tiles
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sQ = base;
-  auto sK = [&](int t) { return base + (uint32_t)(1 + t % 3) * kTileB; };  // K(t): buffer t % 3
-  auto sV = [&](int t) { return base + (uint32_t)(4 + (t & 1)) * kTileB; };  // V(t): buffer t % 2
-  const uint32_t sP = base + 6u * kTileB;
+  auto sK = [&](int t) { return base + (uint32_t)(1 + (t & 1)) * kTileB; };  // K(t): buffer t % 2
+  auto sV = [&](int t) { return base + (uint32_t)(3 + (t & 1)) * kTileB; };  // V(t): buffer t % 2
+  const uint32_t sP = base + 5u * kTileB;     // P_hi, then P_lo one tile further
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool softmax_warp = warp < kMmaWarp;
@@ -174,8 +176,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(&ctl.bar_e[i], kSoftmaxThreads);
       mbar_init(&ctl.vfull[i], 1);
       mbar_init(&ctl.vempty[i], 1);
-    }
-    for (int i = 0; i < 3; ++i) {
       mbar_init(&ctl.kfull[i], 1);
       mbar_init(&ctl.kempty[i], 1);
     }
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       wait(&ctl.bar_a[b], (unsigned)((t >> 1) & 1));
       if (t == 0) wait(&ctl.qfull, 0u);
       for (int u = t == 0 ? 0 : t + 1; u <= t + 1 && u < n_kt; ++u) {
-        wait(&ctl.kfull[u % 3], (unsigned)((u / 3) & 1));
+        wait(&ctl.kfull[u & 1], (unsigned)((u >> 1) & 1));
         tc_fence_after();
         if (lane == 0 && !failed) {
 #pragma unroll
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mma_bf16(tS(u & 1), desc_k(sQ + off), desc_k(sK(u) + off), kIdescS, s > 0 ? 1u : 0u);
           }
           mma_commit(&ctl.bar_s[u & 1]);
-          mma_commit(&ctl.kempty[u % 3]);
+          mma_commit(&ctl.kempty[u & 1]);
         }
         __syncwarp();
       }
@@ -245,8 +245,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
         for (int s = 0; s < kPT / 16; ++s) {
           const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
-          mma_bf16(tO, desc_k(sP + off), desc_mn(sV(t) + (uint32_t)s * 2048u), kIdescPV,
-                   (t > 0 || s > 0) ? 1u : 0u);
+          const uint64_t vd = desc_mn(sV(t) + (uint32_t)s * 2048u);
+          mma_bf16(tO, desc_k(sP + off), vd, kIdescPV, (t > 0 || s > 0) ? 1u : 0u);       // P_hi V
+          mma_bf16(tO, desc_k(sP + (uint32_t)kTileB + off), vd, kIdescPV, 1u);             // P_lo V
         }
         mma_commit(&ctl.bar_o);
         mma_commit(&ctl.vempty[b]);
@@ -254,13 +255,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       __syncwarp();
     }
   } else if (warp == kLoadWarp) {
-    // ---- load warp: lane 0 copies Q once, then K(t) into buffer t % 3 and V(t) into
+    // ---- load warp: lane 0 copies Q once, then K(t) into buffer t % 2 and V(t) into
     //      buffer t % 2 as soon as the tensor cores are done with the tile they held ----
     if (lane == 0 && n_kt > 0) {
       tma_tile(sQ, &tm_q, i0, h, &ctl.qfull);
       for (int t = 0; t < n_kt; ++t) {
-        if (t >= 3) wait(&ctl.kempty[t % 3], (unsigned)(((t - 3) / 3) & 1));
-        if (!failed) tma_tile(sK(t), &tm_k, t * kPT, h, &ctl.kfull[t % 3]);
+        if (t >= 2) wait(&ctl.kempty[t & 1], (unsigned)(((t - 2) >> 1) & 1));
+        if (!failed) tma_tile(sK(t), &tm_k, t * kPT, h, &ctl.kfull[t & 1]);
         if (t >= 2) wait(&ctl.vempty[t & 1], (unsigned)(((t - 2) >> 1) & 1));
         if (!failed) tma_tile(sV(t), &tm_v, t * kPT, h, &ctl.vfull[t & 1]);
       }
@@ -270,7 +271,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // ---- softmax warps ----
     const uint32_t lane_off = (uint32_t)(32 * grp) << 16;  // this warp's TMEM lanes
     const float kScale = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
-    uint8_t* p_row = gbase + 6 * kTileB + hf * 16384 + row * 128;   // this thread's half-row of P
+    uint8_t* p_row = gbase + 5 * kTileB + hf * 16384 + row * 128;   // this thread's half-row of P_hi
+    uint8_t* p_row_lo = p_row + kTileB;                             // ... and of P_lo
     float m_run = -INFINITY, l_half = 0.f;
     for (int t = 0; t < n_kt; ++t) {
       const int b = t & 1, j0 = t * kPT;
@@ -312,14 +314,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         alpha = ex2(m_run - m_tile);
         m_run = m_tile;
       }
-      // weights (fp32 row sum in four partial sums; P rounded to BF16 for the tensor cores)
+      // weights (fp32 row sum in four partial sums; P split into BF16 P_hi + P_lo for the
+      // tensor cores: p - P_hi is exact in fp32, then rounded to BF16)
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pw[32];
+      uint32_t pw[32], pl[32];
+      auto split2 = [&](int e, float p0, float p1) {
+        pw[e] = pack_bf16(p0, p1);
+        pl[e] = pack_bf16(p0 - __uint_as_float(pw[e] << 16), p1 - __uint_as_float(pw[e] & 0xffff0000u));
+      };
       if (full) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const float p0 = ex2(fmaf(sv[2 * e], kScale, -m_run)), p1 = ex2(fmaf(sv[2 * e + 1], kScale, -m_run));
-          pw[e] = pack_bf16(p0, p1);
+          split2(e, p0, p1);
           ls4[e & 3] += p0 + p1;
         }
       } else {
@@ -328,7 +335,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const int i = 2 * e;
           const float p0 = (c_own + i <= qp) ? ex2(fmaf(sv[i], kScale, -m_run)) : 0.f;
           const float p1 = (c_own + i + 1 <= qp) ? ex2(fmaf(sv[i + 1], kScale, -m_run)) : 0.f;
-          pw[e] = pack_bf16(p0, p1);
+          split2(e, p0, p1);
           ls4[e & 3] += p0 + p1;
         }
       }
@@ -350,16 +357,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
 #pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8)  // 16-byte chunk 8 hf + q8 of the row, swizzled
+      for (int q8 = 0; q8 < 8; ++q8) {  // 16-byte chunk 8 hf + q8 of the row, swizzled
         *reinterpret_cast<uint4*>(p_row + ((q8 ^ (row & 7)) << 4)) =
             make_uint4(pw[4 * q8], pw[4 * q8 + 1], pw[4 * q8 + 2], pw[4 * q8 + 3]);
+        *reinterpret_cast<uint4*>(p_row_lo + ((q8 ^ (row & 7)) << 4)) =
+            make_uint4(pl[4 * q8], pl[4 * q8 + 1], pl[4 * q8 + 2], pl[4 * q8 + 3]);
+      }
       // (E) P(t) and the rescaled O are in place: the MMA warp may issue O += P(t) V(t)
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&ctl.bar_e[b]);
     }
     // the last PV, then o = O / l for this thread's half-row; the halves' row sums meet in
-    // the idle P buffer
+    // the idle P_lo buffer
     wait(&ctl.bar_o, (unsigned)((n_kt - 1) & 1));
     tc_fence_after();
     float* lx = reinterpret_cast<float*>(gbase + 6 * kTileB);

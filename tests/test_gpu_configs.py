@@ -23,7 +23,7 @@ import torch
 import bench
 import synth
 from flhelpers import (TOL, Pair, check_topk_valid, compare_encoding, f32, note_elementwise, rel_err,
-                       selection)
+                       selection, u_err)
 from oracle import flashloop_oracle as fo
 from quantized_kv_attention_int4_b200 import abi
 from quantized_kv_attention_int4_b200.cache import FlashLoopCache, round_up
@@ -92,12 +92,13 @@ def test_full_cache_48_layers_sampled_layers_across_flushes():
             check_topk_valid(S3[l][heads], lay.p_tilde, k_sel)
             ref = lay.sparse_loop(3, f32(q[3][l][heads]), S3[l][heads])
             errs[(l, 3)] = rel_err(O123[2][l][heads], ref["o"])
+            o3_ref = ref["o"]
             S4, m4, u4 = selection(cache, l, k_sel)
             check_topk_valid(S4[heads], lay.p_tilde, k_sel)
             ref = lay.sparse_loop(4, f32(q[4][l][heads]), S4[heads])
             errs[(l, 4)] = rel_err(O4[l][heads], ref["o"])
             errs[(l, 4, "m")] = float(np.max(np.abs(m4[heads] - ref["m"]) / ref["m"]))
-            errs[(l, 4, "u")] = rel_err(u4[heads], ref["u"])
+            errs[(l, 4, "u")] = u_err(u4[heads], ref["u"], O123[2][l][heads], o3_ref)
             note_elementwise("cfg3 o", O4[l][heads], ref["o"])
             note_elementwise("cfg3 u", u4[heads], ref["u"])
             _assert_errs(errs)
@@ -122,6 +123,10 @@ def test_layer_32k_prefill_and_256_decode_steps():
         else:
             pair.run_loops(q, tok, fused=True, oracle=False)
     assert pair.cache.n_q == 32704 + 5 * 64 and pair.cache.n_tail == 0
+    # the oracle moves a full tail into its stores at the next append; the GPU's readers
+    # did it inside step 255, so bring the oracle level before comparing the bytes
+    assert pair.oracle.n_tail == 64
+    pair.oracle.flush_tail()
     compare_encoding(pair)
 
 

@@ -3,15 +3,18 @@ oracle.
 
 FlashLoop project page, "The Method", Step 01 (only the active tokens are recomputed)
 and the paragraph after Step 03 (selected tokens gathered into compact buffers so the
-work stays a regular GEMM).  Tolerance, from the arithmetic: the kernel rounds each
-probability to BF16 (relative error <= 2^-9) before the value product and normalises by
-the fp32 sum of the unrounded ones, so |o - o_ref| <= 2^-9 * sum_j p_j |v_j| / sum_j p_j
-<= 2^-9 max|v| per head, plus fp32 accumulation; the test allows 2^-8 max|v|.
+work stays a regular GEMM).  Tolerance: the benchmark spec's bound, 2e-3 of the reference's
+infinity norm -- held here per query row (max over rows of ||o_i - o_ref_i||_inf /
+||o_ref_i||_inf), which is stricter than per head.  The kernel's own error is far below
+it: the logits are exact BF16 products summed in fp32, and the probabilities reach the
+value product as P_hi + P_lo (two BF16 tiles, about 16 significant bits).  The measured
+errors are reported at the end of the run.
 """
 import numpy as np
 import pytest
 import torch
 
+from flhelpers import ELEMENTWISE, note_elementwise
 from oracle import flashloop_oracle as fo
 from quantized_kv_attention_int4_b200 import abi
 
@@ -32,11 +35,22 @@ def _run(q, pos, k, v, status=None, fill=0.0):
     return o.cpu().numpy()
 
 
-def _check(q, pos, k, v, o):
+TOL = 2e-3
+
+
+def _row_err(o, ref) -> float:
+    """max over heads and rows of ||o_i - ref_i||_inf / ||ref_i||_inf."""
+    num = np.abs(o - ref).max(axis=2)
+    den = np.maximum(np.abs(ref).max(axis=2), 1e-30)
+    return float((num / den).max())
+
+
+def _check(q, pos, k, v, o, label="prefill"):
     ref = fo.prefill_attention(q.float().numpy(), np.asarray(pos), k.float().numpy(), v.float().numpy())
-    bound = 2.0 ** -8 * np.abs(v.float().numpy()).max(axis=(1, 2))
-    err = np.abs(o - ref).max(axis=(1, 2))
-    assert np.all(err <= bound), (err, bound)
+    err = _row_err(o, ref)
+    ELEMENTWISE[f"{label} o per row"] = max(ELEMENTWISE.get(f"{label} o per row", 0.0), err)
+    note_elementwise(f"{label} o", o.reshape(o.shape[0], -1), ref.reshape(ref.shape[0], -1))
+    assert err <= TOL, err
     return err
 
 
@@ -58,8 +72,7 @@ def test_all_active_equals_causal_attention():
     q, k, v = _inputs(H, N, np.arange(N), 7)
     o = _run(q, np.arange(N), k, v)
     ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double(), is_causal=True)
-    bound = 2.0 ** -8 * v.float().abs().amax(dim=(1, 2)).numpy()
-    assert np.all(np.abs(o - ref.numpy()).max(axis=(1, 2)) <= bound)
+    assert _row_err(o, ref.numpy()) <= TOL
 
 
 @pytest.mark.gpu
@@ -74,4 +87,4 @@ def test_bad_positions_are_recorded_and_left_unwritten():
     assert np.all(o[0, 2] == 7.0)
     good = [0, 1, 3, 4]
     ref = fo.prefill_attention(q.float().numpy()[:, good], pos[good], k.float().numpy(), v.float().numpy())
-    assert np.abs(o[:, good] - ref).max() <= 2.0 ** -8 * np.abs(v.float().numpy()).max()
+    assert _row_err(o[:, good], ref) <= TOL
