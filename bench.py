@@ -362,13 +362,16 @@ def run_gpu(args, rank, world):
 
     e2e = run_e2e(step, cache, wr, layers, inputs[total_steps:], device) if args.e2e_steps else None
     del inputs, step, cache
+    encode = run_encode(synth.WORKLOADS["layer_h16_n32768_decode256"], device, hbm) if args.encode else None
+    deep = run_deep(device, hbm) if args.deep else None
     tokens = run_token_select(wr, device, hbm) if args.token_select else None
     codecs = run_codecs(w, device, hbm, layers=args.codec_layers) if args.codecs else None
     prefill = run_prefill(wr, device) if args.prefill else None
     return dict(metric_us=metric_us, step_ms=step_ms, seg=mean, clocks=clocks, launches=launches / args.steps,
                 sp_bytes=sp_bytes, sp_launch_us=sp_launch_us, sp_gbs=sp_gbs, d_bytes=d_bytes,
                 d_launch_us=d_launch_us, d_gbs=d_gbs, hbm=hbm, peak_kind=peak_kind, N=N, k_sel=k_sel,
-                layers=layers, setup_s=setup_s, e2e=e2e, w=wr, tokens=tokens, prefill=prefill, codecs=codecs)
+                layers=layers, setup_s=setup_s, e2e=e2e, w=wr, tokens=tokens, prefill=prefill, codecs=codecs,
+                encode=encode, deep=deep)
 
 
 def run_codecs(w, device, hbm, layers=4, warmup=3, steps=5):
@@ -472,6 +475,143 @@ def run_token_select(w, device, hbm, reps=5):
             "select_us_a3": t["a3"] - t["change"]}
 
 
+def run_encode(w, device, hbm, reps=5):
+    """The prefill encode of one 16-head layer of the workload's prompt (BASELINE
+    configuration 2's prefill): the base encoder over every quantised token, then the
+    residual encoder of loops 2..R over their active rows, each timed with CUDA events on the
+    launch stream (a repetition re-encodes the same rows; inputs of 0.5 GB, larger than L2)."""
+    from quantized_kv_attention_int4_b200 import abi
+    from quantized_kv_attention_int4_b200.cache import FlashLoopCache, round_up, split_prefill
+
+    n = w.n_ctx
+    sets = synth.active_sets(w, n)
+    d = synth.prefill_layer(w, 0, device=device, sets=sets)
+    n_q, _ = split_prefill(n)
+    cache = FlashLoopCache(1, w.heads, w.loops, round_up(n + 64), device=device)
+    rows = {r: sets[r][sets[r] < n_q].to(device=device, dtype=torch.int32) for r in range(2, w.loops + 1)}
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(w.loops + 1)]
+    times = {r: [] for r in range(1, w.loops + 1)}
+    for rep in range(reps + 1):
+        ev[0].record()
+        abi.fl_encode_base(cache.dims, cache.buf, 0, 0, d["K"][1][:, :n_q], d["V"][1][:, :n_q])
+        ev[1].record()
+        for r in range(2, w.loops + 1):
+            abi.fl_encode_residual(cache.dims, cache.buf, 0, r, 0, n_q, 0, rows[r], d["K"][r][:, :n_q],
+                                   d["V"][r][:, :n_q], compact=False)
+            ev[r].record()
+        torch.cuda.synchronize()
+        if rep:
+            for r in range(1, w.loops + 1):
+                times[r].append(ev[r - 1].elapsed_time(ev[r]) * 1e3)
+    st, info = cache.status()
+    if st != 0:
+        raise RuntimeError(f"device error in the encode measurement: {info}")
+    out = {}
+    for r in range(1, w.loops + 1):
+        us = float(np.mean(times[r]))
+        if r == 1:
+            nb, name = bytemodel.encode_base_bytes(w.heads, n_q), "encode_base_kernel"
+        else:
+            nb, name = bytemodel.encode_residual_bytes(w.heads, int(rows[r].numel()), r, n_q), "encode_residual_kernel"
+        gbs = nb / (us * 1e-6) / 1e9
+        out[f"loop{r}"] = {"kernel": name, "us_per_launch": us, "bytes_per_launch": nb, "achieved": gbs,
+                           "frac": gbs / hbm, "rows": n_q if r == 1 else int(rows[r].numel())}
+    tot_b = sum(v["bytes_per_launch"] for v in out.values())
+    tot_us = sum(v["us_per_launch"] for v in out.values())
+    del d, cache
+    torch.cuda.empty_cache()
+    return {"bound": "hbm", "kernel": "encode_base_kernel + encode_residual_kernel (loops 2..R)",
+            "workload": f"one {w.heads}-head layer, {n_q} quantised tokens", "achieved": tot_b / (tot_us * 1e-6) / 1e9,
+            "peak": hbm, "unit": "GB/s", "frac": tot_b / (tot_us * 1e-6) / 1e9 / hbm, "us": tot_us,
+            "traffic": {"encode_base_kernel": _kernel_traffic("encode_base_kernel"),
+                        "encode_residual_kernel": _kernel_traffic("encode_residual_kernel")},
+            "launches": out}
+
+
+def run_deep(device, hbm, warmup=3, steps=10):
+    """BASELINE configuration 4 (one 16-head layer at N = 8192, R = 32 loops, geometric
+    retention, 10 % key retention from loop 3): whole decode steps through the step
+    executor with per-loop CUDA events, the algorithmic bytes of each loop taken from an
+    untimed calibration step's selections; the loops <= 8 run the batched sparse reader,
+    loops 9..32 the direct one.  Plus the dense reader at loop 32 alone (the direct dense
+    form: every column with its residual rows of loops 2..32)."""
+    w = synth.WORKLOADS["deep_r32_h16_n8192"]
+    R, H = w.loops, w.heads
+    cache, wr = build_cache(w, 1, 0, device, new_tokens=warmup + steps + 1)
+    inputs = step_inputs(wr, 1, warmup + steps + 1, device)
+    O = torch.zeros(R + 1, 1, H, 128, dtype=torch.float32, device=device)
+    # calibration step (untimed): loop by loop, the bytes each loop's launch moves
+    q, kn, vn = inputs[0]
+    cache.begin_token()
+    k_sel = wr.k_sel(cache.n_cols)
+    loop_bytes = {}
+    for r in range(1, R + 1):
+        cache.step(wr.dense_loops, k_sel, q, O, kn, vn, loop_first=r, loop_last=r, flush=cache.n_tail == 64)
+        torch.cuda.synchronize()
+        if r <= wr.dense_loops:
+            res_rows = sum(cache.n_rows[0][rp] for rp in range(2, r + 1))
+            loop_bytes[r] = bytemodel.dense_bytes(H, cache.n_q, cache.n_tail, res_rows, r == wr.dense_loops)
+        else:
+            loop_bytes[r] = sparse_bytes_from_state(cache, wr, 1, r, k_sel)
+    ev_names = [f"e{i}" for i in range(2 * R + 1)]
+    seg = {r: [] for r in range(1, R + 1)}
+    sel = {r: [] for r in range(1, R + 1)}
+    step_us = []
+    for s in range(1, warmup + steps + 1):
+        q, kn, vn = inputs[s]
+        cache.begin_token()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in ev_names]
+        cache.step(wr.dense_loops, wr.k_sel(cache.n_cols), q, O, kn, vn, events=evs, flush=cache.n_tail == 64)
+        torch.cuda.synchronize()
+        if s > warmup:
+            step_us.append(evs[0].elapsed_time(evs[2 * R]) * 1e3)
+            for r in range(1, R + 1):
+                seg[r].append(evs[2 * r - 1].elapsed_time(evs[2 * r]) * 1e3)
+                sel[r].append(evs[2 * r - 2].elapsed_time(evs[2 * r - 1]) * 1e3)
+    st, info = cache.status()
+    if st != 0:
+        raise RuntimeError(f"device error in the deep-loop measurement: {info}")
+    us = {r: float(np.mean(seg[r])) for r in range(1, R + 1)}
+    groups = {"dense loops 1-2 (dense_staged_kernel)": range(1, wr.dense_loops + 1),
+              "sparse loops 3-8 (sparse_batch_kernel)": range(wr.dense_loops + 1, 9),
+              "sparse loops 9-32 (sparse_kernel, direct)": range(9, R + 1)}
+    out = {}
+    for name, rr in groups.items():
+        b = sum(loop_bytes[r] for r in rr)
+        t = sum(us[r] for r in rr)
+        out[name] = {"us": t, "bytes": b, "achieved": b / (t * 1e-6) / 1e9, "frac": b / (t * 1e-6) / 1e9 / hbm,
+                     "launches": len(rr)}
+    sel_us = sum(float(np.mean(sel[r])) for r in range(wr.dense_loops + 1, R + 1))
+    # the direct dense reader: full attention at loop 32 over every column (one launch)
+    o = torch.empty(H, 128, dtype=torch.float32, device=device)
+    qd = inputs[0][0][R][0].contiguous()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dts = []
+    for rep in range(6):
+        a.record()
+        cache.dense(0, R, qd, o, keep_scores=False)
+        b.record()
+        torch.cuda.synchronize()
+        if rep:
+            dts.append(a.elapsed_time(b) * 1e3)
+    d_us = float(np.mean(dts))
+    d_bytes = bytemodel.dense_bytes(H, cache.n_q, cache.n_tail, sum(cache.n_rows[0][rp] for rp in range(2, R + 1)),
+                                    False)
+    total_b = sum(loop_bytes.values())
+    step_mean = float(np.mean(step_us))
+    del cache, inputs, O
+    torch.cuda.empty_cache()
+    return {"bound": "hbm", "workload": "deep_r32_h16_n8192 (1 layer, 16 heads, N=8192, R=32)",
+            "us_per_step": step_mean, "bytes_per_step": total_b, "achieved": total_b / (step_mean * 1e-6) / 1e9,
+            "peak": hbm, "unit": "GB/s", "frac": total_b / (step_mean * 1e-6) / 1e9 / hbm,
+            "select_us_per_step": sel_us, "readers": out,
+            "dense_direct_loop32": {"kernel": "dense_direct_kernel", "us_per_launch": d_us, "bytes_per_launch": d_bytes,
+                                    "achieved": d_bytes / (d_us * 1e-6) / 1e9,
+                                    "frac": d_bytes / (d_us * 1e-6) / 1e9 / hbm},
+            "traffic": {"sparse_kernel": _kernel_traffic("sparse_kernel"),
+                        "dense_direct_kernel": _kernel_traffic("dense_direct_kernel")}}
+
+
 def _tensor_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -516,38 +656,39 @@ def run_prefill(w, device, reps=5):
 
 
 def run_e2e(step, cache, w, layers, inputs, device):
-    """The metric end to end through the C ABI: each step runs loops 1-3 untimed, then times
-    the loop-4 inputs copied from pinned host memory, the loop-4 selection and sparse
-    readers, and the loop-4 outputs read back to pinned host memory."""
+    """The metric end to end through the C ABI's host-buffer entry point (fl_decode_step_io):
+    each step runs loops 1-3 untimed, then times one call that copies the loop-4 q / k_new /
+    v_new from pinned host memory (one 2-D copy), runs the loop-4 selection and sparse
+    readers, and copies the loop-4 outputs back to pinned host memory."""
+    R, H = w.loops, w.heads
+    qkv = torch.empty(3, R + 1, layers, H, 128, dtype=torch.bfloat16, device=device)
+    hout = torch.empty(1, layers, H, 128, dtype=torch.float32).pin_memory()
     res, parts = [], []
-    H = w.heads
     for q, kn, vn in inputs:
-        hq = q[4].cpu().pin_memory()
-        hk = kn[4].cpu().pin_memory()
-        hv = vn[4].cpu().pin_memory()
-        hout = torch.empty(layers, H, 128, dtype=torch.float32).pin_memory()
-        q[4].zero_()
-        kn[4].zero_()
-        vn[4].zero_()
-        step.run(q, kn, vn, loop_first=1, loop_last=3)
+        hin = torch.stack([q[4], kn[4], vn[4]])[:, None].cpu().pin_memory()   # [3][1][L][H][128]
+        qkv[0].copy_(q)
+        qkv[1].copy_(kn)
+        qkv[2].copy_(vn)
+        qkv[:, 4].zero_()                        # loop 4's inputs arrive from the host
+        step.run(qkv[0], qkv[1], qkv[2], loop_first=1, loop_last=3)
         torch.cuda.synchronize()
-        a, a1, a2, b = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * R + 1)]
+        c = step.c
         a.record()
-        q[4].copy_(hq, non_blocking=True)
-        kn[4].copy_(hk, non_blocking=True)
-        vn[4].copy_(hv, non_blocking=True)
-        a1.record()
-        step.run(q, kn, vn, loop_first=4, loop_last=4)
-        a2.record()
-        hout.copy_(step.O[4], non_blocking=True)
+        c.step_io(w.dense_loops, w.k_sel(c.n_cols), qkv, hin, step.O, hout, loop_first=4, loop_last=4, events=ev,
+                  flush=c.n_tail == 64)
         b.record()
         b.synchronize()
         res.append(a.elapsed_time(b) * 1e3)
-        parts.append((a.elapsed_time(a1) * 1e3, a1.elapsed_time(a2) * 1e3, a2.elapsed_time(b) * 1e3))
+        parts.append((a.elapsed_time(ev[0]) * 1e3, ev[0].elapsed_time(ev[2 * 4]) * 1e3,
+                      ev[2 * 4].elapsed_time(b) * 1e3))
+        assert torch.equal(hout[0], step.O[4].cpu())
     h2d = 3 * layers * H * 128 * 2
     d2h = layers * H * 128 * 4
     seg = np.mean(np.array(parts), axis=0)
     return {"value": float(np.mean(res)), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": "fl_decode_step_io (one call: host -> device copy, loop 4, device -> host copy)",
             "segments_us": {"h2d": float(seg[0]), "select_and_readers": float(seg[1]), "d2h": float(seg[2])}}
 
 
@@ -675,13 +816,98 @@ def oracle_beside(w: synth.Workload, layers: int, codec_layers: int, budget_s: f
     return out
 
 
+def _oracle_worker(args):
+    """One host core's share of the all-cores baseline (a spawned process, one BLAS thread):
+    set up the oracle's state for one (layer, head) of the workload, then time loop-4 steps
+    for about `budget_s` seconds.  Returns (seconds per step, repetitions)."""
+    name, head, budget_s = args
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(limits=1):
+        o = OracleLoop4(synth.WORKLOADS[name], heads=(head,))
+        times = []
+        t_all = time.perf_counter()
+        while not times or (time.perf_counter() - t_all < budget_s and len(times) < 200):
+            times.append(o.run_once())
+    return float(np.mean(times)), len(times)
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def cpu_baseline(w: synth.Workload, layers: int, budget_s: float):
+    """The oracle's loop-4 step (top-K selection + sparse attention) on the host cores: the
+    single-thread figure, and every core at once (one spawned process per core, each with
+    its own (layer, head) sample and one BLAS thread), scaled to the workload's layers x
+    heads pairs by the pairs a second the cores finish together."""
+    import multiprocessing as mp
+
     per_lh, reps = oracle_loop4_sample(w, budget_s)
-    us = per_lh * layers * w.heads * 1e6
-    return {"value": us, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"oracle (NumPy, fp64) loop-4 top-K selection + sparse attention for 1 of "
-                      f"{layers}x{w.heads} (layer, head) pairs at N={w.n_ctx}, {reps} reps, scaled by "
-                      f"{layers * w.heads}"}
+    single_us = per_lh * layers * w.heads * 1e6
+    cores = host_cores()
+    pairs = layers * w.heads
+    with mp.get_context("spawn").Pool(cores) as pool:
+        res = pool.map(_oracle_worker, [(w.name, i % w.heads, budget_s) for i in range(cores)])
+    per_pair = float(np.mean([t for t, _ in res]))      # seconds per pair on one core, all cores busy
+    all_us = pairs * per_pair / cores * 1e6
+    return {"value": all_us, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"oracle (NumPy, fp64) loop-4 top-K selection + sparse attention at N={w.n_ctx}: "
+                      f"{cores} processes at once, one (layer, head) pair each ({sum(n for _, n in res)} steps), "
+                      f"scaled to {layers}x{w.heads} pairs shared by {cores} cores",
+            "single_thread": {"value": single_us, "unit": UNIT, "cores": 1,
+                              "sample": f"1 of {pairs} (layer, head) pairs, {reps} reps, scaled by {pairs}"}}
+
+
+_REF_STATE = {}
+
+
+def _ref_init(name, head):
+    from threadpoolctl import threadpool_limits
+
+    threadpool_limits(limits=1)
+    _REF_STATE["o"] = OracleLoop4(synth.WORKLOADS[name], heads=(head,))
+
+
+def _ref_step(_):
+    return _REF_STATE["o"].run_once()
+
+
+def reference_arm(w: synth.Workload, layers: int, args, config) -> dict:
+    """The oracle as the reference arm, on every host core: one spawned process per core,
+    each holding one (layer, head) pair's state; a step is one loop-4 step (top-K selection
+    + sparse attention) on every process at once, scaled to the workload's layers x heads
+    pairs shared by the cores."""
+    import multiprocessing as mp
+
+    cores = host_cores()
+    pairs = layers * w.heads
+    ctx = mp.get_context("spawn")
+    per_step = []
+    # each process sets up its own pair: the initializer draws a distinct head per process
+    with ctx.Pool(cores, initializer=_ref_init_next, initargs=(w.name, w.heads, ctx.Value("i", 0))) as pool:
+        for _ in range(args.warmup + args.steps):
+            t = pool.map(_ref_step, range(cores), chunksize=1)
+            per_step.append(pairs * float(np.mean(t)) / cores * 1e6)
+    v = float(np.mean(per_step[args.warmup:]))
+    return {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"oracle loop-4 selection + sparse attention, {cores} processes at once with "
+                                       f"one (layer, head) pair each per step, scaled to {pairs} pairs shared by "
+                                       f"{cores} cores"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def _ref_init_next(name, n_heads, counter):
+    with counter.get_lock():
+        i = counter.value
+        counter.value += 1
+    _ref_init(name, i % n_heads)
 
 
 # ----------------------------------------------------------------------------
@@ -703,6 +929,10 @@ def main():
     ap.add_argument("--no-codecs", dest="codecs", action="store_false",
                     help="skip the codec variant (full-state INT4, INT2 residual) measurement")
     ap.add_argument("--codec-layers", type=int, default=4, help="layers of each codec variant's cache")
+    ap.add_argument("--no-encode", dest="encode", action="store_false",
+                    help="skip the prefill encode measurement (one 32K layer)")
+    ap.add_argument("--no-deep", dest="deep", action="store_false",
+                    help="skip the 32-loop workload measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -720,16 +950,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        ora = OracleLoop4(w)
-        per_step = [ora.run_once() * layers * w.heads * 1e6 for _ in range(args.warmup + args.steps)]
-        v = float(np.mean(per_step[args.warmup:]))
-        line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3, "higher_is_better": False,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
-                "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                 "sample": "oracle loop-4 selection + sparse attention, 1 (layer, head) per step, "
-                                           f"scaled by {layers * w.heads}"},
-                "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        line = reference_arm(w, layers, args, config)
         print(json.dumps(line), flush=True)
         return
 
@@ -770,6 +991,8 @@ def main():
         "roofline_dense": {"bound": "hbm", "kernel": "fl_decode_attn_dense (loops 1-2)", "achieved": r["d_gbs"],
                            "peak": hbm, "unit": "GB/s", "frac": r["d_gbs"] / hbm, "traffic": _kernel_traffic("dense_staged_kernel"),
                            "bytes_per_launch": r["d_bytes"], "us_per_launch": r["d_launch_us"]},
+        "roofline_encode": r["encode"],
+        "roofline_cfg4": r["deep"],
         "roofline_token_select": r["tokens"],
         "roofline_prefill": r["prefill"],
         "codec_variants": r["codecs"],

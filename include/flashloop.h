@@ -124,8 +124,9 @@ extern "C" {
 #define FL_GROUP 64
 #define FL_TAIL 64
 #define FL_MAX_LOOPS 32
-/* The selector holds every column's score of one (layer, head) in shared memory. */
-#define FL_MAX_SELECT_COLS 49152
+/* The selector holds every column's key of one (layer, head) in the shared memory of one
+ * thread-block cluster of up to 8 CTAs. */
+#define FL_MAX_SELECT_COLS 385024
 
 typedef enum fl_status {
   FL_OK = 0,
@@ -357,6 +358,21 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
                                int32_t loop_last, const uint16_t* q, const uint16_t* k_new,
                                const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,
                                void* const* events, const fl_flush* flush, void* stream);
+
+/* fl_decode_step_flush fed from and returning to HOST memory in one call, for callers whose
+ * step inputs arrive on the host: copies q, k_new, v_new of loops loop_first..loop_last from
+ * host_qkv (BF16 [3][loop_last - loop_first + 1][L][H][128]: q, then k_new, then v_new) into
+ * the device array qkv (BF16 [3][R+1][L][H][128], the same three arrays fl_decode_step takes
+ * as q, k_new, v_new) with one 2-D copy, runs those loops, and copies o of those loops
+ * (fp32 [loop_last - loop_first + 1][L][H][128]) from the device array o ([R+1][L][H][128])
+ * to host_o -- all enqueued on `stream`, nothing waited for.  Host buffers should be pinned
+ * (page-locked) for the copies to be asynchronous; read host_o after synchronising the
+ * stream.  flush as in fl_decode_step_flush (NULL: none).  Arguments are validated before
+ * anything is enqueued. */
+fl_status fl_decode_step_io(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
+                            int32_t k_sel, int32_t loop_first, int32_t loop_last, uint16_t* qkv, const uint16_t* host_qkv,
+                            float* o, float* host_o, void* ws, size_t ws_bytes, void* const* events,
+                            const fl_flush* flush, void* stream);
 
 /* [Project] Step 01; [Guide] section 3 (cross-loop token-sparse updates: after the dense
  * early loops each loop ranks the tokens updated in the previous loop by normalized

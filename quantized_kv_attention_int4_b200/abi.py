@@ -23,7 +23,7 @@ MAX_LOOPS = 32
 HEAD_DIM = 128
 GROUP = 64
 TAIL = 64
-MAX_SELECT_COLS = 49152
+MAX_SELECT_COLS = 385024
 N_ARRAYS = 14
 ARRAY_NAMES = ("brec", "rrec", "mask", "first", "depth", "tail_k", "tail_v", "score", "tag", "offset", "sel",
                "mass", "unsel", "plan")
@@ -39,7 +39,7 @@ EXPORTED = ("fl_version", "fl_status_string", "fl_cache_layout", "fl_cache_init"
             "fl_workspace_init", "fl_write_tail", "fl_encode_base", "fl_encode_residual",
             "fl_decode_attn_dense", "fl_select_topk", "fl_decode_attn_sparse", "fl_decode_step",
             "fl_read_status", "fl_decode_attn_sparse_noalloc", "fl_decode_step_flush", "fl_select_active",
-            "fl_prefill_attn_sparse", "fl_sparse_splits")
+            "fl_prefill_attn_sparse", "fl_sparse_splits", "fl_decode_step_io")
 
 
 class fl_dims(ctypes.Structure):
@@ -97,6 +97,8 @@ _c_step_flush = _sig("fl_decode_step_flush", _I, _DP, _P, _I, _I, _I, _I, _I, _I
 _c_select_active = _sig("fl_select_active", _I, _P, _P, _I, _I, _L, _P, _I, _I, _P, _P, _P, _P)
 _c_prefill = _sig("fl_prefill_attn_sparse", _I, _P, _P, _I, _P, _P, _I, _I, _L, _L, _P, _L, _P, _P)
 _c_read_status = _sig("fl_read_status", _I, _DP, _P, ctypes.POINTER(ctypes.c_int32), _I, _P)
+_c_step_io = _sig("fl_decode_step_io", _I, _DP, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                   ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(fl_flush), _P)
 _c_sparse_splits = _sig("fl_sparse_splits", _I, _DP, _I, _I, _I, ctypes.POINTER(ctypes.c_int32),
                         ctypes.POINTER(ctypes.c_int32))
 
@@ -142,6 +144,17 @@ def _ptr(t, dtype=None, name="tensor"):
         raise ValueError(f"{name} must be a CUDA tensor")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t, dtype, name):
+    """A host tensor's data pointer (pinned memory keeps the library's copies asynchronous)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if t.dtype != dtype or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous {dtype} host tensor")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -295,6 +308,27 @@ def fl_decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loo
     else:
         _check("fl_decode_step_flush", _c_step_flush(*args, ctypes.byref(flush), _stream(stream)))
 
+
+
+def fl_decode_step_io(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, qkv, host_qkv, o,
+                      host_o, ws, events=None, stream=None, flush=None):
+    """fl_decode_step_flush fed from and returning to host memory in one call.
+
+    qkv: device BF16 [3][R+1][L][H][128] (q, k_new, v_new); host_qkv: host BF16
+    [3][n][L][H][128] with n = loop_last - loop_first + 1; o: device fp32 [R+1][L][H][128];
+    host_o: host fp32 [n][L][H][128] (valid after the stream is synchronised)."""
+    ev = None
+    if events is not None:
+        for e in events:
+            e.record()
+        ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    if not qkv.is_contiguous() or not o.is_contiguous():
+        raise ValueError("qkv and o must be contiguous")
+    _check("fl_decode_step_io", _c_step_io(
+        ctypes.byref(dims), _ptr(cache, torch.uint8, "cache"), n_q, n_tail, dense_loops, k_sel, loop_first, loop_last,
+        _ptr(qkv, torch.bfloat16, "qkv"), _host_ptr(host_qkv, torch.bfloat16, "host_qkv"), _ptr(o, torch.float32, "o"),
+        _host_ptr(host_o, torch.float32, "host_o"), _ptr(ws, torch.uint8, "ws"), ws.numel(), ev,
+        ctypes.byref(flush) if flush is not None else None, _stream(stream)))
 
 def fl_select_active(h_prev, h_cur, rows, k, rows_out, keys, status=None, stream=None):
     """A_r from A_{r-1}: the k tokens of ``rows`` (int32, ascending) whose hidden state

@@ -87,3 +87,18 @@ def sparse_bytes(heads: int, cols_quant: int, res_rows: int, key_groups: int, co
     return (cols_quant * row + res_rows * (2 * res_code_row + VSZ_ROW) + value_rows * (CODE_ROW + VSZ_ROW)
             + key_groups * KSZ_GROUP + cols_tail * TAIL_ROW
             + cols * (4 + 5) + heads * (HEAD_DIM * 2 + 4 + HEAD_DIM * 4 * 2))
+
+
+def encode_base_bytes(heads: int, n_rows: int) -> int:
+    """One base-encoder launch: BF16 keys and values in (512 B per row), the row's 144 B of
+    codes and scales out."""
+    return heads * n_rows * (TAIL_ROW + ROW_BYTES)
+
+
+def encode_residual_bytes(heads: int, n_rows: int, loop: int, n_tokens: int, row_bytes: int = ROW_BYTES) -> int:
+    """One residual-encoder launch of loop ``loop`` over ``n_rows`` active rows of a span of
+    ``n_tokens``: each row's BF16 key and value in, the loop r-1 reconstruction it is taken
+    against (the row's base row and its residual rows of loops 2..r-1, 144 B each), its new
+    row out; plus the span's block metadata (mask 8 B, first slot 4 B per 64 tokens) and
+    depth (1 B per row)."""
+    return heads * n_rows * (TAIL_ROW + ROW_BYTES * (loop - 1) + row_bytes) + (n_tokens // GROUP) * 12 + n_rows

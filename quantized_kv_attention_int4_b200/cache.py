@@ -205,5 +205,23 @@ class FlashLoopCache:
             self._plan = None
             self._flushed(plan)
 
+    def step_io(self, dense_loops, k_sel, qkv, host_qkv, o, host_o, loop_first=1, loop_last=None, events=None,
+                stream=None, flush=False):
+        """``step`` fed from and returning to host memory (fl_decode_step_io): the loops'
+        q / k_new / v_new come from ``host_qkv`` (BF16 [3][n][L][H][128], pinned) into the
+        device array ``qkv`` ([3][R+1][L][H][128]) and their outputs go from ``o`` to
+        ``host_o`` ([n][L][H][128]), n = loop_last - loop_first + 1, in one call."""
+        loop_last = loop_last or self.R
+        plan = None
+        if flush:
+            if self._plan is None or self._plan[0] != self.n_q:
+                self._plan = (self.n_q, self.flush_plan())
+            plan = self._plan[1]
+        abi.fl_decode_step_io(self.dims, self.buf, self.n_q, self.n_tail, dense_loops, k_sel, loop_first, loop_last,
+                              qkv, host_qkv, o, host_o, self.ws, events, stream, flush=plan)
+        if plan is not None and loop_last == self.R:
+            self._plan = None
+            self._flushed(plan)
+
     def status(self, clear=True):
         return abi.fl_read_status(self.dims, self.buf, clear)

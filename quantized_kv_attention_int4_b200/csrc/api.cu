@@ -111,7 +111,7 @@ uint64_t ws_part_bytes(const fl_dims* d) {
 // The split count a sparse launch will use fits the workspace's partials (it always does
 // for k_sel <= max_select; checked before any launch all the same).
 fl_status check_sparse_splits(const fl_dims* d, int loop, int k_sel) {
-  const int n = sparse_launch_splits(d->heads, d->loops, loop, k_sel, device_sms());
+  const int n = sparse_launch_splits(d->heads, d->loops, d->codec, loop, k_sel, device_sms());
   return n <= workspace_splits(d->loops, d->max_select) ? FL_OK : FL_ERR_UNSUPPORTED;
 }
 
@@ -414,7 +414,8 @@ fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_
   if (scratch_bytes((k_sel + cols - 1) / cols) > FL_NOALLOC_SCRATCH_BYTES) return FL_ERR_UNSUPPORTED;
   const int sms = device_sms();
   if (sms <= 0) return FL_ERR_CUDA;
-  if (scratch_bytes(sparse_launch_splits(dims->heads, dims->loops, loop, k_sel, sms)) > FL_NOALLOC_SCRATCH_BYTES)
+  if (scratch_bytes(sparse_launch_splits(dims->heads, dims->loops, dims->codec, loop, k_sel, sms)) >
+      FL_NOALLOC_SCRATCH_BYTES)
     return FL_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FL_ERR_CUDA;
@@ -453,7 +454,7 @@ fl_status fl_sparse_splits(const fl_dims* dims, int32_t loop, int32_t k_sel, int
   if (st != FL_OK) return st;
   if (!splits || loop < 2 || loop > dims->loops || k_sel < 1 || k_sel > dims->max_select || sm_count < 1)
     return FL_ERR_INVALID;
-  *splits = sparse_launch_splits(dims->heads, dims->loops, loop, k_sel, sm_count);
+  *splits = sparse_launch_splits(dims->heads, dims->loops, dims->codec, loop, k_sel, sm_count);
   if (capacity) *capacity = workspace_splits(dims->loops, dims->max_select);
   return FL_OK;
 }
@@ -564,6 +565,38 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
     }
     if (!rec(2 * r)) return FL_ERR_CUDA;
   }
+  return FL_OK;
+}
+
+fl_status fl_decode_step_io(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
+                            int32_t k_sel, int32_t loop_first, int32_t loop_last, uint16_t* qkv, const uint16_t* host_qkv,
+                            float* o, float* host_o, void* ws, size_t ws_bytes, void* const* events,
+                            const fl_flush* flush, void* stream) {
+  fl_status st = check_dims(dims);
+  if (st != FL_OK) return st;
+  if (!qkv || !host_qkv || !o || !host_o) return FL_ERR_INVALID;
+  const int R = dims->loops;
+  if (loop_first < 1 || loop_last > R || loop_first > loop_last) return FL_ERR_INVALID;
+  const size_t slice = (size_t)dims->layers * dims->heads * FL_HEAD_DIM;  // one (loop) slice of L x H x 128
+  const size_t nl = (size_t)(loop_last - loop_first + 1);
+  uint16_t* q = qkv;
+  uint16_t* kn = qkv + (size_t)(R + 1) * slice;
+  uint16_t* vn = qkv + (size_t)2 * (R + 1) * slice;
+  cudaStream_t s = (cudaStream_t)stream;
+  // validate the whole step before anything is enqueued: a step with the same arguments and
+  // no copies must be acceptable (fl_decode_step_flush validates before launching)
+  st = check_reader(dims, cache, 0, 1, n_q, n_tail, q, kn, vn, o, ws, ws_bytes);
+  if (st != FL_OK) return st;
+  // q, k_new, v_new of loops loop_first..loop_last: three equally spaced device rows
+  if (cudaMemcpy2DAsync(q + (size_t)loop_first * slice, (size_t)(R + 1) * slice * 2, host_qkv, nl * slice * 2,
+                        nl * slice * 2, 3, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return FL_ERR_CUDA;
+  st = fl_decode_step_flush(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, kn, vn, o, ws,
+                            ws_bytes, events, flush, stream);
+  if (st != FL_OK) return st;
+  if (cudaMemcpyAsync(host_o, o + (size_t)loop_first * slice, nl * slice * sizeof(float), cudaMemcpyDeviceToHost,
+                      s) != cudaSuccess)
+    return FL_ERR_CUDA;
   return FL_OK;
 }
 

@@ -111,8 +111,9 @@ cudaError_t once_per_device(std::atomic<bool>* done, std::mutex& mu, F&& fn) {
 // Plan entries (selected columns) one sparse-reader CTA holds in shared memory.
 int sparse_cta_columns(int loops);
 // Split-K partitions per head that launch_sparse uses for a loop-r reader over k_sel
-// columns on a device with `sms` SMs: never fewer than ceil(k_sel / sparse_cta_columns).
-int sparse_launch_splits(int heads, int loops, int r, int k_sel, int sms);
+// columns of a cache with codec `codec` on a device with `sms` SMs: never fewer than
+// ceil(k_sel / sparse_cta_columns).
+int sparse_launch_splits(int heads, int loops, int codec, int r, int k_sel, int sms);
 // Split-K partials per head that a workspace for these dims holds: enough for every
 // dense launch and for every sparse launch with k_sel <= max_select.
 int workspace_splits(int loops, int max_select);

@@ -7,32 +7,39 @@
 // flozi guide "FlashLoop: store changes between repeated passes", section 3: each
 // sparse loop ranks key columns by the previous loop's attention statistics.
 //
-// One CTA (1024 threads) per (layer, head), launched for a range of layers at once.
-//   keys:     log2 p~_j = score_j - offset[tag_j], mapped to an order-preserving u32
-//             and kept in shared memory (N <= FL_MAX_SELECT_COLS);
-//   select:   radix select of the K-th largest key over the bits where the keys
-//             differ (the prefix every key shares is skipped), digits of up to 13
-//             bits, each pass a shared-memory histogram over the keys that still match
-//             the prefix and a block-wide scan from the top bin;
-//   compact:  keys above the threshold plus the lowest-index ties, written in index
-//             order (per-warp ballots and a block prefix), so S is ascending;
-//   m, plan:  m = sum_S p~_j; for every j in S its tag, p~_j, the number of stores it
-//             has in loop r (min(r, depth_j); 0 for a BF16 tail column) and its slot in
-//             each residual store (block first slot + popcount of the block mask), so the
-//             sparse reader can issue all of a column's loads at once.
+// Two forms of the same computation, launched for a range of layers at once:
+//   select_cta_kernel      one CTA (1024 threads) per (layer, head), every key of the head
+//                          in its shared memory (N <= 49152);
+//   select_cluster_kernel  one thread-block cluster of cs CTAs (512 threads; cs = 2, 4 or 8
+//                          from N) per (layer, head), CTA rank c owning the columns
+//                          [c span, (c + 1) span), for N up to FL_MAX_SELECT_COLS.
+// Each:
+//   keys:     log2 p~_j = score_j - offset[tag_j], mapped to an order-preserving u32,
+//             kept in shared memory;
+//   select:   radix select of the K-th largest key over the bits where the head's keys
+//             differ (the prefix every key shares is skipped), each pass a shared-memory
+//             histogram of the keys that still match the prefix (in the cluster form summed
+//             bin by bin over the cluster's CTAs through distributed shared memory, so every
+//             CTA reaches the same digit) and a block-wide scan from the top bin;
+//   compact:  keys above the threshold plus the lowest-index ties, written in index order
+//             (per-warp ballots, a block prefix, and in the cluster form the counts of the
+//             lower-ranked CTAs), so S is ascending;
+//   m, plan:  m = sum_S p~_j; for every j in S its tag, p~_j, the number of stores it has
+//             in loop r (min(r, depth_j); 0 for a BF16 tail column) and its slot in each
+//             residual store (block first slot + popcount of the block mask), so the sparse
+//             reader can issue all of a column's loads at once.
 #include "kernels.h"
 
 namespace fl {
 namespace {
 
-constexpr int kThreads = 1024;
+constexpr int kThreads = 512;
 constexpr int kWarpsSel = kThreads / 32;
-constexpr int kDynMax = 194 * 1024;  // dynamic shared memory: keys [, selected columns]
-
-// Selected columns are kept in shared memory after the keys when both fit.
-__host__ __device__ inline bool sel_fits(int N, int K) {
-  return ((size_t)((N + 3) & ~3) + (size_t)K) * sizeof(uint32_t) <= (size_t)kDynMax;
-}
+constexpr int kDigit = 12;                 // bits per radix digit at most
+constexpr int kBins = 1 << kDigit;
+constexpr int kKeysCta = 18432;            // keys per CTA when the cluster has <= 4 CTAs (two CTAs per SM)
+constexpr int kKeysCtaMax = 48128;         // ... and with 8 (one CTA per SM then)
+constexpr int kClusterMax = 8;
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t b = __float_as_uint(f);
@@ -42,7 +49,38 @@ __device__ __forceinline__ float key_value(uint32_t o) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
-// Inclusive block scan of one value per thread (1024 threads).
+// ---- thread-block cluster helpers ----
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// every thread of every CTA of the cluster arrives; shared-memory writes before it are
+// visible to the cluster's CTAs after it
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned; barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// a 32-bit word of CTA `rank`'s shared memory at the address of `p` in this CTA's
+__device__ __forceinline__ uint32_t ld_peer(const void* p, uint32_t rank) {
+  uint32_t a = smem_addr(p), ra, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+struct SelShared {
+  uint32_t hist[2][kBins];   // one per radix pass, alternating: a CTA clears the next one while
+                             // the cluster may still read the current one
+  uint32_t wtot[32];
+  uint32_t wgt[32];
+  uint32_t xchg[8];      // this CTA's contributions the cluster reads: and, or, gt, eq, mass bits
+  uint32_t digit, krem;
+  float offs[kOffStride];
+  float red[kWarpsSel];
+};
+
+// Inclusive block scan of one value per thread (kNT threads).
+template <int kNT>
 __device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* wtot, int lane, int warp) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -53,21 +91,32 @@ __device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* wtot, int l
   if (lane == 31) wtot[warp] = v;
   __syncthreads();
   if (warp == 0) {
-    uint32_t t = wtot[lane];
+    uint32_t t = lane < kNT / 32 ? wtot[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t n = __shfl_up_sync(kFull, t, o);
       if (lane >= o) t += n;
     }
-    wtot[lane] = t;
+    if (lane < kNT / 32) wtot[lane] = t;
   }
   __syncthreads();
   return v + (warp > 0 ? wtot[warp - 1] : 0u);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
+// ---- one CTA per (layer, head) ----
+constexpr int kThreads1 = 1024;
+constexpr int kWarps1 = kThreads1 / 32;
+constexpr int kDynMax1 = 194 * 1024;  // dynamic shared memory: keys [, selected columns]
+constexpr int kCols1 = 49152;         // the keys of one head that fit it
+
+// Selected columns are kept in shared memory after the keys when both fit.
+__host__ __device__ inline bool sel_fits1(int N, int K) {
+  return ((size_t)((N + 3) & ~3) + (size_t)K) * sizeof(uint32_t) <= (size_t)kDynMax1;
+}
+
+__global__ void __launch_bounds__(kThreads1, 1) select_cta_kernel(SelectArgs a) {
   extern __shared__ uint32_t keys[];  // [N] keys, then [K] selected columns when they fit
-  const bool sel_smem = sel_fits(a.n_q + a.n_tail, a.k_sel);
+  const bool sel_smem = sel_fits1(a.n_q + a.n_tail, a.k_sel);
   int32_t* sel_s = reinterpret_cast<int32_t*>(keys + ((a.n_q + a.n_tail + 3) & ~3));
   __shared__ __align__(16) uint32_t hist[8192];
   __shared__ float offs[kOffStride];
@@ -99,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int N4 = N & ~3;
   uint32_t kand = 0xffffffffu, kor = 0u;  // bits common to every key
 #pragma unroll 4
-  for (int j = 4 * tid; j < N4; j += 4 * kThreads) {
+  for (int j = 4 * tid; j < N4; j += 4 * kThreads1) {
     const float4 sc = *reinterpret_cast<const float4*>(score + j);
     const uint32_t tg = *reinterpret_cast<const uint32_t*>(tag + j);
     const uint32_t k0 = key_of(sc.x, (int)(tg & 0xff), j), k1 = key_of(sc.y, (int)((tg >> 8) & 0xff), j + 1);
@@ -111,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     kand &= k0 & k1 & k2 & k3;
     kor |= k0 | k1 | k2 | k3;
   }
-  for (int j = N4 + tid; j < N; j += kThreads) {
+  for (int j = N4 + tid; j < N; j += kThreads1) {
     const uint32_t k = key_of(score[j], tag[j], j);
     keys[j] = k;
     kand &= k;
@@ -149,20 +198,20 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     nbits = shift;
     const int nbins = 1 << wbits;
     const uint32_t dmask = (uint32_t)nbins - 1u;
-    for (int i = tid; i < nbins; i += kThreads) hist[i] = 0u;
+    for (int i = tid; i < nbins; i += kThreads1) hist[i] = 0u;
     __syncthreads();
-    for (int j = tid; j < N; j += kThreads) {
+    for (int j = tid; j < N; j += kThreads1) {
       const uint32_t u = keys[j];
       if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
     }
     __syncthreads();
     // thread t owns bins [nbins - per*(t+1), nbins - per*t), i.e. descending order
-    const int per = nbins / kThreads > 0 ? nbins / kThreads : 1;
+    const int per = nbins / kThreads1 > 0 ? nbins / kThreads1 : 1;
     const int owners = nbins / per;
     uint32_t local = 0u;
     if (tid < owners)
       for (int i = 0; i < per; ++i) local += hist[nbins - per * tid - 1 - i];
-    const uint32_t incl = block_scan(local, wtot, lane, warp);
+    const uint32_t incl = block_scan<kThreads1>(local, wtot, lane, warp);
     const uint32_t excl = incl - local;
     if (tid < owners && excl < krem && krem <= incl) {
       uint32_t cum = excl;
@@ -185,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const uint32_t thr = prefix;  // the K-th largest key; take krem of the keys equal to it
 
   // ---- compaction in index order ----
-  const int chunk = ((((N + kWarpsSel - 1) / kWarpsSel) + 31) / 32) * 32;
+  const int chunk = ((((N + kWarps1 - 1) / kWarps1) + 31) / 32) * 32;
   const int wbeg = warp * chunk;
   const unsigned lt = (1u << lane) - 1u;
   // one pass counts this warp's keys above the threshold and equal to it; the number it
@@ -240,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int r = a.r;
   __syncthreads();
 #pragma unroll 2
-  for (int k = tid; k < K; k += kThreads) {
+  for (int k = tid; k < K; k += kThreads1) {
     const int j = sel_smem ? sel_s[k] : sel[k];
     int lam = tag[j];
     lam = lam < 1 ? 1 : (lam > R ? R : lam);
@@ -267,21 +316,302 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   }
   if (tid == 0) {
     float m = 0.f;
-    for (int w = 0; w < kWarpsSel; ++w) m += red[w];
+    for (int w = 0; w < kWarps1; ++w) m += red[w];
     arr<float>(c, A_MASS, layer)[h] = m;
+  }
+}
+
+
+// ---- one cluster per (layer, head) ----
+__global__ void __launch_bounds__(kThreads, 2) select_cluster_kernel(SelectArgs a, int cs, int span) {
+  extern __shared__ __align__(16) uint32_t keys[];  // [span]
+  __shared__ SelShared sh;
+
+  const uint32_t crank = cluster_rank();
+  const int h = blockIdx.x / cs, layer = a.layer0 + blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const CacheView& c = a.c;
+  const int cap = c.cap, ncb = cap / kG, R = c.R;
+  const int n_q = a.n_q, N = a.n_q + a.n_tail, K = a.k_sel;
+  const int j0 = (int)crank * span;
+  const int nk = max(0, min(span, N - j0));  // this CTA's columns
+
+  const float* score = arr<float>(c, A_SCORE, layer) + (size_t)h * cap;
+  const uint8_t* tag = arr<uint8_t>(c, A_TAG, layer) + (size_t)h * cap;
+  int32_t* sel = arr<int32_t>(c, A_SEL, layer) + (size_t)h * c.max_select;
+
+  if (tid < kOffStride) sh.offs[tid] = arr<float>(c, A_OFFSET, layer)[(size_t)h * kOffStride + tid];
+  __syncthreads();
+
+  // ---- keys, four columns per thread per step (span and cap are multiples of 4 and 64:
+  //      16-byte score and 4-byte tag loads), all of a thread's loads in flight together ----
+  auto key_of = [&](float sc, int t, int j) {
+    if (t < 1 || t > R) {
+      record_error(c.status, FL_DEV_TAG_RANGE, j);
+      t = t < 1 ? 1 : R;
+    }
+    return order_key(sc - sh.offs[t]);
+  };
+  const int nk4 = nk & ~3;
+  uint32_t kand = 0xffffffffu, kor = 0u;
+#pragma unroll 8
+  for (int i = 4 * tid; i < nk4; i += 4 * kThreads) {
+    const float4 sc = *reinterpret_cast<const float4*>(score + j0 + i);
+    const uint32_t tg = *reinterpret_cast<const uint32_t*>(tag + j0 + i);
+    const uint32_t k0 = key_of(sc.x, (int)(tg & 0xff), j0 + i), k1 = key_of(sc.y, (int)((tg >> 8) & 0xff), j0 + i + 1);
+    const uint32_t k2 = key_of(sc.z, (int)((tg >> 16) & 0xff), j0 + i + 2), k3 = key_of(sc.w, (int)(tg >> 24), j0 + i + 3);
+    *reinterpret_cast<uint4*>(keys + i) = make_uint4(k0, k1, k2, k3);
+    kand &= k0 & k1 & k2 & k3;
+    kor |= k0 | k1 | k2 | k3;
+  }
+  for (int i = nk4 + tid; i < nk; i += kThreads) {
+    const uint32_t k = key_of(score[j0 + i], tag[j0 + i], j0 + i);
+    keys[i] = k;
+    kand &= k;
+    kor |= k;
+  }
+  kand = __reduce_and_sync(kFull, kand);
+  kor = __reduce_or_sync(kFull, kor);
+  if (lane == 0) {
+    sh.wtot[warp] = kand;
+    sh.wgt[warp] = kor;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t A = 0xffffffffu, O = 0u;
+    for (int w = 0; w < kWarpsSel; ++w) {
+      A &= sh.wtot[w];
+      O |= sh.wgt[w];
+    }
+    sh.xchg[0] = A;
+    sh.xchg[1] = O;
+  }
+  cluster_sync();
+  kand = 0xffffffffu;
+  kor = 0u;
+  for (int r = 0; r < cs; ++r) {
+    kand &= ld_peer(&sh.xchg[0], r);
+    kor |= ld_peer(&sh.xchg[1], r);
+  }
+
+  // ---- radix select of the K-th largest key of the head, over the bits where keys differ ----
+  const uint32_t diff = kand ^ kor;
+  int nbits = diff ? 32 - __clz(diff) : 0;  // digits cover bits [0, nbits)
+  uint32_t pmask = nbits >= 32 ? 0u : ~((1u << nbits) - 1u);
+  uint32_t prefix = kand & pmask, krem = (uint32_t)K;
+  for (int pass = 0; nbits > 0; ++pass) {
+    uint32_t* hist = sh.hist[pass & 1];
+    const int npass = (nbits + kDigit - 1) / kDigit;
+    const int wbits = (nbits + npass - 1) / npass;  // balanced digits
+    const int shift = nbits - wbits;
+    nbits = shift;
+    const int nbins = 1 << wbits;
+    const uint32_t dmask = (uint32_t)nbins - 1u;
+    for (int i = tid; i < nbins; i += kThreads) hist[i] = 0u;
+    cluster_sync();  // every CTA has cleared this pass's histogram (and is done reading the
+                     // one this buffer held two passes ago)
+    for (int i = tid; i < nk; i += kThreads) {
+      const uint32_t u = keys[i];
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+    }
+    cluster_sync();  // every CTA's histogram is complete
+    // thread t owns bins [nbins - per (t + 1), nbins - per t) of the cluster's histogram,
+    // i.e. descending order
+    const int per = nbins / kThreads > 0 ? nbins / kThreads : 1;
+    const int owners = nbins / per;
+    constexpr int kPer = kBins / kThreads;  // bins per thread at most
+    uint32_t local = 0u;
+    uint32_t binc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      binc[i] = 0u;
+      if (tid < owners && i < per) {
+        const int bin = nbins - per * tid - 1 - i;
+        for (int r = 0; r < cs; ++r) binc[i] += ld_peer(&hist[bin], r);
+        local += binc[i];
+      }
+    }
+    const uint32_t incl = block_scan<kThreads>(local, sh.wtot, lane, warp);
+    const uint32_t excl = incl - local;
+    if (tid < owners && excl < krem && krem <= incl) {
+      uint32_t cum = excl;
+      bool found = false;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        if (!found && i < per && cum + binc[i] >= krem) {
+          sh.digit = (uint32_t)(nbins - per * tid - 1 - i);
+          sh.krem = krem - cum;
+          found = true;
+        }
+        cum += binc[i];
+      }
+    }
+    __syncthreads();
+    prefix |= sh.digit << shift;
+    pmask |= dmask << shift;
+    krem = sh.krem;
+    __syncthreads();
+  }
+  const uint32_t thr = prefix;  // the K-th largest key; take krem of the keys equal to it (index order)
+
+  // ---- compaction in index order: warp w owns keys [w chunk, (w + 1) chunk) ----
+  const int chunk = ((((nk + kWarpsSel - 1) / kWarpsSel) + 31) / 32) * 32;
+  const int wbeg = warp * chunk;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t gtc = 0u, eqc = 0u;
+  for (int i = 0; i < chunk; i += 32) {
+    const int j = wbeg + i + lane;
+    const uint32_t u = j < nk ? keys[j] : 0u;
+    gtc += __popc(__ballot_sync(kFull, j < nk && u > thr));
+    eqc += __popc(__ballot_sync(kFull, j < nk && u == thr));
+  }
+  if (lane == 0) {
+    sh.wtot[warp] = eqc;
+    sh.wgt[warp] = gtc;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t g = 0u, e = 0u;
+    for (int w = 0; w < kWarpsSel; ++w) {
+      g += sh.wgt[w];
+      e += sh.wtot[w];
+    }
+    sh.xchg[2] = g;
+    sh.xchg[3] = e;
+  }
+  cluster_sync();
+  // ties go to the lowest indices: the lower-ranked CTAs' equal keys come first
+  uint32_t eq_before = 0u, sel_before = 0u;
+  for (uint32_t r = 0; r < crank; ++r) {
+    const uint32_t g = ld_peer(&sh.xchg[2], r), e = ld_peer(&sh.xchg[3], r);
+    const uint32_t take = krem > eq_before ? min(krem - eq_before, e) : 0u;
+    sel_before += g + take;
+    eq_before += e;
+  }
+  uint32_t eq_base = eq_before, pos = sel_before;
+  for (int w = 0; w < warp; ++w) {
+    const uint32_t eb = eq_base;
+    eq_base += sh.wtot[w];
+    const uint32_t take = krem > eb ? min(krem - eb, sh.wtot[w]) : 0u;
+    pos += sh.wgt[w] + take;
+  }
+  uint32_t eqrun = eq_base;
+  float mpart = 0.f;
+  for (int i = 0; i < chunk; i += 32) {
+    const int j = wbeg + i + lane;
+    const uint32_t u = j < nk ? keys[j] : 0u;
+    const unsigned be = __ballot_sync(kFull, j < nk && u == thr);
+    const bool s = (j < nk && u > thr) || (j < nk && u == thr && eqrun + __popc(be & lt) < krem);
+    eqrun += __popc(be);
+    const unsigned bs = __ballot_sync(kFull, s);
+    if (s) {
+      sel[pos + __popc(bs & lt)] = j0 + j;
+      mpart += ex2(key_value(u));
+    }
+    pos += __popc(bs);
+  }
+  mpart = warp_sum(mpart);
+  if (lane == 0) sh.red[warp] = mpart;
+  __syncthreads();  // this CTA's part of S is written (global, visible to the block)
+  if (tid == 0) {
+    float m = 0.f;
+    for (int w = 0; w < kWarpsSel; ++w) m += sh.red[w];
+    sh.xchg[4] = __float_as_uint(m);
+  }
+  cluster_sync();  // every CTA's mass part is in place
+  // this CTA's part of S: [sel0, sel1) -- its keys above the threshold plus its share of
+  // the ties
+  const uint32_t sel0 = sel_before;
+  const uint32_t sel1 = sel0 + sh.xchg[2] + (krem > eq_before ? min(krem - eq_before, sh.xchg[3]) : 0u);
+  if (crank == 0 && tid == 0) {
+    float m = 0.f;
+    for (int r = 0; r < cs; ++r) m += __uint_as_float(ld_peer(&sh.xchg[4], r));
+    arr<float>(c, A_MASS, layer)[h] = m;
+  }
+
+  // ---- gather plan of this CTA's part of S: column, tag, stores, p~, residual slots ----
+  const unsigned long long* mask = arr<unsigned long long>(c, A_MASK, layer);
+  const int32_t* first = arr<int32_t>(c, A_FIRST, layer);
+  const uint8_t* depth = arr<uint8_t>(c, A_DEPTH, layer);
+  const int ps = c.plan_stride;
+  int32_t* plan = arr<int32_t>(c, A_PLAN, layer) + (size_t)h * c.max_select * ps;
+  const int r = a.r;
+#pragma unroll 4
+  for (int k = (int)sel0 + tid; k < (int)sel1; k += kThreads) {
+    const int j = sel[k];
+    int lam = tag[j];
+    lam = lam < 1 ? 1 : (lam > R ? R : lam);
+    int stores = 0;
+    if (j < n_q) {
+      const int dep = depth[j];
+      stores = dep < r ? dep : r;
+    }
+    // the entry's words, stored 16 bytes at a time (ps is a multiple of 4; unused words 0)
+    const int b = j >> 6, jt = j & 63;
+    uint4* e = reinterpret_cast<uint4*>(plan + (size_t)k * ps);
+    const int w2 = __float_as_int(ex2(key_value(keys[j - j0])));
+    auto word = [&](int i) -> int {
+      if (i == 0) return j;
+      if (i == 1) return lam | (stores << 8);
+      if (i == 2) return w2;
+      const int rp = i - 1;
+      if (rp > stores) return 0;
+      const unsigned long long mk = mask[(size_t)rp * ncb + b];
+      return c.slot_base[rp] + first[(size_t)rp * ncb + b] + __popcll(mk & ((1ull << jt) - 1ull));
+    };
+    for (int q4 = 0; q4 < ps; q4 += 4)
+      e[q4 >> 2] = make_uint4((uint32_t)word(q4), (uint32_t)word(q4 + 1), (uint32_t)word(q4 + 2), (uint32_t)word(q4 + 3));
+  }
+  cluster_sync();  // no CTA leaves while another may still read its shared memory
+}
+
+// CTAs per cluster and columns per CTA for N columns; cs = 0 when N is too large.
+void select_shape(int N, int* cs, int* span) {
+  *cs = 0;
+  *span = 0;
+  for (int c = 2; c <= kClusterMax; c *= 2) {
+    const int sp = ((N + c - 1) / c + 63) / 64 * 64;
+    if (sp <= (c < kClusterMax ? kKeysCta : kKeysCtaMax)) {
+      *cs = c;
+      *span = sp;
+      return;
+    }
   }
 }
 
 }  // namespace
 
+static_assert(kClusterMax * kKeysCtaMax == FL_MAX_SELECT_COLS, "the header states the selector's column limit");
+
 cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s) {
   const int N = a.n_q + a.n_tail;
-  const size_t smem = ((size_t)((N + 3) & ~3) + (sel_fits(N, a.k_sel) ? (size_t)a.k_sel : 0)) * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynMax);
+  if (N <= kCols1) {
+    const size_t smem = ((size_t)((N + 3) & ~3) + (sel_fits1(N, a.k_sel) ? (size_t)a.k_sel : 0)) * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynMax1);
+    if (e != cudaSuccess) return e;
+    select_cta_kernel<<<dim3(a.c.H, n_layers), kThreads1, smem, s>>>(a);
+    return cudaGetLastError();
+  }
+  int cs = 0, span = 0;
+  select_shape(N, &cs, &span);
+  if (cs == 0) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)span * sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kKeysCtaMax * (int)sizeof(uint32_t));
   if (e != cudaSuccess) return e;
-  dim3 grid(a.c.H, n_layers);
-  select_kernel<<<grid, kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.c.H * cs, n_layers);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, select_cluster_kernel, a, cs, span);
 }
 
 }  // namespace fl

@@ -658,11 +658,13 @@ std::mutex g_attr_mu;
 
 int sparse_cta_columns(int loops) {
   const int ps = (loops + 2 + 3) / 4 * 4;
-  const int staged = kPlanWords / ps, direct = direct_cta_columns(loops);
-  return staged < direct ? staged : direct;
+  int cols = kPlanWords / ps;
+  if (direct_cta_columns(loops) < cols) cols = direct_cta_columns(loops);
+  return cols;
 }
 
-int sparse_launch_splits(int heads, int loops, int r, int k_sel, int sms) {
+int sparse_launch_splits(int heads, int loops, int codec, int r, int k_sel, int sms) {
+  (void)codec;
   if (r <= kStoresMax && sms > 0) {
     const int n = staged_splits(heads, k_sel, (loops + 2 + 3) / 4 * 4, sms);
     if (n <= kMaxSplits) return n;
@@ -678,7 +680,7 @@ int workspace_splits(int loops, int max_select) {
 
 cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s, bool chain) {
   const int sms = device_sms();
-  const int n = sparse_launch_splits(a.c.H, a.c.R, a.r, a.k_sel, sms);
+  const int n = sparse_launch_splits(a.c.H, a.c.R, a.c.codec, a.r, a.k_sel, sms);
   if (a.r > kStoresMax || sms == 0 || n > kMaxSplits) return launch_sparse_direct(a, s, chain);
   const cudaError_t e = once_per_device(g_attr_done, g_attr_mu, [](int) {
     for (auto k : {sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>, sparse_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>,

@@ -19,7 +19,7 @@ def _declared():
 
 def test_every_declared_symbol_is_exported():
     names = _declared()
-    assert len(names) == 19
+    assert len(names) == 20
     for n in names:
         assert hasattr(abi.lib, n), n
     assert set(names) == set(abi.EXPORTED)
@@ -107,8 +107,8 @@ def test_reader_arguments_are_validated_before_launch():
     assert step(ll=5) == abi.FL_ERR_INVALID
     assert step(k_sel=0) == abi.FL_ERR_INVALID
     assert step(dl=0, lf=1) == abi.FL_ERR_INVALID         # first loop cannot be sparse
-    big = _dims(capacity=65536, max_select=10)
-    assert abi._c_select(ctypes.byref(big), FAKE, 0, 1, 3, 49152, 1, 10, None) == abi.FL_ERR_UNSUPPORTED
+    big = _dims(capacity=385024 + 128, max_select=10)
+    assert abi._c_select(ctypes.byref(big), FAKE, 0, 1, 3, 385024, 1, 10, None) == abi.FL_ERR_UNSUPPORTED
 
 
 def test_encoder_arguments_are_validated_before_launch():
@@ -201,10 +201,12 @@ def test_sparse_split_counts_fit_the_plan_copy_and_the_workspace(loops):
     d = abi.Dims(layers=1, heads=16, loops=loops, capacity=cap, max_select=cap,
                  res_capacity={r: cap for r in range(2, loops + 1)})
     L = abi.fl_cache_layout(d)
-    per_cta = 1024 // L.plan_stride
     base_ws = abi.fl_workspace_bytes(d)
     for sms in (1, 148, 160, 1024):
         for loop in sorted({2, 3, min(8, loops), loops}):
+            # the loop <= 8 reader of the method's codec copies 2048 plan words per CTA, the
+            # loop > 8 reader 1024
+            per_cta = (2048 if loop <= 8 else 1024) // L.plan_stride
             for k_sel in (1, 7, 31, 820, 3277, 7168, 7169, 8192, cap):
                 n, capacity = abi.fl_sparse_splits(d, loop, k_sel, sms)
                 assert 1 <= n <= capacity, (sms, loop, k_sel, n, capacity)
@@ -214,6 +216,12 @@ def test_sparse_split_counts_fit_the_plan_copy_and_the_workspace(loops):
     if loops == 32:
         n, capacity = abi.fl_sparse_splits(d, 32, 8192, 148)
         assert n > 256 and capacity >= n
+    # the codec variants read through the loop <= 8 reader of 1024 plan words
+    dv = abi.Dims(layers=1, heads=16, loops=loops, capacity=cap, max_select=cap,
+                  res_capacity={r: cap for r in range(2, loops + 1)}, codec=abi.FL_CODEC_FULL_INT4)
+    for k_sel in (820, 8192):
+        n, capacity = abi.fl_sparse_splits(dv, 3, k_sel, 148)
+        assert -(-k_sel // n) <= 1024 // L.plan_stride and n <= capacity
     with pytest.raises(abi.FlashLoopError):
         abi.fl_sparse_splits(d, 1, 10, 148)          # loop 1 is never sparse
     with pytest.raises(abi.FlashLoopError):

@@ -131,16 +131,18 @@ def test_layer_32k_prefill_and_256_decode_steps():
 
 
 def test_deep_loops_every_column_selected_needs_many_splits():
-    """BASELINE configuration 4's shape (R = 32, N = 8192) with K_sel = N: a CTA holds at
-    most 28 of the 36-word plan entries, so the readers need ~293 split-K partitions per
-    head.  Every sparse loop must then equal the dense attention of its loop (m = 1)."""
+    """BASELINE configuration 4's shape (R = 32, N = 8192) with K_sel = N: a CTA of the
+    loop > 8 reader holds at most 28 of the 36-word plan entries, so it needs ~293 split-K
+    partitions per head (the loop <= 8 reader holds 56: ~147).  Every sparse loop must then
+    equal the dense attention of its loop (m = 1)."""
     w = W["deep_r32_h16_n8192"]
     pair = Pair(w, heads=[0, 11])
     c = pair.cache
     N = c.n_cols
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    n, cap = abi.fl_sparse_splits(c.dims, 3, N, sms)
-    assert n > 256 and n <= cap
+    n3, cap = abi.fl_sparse_splits(c.dims, 3, N, sms)
+    n9, _ = abi.fl_sparse_splits(c.dims, 9, N, sms)
+    assert 146 <= n3 <= cap and 256 < n9 <= cap
     q = synth.queries(w, 0, 0, device="cuda")
     errs = pair.run_loops(q, k_sel=N, label="deep K=N")
     # at K = N the unselected contribution is exactly zero in the oracle: hold u to the
@@ -219,3 +221,15 @@ def test_standalone_reader_calls_back_to_back_match_synchronised_calls():
         assert torch.equal(a.raw(name, 0), pair.cache.raw(name, 0)), name
     for st in (a.status(), b.status()):
         assert st[0] == abi.FL_OK, st
+
+
+@pytest.mark.parametrize("n_ctx", [60000, 100000])
+def test_long_context_selection_through_thread_block_clusters(n_ctx):
+    """Contexts beyond one CTA's shared memory (49152 columns): the selector spreads each
+    (layer, head)'s keys over a cluster of 4 or 8 CTAs; S must still be a valid top-K of the
+    oracle's distribution, and every loop must match the oracle."""
+    w = synth.Workload(name=f"long{n_ctx}", layers=1, heads=2, n_ctx=n_ctx, loops=4,
+                       sigma=(0, 0, 0.5, 0.2, 0.1), frac=(0, 1, 1, 0.25, 0.10), seed=31 + n_ctx)
+    pair = Pair(w)
+    errs = pair.run_loops(synth.queries(w, 0, 0, device="cuda"), label=f"N={n_ctx}")
+    _assert_errs(errs)
