@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libflashloop_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
-SOURCES = ["api.cu", "encode.cu", "dense.cu", "dense_staged.cu", "sparse.cu", "sparse_staged.cu", "select.cu", "tokens.cu", "prefill.cu"]
+SOURCES = ["api.cu", "encode.cu", "dense.cu", "dense_staged.cu", "sparse.cu", "sparse_staged.cu", "sparse_persist.cu", "select.cu", "tokens.cu", "prefill.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

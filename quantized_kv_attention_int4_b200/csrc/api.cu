@@ -104,15 +104,26 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 fl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FL_OK : FL_ERR_CUDA; }
 
-uint64_t ws_part_bytes(const fl_dims* d) {
-  return (uint64_t)d->heads * workspace_splits(d->loops, d->max_select) * kPartStride * sizeof(float);
+// Split-K partials the workspace holds: those of the one-layer launches (per head), or those
+// of a persistent sparse launch over every layer (per layer and head), whichever is more.
+uint64_t ws_partials(const fl_dims* d) {
+  const uint64_t one = (uint64_t)d->heads * workspace_splits(d->loops, d->max_select);
+  const uint64_t all = (uint64_t)d->layers * d->heads * persist_splits(d->max_select, d->loops);
+  return one > all ? one : all;
 }
+uint64_t ws_part_bytes(const fl_dims* d) { return ws_partials(d) * kPartStride * sizeof(float); }
+// completion tickets: one per (layer, head)
+uint64_t ws_ticket_bytes(const fl_dims* d) { return (uint64_t)d->layers * d->heads * sizeof(int32_t); }
 
-// The split count a sparse launch will use fits the workspace's partials (it always does
-// for k_sel <= max_select; checked before any launch all the same).
+// The split counts a sparse launch of `loop` over k_sel columns uses, with and without the
+// fused flush, fit the workspace's partials (they always do for k_sel <= max_select; checked
+// before any launch all the same).
 fl_status check_sparse_splits(const fl_dims* d, int loop, int k_sel) {
-  const int n = sparse_launch_splits(d->heads, d->loops, d->codec, loop, k_sel, device_sms());
-  return n <= workspace_splits(d->loops, d->max_select) ? FL_OK : FL_ERR_UNSUPPORTED;
+  const int sms = device_sms();
+  const uint64_t one = (uint64_t)d->heads * sparse_launch_splits(d->heads, d->loops, d->codec, loop, k_sel, sms, true);
+  const uint64_t all =
+      (uint64_t)d->layers * d->heads * sparse_launch_splits(d->heads, d->loops, d->codec, loop, k_sel, sms, false);
+  return one <= ws_partials(d) && all <= ws_partials(d) ? FL_OK : FL_ERR_UNSUPPORTED;
 }
 
 fl_status check_reader(const fl_dims* d, void* cache, int layer, int loop, int n_q, int n_tail,
@@ -188,15 +199,15 @@ fl_status fl_cache_init(const fl_dims* dims, void* cache, void* stream) {
 
 size_t fl_workspace_bytes(const fl_dims* dims) {
   if (check_dims(dims) != FL_OK) return 0;
-  return ws_part_bytes(dims) + align_up((uint64_t)dims->heads * sizeof(int32_t));
+  return ws_part_bytes(dims) + align_up(ws_ticket_bytes(dims));
 }
 
 fl_status fl_workspace_init(const fl_dims* dims, void* ws, size_t ws_bytes, void* stream) {
   fl_status st = check_dims(dims);
   if (st != FL_OK) return st;
   if (!ws || ws_bytes < fl_workspace_bytes(dims)) return FL_ERR_WORKSPACE;
-  return cuda_status(cudaMemsetAsync(static_cast<uint8_t*>(ws) + ws_part_bytes(dims), 0,
-                                     (size_t)dims->heads * sizeof(int32_t), (cudaStream_t)stream));
+  return cuda_status(cudaMemsetAsync(static_cast<uint8_t*>(ws) + ws_part_bytes(dims), 0, ws_ticket_bytes(dims),
+                                     (cudaStream_t)stream));
 }
 
 fl_status fl_write_tail(const fl_dims* dims, void* cache, int32_t layer, int32_t loop, int32_t row0,
@@ -414,7 +425,7 @@ fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_
   if (scratch_bytes((k_sel + cols - 1) / cols) > FL_NOALLOC_SCRATCH_BYTES) return FL_ERR_UNSUPPORTED;
   const int sms = device_sms();
   if (sms <= 0) return FL_ERR_CUDA;
-  if (scratch_bytes(sparse_launch_splits(dims->heads, dims->loops, dims->codec, loop, k_sel, sms)) >
+  if (scratch_bytes(sparse_launch_splits(dims->heads, dims->loops, dims->codec, loop, k_sel, sms, false)) >
       FL_NOALLOC_SCRATCH_BYTES)
     return FL_ERR_UNSUPPORTED;
   int dev = 0;
@@ -454,8 +465,8 @@ fl_status fl_sparse_splits(const fl_dims* dims, int32_t loop, int32_t k_sel, int
   if (st != FL_OK) return st;
   if (!splits || loop < 2 || loop > dims->loops || k_sel < 1 || k_sel > dims->max_select || sm_count < 1)
     return FL_ERR_INVALID;
-  *splits = sparse_launch_splits(dims->heads, dims->loops, dims->codec, loop, k_sel, sm_count);
-  if (capacity) *capacity = workspace_splits(dims->loops, dims->max_select);
+  *splits = sparse_launch_splits(dims->heads, dims->loops, dims->codec, loop, k_sel, sm_count, false);
+  if (capacity) *capacity = (int32_t)(ws_partials(dims) / ((uint64_t)dims->layers * dims->heads));
   return FL_OK;
 }
 
@@ -551,16 +562,41 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
       if (launch_select(sa, L, s) != cudaSuccess) return FL_ERR_CUDA;
       if (!rec(2 * r - 1)) return FL_ERR_CUDA;
       a.keep = 1;
-      for (int l = 0; l < L; ++l) {
-        const size_t qo = (size_t)r * ostride_r + (size_t)l * row;
-        a.layer = l;
-        a.q = q + qo;
-        a.k_new = k_new ? k_new + qo : nullptr;
-        a.v_new = v_new ? v_new + qo : nullptr;
-        a.o = o + qo;
-        a.o_prev = o + qo - ostride_r;
-        set_flush(a, flush, l, r);
-        if (launch_sparse(a, s) != cudaSuccess) return FL_ERR_CUDA;
+      if (dims->codec == FL_CODEC_RESIDUAL_INT4 && r <= kPersistMaxLoop) {
+        // every layer of the loop through the persistent reader: one launch (per
+        // kFlushLayersMax layers with the fused flush)
+        const int span = flush ? kFlushLayersMax : L;
+        for (int l0 = 0; l0 < L; l0 += span) {
+          const size_t qo = (size_t)r * ostride_r + (size_t)l0 * row;
+          a.layer = l0;
+          a.n_layers = L - l0 < span ? L - l0 : span;
+          a.io_layer_stride = (int64_t)row;
+          a.q = q + qo;
+          a.k_new = k_new ? k_new + qo : nullptr;
+          a.v_new = v_new ? v_new + qo : nullptr;
+          a.o = o + qo;
+          a.o_prev = o + qo - ostride_r;
+          set_flush(a, flush, l0, r);
+          if (flush)
+            for (int i = 0; i < a.n_layers; ++i)
+              a.flush_slot0s[i] = flush->slot0[(size_t)(l0 + i) * (FL_MAX_LOOPS + 1) + r];
+          if (launch_sparse(a, s) != cudaSuccess) return FL_ERR_CUDA;
+        }
+        a.layer = 0;
+        a.n_layers = 1;
+        a.io_layer_stride = 0;
+      } else {
+        for (int l = 0; l < L; ++l) {
+          const size_t qo = (size_t)r * ostride_r + (size_t)l * row;
+          a.layer = l;
+          a.q = q + qo;
+          a.k_new = k_new ? k_new + qo : nullptr;
+          a.v_new = v_new ? v_new + qo : nullptr;
+          a.o = o + qo;
+          a.o_prev = o + qo - ostride_r;
+          set_flush(a, flush, l, r);
+          if (launch_sparse(a, s) != cudaSuccess) return FL_ERR_CUDA;
+        }
       }
     }
     if (!rec(2 * r)) return FL_ERR_CUDA;

@@ -397,6 +397,60 @@ __device__ __forceinline__ void record_to_limbs(uint32_t* rec, const float* q_s,
   }
 }
 
+// record_to_limbs for two records at once (ra, rb), so that their reductions and shared
+// memory round trips overlap; the same words as two calls.
+__device__ __forceinline__ void record_to_limbs2(uint32_t* ra, uint32_t* rb, const float* q_s, int lane) {
+  uint32_t* rec[2] = {ra, rb};
+  const float4 qv = *reinterpret_cast<const float4*>(q_s + 4 * lane);
+  float qs[2][4], cz[2], mx[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(rec[i] + 4 * lane);
+    const float2 s0 = unpack_sz(raw.x), s1 = unpack_sz(raw.y), s2 = unpack_sz(raw.z), s3 = unpack_sz(raw.w);
+    qs[i][0] = qv.x * s0.x;
+    qs[i][1] = qv.y * s1.x;
+    qs[i][2] = qv.z * s2.x;
+    qs[i][3] = qv.w * s3.x;
+    cz[i] = fmaf(qv.x, s0.y, fmaf(qv.y, s1.y, fmaf(qv.z, s2.y, qv.w * s3.y)));
+    mx[i] = fmaxf(fmaxf(fabsf(qs[i][0]), fabsf(qs[i][1])), fmaxf(fabsf(qs[i][2]), fabsf(qs[i][3])));
+  }
+  mx[0] = warp_max(mx[0]);
+  mx[1] = warp_max(mx[1]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    cz[0] += __shfl_xor_sync(kFull, cz[0], o);
+    cz[1] += __shfl_xor_sync(kFull, cz[1], o);
+  }
+  int Q[2][4], E[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    E[i] = mx[i] > 0.f ? min(23 - exp_frexp(mx[i]), 126) : 0;
+    const float sc = pow2i(E[i]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int x = __float2int_rn(qs[i][k] * sc);
+      Q[i][k] = x > 8388607 ? 8388607 : (x < -8388607 ? -8388607 : x);
+    }
+  }
+  __syncwarp();
+  const int w = lane >> 1, hb = (lane & 1) * 2;
+  auto pair = [](int a, int b, int sh) { return (uint16_t)(((a >> sh) & 0xff) | (((b >> sh) & 0xff) << 8)); };
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    uint16_t* lh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(rec[i] + kLimbWords * w) + hb);
+    lh[0] = pair(Q[i][0], Q[i][2], 0);
+    lh[2] = pair(Q[i][0], Q[i][2], 8);
+    lh[4] = pair(Q[i][0], Q[i][2], 16);
+    lh[6] = pair(Q[i][1], Q[i][3], 0);
+    lh[8] = pair(Q[i][1], Q[i][3], 8);
+    lh[10] = pair(Q[i][1], Q[i][3], 16);
+    if (lane == 0) {
+      rec[i][kLimbE] = (uint32_t)E[i];
+      rec[i][kLimbC] = __float_as_uint(cz[i]);
+    }
+  }
+}
+
 // Dot of one 32-channel quarter of a code row (4 code words) with the record's 24 limb
 // words of that quarter (words 24*qq.., held in registers), in units of 2^-E.  Odd
 // channels are taken in place (their nibble x16) and scaled back here.

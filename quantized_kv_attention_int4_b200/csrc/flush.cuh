@@ -26,15 +26,18 @@ namespace fl {
 // earlier in the step.  The new token (tail row 63) comes from k_new / v_new when the
 // step supplies it, since the tail copy of that row is written by another CTA of this
 // same launch.
-static __device__ __forceinline__ void flush_tail(const ReaderArgs& a, int cta, int n_cta, EncodeSmem& sm, int tid,
-                                                  int nt) {
+// The same for layer `layer` with its group's first slot `slot0` and its new token's
+// key / value rows k_new / v_new (a launch over several layers).
+static __device__ __forceinline__ void flush_tail_layer(const ReaderArgs& a, int layer, int slot0,
+                                                        const uint16_t* k_new, const uint16_t* v_new, int cta,
+                                                        int n_cta, EncodeSmem& sm, int tid, int nt) {
   const CacheView& c = a.c;
   const int r = a.r, H = c.H, ncb = c.cap / kG, T = c.total_slots, gb = a.n_q / kG;
   const unsigned long long act = r == 1 ? ~0ull : a.flush_act;
   const int nr = __popcll(act);
-  uint8_t* depth = arr<uint8_t>(c, A_DEPTH, a.layer);
-  unsigned long long* mask = arr<unsigned long long>(c, A_MASK, a.layer);
-  int32_t* first = arr<int32_t>(c, A_FIRST, a.layer);
+  uint8_t* depth = arr<uint8_t>(c, A_DEPTH, layer);
+  unsigned long long* mask = arr<unsigned long long>(c, A_MASK, layer);
+  int32_t* first = arr<int32_t>(c, A_FIRST, layer);
 
   // store r is a residual against stores 1 .. r - 1 of the same rows: those flushes must
   // have run (loops in order); otherwise record the error and write nothing
@@ -62,7 +65,7 @@ static __device__ __forceinline__ void flush_tail(const ReaderArgs& a, int cta, 
         if ((act >> t) & 1ull) depth[a.n_q + t] = (uint8_t)r;
       if (tid == 0) {
         mask[(size_t)r * ncb + gb] = act;
-        first[(size_t)r * ncb + gb] = nr ? a.flush_slot0 : -1;
+        first[(size_t)r * ncb + gb] = nr ? slot0 : -1;
       }
     }
   }
@@ -76,17 +79,17 @@ static __device__ __forceinline__ void flush_tail(const ReaderArgs& a, int cta, 
     sm.g0[rp] = c.slot_base[rp] + __ldcg(first + (size_t)rp * ncb + gb);
   }
 
-  const uint8_t* brec_l = arr<uint8_t>(c, A_BREC, a.layer);
-  const uint8_t* rrec_l = arr<uint8_t>(c, A_RREC, a.layer);
+  const uint8_t* brec_l = arr<uint8_t>(c, A_BREC, layer);
+  const uint8_t* rrec_l = arr<uint8_t>(c, A_RREC, layer);
   for (int u = cta; u < 8 * H; u += n_cta) {
     const int h = u >> 3, qt = u & 3;
     const bool is_v = ((u >> 2) & 1) != 0;
     const uint8_t* bgrp = brec_l + ((size_t)h * ncb + gb) * kRec;
     const uint8_t* rrec = rrec_l + (size_t)h * (T / kG) * kRec;
-    uint8_t* rec = const_cast<uint8_t*>(r == 1 ? bgrp : rrec + (size_t)((c.slot_base[r] + a.flush_slot0) >> 6) * kRec);
+    uint8_t* rec = const_cast<uint8_t*>(r == 1 ? bgrp : rrec + (size_t)((c.slot_base[r] + slot0) >> 6) * kRec);
     const uint16_t* src =
-        arr<uint16_t>(c, is_v ? A_TAILV : A_TAILK, a.layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
-    const uint16_t* xnew = is_v ? a.v_new : a.k_new;
+        arr<uint16_t>(c, is_v ? A_TAILV : A_TAILK, layer) + ((size_t)(r - 1) * H + h) * kTail * kD;
+    const uint16_t* xnew = is_v ? v_new : k_new;
     if (xnew) xnew += (size_t)h * kD;
 
     __syncthreads();  // the row map is in place; the previous unit is done with shared memory
@@ -128,6 +131,12 @@ static __device__ __forceinline__ void flush_tail(const ReaderArgs& a, int cta, 
     if (is_v) group_codes(sm, rec, true, 16 * qt, 16, 0, kD / 8, nr, tid, nt);
     else group_codes(sm, rec, false, 0, kG, 4 * qt, 4, nr, tid, nt);
   }
+}
+
+// Store a.r of the 64 tail rows of layer a.layer (the one-layer launches).
+static __device__ __forceinline__ void flush_tail(const ReaderArgs& a, int cta, int n_cta, EncodeSmem& sm, int tid,
+                                                  int nt) {
+  flush_tail_layer(a, a.layer, a.flush_slot0, a.k_new, a.v_new, cta, n_cta, sm, tid, nt);
 }
 
 }  // namespace fl

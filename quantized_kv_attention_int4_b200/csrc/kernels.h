@@ -25,6 +25,9 @@ struct EncodeResArgs {
   int64_t head_stride;
 };
 
+// Layers one persistent sparse launch can flush (beyond: one launch per layer).
+constexpr int kFlushLayersMax = 256;
+
 struct ReaderArgs {
   CacheView c;
   int layer, r, n_q, n_tail, k_sel, n_splits, keep;
@@ -40,6 +43,12 @@ struct ReaderArgs {
   // group that starts at residual slot flush_slot0
   int flush, flush_slot0;
   unsigned long long flush_act;
+  // a launch over layers [layer, layer + n_layers) (the persistent sparse reader): q, k_new,
+  // v_new, o_prev and o of layer layer + i start io_layer_stride elements * i further
+  int n_layers;
+  int64_t io_layer_stride;
+  // the fused flush of a launch over several layers: flush_slot0 of layer layer + i
+  int32_t flush_slot0s[kFlushLayersMax];
 };
 
 struct SelectArgs {
@@ -110,15 +119,23 @@ cudaError_t once_per_device(std::atomic<bool>* done, std::mutex& mu, F&& fn) {
 
 // Plan entries (selected columns) one sparse-reader CTA holds in shared memory.
 int sparse_cta_columns(int loops);
-// Split-K partitions per head that launch_sparse uses for a loop-r reader over k_sel
-// columns of a cache with codec `codec` on a device with `sms` SMs: never fewer than
-// ceil(k_sel / sparse_cta_columns).
-int sparse_launch_splits(int heads, int loops, int codec, int r, int k_sel, int sms);
-// Split-K partials per head that a workspace for these dims holds: enough for every
-// dense launch and for every sparse launch with k_sel <= max_select.
+// Split-K partitions per (layer, head) that launch_sparse uses for a loop-r reader over
+// k_sel columns of a cache with codec `codec` on a device with `sms` SMs, with or without
+// the fused tail flush: never fewer than the plan copy of one CTA (or work item) needs.
+int sparse_launch_splits(int heads, int loops, int codec, int r, int k_sel, int sms, bool flush);
+// Split-K partials per head that a workspace for these dims holds for the one-layer
+// launches: enough for every dense launch and every sparse launch with k_sel <= max_select.
 int workspace_splits(int loops, int max_select);
 // The direct sparse reader's split count and per-CTA plan capacity (sparse.cu).
 int direct_splits(int heads, int k_sel, int loops, int sms);
 int direct_cta_columns(int loops);
+// The persistent sparse reader (sparse_persist.cu): the method's 4-bit residual stores,
+// loops r <= kPersistMaxLoop, with or without the fused flush; one launch for a range of
+// layers (work items of at most persist_item_columns(loops) selected columns of one
+// (layer, head)), then one launch of its combine.
+constexpr int kPersistMaxLoop = 8;
+int persist_item_columns(int loops);
+int persist_splits(int k_sel, int loops);
+cudaError_t launch_sparse_persist(ReaderArgs a, cudaStream_t s, bool chain);
 
 }  // namespace fl

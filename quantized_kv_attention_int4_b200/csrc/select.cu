@@ -288,14 +288,16 @@ __global__ void __launch_bounds__(kThreads1, 1) select_cta_kernel(SelectArgs a) 
   int32_t* plan = arr<int32_t>(c, A_PLAN, layer) + (size_t)h * c.max_select * ps;
   const int r = a.r;
   __syncthreads();
-#pragma unroll 2
+  // the layer's tags, depths, masks and first slots are read-only here (non-coherent loads
+  // the compiler may issue ahead of the entries' stores)
+#pragma unroll 4
   for (int k = tid; k < K; k += kThreads1) {
     const int j = sel_smem ? sel_s[k] : sel[k];
-    int lam = tag[j];
+    int lam = __ldg(tag + j);
     lam = lam < 1 ? 1 : (lam > R ? R : lam);
     int stores = 0;
     if (j < n_q) {
-      const int dep = depth[j];
+      const int dep = __ldg(depth + j);
       stores = dep < r ? dep : r;
     }
     // the entry's words, stored 16 bytes at a time (ps is a multiple of 4; unused words 0)
@@ -308,8 +310,8 @@ __global__ void __launch_bounds__(kThreads1, 1) select_cta_kernel(SelectArgs a) 
       if (i == 2) return w2;
       const int rp = i - 1;
       if (rp > stores) return 0;
-      const unsigned long long mk = mask[(size_t)rp * ncb + b];
-      return c.slot_base[rp] + first[(size_t)rp * ncb + b] + __popcll(mk & ((1ull << jt) - 1ull));
+      const unsigned long long mk = __ldg(mask + (size_t)rp * ncb + b);
+      return c.slot_base[rp] + __ldg(first + (size_t)rp * ncb + b) + __popcll(mk & ((1ull << jt) - 1ull));
     };
     for (int q4 = 0; q4 < ps; q4 += 4)
       e[q4 >> 2] = make_uint4((uint32_t)word(q4), (uint32_t)word(q4 + 1), (uint32_t)word(q4 + 2), (uint32_t)word(q4 + 3));
@@ -539,11 +541,11 @@ __global__ void __launch_bounds__(kThreads, 2) select_cluster_kernel(SelectArgs 
 #pragma unroll 4
   for (int k = (int)sel0 + tid; k < (int)sel1; k += kThreads) {
     const int j = sel[k];
-    int lam = tag[j];
+    int lam = __ldg(tag + j);
     lam = lam < 1 ? 1 : (lam > R ? R : lam);
     int stores = 0;
     if (j < n_q) {
-      const int dep = depth[j];
+      const int dep = __ldg(depth + j);
       stores = dep < r ? dep : r;
     }
     // the entry's words, stored 16 bytes at a time (ps is a multiple of 4; unused words 0)
@@ -556,8 +558,8 @@ __global__ void __launch_bounds__(kThreads, 2) select_cluster_kernel(SelectArgs 
       if (i == 2) return w2;
       const int rp = i - 1;
       if (rp > stores) return 0;
-      const unsigned long long mk = mask[(size_t)rp * ncb + b];
-      return c.slot_base[rp] + first[(size_t)rp * ncb + b] + __popcll(mk & ((1ull << jt) - 1ull));
+      const unsigned long long mk = __ldg(mask + (size_t)rp * ncb + b);
+      return c.slot_base[rp] + __ldg(first + (size_t)rp * ncb + b) + __popcll(mk & ((1ull << jt) - 1ull));
     };
     for (int q4 = 0; q4 < ps; q4 += 4)
       e[q4 >> 2] = make_uint4((uint32_t)word(q4), (uint32_t)word(q4 + 1), (uint32_t)word(q4 + 2), (uint32_t)word(q4 + 3));
@@ -565,11 +567,12 @@ __global__ void __launch_bounds__(kThreads, 2) select_cluster_kernel(SelectArgs 
   cluster_sync();  // no CTA leaves while another may still read its shared memory
 }
 
-// CTAs per cluster and columns per CTA for N columns; cs = 0 when N is too large.
-void select_shape(int N, int* cs, int* span) {
+// CTAs per cluster (at least `want`, at least 2) and columns per CTA for N columns; cs = 0
+// when N is too large.
+void select_shape(int N, int want, int* cs, int* span) {
   *cs = 0;
   *span = 0;
-  for (int c = 2; c <= kClusterMax; c *= 2) {
+  for (int c = want > 2 ? want : 2; c <= kClusterMax; c *= 2) {
     const int sp = ((N + c - 1) / c + 63) / 64 * 64;
     if (sp <= (c < kClusterMax ? kKeysCta : kKeysCtaMax)) {
       *cs = c;
@@ -585,7 +588,13 @@ static_assert(kClusterMax * kKeysCtaMax == FL_MAX_SELECT_COLS, "the header state
 
 cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s) {
   const int N = a.n_q + a.n_tail;
-  if (N <= kCols1) {
+  // one CTA per (layer, head) when those fill the GPU and the head's keys fit one CTA;
+  // otherwise clusters, as many CTAs per head as it takes to occupy every SM
+  const int sms = device_sms() > 0 ? device_sms() : 148;
+  const long long heads_all = (long long)a.c.H * n_layers;
+  int want = 1;
+  while (want < kClusterMax && heads_all * want < sms) want *= 2;
+  if (N <= kCols1 && want == 1) {
     const size_t smem = ((size_t)((N + 3) & ~3) + (sel_fits1(N, a.k_sel) ? (size_t)a.k_sel : 0)) * sizeof(uint32_t);
     cudaError_t e = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynMax1);
     if (e != cudaSuccess) return e;
@@ -593,7 +602,7 @@ cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s) {
     return cudaGetLastError();
   }
   int cs = 0, span = 0;
-  select_shape(N, &cs, &span);
+  select_shape(N, want, &cs, &span);
   if (cs == 0) return cudaErrorInvalidValue;
   const size_t smem = (size_t)span * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

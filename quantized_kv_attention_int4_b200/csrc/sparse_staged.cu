@@ -663,8 +663,9 @@ int sparse_cta_columns(int loops) {
   return cols;
 }
 
-int sparse_launch_splits(int heads, int loops, int codec, int r, int k_sel, int sms) {
-  (void)codec;
+int sparse_launch_splits(int heads, int loops, int codec, int r, int k_sel, int sms, bool flush) {
+  (void)flush;
+  if (codec == FL_CODEC_RESIDUAL_INT4 && r <= kPersistMaxLoop) return persist_splits(k_sel, loops);
   if (r <= kStoresMax && sms > 0) {
     const int n = staged_splits(heads, k_sel, (loops + 2 + 3) / 4 * 4, sms);
     if (n <= kMaxSplits) return n;
@@ -679,8 +680,14 @@ int workspace_splits(int loops, int max_select) {
 }
 
 cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s, bool chain) {
+  if (a.c.codec == FL_CODEC_RESIDUAL_INT4 && a.r <= kPersistMaxLoop) {
+    if (a.n_layers < 1) a.n_layers = 1;
+    if (a.flush && a.n_layers == 1) a.flush_slot0s[0] = a.flush_slot0;
+    return launch_sparse_persist(a, s, chain);
+  }
+  a.n_layers = 1;  // one layer per launch below
   const int sms = device_sms();
-  const int n = sparse_launch_splits(a.c.H, a.c.R, a.c.codec, a.r, a.k_sel, sms);
+  const int n = sparse_launch_splits(a.c.H, a.c.R, a.c.codec, a.r, a.k_sel, sms, a.flush != 0);
   if (a.r > kStoresMax || sms == 0 || n > kMaxSplits) return launch_sparse_direct(a, s, chain);
   const cudaError_t e = once_per_device(g_attr_done, g_attr_mu, [](int) {
     for (auto k : {sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>, sparse_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>,
