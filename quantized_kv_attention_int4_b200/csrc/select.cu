@@ -40,6 +40,7 @@ constexpr int kBins = 1 << kDigit;
 constexpr int kKeysCta = 18432;            // keys per CTA when the cluster has <= 4 CTAs (two CTAs per SM)
 constexpr int kKeysCtaMax = 48128;         // ... and with 8 (one CTA per SM then)
 constexpr int kClusterMax = 8;
+constexpr int kPlanPer = 4;               // gather-plan entries a thread forms together
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t b = __float_as_uint(f);
@@ -287,23 +288,13 @@ __global__ void __launch_bounds__(kThreads1, 1) select_cta_kernel(SelectArgs a) 
   const int ps = c.plan_stride;
   int32_t* plan = arr<int32_t>(c, A_PLAN, layer) + (size_t)h * c.max_select * ps;
   const int r = a.r;
-  __syncthreads();
-  // the layer's tags, depths, masks and first slots are read-only here (non-coherent loads
-  // the compiler may issue ahead of the entries' stores)
-#pragma unroll 4
-  for (int k = tid; k < K; k += kThreads1) {
-    const int j = sel_smem ? sel_s[k] : sel[k];
-    int lam = __ldg(tag + j);
-    lam = lam < 1 ? 1 : (lam > R ? R : lam);
-    int stores = 0;
-    if (j < n_q) {
-      const int dep = __ldg(depth + j);
-      stores = dep < r ? dep : r;
-    }
-    // the entry's words, stored 16 bytes at a time (ps is a multiple of 4; unused words 0)
+  // one gather-plan entry: column j with tag tg, depth dp and key u, written 16 bytes at a
+  // time (ps is a multiple of 4; unused words 0)
+  auto plan_entry = [&](int32_t* ent, int j, int tg, int dp, uint32_t u) {
+    const int lam = tg < 1 ? 1 : (tg > R ? R : tg);
+    const int stores = dp < r ? dp : r;  // dp = 0 for a tail column
     const int b = j >> 6, jt = j & 63;
-    uint4* e = reinterpret_cast<uint4*>(plan + (size_t)k * ps);
-    const int w2 = __float_as_int(ex2(key_value(keys[j])));
+    const int w2 = __float_as_int(ex2(key_value(u)));
     auto word = [&](int i) -> int {
       if (i == 0) return j;
       if (i == 1) return lam | (stores << 8);
@@ -313,8 +304,30 @@ __global__ void __launch_bounds__(kThreads1, 1) select_cta_kernel(SelectArgs a) 
       const unsigned long long mk = __ldg(mask + (size_t)rp * ncb + b);
       return c.slot_base[rp] + __ldg(first + (size_t)rp * ncb + b) + __popcll(mk & ((1ull << jt) - 1ull));
     };
+    uint4* e = reinterpret_cast<uint4*>(ent);
     for (int q4 = 0; q4 < ps; q4 += 4)
       e[q4 >> 2] = make_uint4((uint32_t)word(q4), (uint32_t)word(q4 + 1), (uint32_t)word(q4 + 2), (uint32_t)word(q4 + 3));
+  };
+  __syncthreads();
+  // the layer's tags, depths, masks and first slots are read-only here (non-coherent loads
+  // the compiler may issue ahead of the entries' stores); kPlanPer entries per thread at a
+  // time, their columns' tags and depths loaded together before any entry is formed
+  for (int k0 = 0; k0 < K; k0 += kPlanPer * kThreads1) {
+    int jj[kPlanPer], tg[kPlanPer], dp[kPlanPer];
+#pragma unroll
+    for (int u = 0; u < kPlanPer; ++u) {
+      const int k = k0 + u * kThreads1 + tid;
+      jj[u] = k < K ? (sel_smem ? sel_s[k] : sel[k]) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kPlanPer; ++u) {
+      const int j = jj[u];
+      tg[u] = j >= 0 ? __ldg(tag + j) : 1;
+      dp[u] = j >= 0 && j < n_q ? __ldg(depth + j) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kPlanPer; ++u)
+      if (jj[u] >= 0) plan_entry(plan + (size_t)(k0 + u * kThreads1 + tid) * ps, jj[u], tg[u], dp[u], keys[jj[u]]);
   }
   if (tid == 0) {
     float m = 0.f;
@@ -538,20 +551,13 @@ __global__ void __launch_bounds__(kThreads, 2) select_cluster_kernel(SelectArgs 
   const int ps = c.plan_stride;
   int32_t* plan = arr<int32_t>(c, A_PLAN, layer) + (size_t)h * c.max_select * ps;
   const int r = a.r;
-#pragma unroll 4
-  for (int k = (int)sel0 + tid; k < (int)sel1; k += kThreads) {
-    const int j = sel[k];
-    int lam = __ldg(tag + j);
-    lam = lam < 1 ? 1 : (lam > R ? R : lam);
-    int stores = 0;
-    if (j < n_q) {
-      const int dep = __ldg(depth + j);
-      stores = dep < r ? dep : r;
-    }
-    // the entry's words, stored 16 bytes at a time (ps is a multiple of 4; unused words 0)
+  // one gather-plan entry: column j with tag tg, depth dp and key u, written 16 bytes at a
+  // time (ps is a multiple of 4; unused words 0)
+  auto plan_entry = [&](int32_t* ent, int j, int tg, int dp, uint32_t u) {
+    const int lam = tg < 1 ? 1 : (tg > R ? R : tg);
+    const int stores = dp < r ? dp : r;  // dp = 0 for a tail column
     const int b = j >> 6, jt = j & 63;
-    uint4* e = reinterpret_cast<uint4*>(plan + (size_t)k * ps);
-    const int w2 = __float_as_int(ex2(key_value(keys[j - j0])));
+    const int w2 = __float_as_int(ex2(key_value(u)));
     auto word = [&](int i) -> int {
       if (i == 0) return j;
       if (i == 1) return lam | (stores << 8);
@@ -561,8 +567,27 @@ __global__ void __launch_bounds__(kThreads, 2) select_cluster_kernel(SelectArgs 
       const unsigned long long mk = __ldg(mask + (size_t)rp * ncb + b);
       return c.slot_base[rp] + __ldg(first + (size_t)rp * ncb + b) + __popcll(mk & ((1ull << jt) - 1ull));
     };
+    uint4* e = reinterpret_cast<uint4*>(ent);
     for (int q4 = 0; q4 < ps; q4 += 4)
       e[q4 >> 2] = make_uint4((uint32_t)word(q4), (uint32_t)word(q4 + 1), (uint32_t)word(q4 + 2), (uint32_t)word(q4 + 3));
+  };
+  for (int k0 = (int)sel0; k0 < (int)sel1; k0 += kPlanPer * kThreads) {
+    int jj[kPlanPer], tg[kPlanPer], dp[kPlanPer];
+#pragma unroll
+    for (int u = 0; u < kPlanPer; ++u) {
+      const int k = k0 + u * kThreads + tid;
+      jj[u] = k < (int)sel1 ? sel[k] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kPlanPer; ++u) {
+      const int j = jj[u];
+      tg[u] = j >= 0 ? __ldg(tag + j) : 1;
+      dp[u] = j >= 0 && j < n_q ? __ldg(depth + j) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kPlanPer; ++u)
+      if (jj[u] >= 0)
+        plan_entry(plan + (size_t)(k0 + u * kThreads + tid) * ps, jj[u], tg[u], dp[u], keys[jj[u] - j0]);
   }
   cluster_sync();  // no CTA leaves while another may still read its shared memory
 }
