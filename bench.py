@@ -584,7 +584,7 @@ def run_deep(device, hbm, warmup=3, steps=10):
         raise RuntimeError(f"device error in the deep-loop measurement: {info}")
     us = {r: float(np.mean(seg[r])) for r in range(1, R + 1)}
     groups = {"dense loops 1-2 (dense_staged_kernel)": range(1, wr.dense_loops + 1),
-              "sparse loops 3-8 (sparse_batch_kernel)": range(wr.dense_loops + 1, 9),
+              "sparse loops 3-8 (sparse_persist_kernel)": range(wr.dense_loops + 1, 9),
               "sparse loops 9-32 (sparse_kernel, direct)": range(9, R + 1)}
     out = {}
     for name, rr in groups.items():
@@ -986,15 +986,19 @@ def main():
             for name, v in r["codecs"].items():
                 v["cpu_baseline"] = beside[name]
     hbm = r["hbm"]
+    sp_layer = _kernel_traffic("sparse_persist_kernel")   # ncu DRAM bytes per layer (8-layer capture)
+    sp_traffic = sp_layer * r["layers"] if sp_layer is not None else None
     line = {
         "metric": METRIC, "value": r["metric_us"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": {**config, "context_at_end": r["N"],
                                                                           "k_sel": r["k_sel"]},
-        "roofline": {"bound": "hbm", "kernel": "fl_decode_attn_sparse (loop 4)", "achieved": r["sp_gbs"],
-                     "peak": hbm, "unit": "GB/s", "frac": r["sp_gbs"] / hbm, "traffic": _kernel_traffic("sparse_staged_kernel"),
-                     "peak_kind": peak_kind_str(r["peak_kind"]), "bytes_per_launch": r["sp_bytes"],
-                     "us_per_launch": r["sp_launch_us"]},
+        "roofline": {"bound": "hbm", "kernel": "sparse_persist_kernel (loop 4: one launch for every layer, then "
+                               "its combine)", "achieved": r["sp_gbs"],
+                     "peak": hbm, "unit": "GB/s", "frac": r["sp_gbs"] / hbm, "traffic": sp_traffic,
+                     "peak_kind": peak_kind_str(r["peak_kind"]), "bytes_per_launch": r["sp_bytes"] * r["layers"],
+                     "us_per_launch": r["sp_launch_us"] * r["layers"], "layers_per_launch": r["layers"],
+                     "bytes_per_layer": r["sp_bytes"], "us_per_layer": r["sp_launch_us"]},
         "roofline_dense": {"bound": "hbm", "kernel": "fl_decode_attn_dense (loops 1-2)", "achieved": r["d_gbs"],
                            "peak": hbm, "unit": "GB/s", "frac": r["d_gbs"] / hbm, "traffic": _kernel_traffic("dense_staged_kernel"),
                            "bytes_per_launch": r["d_bytes"], "us_per_launch": r["d_launch_us"]},
