@@ -384,7 +384,8 @@ __device__ __forceinline__ void record_to_limbs(uint32_t* rec, const float* q_s,
   // channels 4l+1, 4l+3 fill bytes 2*(l&1), 2*(l&1)+1 of the word's limb words.
   const int w = lane >> 1, hb = (lane & 1) * 2;
   uint16_t* lh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(rec + kLimbWords * w) + hb);
-  auto pair = [](int a, int b, int sh) { return (uint16_t)(((a >> sh) & 0xff) | (((b >> sh) & 0xff) << 8)); };
+  // byte sh / 8 of a, then the same byte of b (one byte permute)
+  auto pair = [](int a, int b, int sh) { return (uint16_t)__byte_perm(a, b, (unsigned)((sh >> 3) | ((4 + (sh >> 3)) << 4))); };
   lh[0] = pair(Q0, Q2, 0);
   lh[2] = pair(Q0, Q2, 8);
   lh[4] = pair(Q0, Q2, 16);
@@ -434,7 +435,8 @@ __device__ __forceinline__ void record_to_limbs2(uint32_t* ra, uint32_t* rb, con
   }
   __syncwarp();
   const int w = lane >> 1, hb = (lane & 1) * 2;
-  auto pair = [](int a, int b, int sh) { return (uint16_t)(((a >> sh) & 0xff) | (((b >> sh) & 0xff) << 8)); };
+  // byte sh / 8 of a, then the same byte of b (one byte permute)
+  auto pair = [](int a, int b, int sh) { return (uint16_t)__byte_perm(a, b, (unsigned)((sh >> 3) | ((4 + (sh >> 3)) << 4))); };
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     uint16_t* lh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(rec[i] + kLimbWords * w) + hb);

@@ -165,15 +165,9 @@ __device__ __forceinline__ int scan_incl(int v, int lane) {
   return v;
 }
 
-// acc += a * b on two fp32 lanes at once (fma.rn.f32x2: two independent fma.rn)
-__device__ __forceinline__ void ffma2(float2& acc, float2 a, float2 b) {
-  unsigned long long C, A, B;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(C) : "f"(acc.x), "f"(acc.y));
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(C) : "l"(A), "l"(B));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(acc.x), "=f"(acc.y) : "l"(C));
-}
+// acc += a * b on two fp32 lanes at once (two independent round-to-nearest fmas, one
+// packed instruction)
+__device__ __forceinline__ void ffma2(float2& acc, float2 a, float2 b) { acc = __ffma2_rn(a, b, acc); }
 
 // The eight nibbles of a code word (channel 8w + k in nibble k) as exact fp32 values
 // 1 + n/128, in channel pairs: each nibble is shifted to bits 16..19 (mantissa bits below
