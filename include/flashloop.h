@@ -27,20 +27,24 @@
  *   - All data pointers are DEVICE pointers owned by the caller.  The library never
  *     allocates or frees device memory.  Its only process-wide state is (a) per-device
  *     caches filled on a device's first call (its SM count, the kernels' shared-memory
- *     attributes, the address of the array below), each guarded so that host threads
- *     making their first call at once neither race nor repeat it, and (b) the one static
- *     device array of fl_decode_attn_sparse_noalloc (FL_NOALLOC_SCRATCH_BYTES per device
- *     that loads the library).  The caches do not survive cudaDeviceReset or a context
- *     teardown: reload the library after one.
+ *     attributes, the address of the array below, and the stream fl_decode_step_io copies
+ *     its inputs on), each guarded so that host threads making their first call at once
+ *     neither race nor repeat it, and (b) the one static device array of
+ *     fl_decode_attn_sparse_noalloc (FL_NOALLOC_SCRATCH_BYTES per device that loads the
+ *     library).  The caches do not survive cudaDeviceReset or a context teardown: reload
+ *     the library after one.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
- *     enqueues work on it and returns; calls on one cache must be stream-ordered.
+ *     enqueues work and returns (on `stream`, and for fl_decode_step_io's input copy on
+ *     the library's copy stream, ordered after `stream`'s earlier work and before the
+ *     readers that need it); calls on one cache must be stream-ordered.
  *   - BF16 tensors are passed as uint16_t bit patterns.
  *   - Arguments are validated on the host before any launch: a bad value returns
  *     FL_ERR_INVALID / FL_ERR_UNSUPPORTED / FL_ERR_WORKSPACE and enqueues nothing.
  *     A failed launch returns FL_ERR_CUDA.  Data errors found on the device (rows
  *     out of order, sets that do not nest, a selected index out of range) are
  *     recorded in the cache's status words, read with fl_read_status(); kernels
- *     never trap and never spin-wait.
+ *     never trap, and every wait inside a kernel (the readers' mbarrier hand-offs) is
+ *     bounded: after 2 s of device time it records FL_DEV_TIMEOUT and the kernel drains.
  *   - Numbers: codes, scales and zero points are exact (the quantiser below, fp32
  *     with one IEEE rounding per operation); attention runs in fp32 and returns fp32.
  *
@@ -365,10 +369,14 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
  * the device array qkv (BF16 [3][R+1][L][H][128], the same three arrays fl_decode_step takes
  * as q, k_new, v_new) with one 2-D copy, runs those loops, and copies o of those loops
  * (fp32 [loop_last - loop_first + 1][L][H][128]) from the device array o ([R+1][L][H][128])
- * to host_o -- all enqueued on `stream`, nothing waited for.  Host buffers should be pinned
- * (page-locked) for the copies to be asynchronous; read host_o after synchronising the
- * stream.  flush as in fl_decode_step_flush (NULL: none).  Arguments are validated before
- * anything is enqueued. */
+ * to host_o -- nothing waited for on the host.  The input copy runs on a stream the library
+ * creates once per device, after all work enqueued on `stream` before the call and beside
+ * the first loop's selection (which reads no query); the first reader waits for it, and the
+ * output copy follows the last loop on `stream`.  Host buffers should be pinned
+ * (page-locked) for the copies to be asynchronous; read host_o after synchronising
+ * `stream`.  Calls from several host threads share the copy stream (their copies run one
+ * after another).  flush as in fl_decode_step_flush (NULL: none).  Arguments are validated
+ * before anything is enqueued. */
 fl_status fl_decode_step_io(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
                             int32_t k_sel, int32_t loop_first, int32_t loop_last, uint16_t* qkv, const uint16_t* host_qkv,
                             float* o, float* host_o, void* ws, size_t ws_bytes, void* const* events,

@@ -478,10 +478,14 @@ fl_status fl_decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t 
                               o, ws, ws_bytes, events, nullptr, stream);
 }
 
-fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
-                               int32_t k_sel, int32_t loop_first, int32_t loop_last, const uint16_t* q,
-                               const uint16_t* k_new, const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,
-                               void* const* events, const fl_flush* flush, void* stream) {
+namespace {
+// The executor behind fl_decode_step_flush and fl_decode_step_io: with `inputs_ready`, the
+// stream waits on that event before its first reader (the selection before it reads no
+// query), so a host -> device copy of the inputs can overlap the loop's selection.
+fl_status decode_step(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
+                      int32_t k_sel, int32_t loop_first, int32_t loop_last, const uint16_t* q, const uint16_t* k_new,
+                      const uint16_t* v_new, float* o, void* ws, size_t ws_bytes, void* const* events,
+                      const fl_flush* flush, void* stream, cudaEvent_t inputs_ready, bool validate_only = false) {
   fl_status st = check_reader(dims, cache, 0, 1, n_q, n_tail, q, k_new, v_new, o, ws, ws_bytes);
   if (st != FL_OK) return st;
   const int R = dims->loops, L = dims->layers, H = dims->heads;
@@ -514,6 +518,7 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
       if (st != FL_OK) return st;
     }
   }
+  if (validate_only) return FL_OK;
   fl_layout lay;
   make_layout(dims, &lay);
   cudaStream_t s = (cudaStream_t)stream;
@@ -521,6 +526,11 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
   const size_t ostride_r = (size_t)L * row;                // elements between loops
   auto rec = [&](int i) -> bool {
     return !events || cudaEventRecord((cudaEvent_t)events[i], s) == cudaSuccess;
+  };
+  auto wait_inputs = [&]() -> bool {
+    const bool ok = !inputs_ready || cudaStreamWaitEvent(s, inputs_ready, 0) == cudaSuccess;
+    inputs_ready = nullptr;
+    return ok;
   };
   ReaderArgs a{};
   a.c = make_view(dims, lay, cache);
@@ -540,6 +550,7 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
     if (r <= dense_loops) {
       if (!rec(2 * r - 1)) return FL_ERR_CUDA;
       a.keep = r == dense_loops ? 1 : 0;
+      if (!wait_inputs()) return FL_ERR_CUDA;
       for (int l = 0; l < L; ++l) {
         const size_t qo = (size_t)r * ostride_r + (size_t)l * row;
         a.layer = l;
@@ -561,6 +572,7 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
       sa.k_sel = k_sel;
       if (launch_select(sa, L, s) != cudaSuccess) return FL_ERR_CUDA;
       if (!rec(2 * r - 1)) return FL_ERR_CUDA;
+      if (!wait_inputs()) return FL_ERR_CUDA;
       a.keep = 1;
       if (dims->codec == FL_CODEC_RESIDUAL_INT4 && r <= kPersistMaxLoop) {
         // every layer of the loop through the persistent reader: one launch (per
@@ -604,6 +616,20 @@ fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, in
   return FL_OK;
 }
 
+// per device, the stream fl_decode_step_io copies its inputs on (created on first use)
+std::atomic<bool> g_side_done[kMaxDevices];
+std::mutex g_side_mu;
+cudaStream_t g_side[kMaxDevices];
+}  // namespace
+
+fl_status fl_decode_step_flush(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
+                               int32_t k_sel, int32_t loop_first, int32_t loop_last, const uint16_t* q,
+                               const uint16_t* k_new, const uint16_t* v_new, float* o, void* ws, size_t ws_bytes,
+                               void* const* events, const fl_flush* flush, void* stream) {
+  return decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, k_new, v_new, o, ws,
+                     ws_bytes, events, flush, stream, nullptr);
+}
+
 fl_status fl_decode_step_io(const fl_dims* dims, void* cache, int32_t n_q, int32_t n_tail, int32_t dense_loops,
                             int32_t k_sel, int32_t loop_first, int32_t loop_last, uint16_t* qkv, const uint16_t* host_qkv,
                             float* o, float* host_o, void* ws, size_t ws_bytes, void* const* events,
@@ -619,16 +645,37 @@ fl_status fl_decode_step_io(const fl_dims* dims, void* cache, int32_t n_q, int32
   uint16_t* kn = qkv + (size_t)(R + 1) * slice;
   uint16_t* vn = qkv + (size_t)2 * (R + 1) * slice;
   cudaStream_t s = (cudaStream_t)stream;
-  // validate the whole step before anything is enqueued: a step with the same arguments and
-  // no copies must be acceptable (fl_decode_step_flush validates before launching)
-  st = check_reader(dims, cache, 0, 1, n_q, n_tail, q, kn, vn, o, ws, ws_bytes);
+  // validate the whole step before anything is enqueued
+  st = decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, kn, vn, o, ws, ws_bytes,
+                   events, flush, stream, nullptr, true);
   if (st != FL_OK) return st;
-  // q, k_new, v_new of loops loop_first..loop_last: three equally spaced device rows
-  if (cudaMemcpy2DAsync(q + (size_t)loop_first * slice, (size_t)(R + 1) * slice * 2, host_qkv, nl * slice * 2,
-                        nl * slice * 2, 3, cudaMemcpyHostToDevice, s) != cudaSuccess)
+  // q, k_new, v_new of loops loop_first..loop_last (three equally spaced device rows) are
+  // copied on a side stream once the stream's earlier work is done, beside the first
+  // loop's selection; the first reader waits for them
+  if (once_per_device(g_side_done, g_side_mu, [](int dev) {
+        return cudaStreamCreateWithFlags(&g_side[dev], cudaStreamNonBlocking);
+      }) != cudaSuccess)
     return FL_ERR_CUDA;
-  st = fl_decode_step_flush(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, kn, vn, o, ws,
-                            ws_bytes, events, flush, stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FL_ERR_CUDA;
+  const cudaStream_t side = g_side[dev];
+  cudaEvent_t ev_start = nullptr, ev_copied = nullptr;
+  auto release = [&]() {
+    if (ev_start) cudaEventDestroy(ev_start);
+    if (ev_copied) cudaEventDestroy(ev_copied);
+  };
+  if (cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_copied, cudaEventDisableTiming) != cudaSuccess || cudaEventRecord(ev_start, s) != cudaSuccess ||
+      cudaStreamWaitEvent(side, ev_start, 0) != cudaSuccess ||
+      cudaMemcpy2DAsync(q + (size_t)loop_first * slice, (size_t)(R + 1) * slice * 2, host_qkv, nl * slice * 2,
+                        nl * slice * 2, 3, cudaMemcpyHostToDevice, side) != cudaSuccess ||
+      cudaEventRecord(ev_copied, side) != cudaSuccess) {
+    release();
+    return FL_ERR_CUDA;
+  }
+  st = decode_step(dims, cache, n_q, n_tail, dense_loops, k_sel, loop_first, loop_last, q, kn, vn, o, ws, ws_bytes,
+                   events, flush, stream, ev_copied);
+  release();  // destroyed once their work is done
   if (st != FL_OK) return st;
   if (cudaMemcpyAsync(host_o, o + (size_t)loop_first * slice, nl * slice * sizeof(float), cudaMemcpyDeviceToHost,
                       s) != cudaSuccess)
