@@ -487,8 +487,8 @@ def run_token_select(w, device, hbm, reps=5):
 
 
 def run_encode(w, device, hbm, reps=5):
-    """The prefill encode of one 16-head layer of the workload's prompt (BASELINE
-    configuration 2's prefill): the base encoder over every quantised token, then the
+    """The prefill encode of one 16-head layer of a 32K-token prompt (the layer that then
+    decodes 256 tokens): the base encoder over every quantised token, then the
     residual encoder of loops 2..R over their active rows, each timed with CUDA events on the
     launch stream (a repetition re-encodes the same rows; inputs of 0.5 GB, larger than L2)."""
     from quantized_kv_attention_int4_b200 import abi
@@ -540,10 +540,10 @@ def run_encode(w, device, hbm, reps=5):
 
 
 def run_deep(device, hbm, warmup=3, steps=10):
-    """BASELINE configuration 4 (one 16-head layer at N = 8192, R = 32 loops, geometric
+    """The 32-loop workload (one 16-head layer at N = 8192, R = 32 loops, geometric
     retention, 10 % key retention from loop 3): whole decode steps through the step
     executor with per-loop CUDA events, the algorithmic bytes of each loop taken from an
-    untimed calibration step's selections; the loops <= 8 run the batched sparse reader,
+    untimed calibration step's selections; the loops <= 8 run the persistent sparse reader,
     loops 9..32 the direct one.  Plus the dense reader at loop 32 alone (the direct dense
     form: every column with its residual rows of loops 2..32)."""
     w = synth.WORKLOADS["deep_r32_h16_n8192"]

@@ -39,8 +39,8 @@ def _assert_errs(errs, tol=TOL):
 
 
 def test_full_cache_48_layers_sampled_layers_across_flushes():
-    """BASELINE configuration 3 (Ouro-2.6B-shaped: 48 layers x 16 heads x 128, 32K context,
-    R = 4, per-layer seeds): the bench's own cache and executor."""
+    """The 48-layer cache (Ouro-2.6B-shaped: 48 layers x 16 heads x 128, 32K context, R = 4,
+    per-layer seeds): the bench's own cache and executor."""
     w = W["cache_l48_h16_n32768"]
     L, R = w.layers, w.loops
     steps = 65
@@ -108,7 +108,7 @@ def test_full_cache_48_layers_sampled_layers_across_flushes():
 
 
 def test_layer_32k_prefill_and_256_decode_steps():
-    """BASELINE configuration 2: one 16-head layer at 32K, prefill encode, then 256 decode
+    """One 16-head layer at 32K: prefill encode, then 256 decode
     steps through the step executor (the prompt's full tail flushed by the encoders at the
     first token, then a fused flush whenever the tail fills: steps 63, 127, 191, 255)."""
     w = W["layer_h16_n32768_decode256"]
@@ -131,7 +131,7 @@ def test_layer_32k_prefill_and_256_decode_steps():
 
 
 def test_deep_loops_every_column_selected_needs_many_splits():
-    """BASELINE configuration 4's shape (R = 32, N = 8192) with K_sel = N: a CTA of the
+    """The 32-loop workload's shape (R = 32, N = 8192) with K_sel = N: a CTA of the
     loop > 8 reader holds at most 28 of the 36-word plan entries, so it needs ~293 split-K
     partitions per head (the loop <= 8 reader holds 56: ~147).  Every sparse loop must then
     equal the dense attention of its loop (m = 1)."""
