@@ -114,11 +114,23 @@ constexpr int kCols1 = 49152;         // the keys of one head that fit it
 __host__ __device__ inline bool sel_fits1(int N, int K) {
   return ((size_t)((N + 3) & ~3) + (size_t)K) * sizeof(uint32_t) <= (size_t)kDynMax1;
 }
+// The head's scores and tags are staged in shared memory by two bulk copies (the scores in
+// the key array, turned into keys in place; the tags after it), with the selected columns
+// after those, when all three fit.
+__host__ __device__ inline size_t stage_bytes1(int N, int K) {
+  return (size_t)((N + 3) & ~3) * sizeof(uint32_t) + (size_t)((N + 15) & ~15) + (size_t)K * sizeof(int32_t);
+}
+__host__ __device__ inline bool stage_fits1(int N, int K) { return stage_bytes1(N, K) <= (size_t)kDynMax1; }
 
 __global__ void __launch_bounds__(kThreads1, 1) select_cta_kernel(SelectArgs a) {
-  extern __shared__ uint32_t keys[];  // [N] keys, then [K] selected columns when they fit
-  const bool sel_smem = sel_fits1(a.n_q + a.n_tail, a.k_sel);
-  int32_t* sel_s = reinterpret_cast<int32_t*>(keys + ((a.n_q + a.n_tail + 3) & ~3));
+  // [N] keys, then (staged) the N tags, then [K] selected columns when they fit
+  extern __shared__ __align__(16) uint32_t keys[];
+  const bool staged = stage_fits1(a.n_q + a.n_tail, a.k_sel);
+  const bool sel_smem = staged || sel_fits1(a.n_q + a.n_tail, a.k_sel);
+  uint8_t* tag_s = reinterpret_cast<uint8_t*>(keys + ((a.n_q + a.n_tail + 3) & ~3));
+  int32_t* sel_s = staged ? reinterpret_cast<int32_t*>(tag_s + ((a.n_q + a.n_tail + 15) & ~15))
+                          : reinterpret_cast<int32_t*>(keys + ((a.n_q + a.n_tail + 3) & ~3));
+  __shared__ uint64_t stage_bar;
   __shared__ __align__(16) uint32_t hist[8192];
   __shared__ float offs[kOffStride];
   __shared__ uint32_t wtot[32];
@@ -136,9 +148,29 @@ __global__ void __launch_bounds__(kThreads1, 1) select_cta_kernel(SelectArgs a) 
   int32_t* sel = arr<int32_t>(c, A_SEL, layer) + (size_t)h * c.max_select;
 
   if (tid < kOffStride) offs[tid] = arr<float>(c, A_OFFSET, layer)[(size_t)h * kOffStride + tid];
+  if (staged && tid == 0) {
+    mbar_init(&stage_bar, 1);
+    fence_mbar_init();
+  }
   __syncthreads();
+  if (staged) {
+    // the head's scores and tags in two bulk copies (rows start 256-byte aligned: cap is a
+    // multiple of 64; the copies round up to 16 bytes, within the row's capacity)
+    if (tid == 0) {
+      const unsigned sb = (unsigned)(((N + 3) & ~3) * sizeof(float)), tb = (unsigned)((N + 15) & ~15);
+      mbar_expect_tx(&stage_bar, sb + tb);
+      bulk_g2s(keys, score, sb, &stage_bar);
+      bulk_g2s(tag_s, tag, tb, &stage_bar);
+    }
+    const bool ok = mbar_wait(&stage_bar, 0);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) record_error(c.status, FL_DEV_TIMEOUT, blockIdx.y * gridDim.x + blockIdx.x);
+      return;
+    }
+  }
   // keys, four columns per thread per step (score rows are 16-byte and tag rows 4-byte
-  // aligned: cap is a multiple of 64); loads of several steps are in flight together
+  // aligned: cap is a multiple of 64); from the staged copies, or from global memory with
+  // the loads of several steps in flight together
   auto key_of = [&](float sc, int t, int j) {
     if (t < 1 || t > R) {
       record_error(c.status, FL_DEV_TAG_RANGE, j);
@@ -148,24 +180,32 @@ __global__ void __launch_bounds__(kThreads1, 1) select_cta_kernel(SelectArgs a) 
   };
   const int N4 = N & ~3;
   uint32_t kand = 0xffffffffu, kor = 0u;  // bits common to every key
-#pragma unroll 4
-  for (int j = 4 * tid; j < N4; j += 4 * kThreads1) {
-    const float4 sc = *reinterpret_cast<const float4*>(score + j);
-    const uint32_t tg = *reinterpret_cast<const uint32_t*>(tag + j);
+  auto keys4 = [&](int j, float4 sc, uint32_t tg) {  // columns j .. j + 3 into keys[j .. j + 3]
     const uint32_t k0 = key_of(sc.x, (int)(tg & 0xff), j), k1 = key_of(sc.y, (int)((tg >> 8) & 0xff), j + 1);
     const uint32_t k2 = key_of(sc.z, (int)((tg >> 16) & 0xff), j + 2), k3 = key_of(sc.w, (int)(tg >> 24), j + 3);
-    keys[j] = k0;
-    keys[j + 1] = k1;
-    keys[j + 2] = k2;
-    keys[j + 3] = k3;
+    *reinterpret_cast<uint4*>(keys + j) = make_uint4(k0, k1, k2, k3);
     kand &= k0 & k1 & k2 & k3;
     kor |= k0 | k1 | k2 | k3;
-  }
-  for (int j = N4 + tid; j < N; j += kThreads1) {
-    const uint32_t k = key_of(score[j], tag[j], j);
-    keys[j] = k;
-    kand &= k;
-    kor |= k;
+  };
+  if (staged) {
+    for (int j = 4 * tid; j < N4; j += 4 * kThreads1)  // each thread turns its own scores into keys
+      keys4(j, *reinterpret_cast<const float4*>(keys + j), *reinterpret_cast<const uint32_t*>(tag_s + j));
+    for (int j = N4 + tid; j < N; j += kThreads1) {
+      const uint32_t k = key_of(__uint_as_float(keys[j]), tag_s[j], j);
+      keys[j] = k;
+      kand &= k;
+      kor |= k;
+    }
+  } else {
+#pragma unroll 4
+    for (int j = 4 * tid; j < N4; j += 4 * kThreads1)
+      keys4(j, *reinterpret_cast<const float4*>(score + j), *reinterpret_cast<const uint32_t*>(tag + j));
+    for (int j = N4 + tid; j < N; j += kThreads1) {
+      const uint32_t k = key_of(score[j], tag[j], j);
+      keys[j] = k;
+      kand &= k;
+      kor |= k;
+    }
   }
   kand = __reduce_and_sync(kFull, kand);
   kor = __reduce_or_sync(kFull, kor);
@@ -622,7 +662,9 @@ cudaError_t launch_select(const SelectArgs& a, int n_layers, cudaStream_t s) {
   int want = 1;
   while (want < kClusterMax && heads_all * want < sms) want *= 2;
   if (N <= kCols1) {
-    const size_t smem = ((size_t)((N + 3) & ~3) + (sel_fits1(N, a.k_sel) ? (size_t)a.k_sel : 0)) * sizeof(uint32_t);
+    const size_t smem = stage_fits1(N, a.k_sel)
+                            ? stage_bytes1(N, a.k_sel)
+                            : ((size_t)((N + 3) & ~3) + (sel_fits1(N, a.k_sel) ? (size_t)a.k_sel : 0)) * sizeof(uint32_t);
     cudaError_t e = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynMax1);
     if (e != cudaSuccess) return e;
     select_cta_kernel<<<dim3(a.c.H, n_layers), kThreads1, smem, s>>>(a);
