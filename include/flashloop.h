@@ -317,7 +317,9 @@ fl_status fl_decode_attn_sparse_noalloc(const fl_dims* dims, void* cache, int32_
  * loops up to dense_loops call the dense reader (the last dense loop keeps scores);
  * every later loop first selects k_sel columns for all layers in one launch
  * (fl_select_topk) and then runs each layer's sparse reader with o_prev = that
- * layer's output of the previous loop.  Same arguments and semantics as the individual calls; validated once.
+ * layer's output of the previous loop (for the 4-bit residual codec and loops <= 8,
+ * one persistent launch covers every layer, then one combine launch).  Same arguments
+ * and semantics as the individual calls; validated once.
  *   q, k_new, v_new: BF16 [R+1][L][H][128] (slice r = loop r, slice 0 unused;
  *                    k_new/v_new may be NULL)
  *   o: fp32 [R+1][L][H][128]   (o[r] = loop r's outputs; o[loop_first-1] must hold the

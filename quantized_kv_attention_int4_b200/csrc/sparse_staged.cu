@@ -1,5 +1,7 @@
-// Sparse decode reader, staged form (loops r <= 8): loop-aware sparse attention over
-// the selected columns S.
+// Sparse decode reader, staged form: loop-aware sparse attention over the selected
+// columns S for loops r <= 8 of the codec variants (per-loop KIVI4 full state, INT2
+// residuals); the method's 4-bit residual stores take the persistent reader
+// (sparse_persist.cu).
 //
 // FlashLoop project page, "The Method", Step 02: a sparse loop recomputes attention
 // only for the columns chosen from the preceding loop and keeps their global
@@ -10,7 +12,7 @@
 // with m = sum_{j in S} p~_j.  u and m are formed from the rows this pass gathers
 // anyway (a column's value at loop tag_j is a prefix of its rows at loop r).
 //
-// Work split: grid (splits, heads), three CTAs of 4 warps per SM.  The CTA copies its
+// Work split: grid (splits, heads), three CTAs of 5 warps per SM.  The CTA copies its
 // part of the gather plan (column, tag, stores, p~, residual slots; written by the
 // selector) into shared memory; each warp walks its own run of columns span by span.
 // A span is up to 32 consecutive columns, cut so that it holds at most kMaxRows rows
@@ -690,8 +692,7 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s, bool chain) {
   const int n = sparse_launch_splits(a.c.H, a.c.R, a.c.codec, a.r, a.k_sel, sms, a.flush != 0);
   if (a.r > kStoresMax || sms == 0 || n > kMaxSplits) return launch_sparse_direct(a, s, chain);
   const cudaError_t e = once_per_device(g_attr_done, g_attr_mu, [](int) {
-    for (auto k : {sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>, sparse_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>,
-                   sparse_staged_kernel<false, FL_CODEC_FULL_INT4>, sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>}) {
+    for (auto k : {sparse_staged_kernel<false, FL_CODEC_FULL_INT4>, sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>}) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCta);
       if (e != cudaSuccess) return e;
       e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -702,10 +703,10 @@ cudaError_t launch_sparse(ReaderArgs a, cudaStream_t s, bool chain) {
   if (e != cudaSuccess) return e;
   a.n_splits = n;
   dim3 grid(n, a.c.H);
-  auto kern = a.c.codec == FL_CODEC_FULL_INT4       ? sparse_staged_kernel<false, FL_CODEC_FULL_INT4>
-              : a.c.codec == FL_CODEC_RESIDUAL_INT2 ? sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>
-              : a.flush                             ? sparse_staged_kernel<true, FL_CODEC_RESIDUAL_INT4>
-                                                    : sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT4>;
+  // the variants only (the method's 4-bit residuals went to the persistent reader above;
+  // the variants never take the fused flush)
+  auto kern = a.c.codec == FL_CODEC_FULL_INT4 ? sparse_staged_kernel<false, FL_CODEC_FULL_INT4>
+                                              : sparse_staged_kernel<false, FL_CODEC_RESIDUAL_INT2>;
   return launch_pdl_if(chain, kern, grid, dim3(kNT), (size_t)kSmemCta, s, a);
 }
 
