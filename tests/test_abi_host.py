@@ -109,6 +109,17 @@ def test_reader_arguments_are_validated_before_launch():
     assert step(dl=0, lf=1) == abi.FL_ERR_INVALID         # first loop cannot be sparse
     big = _dims(capacity=385024 + 128, max_select=10)
     assert abi._c_select(ctypes.byref(big), FAKE, 0, 1, 3, 385024, 1, 10, None) == abi.FL_ERR_UNSUPPORTED
+    # the host-buffer step validates the whole step (the same rules) before any copy is enqueued
+    step_io = lambda **k: abi._c_step_io(ctypes.byref(d), FAKE, 64, 1, k.get("dl", 2), k.get("k_sel", 10),
+                                         k.get("lf", 1), k.get("ll", 4), k.get("qkv", FAKE), k.get("hq", FAKE),
+                                         FAKE, k.get("ho", FAKE), FAKE, ws, None, None, None)
+    assert step_io(dl=5) == abi.FL_ERR_INVALID
+    assert step_io(lf=3, ll=2) == abi.FL_ERR_INVALID
+    assert step_io(k_sel=0) == abi.FL_ERR_INVALID
+    assert step_io(dl=0, lf=1) == abi.FL_ERR_INVALID
+    assert step_io(qkv=None) == abi.FL_ERR_INVALID
+    assert step_io(hq=None) == abi.FL_ERR_INVALID
+    assert step_io(ho=None) == abi.FL_ERR_INVALID
 
 
 def test_encoder_arguments_are_validated_before_launch():
