@@ -90,8 +90,7 @@ struct ItemInfo {
 
 struct alignas(16) CtaB {
   ItemInfo item[2];
-  float4 wrow[kRowsMax][2];            // per row: (wS0, wS0, wU0, wU0), the same for half 1;
-                                       // at an item's end, the warps' merge area
+  float4 wrow[kRowsMax][2];            // per row: (wS0, wS0, wU0, wU0), the same for half 1
   float lr[kRowsMax];                  // per row: logit part
   float lcol[kBCols];                  // per column of the batch: logit (-inf: no quantised column)
   float wmax[kCW];                     // per warp: maximum logit of its columns of the batch
@@ -108,7 +107,6 @@ constexpr int kCtaB = (int)((sizeof(CtaB) + 127) / 128 * 128);
 constexpr int kTabB = (int)((sizeof(BatchTab) + 15) / 16 * 16);
 constexpr int kSmemP = kCtaB + 2 * kItemWords * 4 + kTabs * kTabB + 2 * kBufB;
 static_assert(kSmemP <= 113 * 1024, "two CTAs per SM");
-static_assert((int)sizeof(CtaB::wrow) >= kCW * kD * 4, "the merge area holds one sum of every warp");
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
